@@ -1,0 +1,382 @@
+"""Benchmark of the LaCT fast-weight TTT layer forward on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload IDX] [--impl ours|reference]
+
+A step is one full layer forward (every chunk: apply, chunk gradient, rule,
+renorm) over one batch of synthetic inputs already resident in HBM.  The
+default workload is the 760M-shaped language-model layer at 32K context
+(B=2, H=6, d=256, dh=512, chunk 2048, GD, bf16).  Inputs (q, k, v: 604 MB)
+are larger than the 126 MB L2, so no flush is needed between steps.
+With N > 1 (torchrun) every rank runs its own batch (independent problems,
+no data-path collective: weak scaling); time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload (one full-length (batch, head) sequence per step) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from lact_inputs import BF16, RULE_MUON, WORKLOADS, Workload, make_inputs  # noqa: E402
+
+METRIC = "TTT-layer tokens/s (fwd) at 1 B200 and % of bf16 tensor-core peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = 2
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- algorithmic work
+def step_flops(w: Workload) -> float:
+    """18 d dh FLOPs per key token per head (4 forward on k, 2 for W2^T v, 6 for
+    the three gradients) + 6 d dh per query token (apply), plus Newton-Schulz."""
+    per_head = 12.0 * w.d * w.dh * w.T + 6.0 * w.d * w.dh * w.Tq
+    if w.rule == RULE_MUON:
+        m, p = min(w.d, w.dh), max(w.d, w.dh)
+        per_head += w.n_chunks * 3 * 5 * (4.0 * m * m * p + 2.0 * m ** 3)
+    return per_head * w.B * w.H
+
+
+def kernel_work(w: Workload):
+    """Algorithmic work per kernel kind over one step: (bound, amount, unit).
+    FLOPs count 2 per multiply-add; bytes count each tensor read or written once."""
+    BH, d, dh, T, Tq = w.B * w.H, w.d, w.dh, w.T, w.Tq
+    esz = 2 if w.dtype == BF16 else 4
+    ns = 3 * 5 * w.n_chunks * BH if w.rule == RULE_MUON else 0   # NS matrix-iterations
+    planes = 3 * BH * d * dh
+    return {
+        "fwd_query_umma": ("tensor", 4.0 * Tq * d * dh * BH, "FLOP"),
+        "apply_out_umma": ("tensor", 2.0 * Tq * d * dh * BH, "FLOP"),
+        "fwd_key_umma": ("tensor", 6.0 * T * d * dh * BH, "FLOP"),
+        "grad_umma": ("tensor", 6.0 * T * d * dh * BH, "FLOP"),
+        "ns_gram_umma": ("tensor", 2.0 * d * d * dh * ns, "FLOP"),
+        "ns_poly_umma": ("tensor", 2.0 * d ** 3 * ns, "FLOP"),
+        "ns_update_umma": ("tensor", 2.0 * dh * d * d * ns, "FLOP"),
+        "qk_prologue": ("hbm", 2.0 * (Tq + T) * d * esz * BH, "B"),
+        "rule_renorm": ("hbm", w.n_chunks * planes * (4 + 4 + 4 + 2), "B"),
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx.append(float(r[1]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, r[4:8]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w: Workload, inp: dict, budget_s: float, max_heads: int):
+    """Runs the oracle on whole (batch, head) sequences until `budget_s`
+    seconds have passed (at least one).  Returns (tokens, seconds, heads)."""
+    import oracle
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)][:max_heads]
+    tokens, t0, done = 0, time.perf_counter(), 0
+    for b, h in heads:
+        oracle.ttt_layer(inp["q"], inp["k"], inp["v"], inp["lr"], inp["beta"], inp["w1"],
+                         inp["w2"], inp["w3"], w.chunk, w.order, w.rule, heads=[(b, h)])
+        tokens += w.tokens // (w.B * w.H)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return tokens, time.perf_counter() - t0, done
+
+
+def blas_threads():
+    import oracle
+    return oracle.blas_threads()
+
+
+# ---------------------------------------------------------------- helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def workload_config(w: Workload, n_gpus: int) -> dict:
+    in_bytes = (w.B * w.H * (w.Tq + 2 * w.T) * w.d) * (2 if w.dtype == BF16 else 4)
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "Tq": w.Tq, "d": w.d, "dh": w.dh,
+            "chunk": w.chunk, "order": ["apply_then_update", "update_then_apply"][w.order],
+            "rule": ["gd", "momentum", "muon"][w.rule], "tokens_per_step_per_gpu": w.tokens,
+            "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single",
+            "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB > 126 MB), no flush"}
+
+
+def run_reference(args, w: Workload):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = make_inputs(w, seed=0)
+    cores = blas_threads()
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        tok, sec, _ = oracle_sample(w, inp, budget_s=0.0, max_heads=1)
+        if i >= args.warmup:
+            per_step.append((tok, sec))
+    tokens = sum(t for t, _ in per_step)
+    secs = sum(s for _, s in per_step)
+    value = tokens / secs
+    sample = f"one (batch, head) sequence of {w.T} key tokens per step (of {w.B * w.H})"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import chunk_test_b200 as ct
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier_max(x: float) -> float:
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    inp_cpu = make_inputs(w, seed=rank)
+    inp = {k: (None if v is None else v.to(dev)) for k, v in inp_cpu.items()}
+    B, H = w.B, w.H
+    out = torch.empty_like(inp["q"])
+    w_out = (torch.empty((B * H, w.dh, w.d), device=dev), torch.empty((B * H, w.d, w.dh), device=dev),
+             torch.empty((B * H, w.dh, w.d), device=dev))
+    ws = torch.empty(ct.workspace_bytes(inp["q"], inp["k"], inp["w1"], w.chunk, w.order, w.rule),
+                     device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ct.ttt_fwd(inp["q"], inp["k"], inp["v"], inp["lr"], inp["beta"], inp["w1"], inp["w2"],
+                   inp["w3"], w.chunk, w.order, w.rule, out=out, w_out=w_out, workspace=ws,
+                   stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after warm-up")
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    ct.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ct.profile_enable(False)
+    clk = clocks.stop()
+    ms_total = barrier_max(e0.elapsed_time(e1))
+    prof = ct.profile_read()
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after the timed region")
+
+    ms_step = ms_total / args.steps
+    tok_step = w.tokens
+    value = world * tok_step * args.steps / (ms_total / 1e3)
+    hbm, pk_burst, pk_sust, pk_src = peaks()
+    flops = step_flops(w)
+    launches_per_step = ct.launch_count(inp["q"], inp["k"], inp["w1"], w.chunk, w.order, w.rule)
+
+    # ---- roofline of the dominant kernel
+    work = kernel_work(w)
+    dom = max(prof.items(), key=lambda kv: kv[1][1])
+    name, (n_launch, ms_kind) = dom
+    roof = None
+    if name in work:
+        bound, amount, unit = work[name]
+        per_launch = amount * args.steps / n_launch
+        dur_s = ms_kind / n_launch / 1e3
+        if bound == "tensor":
+            achieved = per_launch / dur_s / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
+                    "frac": achieved / pk_sust}
+        else:
+            achieved = per_launch / dur_s / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm}
+        roof.update({"kernel": name, "launches": n_launch, "avg_launch_us": 1e3 * ms_kind / n_launch,
+                     "traffic": traffic_for(name, w), "peak_source": f"{pk_src} sustained bf16"
+                     if bound == "tensor" else f"{pk_src} copy bandwidth"})
+    kernels = {k: {"launches": v[0], "ms": round(v[1], 4),
+                   "share": round(v[1] / sum(x[1] for x in prof.values()), 4)}
+               for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+
+    # ---- end to end: host buffers in, results back, through the C ABI
+    pin = {k: (None if v is None else v.pin_memory()) for k, v in inp_cpu.items()}
+    hout = torch.empty_like(inp_cpu["q"]).pin_memory()
+    hwo = tuple(torch.empty(t.shape, dtype=torch.float32).pin_memory() for t in w_out)
+    hws = torch.empty(ct.host_workspace_bytes(pin["q"], pin["k"], pin["w1"], w.chunk, w.order,
+                                              w.rule), device=dev, dtype=torch.uint8)
+    del ws
+
+    def host_step():
+        ct.ttt_fwd_host(pin["q"], pin["k"], pin["v"], pin["lr"], pin["beta"], pin["w1"], pin["w2"],
+                        pin["w3"], w.chunk, w.order, w.rule, out=hout, w_out=hwo, workspace=hws,
+                        stream=stream)
+
+    for _ in range(args.warmup):
+        host_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for _ in range(args.steps):
+        host_step()
+    h1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = barrier_max(h0.elapsed_time(h1))
+    h2d = sum(t.numel() * t.element_size() for t in pin.values() if t is not None)
+    d2h = hout.numel() * hout.element_size() + sum(t.numel() * 4 for t in hwo)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == BF16 else "f32",
+        "data": "synthetic (seeded normal q/k/v, softplus lr, random-init fast weights)",
+        "config": workload_config(w, world),
+        "tensor_peak_frac": {"algorithmic_tflops": flops / (ms_step / 1e3) / 1e12,
+                             "frac_of_sustained": flops / (ms_step / 1e3) / 1e12 / pk_sust,
+                             "frac_of_burst": flops / (ms_step / 1e3) / 1e12 / pk_burst,
+                             "peak_source": pk_src},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": world * tok_step * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk,
+    }
+    if world == 1 and rank == 0:
+        tok, sec, nh = oracle_sample(w, inp_cpu, args.cpu_budget, max_heads=w.B * w.H)
+        line["cpu_baseline"] = {"value": tok / sec, "unit": UNIT, "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{nh} of {w.B * w.H} (batch, head) sequences, "
+                                          f"{tok} tokens, {sec:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def traffic_for(kernel: str, w: Workload):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
+    was taken on this workload with the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    r = rec.get(f"{kernel}@{w.name}")
+    if not r or r.get("source_hash") != source_hash():
+        return None
+    return r.get("bytes_per_launch")
+
+
+def source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "chunk_test_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    sys.exit(main())

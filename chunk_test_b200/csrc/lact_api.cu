@@ -1,0 +1,777 @@
+// lact_api.cu -- C ABI of the LaCT fast-weight TTT layer forward (see
+// include/lact.h): argument checks, the workspace plan, TMA tensor maps and
+// the per-chunk launch sequence on the caller's stream.
+//
+// Per chunk c (tokens [c0, c0 + nc)), in the order the problem asks for
+// ("LaCT：以大分块更新…" 「更新顺序必须遵守信息可见范围」):
+//   apply  : FwdOp<query>  Hq = silu(q^ W1^T) * (q^ W3^T)
+//            GemmOp        out_c = Hq W2^T
+//   update : FwdOp<key>    E1, Eh, E3 (per-token gradient factors, lr-scaled)
+//            GemmOp        -G_j = E_j^T X_j   (X = k^, v, k^), split over tokens
+//            [Muon]        X0 = -G/||G||, 5 x (A = X^T X; B = bA + cA^2;
+//                          X = aX + XB) on the d-side Gram matrix
+//            k_rule_renorm W <- renorm(W - U)
+// The fp32 path runs the same sequence with CUDA-core kernels.
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/lact.h"
+#include "elem_kernels.cuh"
+#include "simt_kernels.cuh"
+#include "sm100.cuh"
+#include "umma_kernels.cuh"
+
+namespace lact {
+
+static inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+static inline int64_t rup(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+
+constexpr float kNsA = 3.4445f, kNsB = -4.7750f, kNsC = 2.0315f;
+constexpr int kNsSteps = 5;
+constexpr float kNsEps = 1e-7f;
+constexpr int kNsBlocks = 16;  // partial-sum blocks per matrix for ||G||_F
+
+struct Dims {
+  int64_t B, H, BH, T, Tq, d, dh, chunk, nch;
+  int order, rule, dtype, w_shared;
+  int64_t key_rows;  // rows per head of the per-chunk key buffers (E / Z)
+  int64_t q_rows;    // rows per head of the per-chunk query buffer (Hq)
+  int splits;        // token splits of the gradient contraction (bf16)
+  int bn;            // N tile over d (bf16 GEMMs)
+};
+
+static int choose_bn(int64_t d) {
+  if (d <= 256) return static_cast<int>(d);
+  if (d % 256 == 0) return 256;
+  if (d % 192 == 0) return 192;
+  if (d % 128 == 0) return 128;
+  return 64;
+}
+
+static int validate(const lact_problem* p, Dims& D) {
+  if (!p) return LACT_EINVAL;
+  if (p->B < 1 || p->H < 1 || p->T < 1 || p->Tq < 1 || p->d < 1 || p->dh < 1 || p->chunk < 1)
+    return LACT_EINVAL;
+  if (p->order != LACT_APPLY_THEN_UPDATE && p->order != LACT_UPDATE_THEN_APPLY) return LACT_EINVAL;
+  if (p->rule < LACT_RULE_GD || p->rule > LACT_RULE_MUON) return LACT_EINVAL;
+  if (p->dtype != LACT_F32 && p->dtype != LACT_BF16) return LACT_EINVAL;
+  if (p->w_shared != 0 && p->w_shared != 1) return LACT_EINVAL;
+  D.B = p->B; D.H = p->H; D.BH = p->B * p->H; D.T = p->T; D.Tq = p->Tq; D.d = p->d; D.dh = p->dh;
+  D.chunk = p->chunk < p->T ? p->chunk : p->T;
+  D.nch = cdiv(p->T, D.chunk);
+  D.order = p->order; D.rule = p->rule; D.dtype = p->dtype; D.w_shared = p->w_shared;
+  if (D.nch > 1 && D.Tq != D.T) return LACT_EINVAL;
+  if (D.d > 512 || D.dh > 4096) return LACT_EINVAL;
+  if (D.BH > 4096 || D.T > (int64_t(1) << 30) || D.Tq > (int64_t(1) << 30)) return LACT_EINVAL;
+  if (D.dtype == LACT_BF16 && (D.d % 64 != 0 || D.dh % 64 != 0)) return LACT_EINVAL;
+  D.key_rows = rup(D.chunk, 128);
+  D.q_rows = rup(D.nch == 1 ? D.Tq : D.chunk, 128);
+  if (D.key_rows / 128 > 65535 || D.q_rows / 128 > 65535) return LACT_EINVAL;
+  D.bn = choose_bn(D.d);
+  // Token splits of the gradient contraction: fill ~2 waves of 148 SMs when
+  // the output tiles alone do not.
+  const int64_t tiles = (D.d / D.bn) * cdiv(D.dh, 128) * 3 * D.BH;
+  int64_t s = tiles >= 120 ? 1 : cdiv(296, tiles);
+  const int64_t kbt = cdiv(D.chunk, 64);
+  if (s > kbt) s = kbt;
+  if (s * 3 * D.BH > 65535) s = 65535 / (3 * D.BH);
+  D.splits = static_cast<int>(s < 1 ? 1 : s);
+  if (3 * D.BH * D.splits > 65535) return LACT_EINVAL;
+  return LACT_OK;
+}
+
+struct Bufs {
+  void* qh; void* kh;
+  float* Wm; __nv_bfloat16* Ws; float* P; float* Mm; float* bbar;
+  void* E; void* Hq; float* Z;
+  float* Yf[2]; __nv_bfloat16* Yb[2];
+  float* Af; __nv_bfloat16* Ab; float* Bf; __nv_bfloat16* Bb; float* part;
+};
+
+struct Bump {
+  uintptr_t base, off;
+  template <class T> T* take(int64_t count) {
+    off = static_cast<uintptr_t>(rup(static_cast<int64_t>(off), 256));
+    T* r = reinterpret_cast<T*>(base + off);
+    off += static_cast<uintptr_t>(count) * sizeof(T);
+    return r;
+  }
+};
+
+static void plan(const Dims& D, Bump& bp, Bufs& b) {
+  std::memset(&b, 0, sizeof(b));
+  const bool bf = D.dtype == LACT_BF16;
+  const int64_t esz = bf ? 2 : 4;
+  const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane;
+  b.qh = bp.take<uint8_t>(D.BH * D.Tq * D.d * esz);
+  b.kh = bp.take<uint8_t>(D.BH * D.T * D.d * esz);
+  b.Wm = bp.take<float>(planes);
+  if (bf) b.Ws = bp.take<__nv_bfloat16>(planes);
+  b.P = bp.take<float>((bf ? D.splits : 1) * planes);
+  if (D.rule == LACT_RULE_MOMENTUM) {
+    b.Mm = bp.take<float>(planes);
+    b.bbar = bp.take<float>(D.BH * D.nch);
+  }
+  b.E = bp.take<uint8_t>(3 * D.BH * D.key_rows * D.dh * esz);
+  b.Hq = bp.take<uint8_t>(D.BH * D.q_rows * D.dh * esz);
+  if (!bf) b.Z = bp.take<float>(3 * D.BH * (D.key_rows > D.q_rows ? D.key_rows : D.q_rows) * D.dh);
+  if (D.rule == LACT_RULE_MUON) {
+    for (int i = 0; i < 2; ++i) {
+      b.Yf[i] = bp.take<float>(planes);
+      if (bf) b.Yb[i] = bp.take<__nv_bfloat16>(planes);
+    }
+    b.Af = bp.take<float>(3 * D.BH * D.d * D.d);
+    if (bf) {
+      b.Ab = bp.take<__nv_bfloat16>(3 * D.BH * D.d * D.d);
+      b.Bb = bp.take<__nv_bfloat16>(3 * D.BH * D.d * D.d);
+    } else {
+      b.Bf = bp.take<float>(3 * D.BH * D.d * D.d);
+    }
+    b.part = bp.take<float>(3 * D.BH * kNsBlocks);
+  }
+}
+
+static size_t workspace_bytes(const Dims& D) {
+  Bump bp{0, 0};
+  Bufs b;
+  plan(D, bp, b);
+  return static_cast<size_t>(rup(static_cast<int64_t>(bp.off), 256));
+}
+
+// ------------------------------------------------------------------ TMA maps
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over [batch][rows][inner] (dense), 128-byte swizzle,
+// out-of-bounds elements read as zero.
+static bool map3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint64_t batch,
+                  uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ launches
+template <class Op>
+static cudaError_t launch_umma(dim3 grid, const typename Op::Params& p, cudaStream_t st) {
+  constexpr int smem = umma_smem_bytes<Op>();
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(umma_kernel<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  umma_kernel<Op><<<grid, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <bool A_MN, bool B_MN>
+static cudaError_t launch_gemm(int bn, dim3 grid, const GemmParams& p, cudaStream_t st) {
+  switch (bn) {
+    case 64: return launch_umma<GemmOp<A_MN, B_MN, 64>>(grid, p, st);
+    case 128: return launch_umma<GemmOp<A_MN, B_MN, 128>>(grid, p, st);
+    case 192: return launch_umma<GemmOp<A_MN, B_MN, 192>>(grid, p, st);
+    case 256: return launch_umma<GemmOp<A_MN, B_MN, 256>>(grid, p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Kernel kinds, for the launch profiler (lact_profile_*).
+enum Kind {
+  K_INIT, K_PROLOGUE, K_BETA_MEAN, K_FWD_QUERY, K_APPLY_OUT, K_FWD_KEY, K_GRAD, K_NS_SUMSQ,
+  K_NS_SCALE, K_NS_GRAM, K_NS_POLY, K_NS_UPDATE, K_RULE, K_FINALIZE, K_SIMT_GEMM, K_FWD_ELEM_F32,
+  K_COUNT
+};
+static const char* const kKindNames[K_COUNT] = {
+    "init_state", "qk_prologue", "beta_mean", "fwd_query_umma", "apply_out_umma", "fwd_key_umma",
+    "grad_umma", "ns_sumsq", "ns_scale", "ns_gram_umma", "ns_poly_umma", "ns_update_umma",
+    "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32"};
+
+// Optional per-launch CUDA-event pairs on the launching stream.
+struct ProfRec { int kind; cudaEvent_t a, b; };
+static std::mutex g_prof_mu;
+static bool g_prof_on = false;
+static std::vector<ProfRec> g_prof;
+static std::vector<cudaEvent_t> g_event_pool;
+
+static cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+struct Launcher {
+  bool dry;
+  cudaStream_t st = nullptr;
+  int64_t count = 0;
+  int err = LACT_OK;
+  template <class F> void operator()(int kind, F&& f) {
+    ++count;
+    if (dry || err != LACT_OK) return;
+    cudaEvent_t a = nullptr, b = nullptr;
+    std::unique_lock<std::mutex> lk(g_prof_mu, std::defer_lock);
+    if (g_prof_on) {
+      lk.lock();
+      a = take_event();
+      b = take_event();
+      if (a && b) cudaEventRecord(a, st);
+    }
+    if (f() != cudaSuccess) err = LACT_ECUDA;
+    if (a && b) {
+      cudaEventRecord(b, st);
+      g_prof.push_back({kind, a, b});
+    }
+  }
+};
+
+struct Inputs {
+  const void *q, *k, *v;
+  const float *lr, *beta, *w1, *w2, *w3;
+  void* out;
+  float *w1o, *w2o, *w3o;
+};
+
+static GemmParams gemm_params() {
+  GemmParams g;
+  std::memset(&g, 0, sizeof(g));
+  g.alt_group = -1;
+  g.alpha = 1.0f;
+  return g;
+}
+
+static SimtGemmParams simt_params() {
+  SimtGemmParams s;
+  std::memset(&s, 0, sizeof(s));
+  s.alt_a = -1;
+  s.alt_b = -1;
+  s.za_mod = 1 << 30;
+  s.zb_mod = 1 << 30;
+  s.alpha = 1.0f;
+  return s;
+}
+
+static cudaError_t simt(const SimtGemmParams& p, int items, cudaStream_t st) {
+  k_simt_gemm<<<dim3(cdiv(p.N, 64), cdiv(p.M, 64), items), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st, Launcher& L) {
+  const bool bf = D.dtype == LACT_BF16;
+  const int BH = static_cast<int>(D.BH), d = static_cast<int>(D.d), dh = static_cast<int>(D.dh);
+  const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane;
+  const dim3 tile_grid(cdiv(d, 32), cdiv(dh, 32), 3 * BH), tile_block(32, 8);
+
+  // Fast-weight masters (+ bf16 shadows), momentum = 0.
+  L(K_INIT, [&] {
+    k_init_state<<<tile_grid, tile_block, 0, st>>>(in.w1, in.w2, in.w3, static_cast<int>(D.H),
+                                                   D.w_shared, BH, d, dh, b.Wm, b.Ws, b.Mm);
+    return cudaGetLastError();
+  });
+  // q^, k^ = silu + L2 norm rows.
+  L(K_PROLOGUE, [&] {
+    const int64_t rows = D.BH * D.Tq + D.BH * D.T;
+    const unsigned blocks = static_cast<unsigned>(cdiv(rows * 32, 256));
+    if (bf)
+      k_qk_prologue<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(in.q), static_cast<__nv_bfloat16*>(b.qh), D.BH * D.Tq,
+          static_cast<const __nv_bfloat16*>(in.k), static_cast<__nv_bfloat16*>(b.kh), D.BH * D.T, d);
+    else
+      k_qk_prologue<float><<<blocks, 256, 0, st>>>(
+          static_cast<const float*>(in.q), static_cast<float*>(b.qh), D.BH * D.Tq,
+          static_cast<const float*>(in.k), static_cast<float*>(b.kh), D.BH * D.T, d);
+    return cudaGetLastError();
+  });
+  if (D.rule == LACT_RULE_MOMENTUM) {
+    L(K_BETA_MEAN, [&] {
+      const int64_t w = D.BH * D.nch;
+      k_beta_mean<<<static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st>>>(in.beta, BH, D.T, D.chunk,
+                                                                            static_cast<int>(D.nch), b.bbar);
+      return cudaGetLastError();
+    });
+  }
+
+  for (int64_t c = 0; c < D.nch; ++c) {
+    const int64_t c0 = c * D.chunk;
+    const int nc = static_cast<int>((c0 + D.chunk < D.T ? c0 + D.chunk : D.T) - c0);
+    const int64_t qr0 = D.nch == 1 ? 0 : c0;
+    const int nq = static_cast<int>(D.nch == 1 ? D.Tq : nc);
+
+    auto apply = [&] {
+      if (bf) {
+        L(K_FWD_QUERY, [&] {
+          FwdParams f;
+          std::memset(&f, 0, sizeof(f));
+          if (!map3d(&f.tmX, b.qh, d, D.Tq, BH, 64, 128) || !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 64))
+            return cudaErrorInvalidValue;
+          f.bh_count = BH; f.x_row0 = static_cast<int>(qr0); f.rows_valid = nq; f.kb_count = d / 64;
+          f.dh = dh; f.T = static_cast<int>(D.T); f.hq = static_cast<__nv_bfloat16*>(b.Hq);
+          f.buf_rows = D.q_rows; f.lr = in.lr;
+          return launch_umma<FwdOp<false>>(dim3(dh / 64, cdiv(nq, 128), BH), f, st);
+        });
+        L(K_APPLY_OUT, [&] {
+          GemmParams g = gemm_params();
+          if (!map3d(&g.tmA, b.Hq, dh, D.q_rows, BH, 64, 128) || !map3d(&g.tmB, b.Ws, d, dh, 3 * BH, 64, 64))
+            return cudaErrorInvalidValue;
+          g.items = BH; g.kb_count = dh / 64; g.kb_total = g.kb_count;
+          g.zb_mod = BH; g.zb_add = BH; g.m_valid = nq;
+          g.outb = static_cast<__nv_bfloat16*>(in.out) + qr0 * d;
+          g.item_stride = D.Tq * D.d; g.ld = d;
+          return launch_gemm<false, true>(D.bn, dim3(d / D.bn, cdiv(nq, 128), BH), g, st);
+        });
+      } else {
+        float* Z = b.Z;
+        const int64_t zpl = D.BH * D.q_rows * D.dh;
+        for (int j = 0; j < 3; j += 2) {
+          L(K_SIMT_GEMM, [&] {
+            SimtGemmParams s = simt_params();
+            s.A = static_cast<const float*>(b.qh) + qr0 * d; s.a_item = D.Tq * D.d; s.a_m = d; s.a_k = 1;
+            s.B = b.Wm + j * D.BH * plane; s.b_item = plane; s.b_n = d; s.b_k = 1;
+            s.M = nq; s.N = dh; s.K = d;
+            s.outf = Z + j * zpl; s.item_stride = D.q_rows * D.dh; s.ld = dh;
+            return simt(s, BH, st);
+          });
+        }
+        L(K_FWD_ELEM_F32, [&] {
+          const int64_t n = zpl;
+          k_fwd_elem_f32<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, st>>>(
+              Z, BH, D.q_rows, dh, nq, 0, nullptr, D.T, 0, static_cast<float*>(b.Hq));
+          return cudaGetLastError();
+        });
+        L(K_SIMT_GEMM, [&] {
+          SimtGemmParams s = simt_params();
+          s.A = static_cast<const float*>(b.Hq); s.a_item = D.q_rows * D.dh; s.a_m = dh; s.a_k = 1;
+          s.B = b.Wm + D.BH * plane; s.b_item = plane; s.b_n = 1; s.b_k = d;
+          s.M = nq; s.N = d; s.K = dh;
+          s.outf = static_cast<float*>(in.out) + qr0 * d; s.item_stride = D.Tq * D.d; s.ld = d;
+          return simt(s, BH, st);
+        });
+      }
+    };
+
+    auto update = [&] {
+      int splits = 1;
+      if (bf) {
+        L(K_FWD_KEY, [&] {
+          FwdParams f;
+          std::memset(&f, 0, sizeof(f));
+          if (!map3d(&f.tmX, b.kh, d, D.T, BH, 64, 128) || !map3d(&f.tmV, in.v, d, D.T, BH, 64, 128) ||
+              !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 64))
+            return cudaErrorInvalidValue;
+          f.bh_count = BH; f.x_row0 = static_cast<int>(c0); f.rows_valid = nc; f.kb_count = d / 64;
+          f.dh = dh; f.T = static_cast<int>(D.T); f.e = static_cast<__nv_bfloat16*>(b.E);
+          f.buf_rows = D.key_rows; f.lr = in.lr;
+          return launch_umma<FwdOp<true>>(dim3(dh / 64, cdiv(nc, 128), BH), f, st);
+        });
+        const int kbt = static_cast<int>(cdiv(nc, 64));
+        const int kbp = static_cast<int>(cdiv(kbt, D.splits));
+        splits = static_cast<int>(cdiv(kbt, kbp));
+        L(K_GRAD, [&] {
+          GemmParams g = gemm_params();
+          if (!map3d(&g.tmA, b.E, dh, D.key_rows, 3 * BH, 64, 64) || !map3d(&g.tmB, b.kh, d, D.T, BH, 64, 64) ||
+              !map3d(&g.tmB2, in.v, d, D.T, BH, 64, 64))
+            return cudaErrorInvalidValue;
+          g.items = 3 * BH; g.kb_count = kbp; g.kb_total = kbt;
+          g.a_k0 = 0; g.b_k0 = static_cast<int>(c0);
+          g.zb_mod = BH; g.zb_add = 0; g.alt_group = 1; g.m_valid = dh;
+          g.outf = b.P; g.item_stride = plane; g.ld = d;
+          return launch_gemm<true, true>(D.bn, dim3(d / D.bn, cdiv(dh, 128), splits * 3 * BH), g, st);
+        });
+      } else {
+        const int64_t zpl = D.BH * D.key_rows * D.dh;
+        for (int j = 0; j < 3; ++j) {
+          L(K_SIMT_GEMM, [&] {
+            SimtGemmParams s = simt_params();
+            s.A = (j == 1 ? static_cast<const float*>(in.v) : static_cast<const float*>(b.kh)) + c0 * d;
+            s.a_item = D.T * D.d; s.a_m = d; s.a_k = 1;
+            s.B = b.Wm + j * D.BH * plane; s.b_item = plane; s.b_n = d; s.b_k = 1;
+            s.M = nc; s.N = dh; s.K = d;
+            s.outf = b.Z + j * zpl; s.item_stride = D.key_rows * D.dh; s.ld = dh;
+            return simt(s, BH, st);
+          });
+        }
+        L(K_FWD_ELEM_F32, [&] {
+          k_fwd_elem_f32<<<static_cast<unsigned>(cdiv(zpl, 256)), 256, 0, st>>>(
+              b.Z, BH, D.key_rows, dh, nc, 1, in.lr, D.T, c0, static_cast<float*>(b.E));
+          return cudaGetLastError();
+        });
+        L(K_SIMT_GEMM, [&] {
+          SimtGemmParams s = simt_params();
+          s.A = static_cast<const float*>(b.E); s.a_item = D.key_rows * D.dh; s.a_m = 1; s.a_k = dh;
+          s.B = static_cast<const float*>(b.kh) + c0 * d; s.B2 = static_cast<const float*>(in.v) + c0 * d;
+          s.b_item = D.T * D.d; s.b_n = 1; s.b_k = d; s.zb_mod = BH; s.alt_b = 1;
+          s.M = dh; s.N = d; s.K = nc;
+          s.outf = b.P; s.item_stride = plane; s.ld = d;
+          return simt(s, 3 * BH, st);
+        });
+      }
+
+      const float* dir = b.P;
+      int dir_splits = splits;
+      if (D.rule == LACT_RULE_MUON) {
+        L(K_NS_SUMSQ, [&] {
+          k_ns_sumsq<<<dim3(kNsBlocks, 3 * BH), 256, 0, st>>>(b.P, splits, planes, plane, b.Yf[0], b.part);
+          return cudaGetLastError();
+        });
+        L(K_NS_SCALE, [&] {
+          k_ns_scale<<<dim3(kNsBlocks, 3 * BH), 256, 0, st>>>(b.Yf[0], b.Yb[0], plane, b.part, kNsBlocks,
+                                                              kNsEps);
+          return cudaGetLastError();
+        });
+        for (int it = 0; it < kNsSteps; ++it) {
+          const int cur = it & 1, nxt = cur ^ 1;
+          if (bf) {
+            L(K_NS_GRAM, [&] {  // A = X^T X  (d x d, K = dh)
+              GemmParams g = gemm_params();
+              if (!map3d(&g.tmA, b.Yb[cur], d, dh, 3 * BH, 64, 64)) return cudaErrorInvalidValue;
+              g.tmB = g.tmA;
+              g.items = 3 * BH; g.kb_count = g.kb_total = static_cast<int>(cdiv(dh, 64));
+              g.zb_mod = 3 * BH; g.m_valid = d;
+              g.outf = b.Af; g.outb = b.Ab; g.item_stride = D.d * D.d; g.ld = d;
+              return launch_gemm<true, true>(D.bn, dim3(d / D.bn, cdiv(d, 128), 3 * BH), g, st);
+            });
+            L(K_NS_POLY, [&] {  // B = b A + c A A
+              GemmParams g = gemm_params();
+              if (!map3d(&g.tmA, b.Ab, d, d, 3 * BH, 64, 128) || !map3d(&g.tmB, b.Ab, d, d, 3 * BH, 64, D.bn))
+                return cudaErrorInvalidValue;
+              g.items = 3 * BH; g.kb_count = g.kb_total = d / 64;
+              g.zb_mod = 3 * BH; g.m_valid = d;
+              g.alpha = kNsC; g.beta = kNsB; g.cin = b.Af;
+              g.outb = b.Bb; g.item_stride = D.d * D.d; g.ld = d;
+              return launch_gemm<false, false>(D.bn, dim3(d / D.bn, cdiv(d, 128), 3 * BH), g, st);
+            });
+            L(K_NS_UPDATE, [&] {  // X <- a X + X B
+              GemmParams g = gemm_params();
+              if (!map3d(&g.tmA, b.Yb[cur], d, dh, 3 * BH, 64, 128) ||
+                  !map3d(&g.tmB, b.Bb, d, d, 3 * BH, 64, D.bn))
+                return cudaErrorInvalidValue;
+              g.items = 3 * BH; g.kb_count = g.kb_total = d / 64;
+              g.zb_mod = 3 * BH; g.m_valid = dh;
+              g.alpha = 1.0f; g.beta = kNsA; g.cin = b.Yf[cur];
+              g.outf = b.Yf[nxt]; g.outb = b.Yb[nxt]; g.item_stride = plane; g.ld = d;
+              return launch_gemm<false, false>(D.bn, dim3(d / D.bn, cdiv(dh, 128), 3 * BH), g, st);
+            });
+          } else {
+            L(K_SIMT_GEMM, [&] {
+              SimtGemmParams s = simt_params();
+              s.A = b.Yf[cur]; s.a_item = plane; s.a_m = 1; s.a_k = d;
+              s.B = b.Yf[cur]; s.b_item = plane; s.b_n = 1; s.b_k = d;
+              s.M = d; s.N = d; s.K = dh;
+              s.outf = b.Af; s.item_stride = D.d * D.d; s.ld = d;
+              return simt(s, 3 * BH, st);
+            });
+            L(K_SIMT_GEMM, [&] {
+              SimtGemmParams s = simt_params();
+              s.A = b.Af; s.a_item = D.d * D.d; s.a_m = d; s.a_k = 1;
+              s.B = b.Af; s.b_item = D.d * D.d; s.b_n = 1; s.b_k = d;
+              s.M = d; s.N = d; s.K = d;
+              s.alpha = kNsC; s.beta = kNsB; s.cin = b.Af;
+              s.outf = b.Bf; s.item_stride = D.d * D.d; s.ld = d;
+              return simt(s, 3 * BH, st);
+            });
+            L(K_SIMT_GEMM, [&] {
+              SimtGemmParams s = simt_params();
+              s.A = b.Yf[cur]; s.a_item = plane; s.a_m = d; s.a_k = 1;
+              s.B = b.Bf; s.b_item = D.d * D.d; s.b_n = 1; s.b_k = d;
+              s.M = dh; s.N = d; s.K = d;
+              s.alpha = 1.0f; s.beta = kNsA; s.cin = b.Yf[cur];
+              s.outf = b.Yf[nxt]; s.item_stride = plane; s.ld = d;
+              return simt(s, 3 * BH, st);
+            });
+          }
+        }
+        dir = b.Yf[kNsSteps & 1];
+        dir_splits = 1;
+      }
+      L(K_RULE, [&] {
+        RuleParams r;
+        std::memset(&r, 0, sizeof(r));
+        r.Wm = b.Wm; r.Ws = b.Ws; r.S = dir; r.splits = dir_splits; r.split_stride = planes;
+        r.Mm = b.Mm; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c);
+        r.rule = D.rule; r.BH = BH; r.dh = dh; r.d = d;
+        r.row_blocks = static_cast<int>(cdiv(2 * D.BH * D.dh * 32, 256));
+        const unsigned grid = static_cast<unsigned>(r.row_blocks + D.BH * cdiv(d, 32));
+        k_rule_renorm<<<grid, 256, 0, st>>>(r);
+        return cudaGetLastError();
+      });
+    };
+
+    if (D.order == LACT_APPLY_THEN_UPDATE) {
+      apply();
+      update();
+    } else {
+      update();
+      apply();
+    }
+  }
+
+  L(K_FINALIZE, [&] {
+    k_finalize_state<<<tile_grid, tile_block, 0, st>>>(b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o);
+    return cudaGetLastError();
+  });
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+static int check_pointers(const Dims& D, const Inputs& in) {
+  const void* need[] = {in.q, in.k, in.v, in.lr, in.w1, in.w2, in.w3, in.out, in.w1o, in.w2o, in.w3o};
+  for (const void* p : need)
+    if (!p || !aligned16(p)) return LACT_EINVAL;
+  if (D.rule == LACT_RULE_MOMENTUM && (!in.beta || !aligned16(in.beta))) return LACT_EINVAL;
+  const size_t wn = static_cast<size_t>((D.w_shared ? D.H : D.BH) * D.d * D.dh) * 4;
+  const size_t won = static_cast<size_t>(D.BH * D.d * D.dh) * 4;
+  const float* ins[3] = {in.w1, in.w2, in.w3};
+  const float* outs[3] = {in.w1o, in.w2o, in.w3o};
+  for (int i = 0; i < 3; ++i)
+    for (int j = 0; j < 3; ++j) {
+      if (!overlaps(outs[i], won, ins[j], wn)) continue;
+      // Exact in-place aliasing of the matching matrix is allowed for
+      // per-(b,h) initial states; any other overlap is rejected.
+      if (!(i == j && outs[i] == ins[j] && wn == won)) return LACT_EINVAL;
+    }
+  for (int i = 0; i < 3; ++i)
+    for (int j = i + 1; j < 3; ++j)
+      if (overlaps(outs[i], won, outs[j], won)) return LACT_EINVAL;
+  const size_t on = static_cast<size_t>(D.BH * D.Tq * D.d) * (D.dtype == LACT_BF16 ? 2 : 4);
+  for (int i = 0; i < 3; ++i)
+    if (overlaps(in.out, on, outs[i], won)) return LACT_EINVAL;
+  return LACT_OK;
+}
+
+static int input_bytes(const Dims& D, size_t sz[8]) {
+  const size_t e = D.dtype == LACT_BF16 ? 2 : 4;
+  const size_t hw = static_cast<size_t>(D.w_shared ? D.H : D.BH);
+  sz[0] = static_cast<size_t>(D.BH * D.Tq * D.d) * e;
+  sz[1] = static_cast<size_t>(D.BH * D.T * D.d) * e;
+  sz[2] = sz[1];
+  sz[3] = static_cast<size_t>(D.BH * D.T * 3) * 4;
+  sz[4] = D.rule == LACT_RULE_MOMENTUM ? static_cast<size_t>(D.BH * D.T) * 4 : 0;
+  sz[5] = hw * D.dh * D.d * 4;
+  sz[6] = sz[5];
+  sz[7] = sz[5];
+  return 0;
+}
+
+// One thread waits on a barrier that expects one arrival nobody makes.
+__global__ void k_selftest_wait() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait(&bar, 0);
+  }
+}
+
+}  // namespace lact
+
+using namespace lact;
+
+extern "C" {
+
+size_t lact_ttt_workspace_bytes(const lact_problem* p) {
+  Dims D;
+  if (validate(p, D) != LACT_OK) return 0;
+  return workspace_bytes(D);
+}
+
+int64_t lact_ttt_launch_count(const lact_problem* p) {
+  Dims D;
+  if (validate(p, D) != LACT_OK) return 0;
+  Bump bp{0, 0};
+  Bufs b;
+  plan(D, bp, b);
+  Inputs in;
+  std::memset(&in, 0, sizeof(in));
+  Launcher L{true, nullptr};
+  run(D, b, in, nullptr, L);
+  return L.count;
+}
+
+int lact_ttt_fwd(const lact_problem* p, const void* q, const void* k, const void* v, const float* lr,
+                 const float* beta, const float* w1, const float* w2, const float* w3, void* out,
+                 float* w1_out, float* w2_out, float* w3_out, void* workspace, size_t workspace_bytes_,
+                 void* stream) {
+  Dims D;
+  int rc = validate(p, D);
+  if (rc != LACT_OK) return rc;
+  Inputs in{q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out};
+  rc = check_pointers(D, in);
+  if (rc != LACT_OK) return rc;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LACT_EINVAL;
+  if (workspace_bytes_ < workspace_bytes(D)) return LACT_ENOSPC;
+  if (D.dtype == LACT_BF16 && !encode_fn()) return LACT_ECUDA;
+  Bump bp{reinterpret_cast<uintptr_t>(workspace), 0};
+  Bufs b;
+  plan(D, bp, b);
+  Launcher L{false, static_cast<cudaStream_t>(stream)};
+  run(D, b, in, static_cast<cudaStream_t>(stream), L);
+  return L.err;
+}
+
+size_t lact_ttt_host_workspace_bytes(const lact_problem* p) {
+  Dims D;
+  if (validate(p, D) != LACT_OK) return 0;
+  size_t sz[8];
+  input_bytes(D, sz);
+  size_t total = workspace_bytes(D);
+  for (size_t s : sz) total += (s + 255) / 256 * 256;
+  const size_t e = D.dtype == LACT_BF16 ? 2 : 4;
+  total += (static_cast<size_t>(D.BH * D.Tq * D.d) * e + 255) / 256 * 256;
+  total += 3 * ((static_cast<size_t>(D.BH * D.d * D.dh) * 4 + 255) / 256 * 256);
+  return total;
+}
+
+int lact_ttt_fwd_host(const lact_problem* p, const void* q, const void* k, const void* v,
+                      const float* lr, const float* beta, const float* w1, const float* w2,
+                      const float* w3, void* out, float* w1_out, float* w2_out, float* w3_out,
+                      void* workspace, size_t workspace_bytes_, void* stream) {
+  Dims D;
+  int rc = validate(p, D);
+  if (rc != LACT_OK) return rc;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LACT_EINVAL;
+  if (workspace_bytes_ < lact_ttt_host_workspace_bytes(p)) return LACT_ENOSPC;
+  const void* hin[8] = {q, k, v, lr, beta, w1, w2, w3};
+  size_t sz[8];
+  input_bytes(D, sz);
+  for (int i = 0; i < 8; ++i)
+    if (sz[i] && !hin[i]) return LACT_EINVAL;
+  if (!out || !w1_out || !w2_out || !w3_out) return LACT_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Bump bp{reinterpret_cast<uintptr_t>(workspace), static_cast<uintptr_t>(workspace_bytes(D))};
+  void* dev[8];
+  for (int i = 0; i < 8; ++i) dev[i] = sz[i] ? bp.take<uint8_t>(static_cast<int64_t>(sz[i])) : nullptr;
+  const size_t e = D.dtype == LACT_BF16 ? 2 : 4;
+  const size_t osz = static_cast<size_t>(D.BH * D.Tq * D.d) * e;
+  const size_t wsz = static_cast<size_t>(D.BH * D.d * D.dh) * 4;
+  void* dout = bp.take<uint8_t>(static_cast<int64_t>(osz));
+  float* dw[3];
+  for (int i = 0; i < 3; ++i) dw[i] = bp.take<float>(D.BH * D.d * D.dh);
+  for (int i = 0; i < 8; ++i)
+    if (sz[i] && cudaMemcpyAsync(dev[i], hin[i], sz[i], cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return LACT_ECUDA;
+  rc = lact_ttt_fwd(p, dev[0], dev[1], dev[2], static_cast<const float*>(dev[3]),
+                    static_cast<const float*>(dev[4]), static_cast<const float*>(dev[5]),
+                    static_cast<const float*>(dev[6]), static_cast<const float*>(dev[7]), dout, dw[0],
+                    dw[1], dw[2], workspace, workspace_bytes(D), stream);
+  if (rc != LACT_OK) return rc;
+  if (cudaMemcpyAsync(out, dout, osz, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(w1_out, dw[0], wsz, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(w2_out, dw[1], wsz, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(w3_out, dw[2], wsz, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return LACT_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LACT_ECUDA;
+  return LACT_OK;
+}
+
+int lact_ttt_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LACT_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return LACT_ECUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return LACT_ECUDA;
+    return LACT_ETIMEOUT;
+  }
+  return LACT_OK;
+}
+
+int lact_device_check(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LACT_ECUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LACT_ECUDA;
+  return (prop.major == 10 && prop.minor == 0) ? LACT_OK : LACT_ENODEV;
+}
+
+int lact_selftest_wait_timeout(int64_t budget_cycles, void* stream) {
+  if (budget_cycles < 1 || budget_cycles > (int64_t(1) << 31)) return LACT_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long normal = kDefaultWaitBudget, b = budget_cycles;
+  if (cudaMemcpyToSymbolAsync(g_wait_budget, &b, sizeof(b), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return LACT_ECUDA;
+  k_selftest_wait<<<1, 32, 0, st>>>();
+  const cudaError_t e = cudaGetLastError();
+  if (cudaMemcpyToSymbolAsync(g_wait_budget, &normal, sizeof(normal), 0, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return LACT_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LACT_ECUDA;
+  return e == cudaSuccess ? LACT_OK : LACT_ECUDA;
+}
+
+int lact_kernel_kinds(void) { return K_COUNT; }
+
+const char* lact_kernel_name(int kind) {
+  return (kind >= 0 && kind < K_COUNT) ? kKindNames[kind] : "unknown";
+}
+
+int lact_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return LACT_OK;
+}
+
+int lact_profile_read(int64_t* launches, double* ms, int nkinds) {
+  if (!launches || !ms || nkinds < K_COUNT) return LACT_EINVAL;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (int i = 0; i < nkinds; ++i) {
+    launches[i] = 0;
+    ms[i] = 0.0;
+  }
+  int rc = LACT_OK;
+  for (const ProfRec& r : g_prof) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      rc = LACT_ECUDA;
+    launches[r.kind] += 1;
+    ms[r.kind] += t;
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  return rc;
+}
+
+const char* lact_status_string(int code) {
+  switch (code) {
+    case LACT_OK: return "ok";
+    case LACT_EINVAL: return "invalid argument";
+    case LACT_ENOSPC: return "workspace too small";
+    case LACT_ECUDA: return "CUDA error";
+    case LACT_ETIMEOUT: return "a bounded device wait gave up";
+    case LACT_ENODEV: return "not an sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

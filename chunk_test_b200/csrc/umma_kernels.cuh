@@ -1,0 +1,398 @@
+// umma_kernels.cuh -- tcgen05 (sm_100a) tensor-core kernels of the bf16 path.
+//
+// Every kernel here is one output tile of 128 rows per CTA, 192 threads:
+//   warp 0      TMA producer (one elected lane), STAGES-deep smem ring
+//   warp 1      TMEM allocator + MMA issuer (one elected lane)
+//   warps 2..5  epilogue: tcgen05.ld of one 32-lane TMEM quarter each, fused
+//               elementwise math, stores to global memory
+// Operands are bf16 in 128-byte-swizzled smem tiles fed by TMA, accumulators
+// fp32 in TMEM.  K is consumed in blocks of 64 (one 128-byte swizzle row).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace lact {
+
+constexpr int kBM = 128;  // rows of every output tile (one TMEM lane per row)
+constexpr int kBK = 64;   // K elements per stage (128 bytes of bf16)
+constexpr int kThreads = 192;
+
+template <int N>
+struct TmemCols {
+  static constexpr int value = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : N <= 256 ? 256 : 512;
+};
+
+// The shared pipeline: Op supplies kStages, kStageBytes, kTmemCols, Tile,
+// map_tile(), num_kb(), load(), mma(), epilogue().
+template <class Op>
+__global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant__ typename Op::Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int S = Op::kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Op::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tmem_full = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+
+  // Once a bounded wait anywhere has given up, later CTAs do no work (the
+  // results are already invalid and flagged); decided once per CTA.
+  __shared__ int abort_cta;
+  if (threadIdx.x == 0) abort_cta = *reinterpret_cast<volatile int*>(&g_status);
+  __syncthreads();
+  if (abort_cta) return;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const typename Op::Tile tile = Op::map_tile(p);
+  const int nkb = Op::num_kb(p, tile);
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tmem_full, 1);
+    fence_barrier_init();
+    Op::prefetch(p);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Op::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % S;
+        if (kb >= S && !mbar_wait(&empty[s], ((kb / S) - 1) & 1)) break;
+        mbar_arrive_expect_tx(&full[s], Op::stage_bytes(p, tile));
+        Op::load(p, tile, kb, smem + s * Op::kStageBytes, &full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % S;
+        if (!mbar_wait(&full[s], (kb / S) & 1)) break;
+        tc_fence_after();
+        Op::mma(p, tile, smem_u32(smem + s * Op::kStageBytes), tmem, kb);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(tmem_full);
+    }
+  } else {
+    const bool ok = mbar_wait(tmem_full, 0);
+    tc_fence_after();
+    if (ok) Op::epilogue(p, tile, tmem, warp & 3, lane);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, Op::kTmemCols);
+  }
+}
+
+// Issue the 4 UMMAs (K = 16 each) of one 64-wide K block.
+// a_mn / b_mn: operand is MN-major (64-element MN blocks `*_lbo` bytes apart,
+// 16 K rows = 2048 bytes per step) or K-major (32 bytes per step).
+template <bool A_MN, bool B_MN>
+__device__ __forceinline__ void mma_kblock(uint32_t d_tmem, uint32_t a_base, uint32_t a_lbo,
+                                           uint32_t b_base, uint32_t b_lbo, uint32_t idesc,
+                                           bool first) {
+#pragma unroll
+  for (int k = 0; k < kBK / 16; ++k) {
+    const uint32_t ao = A_MN ? k * 2048u : k * 32u;
+    const uint32_t bo = B_MN ? k * 2048u : k * 32u;
+    const uint64_t ad = smem_desc_sw128(a_base + ao, A_MN ? a_lbo : 16u, 1024u);
+    const uint64_t bd = smem_desc_sw128(b_base + bo, B_MN ? b_lbo : 16u, 1024u);
+    umma_bf16(d_tmem, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fast-net forward on one chunk, one (128-token x 64-hidden-unit) tile.
+//   Z1 = X W1^T, Z3 = X W3^T   (X = q^ or k^ rows, K = d)      -> TMEM [0,128)
+//   KMODE also: DH = V (W2^T)^T = V W2                           -> TMEM [128,192)
+// Epilogue, per token t and hidden unit r (s1 = sigmoid(z1)):
+//   query tile: Hq = silu(z1) z3                                  (bf16)
+//   key tile:   E1 = lr1 dh z3 s1 (1 + z1 (1 - s1))               (d<f,v>/dz1)
+//               Eh = lr2 silu(z1) z3                              (h, for G2)
+//               E3 = lr3 dh silu(z1)                              (d<f,v>/dz3)
+// so that the negated chunk gradients are  -G1 = E1^T k^,  -G3 = E3^T k^,
+// -G2^T = Eh^T v  ("大块测试时训练（LaCT）技术解析" §2.1 eqs. 4-5; loss and
+// per-token rates of "LaCT：以大分块更新…" 「局部注意力与非线性记忆相互补充」).
+// Rows past the chunk's end are written as zeros (key tiles) or skipped.
+// ---------------------------------------------------------------------------
+struct FwdParams {
+  CUtensorMap tmX;   // q^ or k^ [BH, rows, d] bf16, box {64, 128, 1}
+  CUtensorMap tmV;   // v [BH, T, d] bf16, box {64, 128, 1}          (key tiles)
+  CUtensorMap tmW;   // bf16 shadows [3*BH, dh, d] (W1, W2^T, W3), box {64, 64, 1}
+  int bh_count;      // B*H
+  int x_row0;        // first token of the chunk in tmX / tmV
+  int rows_valid;    // tokens in this chunk
+  int kb_count;      // d / 64
+  int dh;
+  int T;             // rows of lr per head
+  __nv_bfloat16* hq; // query tiles: Hq [BH, buf_rows, dh]
+  __nv_bfloat16* e;  // key tiles:   E [3][BH][buf_rows][dh]  (E1, Eh, E3)
+  int64_t buf_rows;
+  const float* lr;   // [BH, T, 3]
+};
+
+template <bool KMODE>
+struct FwdOp {
+  using Params = FwdParams;
+  static constexpr int kXBytes = kBM * kBK * 2;           // 16 KB
+  static constexpr int kWBytes = 64 * kBK * 2;            // 8 KB per 64-row slice
+  static constexpr int kStageBytes = KMODE ? (2 * kXBytes + 3 * kWBytes) : (kXBytes + 2 * kWBytes);
+  static constexpr int kStages = KMODE ? 3 : 4;
+  static constexpr int kTmemCols = KMODE ? 256 : 128;
+  struct Tile { int slice, row0, bh; };
+
+  __device__ static Tile map_tile(const Params&) {
+    return Tile{static_cast<int>(blockIdx.x), static_cast<int>(blockIdx.y) * kBM,
+                static_cast<int>(blockIdx.z)};
+  }
+  __device__ static int num_kb(const Params& p, const Tile&) { return p.kb_count; }
+  __device__ static uint32_t stage_bytes(const Params&, const Tile&) { return kStageBytes; }
+  __device__ static void prefetch(const Params& p) {
+    tma_prefetch_map(&p.tmX);
+    tma_prefetch_map(&p.tmW);
+    if (KMODE) tma_prefetch_map(&p.tmV);
+  }
+  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
+    const int k = kb * kBK, row = p.x_row0 + t.row0, hs = t.slice * 64;
+    tma_load_3d(st, &p.tmX, bar, k, row, t.bh);
+    tma_load_3d(st + kXBytes, &p.tmW, bar, k, hs, t.bh);                              // W1
+    tma_load_3d(st + kXBytes + kWBytes, &p.tmW, bar, k, hs, 2 * p.bh_count + t.bh);   // W3
+    if (KMODE) {
+      tma_load_3d(st + kXBytes + 2 * kWBytes, &p.tmV, bar, k, row, t.bh);
+      tma_load_3d(st + 2 * kXBytes + 2 * kWBytes, &p.tmW, bar, k, hs, p.bh_count + t.bh);  // W2^T
+    }
+  }
+  __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {
+    constexpr uint32_t id0 = idesc_bf16(kBM, 128, false, false);
+    mma_kblock<false, false>(tmem, st, 0, st + kXBytes, 0, id0, kb == 0);
+    if (KMODE) {
+      constexpr uint32_t id1 = idesc_bf16(kBM, 64, false, false);
+      mma_kblock<false, false>(tmem + 128, st + kXBytes + 2 * kWBytes, 0,
+                               st + 2 * kXBytes + 2 * kWBytes, 0, id1, kb == 0);
+    }
+  }
+  __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
+                                  int lane) {
+    const int r = quarter * 32 + lane;
+    const int grow = t.row0 + r;
+    const bool valid = grow < p.rows_valid;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int64_t col0 = static_cast<int64_t>(t.slice) * 64;
+    if (!KMODE) {
+      __nv_bfloat16* dst = p.hq + (static_cast<int64_t>(t.bh) * p.buf_rows + grow) * p.dh + col0;
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float z1[16], z3[16];
+        __syncwarp();
+        tmem_ld16(tq + j, z1);
+        tmem_ld16(tq + 64 + j, z3);
+        tmem_ld_wait();
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float h0 = z1[2 * i] * sigmoidf_(z1[2 * i]) * z3[2 * i];
+          const float h1 = z1[2 * i + 1] * sigmoidf_(z1[2 * i + 1]) * z3[2 * i + 1];
+          w[i] = pack_bf16x2(h0, h1);
+        }
+        if (valid) {
+          st_global_v4(dst + j, w[0], w[1], w[2], w[3]);
+          st_global_v4(dst + j + 8, w[4], w[5], w[6], w[7]);
+        }
+      }
+    } else {
+      float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
+      if (valid) {
+        const float* l = p.lr + (static_cast<int64_t>(t.bh) * p.T + p.x_row0 + grow) * 3;
+        eta0 = l[0];
+        eta1 = l[1];
+        eta2 = l[2];
+      }
+      const int64_t plane = static_cast<int64_t>(p.bh_count) * p.buf_rows * p.dh;
+      __nv_bfloat16* d1 = p.e + (static_cast<int64_t>(t.bh) * p.buf_rows + grow) * p.dh + col0;
+      __nv_bfloat16* dh2 = d1 + plane;
+      __nv_bfloat16* d3 = d1 + 2 * plane;
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float z1[16], z3[16], u[16];
+        __syncwarp();
+        tmem_ld16(tq + j, z1);
+        tmem_ld16(tq + 64 + j, z3);
+        tmem_ld16(tq + 128 + j, u);
+        tmem_ld_wait();
+        uint32_t w1[8], w2[8], w3[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float e1[2], eh[2], e3[2];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const float a = z1[2 * i + c], b = z3[2 * i + c], g = u[2 * i + c];
+            const float s = sigmoidf_(a);
+            const float sa = a * s;
+            e1[c] = eta0 * g * b * (s * (1.0f + a * (1.0f - s)));
+            eh[c] = eta1 * sa * b;
+            e3[c] = eta2 * g * sa;
+          }
+          w1[i] = pack_bf16x2(e1[0], e1[1]);
+          w2[i] = pack_bf16x2(eh[0], eh[1]);
+          w3[i] = pack_bf16x2(e3[0], e3[1]);
+        }
+        st_global_v4(d1 + j, w1[0], w1[1], w1[2], w1[3]);
+        st_global_v4(d1 + j + 8, w1[4], w1[5], w1[6], w1[7]);
+        st_global_v4(dh2 + j, w2[0], w2[1], w2[2], w2[3]);
+        st_global_v4(dh2 + j + 8, w2[4], w2[5], w2[6], w2[7]);
+        st_global_v4(d3 + j, w3[0], w3[1], w3[2], w3[3]);
+        st_global_v4(d3 + j + 8, w3[4], w3[5], w3[6], w3[7]);
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Generic batched GEMM with a fused affine epilogue:
+//   C[m][n] = alpha * sum_k A(m,k) B(n,k) + beta * Cin[m][n]
+// stored as fp32 (outf) and/or bf16 (outb) at
+//   base + item * item_stride + m * ld + n,  rows m < m_valid.
+// A is K-major (rows of A in memory) or MN-major (A^T rows in memory), same
+// for B.  Batch index z = split * items + item; split s covers K blocks
+// [s*kb_count, (s+1)*kb_count) and writes output item (s*items + item).
+// B's batch coordinate is (item % zb_mod) + zb_add, read from tmB2 instead of
+// tmB when item / zb_mod == alt_group.
+// Used for: the apply output (Hq W2), the chunk gradients (E^T X), and the
+// three Newton-Schulz products.
+// ---------------------------------------------------------------------------
+struct GemmParams {
+  CUtensorMap tmA, tmB, tmB2;
+  int items;
+  int kb_count;           // K blocks per split
+  int kb_total;           // K blocks in all (the last split may hold fewer)
+  int a_k0, b_k0;
+  int zb_mod, zb_add, alt_group;
+  int m_valid;
+  float alpha, beta;
+  const float* cin;
+  float* outf;
+  __nv_bfloat16* outb;
+  int64_t item_stride, ld;
+};
+
+template <bool A_MN, bool B_MN, int BN>
+struct GemmOp {
+  using Params = GemmParams;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = kStageBytes <= 32768 ? 6 : 4;
+  static constexpr int kTmemCols = TmemCols<BN>::value;
+  struct Tile { int m0, n0, item, out_item, split, zb; bool alt; };
+
+  __device__ static Tile map_tile(const Params& p) {
+    Tile t;
+    t.n0 = blockIdx.x * BN;
+    t.m0 = blockIdx.y * kBM;
+    t.item = blockIdx.z % p.items;
+    t.split = blockIdx.z / p.items;
+    t.out_item = blockIdx.z;
+    t.zb = (t.item % p.zb_mod) + p.zb_add;
+    t.alt = p.alt_group >= 0 && (t.item / p.zb_mod) == p.alt_group;
+    return t;
+  }
+  __device__ static int num_kb(const Params& p, const Tile& t) {
+    const int left = p.kb_total - t.split * p.kb_count;
+    return left < p.kb_count ? left : p.kb_count;
+  }
+  __device__ static uint32_t stage_bytes(const Params&, const Tile&) { return kStageBytes; }
+  __device__ static void prefetch(const Params& p) {
+    tma_prefetch_map(&p.tmA);
+    tma_prefetch_map(&p.tmB);
+    if (p.alt_group >= 0) tma_prefetch_map(&p.tmB2);
+  }
+  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
+    const int kk = (t.split * p.kb_count + kb) * kBK;
+    const int ak = p.a_k0 + kk, bk = p.b_k0 + kk;
+    if (A_MN) {
+      tma_load_3d(st, &p.tmA, bar, t.m0, ak, t.item);
+      tma_load_3d(st + 8192, &p.tmA, bar, t.m0 + 64, ak, t.item);
+    } else {
+      tma_load_3d(st, &p.tmA, bar, ak, t.m0, t.item);
+    }
+    const CUtensorMap* mb = t.alt ? &p.tmB2 : &p.tmB;
+    if (B_MN) {
+#pragma unroll
+      for (int b = 0; b < BN / 64; ++b) tma_load_3d(st + kABytes + b * 8192, mb, bar, t.n0 + b * 64, bk, t.zb);
+    } else {
+      tma_load_3d(st + kABytes, mb, bar, bk, t.n0, t.zb);
+    }
+  }
+  __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {
+    constexpr uint32_t id = idesc_bf16(kBM, BN, A_MN, B_MN);
+    mma_kblock<A_MN, B_MN>(tmem, st, 8192u, st + kABytes, 8192u, id, kb == 0);
+  }
+  __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
+                                  int lane) {
+    const int r = quarter * 32 + lane;
+    const int grow = t.m0 + r;
+    const bool valid = grow < p.m_valid;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int64_t off = static_cast<int64_t>(t.out_item) * p.item_stride +
+                        static_cast<int64_t>(grow) * p.ld + t.n0;
+#pragma unroll 1
+    for (int j = 0; j < BN; j += 16) {
+      float v[16];
+      __syncwarp();
+      tmem_ld16(tq + j, v);
+      tmem_ld_wait();
+      if (valid) {
+        if (p.cin) {
+          const float4* c = reinterpret_cast<const float4*>(p.cin + off + j);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 x = c[i];
+            v[4 * i + 0] = p.alpha * v[4 * i + 0] + p.beta * x.x;
+            v[4 * i + 1] = p.alpha * v[4 * i + 1] + p.beta * x.y;
+            v[4 * i + 2] = p.alpha * v[4 * i + 2] + p.beta * x.z;
+            v[4 * i + 3] = p.alpha * v[4 * i + 3] + p.beta * x.w;
+          }
+        } else if (p.alpha != 1.0f) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] *= p.alpha;
+        }
+        if (p.outf) {
+          float* o = p.outf + off + j;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            st_global_v4(o + 4 * i, __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
+                         __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
+        }
+        if (p.outb) {
+          __nv_bfloat16* o = p.outb + off + j;
+          st_global_v4(o, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                       pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+          st_global_v4(o + 8, pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                       pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+        }
+      }
+    }
+  }
+};
+
+template <class Op>
+constexpr int umma_smem_bytes() {
+  return Op::kStages * Op::kStageBytes + (2 * Op::kStages + 1) * 8 + 16 + 1024;
+}
+
+}  // namespace lact

@@ -1,0 +1,133 @@
+"""torch-facing wrapper of the LaCT TTT layer forward.
+
+torch provides device memory and the stream; the CUDA library does all the
+work.  Shapes follow include/lact.h:
+  q [B,H,Tq,d], k, v [B,H,T,d] (fp32 or bf16), lr [B,H,T,3] fp32,
+  beta [B,H,T] fp32 (momentum only), w1, w3 [Hw,dh,d], w2 [Hw,d,dh] fp32 with
+  Hw = H (shared initial state) or B*H.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import LactError
+
+_DT = {torch.float32: _abi.LACT_F32, torch.bfloat16: _abi.LACT_BF16}
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def make_problem(q, k, w1, chunk, order, rule) -> _abi.LactProblem:
+    B, H, Tq, d = q.shape
+    T = k.shape[2]
+    dh = w1.shape[1]
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    if w1.shape[0] == B * H:
+        w_shared = 0
+    elif w1.shape[0] == H:
+        w_shared = 1
+    else:
+        raise ValueError("w1/w2/w3 must hold H (shared) or B*H initial states")
+    return _abi.problem(B, H, T, Tq, d, dh, chunk, order, rule, _DT[q.dtype], w_shared)
+
+
+def _check(q, k, v, lr, beta, w1, w2, w3, device_kind):
+    for name, t in (("q", q), ("k", k), ("v", v), ("lr", lr), ("w1", w1), ("w2", w2), ("w3", w3),
+                    ("beta", beta)):
+        if t is None:
+            continue
+        if t.device.type != device_kind:
+            raise ValueError(f"{name} must be on {device_kind}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    for name, t in (("lr", lr), ("beta", beta), ("w1", w1), ("w2", w2), ("w3", w3)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+
+
+def workspace_bytes(q, k, w1, chunk, order, rule) -> int:
+    return _abi.workspace_bytes(make_problem(q, k, w1, chunk, order, rule))
+
+
+def launch_count(q, k, w1, chunk, order, rule) -> int:
+    return _abi.launch_count(make_problem(q, k, w1, chunk, order, rule))
+
+
+def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_out=None,
+            workspace=None, stream=None):
+    """Runs the layer on the current CUDA device.  Returns (out, w1o, w2o, w3o).
+    Optional `out`, `w_out` (a 3-tuple) and `workspace` (uint8 tensor) avoid
+    allocations; `stream` defaults to torch's current stream."""
+    _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
+    p = make_problem(q, k, w1, chunk, order, rule)
+    B, H, Tq, d = q.shape
+    dh = w1.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if w_out is None:
+        w_out = (torch.empty((B * H, dh, d), device=q.device, dtype=torch.float32),
+                 torch.empty((B * H, d, dh), device=q.device, dtype=torch.float32),
+                 torch.empty((B * H, dh, d), device=q.device, dtype=torch.float32))
+    need = _abi.workspace_bytes(p)
+    if need == 0:
+        raise LactError(_abi.LACT_EINVAL, "lact_ttt_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = _abi.lib().lact_ttt_fwd(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(beta), _ptr(w1), _ptr(w2),
+        _ptr(w3), _ptr(out), _ptr(w_out[0]), _ptr(w_out[1]), _ptr(w_out[2]), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
+    if rc != _abi.LACT_OK:
+        raise LactError(rc, "lact_ttt_fwd")
+    return out, w_out[0], w_out[1], w_out[2]
+
+
+def ttt_fwd_host(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out, w_out, workspace,
+                 stream=None):
+    """The same forward from HOST tensors (pinned for full-speed copies): the
+    library copies in, runs, copies `out` and `w_out` back and returns when
+    they are valid.  `workspace` is a device uint8 tensor of
+    host_workspace_bytes() bytes."""
+    _check(q, k, v, lr, beta, w1, w2, w3, "cpu")
+    p = make_problem(q, k, w1, chunk, order, rule)
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device)
+    rc = _abi.lib().lact_ttt_fwd_host(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(beta), _ptr(w1), _ptr(w2),
+        _ptr(w3), _ptr(out), _ptr(w_out[0]), _ptr(w_out[1]), _ptr(w_out[2]), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
+    if rc != _abi.LACT_OK:
+        raise LactError(rc, "lact_ttt_fwd_host")
+    return out, w_out[0], w_out[1], w_out[2]
+
+
+def host_workspace_bytes(q, k, w1, chunk, order, rule) -> int:
+    return _abi.host_workspace_bytes(make_problem(q, k, w1, chunk, order, rule))
+
+
+def status(stream=None) -> int:
+    """Waits for the stream and returns (and clears) the device status word."""
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(_abi.lib().lact_ttt_status(ctypes.c_void_p(stream.cuda_stream)))
+
+
+def device_check() -> int:
+    return int(_abi.lib().lact_device_check())
+
+
+def selftest_wait_timeout(budget_cycles: int, stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(_abi.lib().lact_selftest_wait_timeout(int(budget_cycles),
+                                                    ctypes.c_void_p(stream.cuda_stream)))

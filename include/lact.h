@@ -1,0 +1,171 @@
+/*
+ * lact.h -- C ABI of the B200 (sm_100a) LaCT fast-weight TTT layer forward.
+ *
+ * The layer (Large-Chunk Test-Time Training).  Sources are cited by page
+ * title and section:
+ *   [P1] "LaCT架构核心思想解析" (gsyq.cn) §1.2, §2.1, §2.2
+ *   [P2] "大块测试时训练（LaCT）技术解析" (dpshk.com) §2.1, §2.2.1
+ *   [P3] "LaCT：以大分块更新人工智能的临时记忆" (iplexlaw.co.kr), sections
+ *        「局部注意力与非线性记忆相互补充」 and 「更新顺序必须遵守信息可见范围」
+ *
+ * Per (batch b, head h) the layer keeps a SwiGLU fast-weight net
+ *     f_W(x) = W2 (silu(W1 x) * (W3 x)),   W1, W3: [dh, d],  W2: [d, dh]
+ * ([P3] three-matrix SwiGLU memory; [P1 §1.2] shapes).  Queries and keys are
+ * first mapped to silu(x)/||silu(x)|| over the head dim ([P1 §1.2]).  The
+ * sequence is cut into chunks of `chunk` tokens (the last one may be
+ * shorter).  For each chunk c:
+ *   apply   o_t = f_W(q_t) for the chunk's queries ([P2 §2.1], eq. 2);
+ *   update  G_j = d/dW_j [ -sum_{i in c} lr[i,j] <f_W(k_i), v_i> ]
+ *           (chunk-summed, per-token rates; j = 0: W1, 1: W2, 2: W3;
+ *           [P2 §2.1] eqs. 4-5, [P3]), then a rule
+ *             GD:        U = G
+ *             momentum:  M <- mean_{i in c}(beta_i) M + G, U = M   [P1 §1.2]
+ *             Muon:      U = NewtonSchulz5(G / (||G||_F + 1e-7)),
+ *                        quintic (3.4445, -4.7750, 2.0315)         [P2 §2.2.1]
+ *           and W_j <- W_j - U_j with every row of W_j scaled back to its
+ *           norm before the update ([P2 §2.2.1] eq. 8; rows of W1/W3 have
+ *           length d, rows of W2 length dh).
+ * Order ([P3] 「更新顺序…」, [P1 §2.2]): LACT_APPLY_THEN_UPDATE (causal
+ * sequences: chunk c reads the state left by chunks < c) or
+ * LACT_UPDATE_THEN_APPLY (sets: chunk c reads the state after itself).
+ *
+ * Memory: every pointer passed to lact_ttt_fwd is a DEVICE pointer owned by
+ * the caller; the library allocates nothing.  Calls are asynchronous on the
+ * caller's CUDA stream (`stream` is a cudaStream_t, NULL = legacy default).
+ * Layouts (all dense, row-major, no padding):
+ *   q      [B, H, Tq, d]  dtype        raw queries (the prologue runs inside)
+ *   k, v   [B, H, T, d]   dtype        raw keys, values
+ *   lr     [B, H, T, 3]   float32      per-token rates, already softplus-ed,
+ *                                      columns (W1, W2, W3)
+ *   beta   [B, H, T]      float32      per-token momentum, already sigmoid-ed;
+ *                                      read only when rule == MOMENTUM
+ *   w1, w3 [Hw, dh, d]    float32      initial fast weights, Hw = H (shared
+ *   w2     [Hw, d, dh]    float32        by the batch, w_shared = 1) or B*H
+ *   out    [B, H, Tq, d]  dtype        layer output
+ *   w1_out, w3_out [B*H, dh, d], w2_out [B*H, d, dh]  float32  final state;
+ *          each may alias the matching input exactly (in-place update,
+ *          only when w_shared = 0); any other overlap is rejected.
+ *   dtype = LACT_F32 (fp32 path, SIMT kernels) or LACT_BF16 (bf16 tensor-core
+ *   path; fp32 fast-weight masters, fp32 accumulation).
+ * Alignment: all device pointers 16-byte aligned.
+ * Limits: 1 <= d <= 512, 1 <= dh <= 4096 (bf16 path: both multiples of 64);
+ *   B*H <= 4096; 1 <= T, Tq <= 2^30; chunk >= 1 (a chunk >= T means one
+ *   chunk); Tq == T unless there is a single chunk.
+ *
+ * Errors: every entry point returns LACT_OK (0) or a negative code.  Argument
+ * errors (LACT_EINVAL, LACT_ENOSPC) are found before anything is enqueued.
+ * LACT_ECUDA means a launch failed part way; the outputs are then undefined.
+ * Device-side failures (a bounded wait inside a kernel that gave up) are
+ * recorded in a device status word and reported by lact_ttt_status().
+ */
+#ifndef LACT_H
+#define LACT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  LACT_OK = 0,
+  LACT_EINVAL = -1,       /* bad shape, dtype, order, rule, null or misaligned
+                             pointer, partial aliasing, unsupported size */
+  LACT_ENOSPC = -2,       /* workspace smaller than lact_ttt_workspace_bytes() */
+  LACT_ECUDA = -3,        /* a CUDA runtime call or kernel launch failed */
+  LACT_ETIMEOUT = -4,     /* a bounded device wait gave up (see lact_ttt_status) */
+  LACT_ENODEV = -5        /* the current device is not an sm_100 GPU */
+};
+
+enum { LACT_F32 = 0, LACT_BF16 = 1 };
+enum { LACT_APPLY_THEN_UPDATE = 0, LACT_UPDATE_THEN_APPLY = 1 };
+enum { LACT_RULE_GD = 0, LACT_RULE_MOMENTUM = 1, LACT_RULE_MUON = 2 };
+
+/* Problem description shared by every entry point. */
+typedef struct lact_problem {
+  int64_t B, H;     /* batch, heads */
+  int64_t T;        /* key/value tokens per (b, h) */
+  int64_t Tq;       /* query tokens per (b, h) */
+  int64_t d, dh;    /* head dim, fast-net hidden dim */
+  int64_t chunk;    /* tokens per update (the last chunk may be shorter) */
+  int32_t order;    /* LACT_APPLY_THEN_UPDATE or LACT_UPDATE_THEN_APPLY */
+  int32_t rule;     /* LACT_RULE_GD, LACT_RULE_MOMENTUM or LACT_RULE_MUON */
+  int32_t dtype;    /* LACT_F32 or LACT_BF16: q, k, v and out */
+  int32_t w_shared; /* 1: w1/w2/w3 hold H states shared over the batch; 0: B*H */
+} lact_problem;
+
+/* Device scratch bytes lact_ttt_fwd needs for problem *p (0 if *p is invalid).
+ * Pure host arithmetic; needs no GPU. */
+size_t lact_ttt_workspace_bytes(const lact_problem* p);
+
+/* The layer forward, enqueued on `stream`.  All tensor pointers are device
+ * pointers in the layouts above; `workspace` is device scratch of at least
+ * lact_ttt_workspace_bytes(p) bytes, 256-byte aligned, owned by the caller
+ * and not touched by anything else until the stream reaches the end of this
+ * call.  beta may be NULL unless rule == LACT_RULE_MOMENTUM. */
+int lact_ttt_fwd(const lact_problem* p,
+                 const void* q, const void* k, const void* v,
+                 const float* lr, const float* beta,
+                 const float* w1, const float* w2, const float* w3,
+                 void* out, float* w1_out, float* w2_out, float* w3_out,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Device scratch bytes lact_ttt_fwd_host needs: lact_ttt_workspace_bytes(p)
+ * plus room for device copies of every input and output. */
+size_t lact_ttt_host_workspace_bytes(const lact_problem* p);
+
+/* The same forward with every tensor pointer a HOST pointer (pinned memory
+ * gives full-speed copies).  Copies the inputs into `workspace` (device
+ * memory of lact_ttt_host_workspace_bytes(p) bytes), runs lact_ttt_fwd on
+ * `stream`, copies out and w*_out back to the host, and returns after the
+ * stream has reached that point (the host buffers are then valid). */
+int lact_ttt_fwd_host(const lact_problem* p,
+                      const void* q, const void* k, const void* v,
+                      const float* lr, const float* beta,
+                      const float* w1, const float* w2, const float* w3,
+                      void* out, float* w1_out, float* w2_out, float* w3_out,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Waits for `stream`, then returns and clears the device status word of the
+ * current device: LACT_OK, or LACT_ETIMEOUT if a bounded wait inside one of
+ * this library's kernels gave up since the last call (its results are then
+ * invalid), or LACT_ECUDA if the stream reported an error. */
+int lact_ttt_status(void* stream);
+
+/* LACT_OK if the current CUDA device is an sm_100 part this library was
+ * built for, LACT_ENODEV otherwise (or LACT_ECUDA if there is no device). */
+int lact_device_check(void);
+
+/* Kernel launches one lact_ttt_fwd call of problem *p enqueues (0 if *p is
+ * invalid).  Pure host arithmetic. */
+int64_t lact_ttt_launch_count(const lact_problem* p);
+
+/* Failure-path self-test: launches one block whose thread waits on a shared
+ * memory barrier that nothing ever completes, with a wait budget of
+ * `budget_cycles` SM clock cycles (1 <= budget_cycles <= 2^31).  The wait
+ * gives up, records LACT_ETIMEOUT in the device status word and the kernel
+ * returns; the context stays usable.  Returns the launch status; read the
+ * outcome with lact_ttt_status(stream).  Restores the normal budget after
+ * the launch. */
+int lact_selftest_wait_timeout(int64_t budget_cycles, void* stream);
+
+/* Launch profiler.  While enabled, every kernel launch of lact_ttt_fwd is
+ * bracketed by a pair of CUDA events recorded on the launching stream.
+ * lact_profile_read waits for those events, returns per kernel kind the
+ * number of launches and the summed device milliseconds since the last read
+ * (arrays of lact_kernel_kinds() entries), and forgets them.  Off by default;
+ * not meant for use while a stream is being captured. */
+int lact_profile_enable(int on);
+int lact_profile_read(int64_t* launches, double* ms, int nkinds);
+int lact_kernel_kinds(void);
+const char* lact_kernel_name(int kind);
+
+/* Static text for a status code. */
+const char* lact_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LACT_H */

@@ -1,0 +1,103 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and its host logic (argument checks, workspace plan, launch
+count) behaves.  No call here touches a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunk_test_b200 as ct
+from chunk_test_b200 import _abi
+from lact_inputs import WORKLOADS, BF16
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "lact.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lact_\w+)\s*\(", src)))
+
+
+def test_library_builds_and_loads():
+    from chunk_test_b200 import build
+    build.build()
+    assert os.path.exists(_abi.LIB_PATH)
+    assert ct.lib() is not None
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = _declared()
+    assert "lact_ttt_fwd" in names and "lact_ttt_workspace_bytes" in names
+    handle = ctypes.CDLL(_abi.LIB_PATH)
+    for n in names:
+        assert hasattr(handle, n), n
+    assert set(names) == set(_abi.SIGNATURES), "binding and header disagree"
+
+
+def _prob(w, **kw):
+    args = dict(B=w.B, H=w.H, T=w.T, Tq=w.Tq, d=w.d, dh=w.dh, chunk=w.chunk, order=w.order,
+                rule=w.rule, dtype=1 if w.dtype == BF16 else 0, w_shared=1)
+    args.update(kw)
+    return _abi.problem(**args)
+
+
+@pytest.mark.parametrize("idx", sorted(WORKLOADS))
+def test_workspace_and_launch_count_for_each_workload(idx):
+    w = WORKLOADS[idx]
+    p = _prob(w)
+    ws = _abi.workspace_bytes(p)
+    assert ws > 0 and ws % 256 == 0
+    assert _abi.host_workspace_bytes(p) > ws
+    n = _abi.launch_count(p)
+    per_chunk = {0: 5, 1: 5, 2: 22}[w.rule] if w.dtype == BF16 else None
+    if per_chunk is not None:
+        fixed = 3 + (1 if w.rule == 1 else 0)
+        assert n == fixed + per_chunk * w.n_chunks
+
+
+@pytest.mark.parametrize("bad", [
+    dict(B=0), dict(H=0), dict(T=0), dict(d=0), dict(dh=0), dict(chunk=0), dict(order=2),
+    dict(rule=3), dict(dtype=7), dict(w_shared=2), dict(Tq=100),   # Tq != T with many chunks
+    dict(d=96), dict(dh=100), dict(d=576, dh=1024),               # bf16 tile limits
+])
+def test_invalid_problems_are_rejected_by_the_host(bad):
+    p = _prob(WORKLOADS[2], **bad)
+    assert _abi.workspace_bytes(p) == 0
+    assert _abi.launch_count(p) == 0
+    nul = ctypes.c_void_p(0)
+    rc = ct.lib().lact_ttt_fwd(ctypes.byref(p), *([nul] * 12), nul, ctypes.c_size_t(0), nul)
+    assert rc == ct.LACT_EINVAL
+
+
+def test_null_and_misaligned_pointers_are_rejected_without_a_gpu():
+    p = _prob(WORKLOADS[1])
+    fake = [ctypes.c_void_p((1 << 30) * (i + 1)) for i in range(12)]
+    ws = ctypes.c_void_p(1 << 40)
+    lib = ct.lib()
+    args = list(fake)
+    args[0] = ctypes.c_void_p(0)
+    assert lib.lact_ttt_fwd(ctypes.byref(p), *args, ws, ctypes.c_size_t(1 << 40), None) == ct.LACT_EINVAL
+    args = list(fake)
+    args[2] = ctypes.c_void_p((3 << 30) + 8)                   # v not 16-byte aligned
+    assert lib.lact_ttt_fwd(ctypes.byref(p), *args, ws, ctypes.c_size_t(1 << 40), None) == ct.LACT_EINVAL
+    # workspace too small
+    assert lib.lact_ttt_fwd(ctypes.byref(p), *fake, ws, ctypes.c_size_t(16), None) == ct.LACT_ENOSPC
+    # w2_out overlapping w3_out
+    args = list(fake)
+    args[10] = ctypes.c_void_p(args[11].value)
+    assert lib.lact_ttt_fwd(ctypes.byref(p), *args, ws, ctypes.c_size_t(1 << 40), None) == ct.LACT_EINVAL
+
+
+def test_ragged_and_single_chunk_problems_are_accepted():
+    base = WORKLOADS[1]
+    assert _abi.workspace_bytes(_prob(base, T=1000, Tq=1000, chunk=384)) > 0
+    assert _abi.workspace_bytes(_prob(base, T=1000, Tq=77, chunk=1000)) > 0
+    assert _abi.workspace_bytes(_prob(base, T=1000, Tq=77, chunk=4096)) > 0
+    assert _abi.workspace_bytes(_prob(base, d=5, dh=7, dtype=0)) > 0      # fp32: any size
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5):
+        assert isinstance(ct.status_string(code), str) and ct.status_string(code)
