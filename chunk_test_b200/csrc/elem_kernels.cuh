@@ -34,10 +34,13 @@ __device__ __forceinline__ float warp_sum(float v) {
 // ---------------------------------------------------------------------------
 constexpr int kMaxRowPerLane = 16;  // d <= 512
 
+// With kh_lo (bf16 only) the keys are also written as the lo part of a
+// split-bf16 pair (kh_lo = bf16(k^ - kh)).
 template <typename T>
 __global__ void __launch_bounds__(256) k_qk_prologue(const T* __restrict__ q, T* __restrict__ qh,
                                                      int64_t q_rows, const T* __restrict__ k,
-                                                     T* __restrict__ kh, int64_t k_rows, int d) {
+                                                     T* __restrict__ kh, int64_t k_rows, int d,
+                                                     T* __restrict__ kh_lo) {
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= q_rows + k_rows) return;
@@ -56,11 +59,25 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const T* __restrict__ q, T*
   }
   ss = warp_sum(ss);
   const float inv = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+  T* dst_lo = (kh_lo && row >= q_rows) ? kh_lo + (row - q_rows) * d : nullptr;
 #pragma unroll
   for (int i = 0; i < kMaxRowPerLane; ++i) {
     const int c = lane + 32 * i;
-    if (c < d) dst[c] = from_f<T>(s[i] * inv);
+    if (c < d) {
+      const float y = s[i] * inv;
+      const T hi = from_f<T>(y);
+      dst[c] = hi;
+      if (dst_lo) dst_lo[c] = from_f<T>(y - to_f(hi));
+    }
   }
+}
+
+// bf16 shadow of an fp32 value, and its split-bf16 lo part when asked for.
+__device__ __forceinline__ void store_shadow(__nv_bfloat16* hi, __nv_bfloat16* lo, int64_t o, float x) {
+  if (!hi) return;
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  hi[o] = h;
+  if (lo) lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
 }
 
 // ---------------------------------------------------------------------------
@@ -74,6 +91,7 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
                                                     int w_shared, int BH, int d, int dh,
                                                     float* __restrict__ Wm,
                                                     __nv_bfloat16* __restrict__ Ws,
+                                                    __nv_bfloat16* __restrict__ Ws_lo,
                                                     float* __restrict__ Mm) {
   __shared__ float tile[32][33];
   const int j = blockIdx.z / BH, bh = blockIdx.z % BH;
@@ -95,7 +113,7 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
         const int64_t o = (static_cast<int64_t>(j) * BH + bh) * plane + static_cast<int64_t>(r) * d + c;
         const float x = tile[tx][i];
         Wm[o] = x;
-        if (Ws) Ws[o] = __float2bfloat16_rn(x);
+        store_shadow(Ws, Ws_lo, o, x);
         if (Mm) Mm[o] = 0.f;
       }
     }
@@ -107,7 +125,7 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
         const int64_t o = (static_cast<int64_t>(j) * BH + bh) * plane + static_cast<int64_t>(r) * d + c;
         const float x = s[static_cast<int64_t>(r) * d + c];
         Wm[o] = x;
-        if (Ws) Ws[o] = __float2bfloat16_rn(x);
+        store_shadow(Ws, Ws_lo, o, x);
         if (Mm) Mm[o] = 0.f;
       }
     }
@@ -176,6 +194,7 @@ __global__ void __launch_bounds__(256) k_beta_mean(const float* __restrict__ bet
 struct RuleParams {
   float* Wm;
   __nv_bfloat16* Ws;      // bf16 shadow or null
+  __nv_bfloat16* Ws_lo;   // split-bf16 lo part of the shadow or null
   const float* S;         // [splits][3][BH][dh][d]
   int splits;
   int64_t split_stride;   // elements between partial planes
@@ -224,7 +243,7 @@ __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
     for (int c = lane; c < p.d; c += 32) {
       const float w = p.Wm[base + c] * sc;
       p.Wm[base + c] = w;
-      if (p.Ws) p.Ws[base + c] = __float2bfloat16_rn(w);
+      store_shadow(p.Ws, p.Ws_lo, base + c, w);
     }
   } else {
     __shared__ float red_o[8][32], red_n[8][32], scale[32];
@@ -264,7 +283,7 @@ __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
         const int64_t o = base + static_cast<int64_t>(r) * p.d + c;
         const float w = p.Wm[o] * sc;
         p.Wm[o] = w;
-        if (p.Ws) p.Ws[o] = __float2bfloat16_rn(w);
+        store_shadow(p.Ws, p.Ws_lo, o, w);
       }
     }
   }
@@ -313,7 +332,8 @@ __global__ void __launch_bounds__(256) k_ns_sumsq(const float* __restrict__ S, i
 }
 
 __global__ void __launch_bounds__(256) k_ns_scale(float* __restrict__ Y,
-                                                  __nv_bfloat16* __restrict__ Yb, int64_t plane,
+                                                  __nv_bfloat16* __restrict__ Yb,
+                                                  __nv_bfloat16* __restrict__ Yb_lo, int64_t plane,
                                                   const float* __restrict__ part, int nblk,
                                                   float eps) {
   __shared__ float sc;
@@ -330,7 +350,7 @@ __global__ void __launch_bounds__(256) k_ns_scale(float* __restrict__ Y,
   for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
     const float y = Y[base + e] * sc;
     Y[base + e] = y;
-    if (Yb) Yb[base + e] = __float2bfloat16_rn(y);
+    store_shadow(Yb, Yb_lo, base + e, y);
   }
 }
 

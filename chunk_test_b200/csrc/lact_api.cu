@@ -41,6 +41,7 @@ struct Dims {
   int64_t q_rows;    // rows per head of the per-chunk query buffer (Hq)
   int splits;        // token splits of the gradient contraction (bf16)
   int bn;            // N tile over d (bf16 GEMMs)
+  bool split;        // split-bf16 update path (bf16 + Muon)
 };
 
 static int choose_bn(int64_t d) {
@@ -71,6 +72,7 @@ static int validate(const lact_problem* p, Dims& D) {
   D.q_rows = rup(D.nch == 1 ? D.Tq : D.chunk, 128);
   if (D.key_rows / 128 > 65535 || D.q_rows / 128 > 65535) return LACT_EINVAL;
   D.bn = choose_bn(D.d);
+  D.split = D.dtype == LACT_BF16 && D.rule == LACT_RULE_MUON;
   // Token splits of the gradient contraction: fill ~2 waves of 148 SMs when
   // the output tiles alone do not.
   const int64_t tiles = (D.d / D.bn) * cdiv(D.dh, 128) * 3 * D.BH;
@@ -84,11 +86,12 @@ static int validate(const lact_problem* p, Dims& D) {
 }
 
 struct Bufs {
-  void* qh; void* kh;
-  float* Wm; __nv_bfloat16* Ws; float* P; float* Mm; float* bbar;
-  void* E; void* Hq; float* Z;
-  float* Yf[2]; __nv_bfloat16* Yb[2];
-  float* Af; __nv_bfloat16* Ab; float* Bf; __nv_bfloat16* Bb; float* part;
+  void* qh; void* kh; __nv_bfloat16* kh_lo;
+  float* Wm; __nv_bfloat16* Ws; __nv_bfloat16* Ws_lo; float* P; float* Mm; float* bbar;
+  void* E; void* E_lo; void* Hq; float* Z;
+  float* Yf[2]; __nv_bfloat16* Yb[2]; __nv_bfloat16* Yb_lo[2];
+  float* Af; __nv_bfloat16* Ab; __nv_bfloat16* Ab_lo; float* Bf; __nv_bfloat16* Bb;
+  __nv_bfloat16* Bb_lo; float* part;
 };
 
 struct Bump {
@@ -108,25 +111,33 @@ static void plan(const Dims& D, Bump& bp, Bufs& b) {
   const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane;
   b.qh = bp.take<uint8_t>(D.BH * D.Tq * D.d * esz);
   b.kh = bp.take<uint8_t>(D.BH * D.T * D.d * esz);
+  if (D.split) b.kh_lo = bp.take<__nv_bfloat16>(D.BH * D.T * D.d);
   b.Wm = bp.take<float>(planes);
   if (bf) b.Ws = bp.take<__nv_bfloat16>(planes);
+  if (D.split) b.Ws_lo = bp.take<__nv_bfloat16>(planes);
   b.P = bp.take<float>((bf ? D.splits : 1) * planes);
   if (D.rule == LACT_RULE_MOMENTUM) {
     b.Mm = bp.take<float>(planes);
     b.bbar = bp.take<float>(D.BH * D.nch);
   }
   b.E = bp.take<uint8_t>(3 * D.BH * D.key_rows * D.dh * esz);
+  if (D.split) b.E_lo = bp.take<uint8_t>(3 * D.BH * D.key_rows * D.dh * esz);
   b.Hq = bp.take<uint8_t>(D.BH * D.q_rows * D.dh * esz);
   if (!bf) b.Z = bp.take<float>(3 * D.BH * (D.key_rows > D.q_rows ? D.key_rows : D.q_rows) * D.dh);
   if (D.rule == LACT_RULE_MUON) {
     for (int i = 0; i < 2; ++i) {
       b.Yf[i] = bp.take<float>(planes);
       if (bf) b.Yb[i] = bp.take<__nv_bfloat16>(planes);
+      if (D.split) b.Yb_lo[i] = bp.take<__nv_bfloat16>(planes);
     }
     b.Af = bp.take<float>(3 * D.BH * D.d * D.d);
     if (bf) {
       b.Ab = bp.take<__nv_bfloat16>(3 * D.BH * D.d * D.d);
       b.Bb = bp.take<__nv_bfloat16>(3 * D.BH * D.d * D.d);
+      if (D.split) {
+        b.Ab_lo = bp.take<__nv_bfloat16>(3 * D.BH * D.d * D.d);
+        b.Bb_lo = bp.take<__nv_bfloat16>(3 * D.BH * D.d * D.d);
+      }
     } else {
       b.Bf = bp.take<float>(3 * D.BH * D.d * D.d);
     }
@@ -187,15 +198,20 @@ static cudaError_t launch_umma(dim3 grid, const typename Op::Params& p, cudaStre
   return cudaGetLastError();
 }
 
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, bool SPLIT = false>
 static cudaError_t launch_gemm(int bn, dim3 grid, const GemmParams& p, cudaStream_t st) {
   switch (bn) {
-    case 64: return launch_umma<GemmOp<A_MN, B_MN, 64>>(grid, p, st);
-    case 128: return launch_umma<GemmOp<A_MN, B_MN, 128>>(grid, p, st);
-    case 192: return launch_umma<GemmOp<A_MN, B_MN, 192>>(grid, p, st);
-    case 256: return launch_umma<GemmOp<A_MN, B_MN, 256>>(grid, p, st);
+    case 64: return launch_umma<GemmOp<A_MN, B_MN, 64, SPLIT>>(grid, p, st);
+    case 128: return launch_umma<GemmOp<A_MN, B_MN, 128, SPLIT>>(grid, p, st);
+    case 192: return launch_umma<GemmOp<A_MN, B_MN, 192, SPLIT>>(grid, p, st);
+    case 256: return launch_umma<GemmOp<A_MN, B_MN, 256, SPLIT>>(grid, p, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <bool A_MN, bool B_MN>
+static cudaError_t launch_gemm_any(bool split, int bn, dim3 grid, const GemmParams& p, cudaStream_t st) {
+  return split ? launch_gemm<A_MN, B_MN, true>(bn, grid, p, st) : launch_gemm<A_MN, B_MN, false>(bn, grid, p, st);
 }
 
 // Kernel kinds, for the launch profiler (lact_profile_*).
@@ -291,7 +307,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
   // Fast-weight masters (+ bf16 shadows), momentum = 0.
   L(K_INIT, [&] {
     k_init_state<<<tile_grid, tile_block, 0, st>>>(in.w1, in.w2, in.w3, static_cast<int>(D.H),
-                                                   D.w_shared, BH, d, dh, b.Wm, b.Ws, b.Mm);
+                                                   D.w_shared, BH, d, dh, b.Wm, b.Ws, b.Ws_lo, b.Mm);
     return cudaGetLastError();
   });
   // q^, k^ = silu + L2 norm rows.
@@ -301,11 +317,12 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
     if (bf)
       k_qk_prologue<__nv_bfloat16><<<blocks, 256, 0, st>>>(
           static_cast<const __nv_bfloat16*>(in.q), static_cast<__nv_bfloat16*>(b.qh), D.BH * D.Tq,
-          static_cast<const __nv_bfloat16*>(in.k), static_cast<__nv_bfloat16*>(b.kh), D.BH * D.T, d);
+          static_cast<const __nv_bfloat16*>(in.k), static_cast<__nv_bfloat16*>(b.kh), D.BH * D.T, d,
+          b.kh_lo);
     else
       k_qk_prologue<float><<<blocks, 256, 0, st>>>(
           static_cast<const float*>(in.q), static_cast<float*>(b.qh), D.BH * D.Tq,
-          static_cast<const float*>(in.k), static_cast<float*>(b.kh), D.BH * D.T, d);
+          static_cast<const float*>(in.k), static_cast<float*>(b.kh), D.BH * D.T, d, nullptr);
     return cudaGetLastError();
   });
   if (D.rule == LACT_RULE_MOMENTUM) {
@@ -384,10 +401,15 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           if (!map3d(&f.tmX, b.kh, d, D.T, BH, 64, 128) || !map3d(&f.tmV, in.v, d, D.T, BH, 64, 128) ||
               !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 64))
             return cudaErrorInvalidValue;
+          if (D.split && (!map3d(&f.tmXlo, b.kh_lo, d, D.T, BH, 64, 128) ||
+                          !map3d(&f.tmWlo, b.Ws_lo, d, dh, 3 * BH, 64, 64)))
+            return cudaErrorInvalidValue;
           f.bh_count = BH; f.x_row0 = static_cast<int>(c0); f.rows_valid = nc; f.kb_count = d / 64;
           f.dh = dh; f.T = static_cast<int>(D.T); f.e = static_cast<__nv_bfloat16*>(b.E);
+          f.e_lo = static_cast<__nv_bfloat16*>(b.E_lo);
           f.buf_rows = D.key_rows; f.lr = in.lr;
-          return launch_umma<FwdOp<true>>(dim3(dh / 64, cdiv(nc, 128), BH), f, st);
+          const dim3 grid(dh / 64, cdiv(nc, 128), BH);
+          return D.split ? launch_umma<FwdOp<true, true>>(grid, f, st) : launch_umma<FwdOp<true>>(grid, f, st);
         });
         const int kbt = static_cast<int>(cdiv(nc, 64));
         const int kbp = static_cast<int>(cdiv(kbt, D.splits));
@@ -397,11 +419,14 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           if (!map3d(&g.tmA, b.E, dh, D.key_rows, 3 * BH, 64, 64) || !map3d(&g.tmB, b.kh, d, D.T, BH, 64, 64) ||
               !map3d(&g.tmB2, in.v, d, D.T, BH, 64, 64))
             return cudaErrorInvalidValue;
+          if (D.split && (!map3d(&g.tmAlo, b.E_lo, dh, D.key_rows, 3 * BH, 64, 64) ||
+                          !map3d(&g.tmBlo, b.kh_lo, d, D.T, BH, 64, 64)))
+            return cudaErrorInvalidValue;
           g.items = 3 * BH; g.kb_count = kbp; g.kb_total = kbt;
           g.a_k0 = 0; g.b_k0 = static_cast<int>(c0);
           g.zb_mod = BH; g.zb_add = 0; g.alt_group = 1; g.m_valid = dh;
           g.outf = b.P; g.item_stride = plane; g.ld = d;
-          return launch_gemm<true, true>(D.bn, dim3(d / D.bn, cdiv(dh, 128), splits * 3 * BH), g, st);
+          return launch_gemm_any<true, true>(D.split, D.bn, dim3(d / D.bn, cdiv(dh, 128), splits * 3 * BH), g, st);
         });
       } else {
         const int64_t zpl = D.BH * D.key_rows * D.dh;
@@ -440,8 +465,8 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           return cudaGetLastError();
         });
         L(K_NS_SCALE, [&] {
-          k_ns_scale<<<dim3(kNsBlocks, 3 * BH), 256, 0, st>>>(b.Yf[0], b.Yb[0], plane, b.part, kNsBlocks,
-                                                              kNsEps);
+          k_ns_scale<<<dim3(kNsBlocks, 3 * BH), 256, 0, st>>>(b.Yf[0], b.Yb[0], b.Yb_lo[0], plane, b.part,
+                                                              kNsBlocks, kNsEps);
           return cudaGetLastError();
         });
         for (int it = 0; it < kNsSteps; ++it) {
@@ -451,31 +476,41 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
               GemmParams g = gemm_params();
               if (!map3d(&g.tmA, b.Yb[cur], d, dh, 3 * BH, 64, 64)) return cudaErrorInvalidValue;
               g.tmB = g.tmA;
+              if (D.split) {
+                if (!map3d(&g.tmAlo, b.Yb_lo[cur], d, dh, 3 * BH, 64, 64)) return cudaErrorInvalidValue;
+                g.tmBlo = g.tmAlo;
+              }
               g.items = 3 * BH; g.kb_count = g.kb_total = static_cast<int>(cdiv(dh, 64));
               g.zb_mod = 3 * BH; g.m_valid = d;
-              g.outf = b.Af; g.outb = b.Ab; g.item_stride = D.d * D.d; g.ld = d;
-              return launch_gemm<true, true>(D.bn, dim3(d / D.bn, cdiv(d, 128), 3 * BH), g, st);
+              g.outf = b.Af; g.outb = b.Ab; g.outb_lo = b.Ab_lo; g.item_stride = D.d * D.d; g.ld = d;
+              return launch_gemm_any<true, true>(D.split, D.bn, dim3(d / D.bn, cdiv(d, 128), 3 * BH), g, st);
             });
             L(K_NS_POLY, [&] {  // B = b A + c A A
               GemmParams g = gemm_params();
               if (!map3d(&g.tmA, b.Ab, d, d, 3 * BH, 64, 128) || !map3d(&g.tmB, b.Ab, d, d, 3 * BH, 64, D.bn))
                 return cudaErrorInvalidValue;
+              if (D.split && (!map3d(&g.tmAlo, b.Ab_lo, d, d, 3 * BH, 64, 128) ||
+                              !map3d(&g.tmBlo, b.Ab_lo, d, d, 3 * BH, 64, D.bn)))
+                return cudaErrorInvalidValue;
               g.items = 3 * BH; g.kb_count = g.kb_total = d / 64;
               g.zb_mod = 3 * BH; g.m_valid = d;
               g.alpha = kNsC; g.beta = kNsB; g.cin = b.Af;
-              g.outb = b.Bb; g.item_stride = D.d * D.d; g.ld = d;
-              return launch_gemm<false, false>(D.bn, dim3(d / D.bn, cdiv(d, 128), 3 * BH), g, st);
+              g.outb = b.Bb; g.outb_lo = b.Bb_lo; g.item_stride = D.d * D.d; g.ld = d;
+              return launch_gemm_any<false, false>(D.split, D.bn, dim3(d / D.bn, cdiv(d, 128), 3 * BH), g, st);
             });
             L(K_NS_UPDATE, [&] {  // X <- a X + X B
               GemmParams g = gemm_params();
               if (!map3d(&g.tmA, b.Yb[cur], d, dh, 3 * BH, 64, 128) ||
                   !map3d(&g.tmB, b.Bb, d, d, 3 * BH, 64, D.bn))
                 return cudaErrorInvalidValue;
+              if (D.split && (!map3d(&g.tmAlo, b.Yb_lo[cur], d, dh, 3 * BH, 64, 128) ||
+                              !map3d(&g.tmBlo, b.Bb_lo, d, d, 3 * BH, 64, D.bn)))
+                return cudaErrorInvalidValue;
               g.items = 3 * BH; g.kb_count = g.kb_total = d / 64;
               g.zb_mod = 3 * BH; g.m_valid = dh;
               g.alpha = 1.0f; g.beta = kNsA; g.cin = b.Yf[cur];
-              g.outf = b.Yf[nxt]; g.outb = b.Yb[nxt]; g.item_stride = plane; g.ld = d;
-              return launch_gemm<false, false>(D.bn, dim3(d / D.bn, cdiv(dh, 128), 3 * BH), g, st);
+              g.outf = b.Yf[nxt]; g.outb = b.Yb[nxt]; g.outb_lo = b.Yb_lo[nxt]; g.item_stride = plane; g.ld = d;
+              return launch_gemm_any<false, false>(D.split, D.bn, dim3(d / D.bn, cdiv(dh, 128), 3 * BH), g, st);
             });
           } else {
             L(K_SIMT_GEMM, [&] {
@@ -512,7 +547,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
       L(K_RULE, [&] {
         RuleParams r;
         std::memset(&r, 0, sizeof(r));
-        r.Wm = b.Wm; r.Ws = b.Ws; r.S = dir; r.splits = dir_splits; r.split_stride = planes;
+        r.Wm = b.Wm; r.Ws = b.Ws; r.Ws_lo = b.Ws_lo; r.S = dir; r.splits = dir_splits; r.split_stride = planes;
         r.Mm = b.Mm; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c);
         r.rule = D.rule; r.BH = BH; r.dh = dh; r.d = d;
         r.row_blocks = static_cast<int>(cdiv(2 * D.BH * D.dh * 32, 256));

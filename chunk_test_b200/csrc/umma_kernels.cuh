@@ -115,6 +115,17 @@ __device__ __forceinline__ void mma_kblock(uint32_t d_tmem, uint32_t a_base, uin
   }
 }
 
+// Split-bf16 ("3-product") mode.  An fp32 value x is carried as
+// x_hi = bf16(x) and x_lo = bf16(x - x_hi); a product is accumulated as
+// x_hi*y_hi + x_hi*y_lo + x_lo*y_hi (fp32 accumulate), which keeps about 16
+// mantissa bits.  Used for the update path of the Muon rule, whose O(1)
+// orthogonalised updates carry operand rounding from chunk to chunk.  An
+// operand that is an exact bf16 input (v) has no lo part and takes 2 products.
+__device__ __forceinline__ uint32_t pack_lo_bf16x2(float a, float b, uint32_t hi) {
+  const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&hi);
+  return pack_bf16x2(a - __low2float(h), b - __high2float(h));
+}
+
 // ---------------------------------------------------------------------------
 // Fast-net forward on one chunk, one (128-token x 64-hidden-unit) tile.
 //   Z1 = X W1^T, Z3 = X W3^T   (X = q^ or k^ rows, K = d)      -> TMEM [0,128)
@@ -128,11 +139,15 @@ __device__ __forceinline__ void mma_kblock(uint32_t d_tmem, uint32_t a_base, uin
 // -G2^T = Eh^T v  ("大块测试时训练（LaCT）技术解析" §2.1 eqs. 4-5; loss and
 // per-token rates of "LaCT：以大分块更新…" 「局部注意力与非线性记忆相互补充」).
 // Rows past the chunk's end are written as zeros (key tiles) or skipped.
+// SPLIT (key tiles only): k^ and the weight shadows come as hi/lo pairs, the
+// E factors are written as hi/lo pairs.
 // ---------------------------------------------------------------------------
 struct FwdParams {
   CUtensorMap tmX;   // q^ or k^ [BH, rows, d] bf16, box {64, 128, 1}
+  CUtensorMap tmXlo; // k^ lo part (split)
   CUtensorMap tmV;   // v [BH, T, d] bf16, box {64, 128, 1}          (key tiles)
   CUtensorMap tmW;   // bf16 shadows [3*BH, dh, d] (W1, W2^T, W3), box {64, 64, 1}
+  CUtensorMap tmWlo; // shadow lo parts (split)
   int bh_count;      // B*H
   int x_row0;        // first token of the chunk in tmX / tmV
   int rows_valid;    // tokens in this chunk
@@ -141,17 +156,25 @@ struct FwdParams {
   int T;             // rows of lr per head
   __nv_bfloat16* hq; // query tiles: Hq [BH, buf_rows, dh]
   __nv_bfloat16* e;  // key tiles:   E [3][BH][buf_rows][dh]  (E1, Eh, E3)
+  __nv_bfloat16* e_lo;  // split: lo parts, same layout
   int64_t buf_rows;
   const float* lr;   // [BH, T, 3]
 };
 
-template <bool KMODE>
+template <bool KMODE, bool SPLIT = false>
 struct FwdOp {
+  static_assert(KMODE || !SPLIT, "split mode is for key tiles");
   using Params = FwdParams;
   static constexpr int kXBytes = kBM * kBK * 2;           // 16 KB
   static constexpr int kWBytes = 64 * kBK * 2;            // 8 KB per 64-row slice
-  static constexpr int kStageBytes = KMODE ? (2 * kXBytes + 3 * kWBytes) : (kXBytes + 2 * kWBytes);
-  static constexpr int kStages = KMODE ? 3 : 4;
+  // stage layout: X [X_lo] [V] W1 W3 [W1_lo W3_lo] [W2^T [W2^T_lo]]
+  static constexpr int kOffXlo = kXBytes;
+  static constexpr int kOffV = kXBytes * (SPLIT ? 2 : 1);
+  static constexpr int kOffW = kOffV + (KMODE ? kXBytes : 0);
+  static constexpr int kOffWlo = kOffW + 2 * kWBytes;
+  static constexpr int kOffW2 = kOffW + (SPLIT ? 4 : 2) * kWBytes;
+  static constexpr int kStageBytes = kOffW2 + (KMODE ? (SPLIT ? 2 : 1) * kWBytes : 0);
+  static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
   static constexpr int kTmemCols = KMODE ? 256 : 128;
   struct Tile { int slice, row0, bh; };
 
@@ -165,24 +188,40 @@ struct FwdOp {
     tma_prefetch_map(&p.tmX);
     tma_prefetch_map(&p.tmW);
     if (KMODE) tma_prefetch_map(&p.tmV);
+    if (SPLIT) {
+      tma_prefetch_map(&p.tmXlo);
+      tma_prefetch_map(&p.tmWlo);
+    }
   }
   __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
     const int k = kb * kBK, row = p.x_row0 + t.row0, hs = t.slice * 64;
+    const int z1 = t.bh, z2 = p.bh_count + t.bh, z3 = 2 * p.bh_count + t.bh;
     tma_load_3d(st, &p.tmX, bar, k, row, t.bh);
-    tma_load_3d(st + kXBytes, &p.tmW, bar, k, hs, t.bh);                              // W1
-    tma_load_3d(st + kXBytes + kWBytes, &p.tmW, bar, k, hs, 2 * p.bh_count + t.bh);   // W3
+    tma_load_3d(st + kOffW, &p.tmW, bar, k, hs, z1);                 // W1
+    tma_load_3d(st + kOffW + kWBytes, &p.tmW, bar, k, hs, z3);       // W3
+    if (SPLIT) {
+      tma_load_3d(st + kOffXlo, &p.tmXlo, bar, k, row, t.bh);
+      tma_load_3d(st + kOffWlo, &p.tmWlo, bar, k, hs, z1);
+      tma_load_3d(st + kOffWlo + kWBytes, &p.tmWlo, bar, k, hs, z3);
+    }
     if (KMODE) {
-      tma_load_3d(st + kXBytes + 2 * kWBytes, &p.tmV, bar, k, row, t.bh);
-      tma_load_3d(st + 2 * kXBytes + 2 * kWBytes, &p.tmW, bar, k, hs, p.bh_count + t.bh);  // W2^T
+      tma_load_3d(st + kOffV, &p.tmV, bar, k, row, t.bh);
+      tma_load_3d(st + kOffW2, &p.tmW, bar, k, hs, z2);              // W2^T
+      if (SPLIT) tma_load_3d(st + kOffW2 + kWBytes, &p.tmWlo, bar, k, hs, z2);
     }
   }
   __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {
     constexpr uint32_t id0 = idesc_bf16(kBM, 128, false, false);
-    mma_kblock<false, false>(tmem, st, 0, st + kXBytes, 0, id0, kb == 0);
+    const bool f = kb == 0;
+    mma_kblock<false, false>(tmem, st, 0, st + kOffW, 0, id0, f);
+    if (SPLIT) {
+      mma_kblock<false, false>(tmem, st, 0, st + kOffWlo, 0, id0, false);
+      mma_kblock<false, false>(tmem, st + kOffXlo, 0, st + kOffW, 0, id0, false);
+    }
     if (KMODE) {
       constexpr uint32_t id1 = idesc_bf16(kBM, 64, false, false);
-      mma_kblock<false, false>(tmem + 128, st + kXBytes + 2 * kWBytes, 0,
-                               st + 2 * kXBytes + 2 * kWBytes, 0, id1, kb == 0);
+      mma_kblock<false, false>(tmem + 128, st + kOffV, 0, st + kOffW2, 0, id1, f);
+      if (SPLIT) mma_kblock<false, false>(tmem + 128, st + kOffV, 0, st + kOffW2 + kWBytes, 0, id1, false);
     }
   }
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
@@ -222,9 +261,7 @@ struct FwdOp {
         eta2 = l[2];
       }
       const int64_t plane = static_cast<int64_t>(p.bh_count) * p.buf_rows * p.dh;
-      __nv_bfloat16* d1 = p.e + (static_cast<int64_t>(t.bh) * p.buf_rows + grow) * p.dh + col0;
-      __nv_bfloat16* dh2 = d1 + plane;
-      __nv_bfloat16* d3 = d1 + 2 * plane;
+      const int64_t off = (static_cast<int64_t>(t.bh) * p.buf_rows + grow) * p.dh + col0;
 #pragma unroll 1
       for (int j = 0; j < 64; j += 16) {
         float z1[16], z3[16], u[16];
@@ -233,29 +270,33 @@ struct FwdOp {
         tmem_ld16(tq + 64 + j, z3);
         tmem_ld16(tq + 128 + j, u);
         tmem_ld_wait();
-        uint32_t w1[8], w2[8], w3[8];
+        float e[3][16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float e1[2], eh[2], e3[2];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const float a = z1[2 * i + c], b = z3[2 * i + c], g = u[2 * i + c];
-            const float s = sigmoidf_(a);
-            const float sa = a * s;
-            e1[c] = eta0 * g * b * (s * (1.0f + a * (1.0f - s)));
-            eh[c] = eta1 * sa * b;
-            e3[c] = eta2 * g * sa;
-          }
-          w1[i] = pack_bf16x2(e1[0], e1[1]);
-          w2[i] = pack_bf16x2(eh[0], eh[1]);
-          w3[i] = pack_bf16x2(e3[0], e3[1]);
+        for (int i = 0; i < 16; ++i) {
+          const float a = z1[i], b = z3[i], g = u[i];
+          const float s = sigmoidf_(a);
+          const float sa = a * s;
+          e[0][i] = eta0 * g * b * (s * (1.0f + a * (1.0f - s)));
+          e[1][i] = eta1 * sa * b;
+          e[2][i] = eta2 * g * sa;
         }
-        st_global_v4(d1 + j, w1[0], w1[1], w1[2], w1[3]);
-        st_global_v4(d1 + j + 8, w1[4], w1[5], w1[6], w1[7]);
-        st_global_v4(dh2 + j, w2[0], w2[1], w2[2], w2[3]);
-        st_global_v4(dh2 + j + 8, w2[4], w2[5], w2[6], w2[7]);
-        st_global_v4(d3 + j, w3[0], w3[1], w3[2], w3[3]);
-        st_global_v4(d3 + j + 8, w3[4], w3[5], w3[6], w3[7]);
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          uint32_t hw[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) hw[i] = pack_bf16x2(e[m][2 * i], e[m][2 * i + 1]);
+          __nv_bfloat16* d = p.e + m * plane + off + j;
+          st_global_v4(d, hw[0], hw[1], hw[2], hw[3]);
+          st_global_v4(d + 8, hw[4], hw[5], hw[6], hw[7]);
+          if (SPLIT) {
+            uint32_t lw[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) lw[i] = pack_lo_bf16x2(e[m][2 * i], e[m][2 * i + 1], hw[i]);
+            __nv_bfloat16* dl = p.e_lo + m * plane + off + j;
+            st_global_v4(dl, lw[0], lw[1], lw[2], lw[3]);
+            st_global_v4(dl + 8, lw[4], lw[5], lw[6], lw[7]);
+          }
+        }
       }
     }
   }
@@ -264,18 +305,20 @@ struct FwdOp {
 // ---------------------------------------------------------------------------
 // Generic batched GEMM with a fused affine epilogue:
 //   C[m][n] = alpha * sum_k A(m,k) B(n,k) + beta * Cin[m][n]
-// stored as fp32 (outf) and/or bf16 (outb) at
+// stored as fp32 (outf) and/or bf16 (outb [+ outb_lo in split mode]) at
 //   base + item * item_stride + m * ld + n,  rows m < m_valid.
 // A is K-major (rows of A in memory) or MN-major (A^T rows in memory), same
 // for B.  Batch index z = split * items + item; split s covers K blocks
 // [s*kb_count, (s+1)*kb_count) and writes output item (s*items + item).
 // B's batch coordinate is (item % zb_mod) + zb_add, read from tmB2 instead of
-// tmB when item / zb_mod == alt_group.
+// tmB when item / zb_mod == alt_group (tmB2 is an exact bf16 input in split
+// mode: no lo part).
 // Used for: the apply output (Hq W2), the chunk gradients (E^T X), and the
 // three Newton-Schulz products.
 // ---------------------------------------------------------------------------
 struct GemmParams {
   CUtensorMap tmA, tmB, tmB2;
+  CUtensorMap tmAlo, tmBlo;  // split mode
   int items;
   int kb_count;           // K blocks per split
   int kb_total;           // K blocks in all (the last split may hold fewer)
@@ -286,17 +329,20 @@ struct GemmParams {
   const float* cin;
   float* outf;
   __nv_bfloat16* outb;
+  __nv_bfloat16* outb_lo;  // split mode
   int64_t item_stride, ld;
 };
 
-template <bool A_MN, bool B_MN, int BN>
+template <bool A_MN, bool B_MN, int BN, bool SPLIT = false>
 struct GemmOp {
   using Params = GemmParams;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = kStageBytes <= 32768 ? 6 : 4;
+  // stage layout: A [A_lo] B [B_lo]
+  static constexpr int kOffB = kABytes * (SPLIT ? 2 : 1);
+  static constexpr int kStageBytes = kOffB + kBBytes * (SPLIT ? 2 : 1);
+  static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
   static constexpr int kTmemCols = TmemCols<BN>::value;
   struct Tile { int m0, n0, item, out_item, split, zb; bool alt; };
 
@@ -315,32 +361,51 @@ struct GemmOp {
     const int left = p.kb_total - t.split * p.kb_count;
     return left < p.kb_count ? left : p.kb_count;
   }
-  __device__ static uint32_t stage_bytes(const Params&, const Tile&) { return kStageBytes; }
+  __device__ static uint32_t stage_bytes(const Params&, const Tile& t) {
+    return kABytes * (SPLIT ? 2 : 1) + kBBytes * ((SPLIT && !t.alt) ? 2 : 1);
+  }
   __device__ static void prefetch(const Params& p) {
     tma_prefetch_map(&p.tmA);
     tma_prefetch_map(&p.tmB);
     if (p.alt_group >= 0) tma_prefetch_map(&p.tmB2);
+    if (SPLIT) {
+      tma_prefetch_map(&p.tmAlo);
+      tma_prefetch_map(&p.tmBlo);
+    }
+  }
+  __device__ static void load_a(const CUtensorMap* m, uint8_t* dst, uint64_t* bar, int m0, int ak, int z) {
+    if (A_MN) {
+      tma_load_3d(dst, m, bar, m0, ak, z);
+      tma_load_3d(dst + 8192, m, bar, m0 + 64, ak, z);
+    } else {
+      tma_load_3d(dst, m, bar, ak, m0, z);
+    }
+  }
+  __device__ static void load_b(const CUtensorMap* m, uint8_t* dst, uint64_t* bar, int n0, int bk, int z) {
+    if (B_MN) {
+#pragma unroll
+      for (int b = 0; b < BN / 64; ++b) tma_load_3d(dst + b * 8192, m, bar, n0 + b * 64, bk, z);
+    } else {
+      tma_load_3d(dst, m, bar, bk, n0, z);
+    }
   }
   __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
     const int kk = (t.split * p.kb_count + kb) * kBK;
     const int ak = p.a_k0 + kk, bk = p.b_k0 + kk;
-    if (A_MN) {
-      tma_load_3d(st, &p.tmA, bar, t.m0, ak, t.item);
-      tma_load_3d(st + 8192, &p.tmA, bar, t.m0 + 64, ak, t.item);
-    } else {
-      tma_load_3d(st, &p.tmA, bar, ak, t.m0, t.item);
-    }
-    const CUtensorMap* mb = t.alt ? &p.tmB2 : &p.tmB;
-    if (B_MN) {
-#pragma unroll
-      for (int b = 0; b < BN / 64; ++b) tma_load_3d(st + kABytes + b * 8192, mb, bar, t.n0 + b * 64, bk, t.zb);
-    } else {
-      tma_load_3d(st + kABytes, mb, bar, bk, t.n0, t.zb);
+    load_a(&p.tmA, st, bar, t.m0, ak, t.item);
+    load_b(t.alt ? &p.tmB2 : &p.tmB, st + kOffB, bar, t.n0, bk, t.zb);
+    if (SPLIT) {
+      load_a(&p.tmAlo, st + kABytes, bar, t.m0, ak, t.item);
+      if (!t.alt) load_b(&p.tmBlo, st + kOffB + kBBytes, bar, t.n0, bk, t.zb);
     }
   }
-  __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {
+  __device__ static void mma(const Params&, const Tile& t, uint32_t st, uint32_t tmem, int kb) {
     constexpr uint32_t id = idesc_bf16(kBM, BN, A_MN, B_MN);
-    mma_kblock<A_MN, B_MN>(tmem, st, 8192u, st + kABytes, 8192u, id, kb == 0);
+    mma_kblock<A_MN, B_MN>(tmem, st, 8192u, st + kOffB, 8192u, id, kb == 0);
+    if (SPLIT) {
+      if (!t.alt) mma_kblock<A_MN, B_MN>(tmem, st, 8192u, st + kOffB + kBBytes, 8192u, id, false);
+      mma_kblock<A_MN, B_MN>(tmem, st + kABytes, 8192u, st + kOffB, 8192u, id, false);
+    }
   }
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
                                   int lane) {
@@ -379,11 +444,20 @@ struct GemmOp {
                          __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
         }
         if (p.outb) {
+          uint32_t hw[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) hw[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
           __nv_bfloat16* o = p.outb + off + j;
-          st_global_v4(o, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                       pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-          st_global_v4(o + 8, pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                       pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+          st_global_v4(o, hw[0], hw[1], hw[2], hw[3]);
+          st_global_v4(o + 8, hw[4], hw[5], hw[6], hw[7]);
+          if (SPLIT) {
+            uint32_t lw[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) lw[i] = pack_lo_bf16x2(v[2 * i], v[2 * i + 1], hw[i]);
+            __nv_bfloat16* ol = p.outb_lo + off + j;
+            st_global_v4(ol, lw[0], lw[1], lw[2], lw[3]);
+            st_global_v4(ol + 8, lw[4], lw[5], lw[6], lw[7]);
+          }
         }
       }
     }
