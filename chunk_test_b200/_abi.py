@@ -10,6 +10,8 @@ import os
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblact_b200.so")
 
 LACT_OK, LACT_EINVAL, LACT_ENOSPC, LACT_ECUDA, LACT_ETIMEOUT, LACT_ENODEV = 0, -1, -2, -3, -4, -5
+LACT_ETOOBIG = -6
+NOALLOC_SCRATCH_BYTES = 32 << 20  # LACT_NOALLOC_SCRATCH_BYTES
 LACT_F32, LACT_BF16 = 0, 1
 APPLY_THEN_UPDATE, UPDATE_THEN_APPLY = 0, 1
 RULE_GD, RULE_MOMENTUM, RULE_MUON = 0, 1, 2
@@ -36,6 +38,7 @@ _vp = ctypes.c_void_p
 SIGNATURES = {
     "lact_ttt_workspace_bytes": (ctypes.c_size_t, [_P]),
     "lact_ttt_fwd": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]),
+    "lact_ttt_fwd_noalloc": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp]),
     "lact_ttt_host_workspace_bytes": (ctypes.c_size_t, [_P]),
     "lact_ttt_fwd_host": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_status": (ctypes.c_int, [_vp]),

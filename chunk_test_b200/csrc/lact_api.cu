@@ -618,6 +618,29 @@ static int input_bytes(const Dims& D, size_t sz[8]) {
   return 0;
 }
 
+// Scratch of lact_ttt_fwd_noalloc: a file-scope device buffer, so callers
+// that may not allocate still get a workspace.  Host code must not use the
+// symbol itself as a device address; the address is looked up per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[LACT_NOALLOC_SCRATCH_BYTES];
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_addr[64];
+
+// Device address of g_noalloc_scratch on the current device (looked up once
+// per device, with that device current).
+static int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LACT_ECUDA;
+  if (dev < 0 || dev >= 64) return LACT_ENODEV;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LACT_ECUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return LACT_OK;
+}
+
 // One thread waits on a barrier that expects one arrival nobody makes.
 __global__ void k_selftest_wait() {
   __shared__ uint64_t bar;
@@ -672,6 +695,21 @@ int lact_ttt_fwd(const lact_problem* p, const void* q, const void* k, const void
   Launcher L{false, static_cast<cudaStream_t>(stream)};
   run(D, b, in, static_cast<cudaStream_t>(stream), L);
   return L.err;
+}
+
+int lact_ttt_fwd_noalloc(const lact_problem* p, const void* q, const void* k, const void* v,
+                         const float* lr, const float* beta, const float* w1, const float* w2,
+                         const float* w3, void* out, float* w1_out, float* w2_out, float* w3_out,
+                         void* stream) {
+  Dims D;
+  int rc = validate(p, D);
+  if (rc != LACT_OK) return rc;
+  if (workspace_bytes(D) > LACT_NOALLOC_SCRATCH_BYTES) return LACT_ETOOBIG;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != LACT_OK) return rc;
+  return lact_ttt_fwd(p, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, scratch,
+                      LACT_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 size_t lact_ttt_host_workspace_bytes(const lact_problem* p) {
@@ -805,6 +843,9 @@ const char* lact_status_string(int code) {
     case LACT_ECUDA: return "CUDA error";
     case LACT_ETIMEOUT: return "a bounded device wait gave up";
     case LACT_ENODEV: return "not an sm_100 device";
+    case LACT_ETOOBIG:
+      return "problem needs more scratch than lact_ttt_fwd_noalloc's built-in buffer "
+             "(LACT_NOALLOC_SCRATCH_BYTES) holds; use lact_ttt_fwd with a caller workspace";
     default: return "unknown status";
   }
 }

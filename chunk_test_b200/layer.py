@@ -92,6 +92,25 @@ def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_ou
     return out, w_out[0], w_out[1], w_out[2]
 
 
+def ttt_fwd_noalloc(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out, w_out,
+                    stream=None):
+    """The forward for callers that cannot allocate device memory: no
+    workspace argument, the library's built-in scratch buffer is used (see
+    lact_ttt_fwd_noalloc in include/lact.h for its size and sharing rules).
+    `out` and `w_out` must be given (pre-allocated by the caller)."""
+    _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
+    p = make_problem(q, k, w1, chunk, order, rule)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = _abi.lib().lact_ttt_fwd_noalloc(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(beta), _ptr(w1), _ptr(w2),
+        _ptr(w3), _ptr(out), _ptr(w_out[0]), _ptr(w_out[1]), _ptr(w_out[2]),
+        ctypes.c_void_p(stream.cuda_stream))
+    if rc != _abi.LACT_OK:
+        raise LactError(rc, "lact_ttt_fwd_noalloc")
+    return out, w_out[0], w_out[1], w_out[2]
+
+
 def ttt_fwd_host(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out, w_out, workspace,
                  stream=None):
     """The same forward from HOST tensors (pinned for full-speed copies): the

@@ -75,7 +75,9 @@ enum {
   LACT_ENOSPC = -2,       /* workspace smaller than lact_ttt_workspace_bytes() */
   LACT_ECUDA = -3,        /* a CUDA runtime call or kernel launch failed */
   LACT_ETIMEOUT = -4,     /* a bounded device wait gave up (see lact_ttt_status) */
-  LACT_ENODEV = -5        /* the current device is not an sm_100 GPU */
+  LACT_ENODEV = -5,       /* the current device is not an sm_100 GPU */
+  LACT_ETOOBIG = -6       /* the problem needs more scratch than the built-in
+                             buffer of lact_ttt_fwd_noalloc holds */
 };
 
 enum { LACT_F32 = 0, LACT_BF16 = 1 };
@@ -110,6 +112,38 @@ int lact_ttt_fwd(const lact_problem* p,
                  const float* w1, const float* w2, const float* w3,
                  void* out, float* w1_out, float* w2_out, float* w3_out,
                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Size of the library's built-in device scratch buffer used by
+ * lact_ttt_fwd_noalloc (32 MiB). */
+#define LACT_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* The same forward as lact_ttt_fwd for callers that cannot allocate device
+ * memory.  The pages describe no such entry point; it exists for code that
+ * must not call the CUDA allocator: cudaMalloc/cudaFree synchronise the
+ * whole device, so latency-bound loops (a serving engine's decode step)
+ * avoid them, and a plugin inside a host framework that owns the device
+ * memory budget may be given no allocator at all.
+ *
+ * Instead of a caller workspace it uses one library-owned, file-scope
+ * device buffer of LACT_NOALLOC_SCRATCH_BYTES bytes, which every GPU that
+ * loads the library holds until the process exits.  Inputs and outputs are
+ * still the caller's device buffers (same layouts as lact_ttt_fwd).  Returns
+ * LACT_ETOOBIG, before enqueuing anything, when lact_ttt_workspace_bytes(p)
+ * exceeds the buffer.  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *
+ * The first call on a device looks up the buffer's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one buffer and it keeps
+ * the previous call's contents (the forward never relies on its contents at
+ * entry): calls that can overlap on the GPU (different streams, or several
+ * host threads) race on it and must be serialised by the caller. */
+int lact_ttt_fwd_noalloc(const lact_problem* p,
+                         const void* q, const void* k, const void* v,
+                         const float* lr, const float* beta,
+                         const float* w1, const float* w2, const float* w3,
+                         void* out, float* w1_out, float* w2_out, float* w3_out,
+                         void* stream);
 
 /* Device scratch bytes lact_ttt_fwd_host needs: lact_ttt_workspace_bytes(p)
  * plus room for device copies of every input and output. */
