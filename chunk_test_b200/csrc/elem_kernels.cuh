@@ -3,10 +3,10 @@
 // write-back, per-chunk mean of beta, the update rule with the row-wise
 // renorm, and the Frobenius normalisation that starts Newton-Schulz.
 //
-// Internal fast-weight layout ("hidden-major"): three fp32 masters per
-// (b, h), each [dh, d]:  plane 0 = W1, plane 1 = W2^T, plane 2 = W3, stored
-// as Wm[j][bh][dh][d].  Renorm rows of W1/W3 are rows of their planes; rows
-// of W2 are COLUMNS of plane 1.
+// Internal fast-weight layout: three fp32 masters per (b, h) in their
+// natural layouts, Wm[j][bh]: plane 0 = W1 [dh, d], plane 1 = W2 [d, dh],
+// plane 2 = W3 [dh, d] (dh*d elements each).  Every renorm row (rows of W1
+// and W3 of length d, rows of W2 of length dh) is a contiguous row.
 #pragma once
 
 #include "sm100.cuh"
@@ -29,45 +29,86 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ---------------------------------------------------------------------------
 // q, k <- silu(q)/||silu(q)||, silu(k)/||silu(k)|| over the head dim
-// ("LaCT架构核心思想解析" §1.2).  One warp per row; rows of q first, then k.
-// An all-zero row stays zero.
+// ("LaCT架构核心思想解析" §1.2).  Rows of q first, then k.  S threads share a
+// row (S a power of two <= 32, so a row's reduction stays inside its warp);
+// each thread moves 16-byte vectors of VEC elements.  An all-zero row stays
+// zero.  With kh_lo (bf16 only) the keys are also written as the lo part of
+// a split-bf16 pair (kh_lo = bf16(k^ - kh)).
 // ---------------------------------------------------------------------------
-constexpr int kMaxRowPerLane = 16;  // d <= 512
+template <typename T, int VEC> struct Vec;
+template <> struct Vec<__nv_bfloat16, 8> {
+  uint4 u;
+  __device__ float get(int i) const {
+    const __nv_bfloat162 h = reinterpret_cast<const __nv_bfloat162*>(&u)[i >> 1];
+    return (i & 1) ? __high2float(h) : __low2float(h);
+  }
+  __device__ void set(int i, float x) {
+    __nv_bfloat16* b = reinterpret_cast<__nv_bfloat16*>(&u);
+    b[i] = __float2bfloat16_rn(x);
+  }
+};
+template <> struct Vec<float, 4> {
+  float4 u;
+  __device__ float get(int i) const { return reinterpret_cast<const float*>(&u)[i]; }
+  __device__ void set(int i, float x) { reinterpret_cast<float*>(&u)[i] = x; }
+};
+template <> struct Vec<float, 1> {
+  float u;
+  __device__ float get(int) const { return u; }
+  __device__ void set(int, float x) { u = x; }
+};
 
-// With kh_lo (bf16 only) the keys are also written as the lo part of a
-// split-bf16 pair (kh_lo = bf16(k^ - kh)).
-template <typename T>
+template <typename T, int VEC, int S, int MAXV>
 __global__ void __launch_bounds__(256) k_qk_prologue(const T* __restrict__ q, T* __restrict__ qh,
                                                      int64_t q_rows, const T* __restrict__ k,
                                                      T* __restrict__ kh, int64_t k_rows, int d,
                                                      T* __restrict__ kh_lo) {
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (row >= q_rows + k_rows) return;
-  const T* src = row < q_rows ? q + row * d : k + (row - q_rows) * d;
-  T* dst = row < q_rows ? qh + row * d : kh + (row - q_rows) * d;
-  float s[kMaxRowPerLane];
+  using V = Vec<T, VEC>;
+  using U = decltype(V::u);
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = gtid / S;
+  const int sl = static_cast<int>(gtid % S);
+  const bool active = row < q_rows + k_rows;
+  const bool is_q = row < q_rows;
+  const int nv = d / VEC;
+  const T* src = is_q ? q + row * d : k + (row - q_rows) * d;
+  float y[MAXV][VEC];
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxRowPerLane; ++i) {
-    const int c = lane + 32 * i;
-    float x = 0.f;
-    if (c < d) x = to_f(src[c]);
-    const float y = x / (1.0f + __expf(-x));
-    s[i] = y;
-    ss += y * y;
-  }
-  ss = warp_sum(ss);
-  const float inv = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
-  T* dst_lo = (kh_lo && row >= q_rows) ? kh_lo + (row - q_rows) * d : nullptr;
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = sl + i * S;
+    V in;
+    if (active && v < nv) in.u = reinterpret_cast<const U*>(src)[v];
 #pragma unroll
-  for (int i = 0; i < kMaxRowPerLane; ++i) {
-    const int c = lane + 32 * i;
-    if (c < d) {
-      const float y = s[i] * inv;
-      const T hi = from_f<T>(y);
-      dst[c] = hi;
-      if (dst_lo) dst_lo[c] = from_f<T>(y - to_f(hi));
+    for (int e = 0; e < VEC; ++e) {
+      float t = 0.f;
+      if (active && v < nv) {
+        const float a = in.get(e);
+        t = __fdividef(a, 1.0f + __expf(-a));
+      }
+      y[i][e] = t;
+      ss += t * t;
+    }
+  }
+#pragma unroll
+  for (int o = S / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (!active) return;
+  const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+  T* dst = is_q ? qh + row * d : kh + (row - q_rows) * d;
+  T* dst_lo = (kh_lo && !is_q) ? kh_lo + (row - q_rows) * d : nullptr;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = sl + i * S;
+    if (v < nv) {
+      V hi, lo;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float val = y[i][e] * inv;
+        hi.set(e, val);
+        lo.set(e, val - hi.get(e));
+      }
+      reinterpret_cast<U*>(dst)[v] = hi.u;
+      if (dst_lo) reinterpret_cast<U*>(dst_lo)[v] = lo.u;
     }
   }
 }
@@ -81,9 +122,9 @@ __device__ __forceinline__ void store_shadow(__nv_bfloat16* hi, __nv_bfloat16* l
 }
 
 // ---------------------------------------------------------------------------
-// State set-up: Wm[j][bh] from the caller's initial weights (plane 1 is the
-// transpose of W2), optional bf16 shadow, momentum zeroed.  32x32 tiles of
-// the [dh, d] planes; grid (ceil(d/32), ceil(dh/32), 3*BH), block (32, 8).
+// State set-up: Wm[j][bh] = the caller's initial weights (state h of the H
+// shared ones, or state bh), plus the bf16 shadow (and its split lo part);
+// momentum zeroed.  Grid-stride over 3 * BH * dh * d elements.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1,
                                                     const float* __restrict__ w2,
@@ -93,73 +134,33 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
                                                     __nv_bfloat16* __restrict__ Ws,
                                                     __nv_bfloat16* __restrict__ Ws_lo,
                                                     float* __restrict__ Mm) {
-  __shared__ float tile[32][33];
-  const int j = blockIdx.z / BH, bh = blockIdx.z % BH;
-  const int src_h = w_shared ? bh % H : bh;
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;
   const int64_t plane = static_cast<int64_t>(dh) * d;
-  if (j == 1) {
-    // W2 [d, dh]: read rows c (= output column) coalesced along dh.
-    const float* s = w2 + static_cast<int64_t>(src_h) * plane;
-    for (int i = ty; i < 32; i += 8) {
-      const int c = c0 + i, r = r0 + tx;
-      tile[i][tx] = (c < d && r < dh) ? s[static_cast<int64_t>(c) * dh + r] : 0.f;
-    }
-    __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-      const int r = r0 + i, c = c0 + tx;
-      if (r < dh && c < d) {
-        const int64_t o = (static_cast<int64_t>(j) * BH + bh) * plane + static_cast<int64_t>(r) * d + c;
-        const float x = tile[tx][i];
-        Wm[o] = x;
-        store_shadow(Ws, Ws_lo, o, x);
-        if (Mm) Mm[o] = 0.f;
-      }
-    }
-  } else {
-    const float* s = (j == 0 ? w1 : w3) + static_cast<int64_t>(src_h) * plane;
-    for (int i = ty; i < 32; i += 8) {
-      const int r = r0 + i, c = c0 + tx;
-      if (r < dh && c < d) {
-        const int64_t o = (static_cast<int64_t>(j) * BH + bh) * plane + static_cast<int64_t>(r) * d + c;
-        const float x = s[static_cast<int64_t>(r) * d + c];
-        Wm[o] = x;
-        store_shadow(Ws, Ws_lo, o, x);
-        if (Mm) Mm[o] = 0.f;
-      }
-    }
+  const int64_t total = 3 * BH * plane;
+  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < total;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t jb = o / plane, e = o % plane;
+    const int j = static_cast<int>(jb / BH), bh = static_cast<int>(jb % BH);
+    const int src_h = w_shared ? bh % H : bh;
+    const float* src = j == 0 ? w1 : (j == 1 ? w2 : w3);
+    const float x = src[static_cast<int64_t>(src_h) * plane + e];
+    Wm[o] = x;
+    store_shadow(Ws, Ws_lo, o, x);
+    if (Mm) Mm[o] = 0.f;
   }
 }
 
-// Write-back: w1_out, w3_out from planes 0, 2; w2_out = plane 1 transposed.
+// Write-back of the final state into w1_out, w2_out, w3_out.
 __global__ void __launch_bounds__(256) k_finalize_state(const float* __restrict__ Wm, int BH, int d,
                                                         int dh, float* __restrict__ w1o,
                                                         float* __restrict__ w2o,
                                                         float* __restrict__ w3o) {
-  __shared__ float tile[32][33];
-  const int j = blockIdx.z / BH, bh = blockIdx.z % BH;
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;
   const int64_t plane = static_cast<int64_t>(dh) * d;
-  const float* s = Wm + (static_cast<int64_t>(j) * BH + bh) * plane;
-  if (j == 1) {
-    for (int i = ty; i < 32; i += 8) {
-      const int r = r0 + i, c = c0 + tx;
-      tile[i][tx] = (r < dh && c < d) ? s[static_cast<int64_t>(r) * d + c] : 0.f;
-    }
-    __syncthreads();
-    float* o = w2o + static_cast<int64_t>(bh) * plane;
-    for (int i = ty; i < 32; i += 8) {
-      const int c = c0 + i, r = r0 + tx;
-      if (c < d && r < dh) o[static_cast<int64_t>(c) * dh + r] = tile[tx][i];
-    }
-  } else {
-    float* o = (j == 0 ? w1o : w3o) + static_cast<int64_t>(bh) * plane;
-    for (int i = ty; i < 32; i += 8) {
-      const int r = r0 + i, c = c0 + tx;
-      if (r < dh && c < d) o[static_cast<int64_t>(r) * d + c] = s[static_cast<int64_t>(r) * d + c];
-    }
+  const int64_t per = BH * plane;
+  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < 3 * per;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(o / per);
+    float* dst = j == 0 ? w1o : (j == 1 ? w2o : w3o);
+    dst[o - j * per] = Wm[o];
   }
 }
 
@@ -188,14 +189,14 @@ __global__ void __launch_bounds__(256) k_beta_mean(const float* __restrict__ bet
 //   GD / Muon:  U' = S
 //   momentum:   M' <- beta_bar M' + S,  U' = M'       (M' = -M)
 //   W' = W + U', then each renorm row of W' scaled to its norm before.
-// Blocks [0, row_blocks): rows of planes 0 and 2 (one warp per row, length d).
-// Blocks [row_blocks, ...): plane 1 in groups of 32 columns (length dh each).
+// One warp per row: BH*dh rows of W1 (length d), BH*d rows of W2 (length
+// dh), BH*dh rows of W3 (length d), in plane order.
 // ---------------------------------------------------------------------------
 struct RuleParams {
   float* Wm;
   __nv_bfloat16* Ws;      // bf16 shadow or null
   __nv_bfloat16* Ws_lo;   // split-bf16 lo part of the shadow or null
-  const float* S;         // [splits][3][BH][dh][d]
+  const float* S;         // [splits][3][BH][plane]
   int splits;
   int64_t split_stride;   // elements between partial planes
   float* Mm;              // momentum (rule 1) or null
@@ -203,89 +204,46 @@ struct RuleParams {
   int nch, chunk_idx;
   int rule;
   int BH, dh, d;
-  int row_blocks;
 };
 
-__device__ __forceinline__ float rule_dir(const RuleParams& p, int64_t o, float bb) {
-  float s = 0.f;
-  for (int i = 0; i < p.splits; ++i) s += p.S[i * p.split_stride + o];
-  if (p.rule == 1) {
-    s = bb * p.Mm[o] + s;
-    p.Mm[o] = s;
-  }
-  return s;
-}
-
 __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t r13 = static_cast<int64_t>(p.BH) * p.dh, r2 = static_cast<int64_t>(p.BH) * p.d;
+  if (row >= 2 * r13 + r2) return;
   const int64_t plane = static_cast<int64_t>(p.dh) * p.d;
-  if (static_cast<int>(blockIdx.x) < p.row_blocks) {
-    const int64_t row = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int64_t rows_per_plane = static_cast<int64_t>(p.BH) * p.dh;
-    if (row >= 2 * rows_per_plane) return;
-    const int j = row < rows_per_plane ? 0 : 2;
-    const int64_t rr = row % rows_per_plane;  // bh * dh + r
-    const int bh = static_cast<int>(rr / p.dh);
-    const float bb = p.rule == 1 ? p.beta_bar[bh * p.nch + p.chunk_idx] : 0.f;
-    const int64_t base = static_cast<int64_t>(j) * p.BH * plane + rr * p.d;
-    float on = 0.f, nn = 0.f;
-    for (int c = lane; c < p.d; c += 32) {
-      const float w = p.Wm[base + c];
-      const float wn = w + rule_dir(p, base + c, bb);
-      p.Wm[base + c] = wn;
-      on += w * w;
-      nn += wn * wn;
+  int j;
+  int64_t rr;
+  if (row < r13) { j = 0; rr = row; }
+  else if (row < r13 + r2) { j = 1; rr = row - r13; }
+  else { j = 2; rr = row - r13 - r2; }
+  const int len = j == 1 ? p.dh : p.d;
+  const int bh = static_cast<int>(rr / (j == 1 ? p.d : p.dh));
+  const int64_t base = static_cast<int64_t>(j) * p.BH * plane + rr * len;
+  const float bb = p.rule == 1 ? p.beta_bar[bh * p.nch + p.chunk_idx] : 0.f;
+  float on = 0.f, nn = 0.f;
+  for (int c = lane; c < len; c += 32) {
+    const int64_t o = base + c;
+    float s = 0.f;
+    for (int i = 0; i < p.splits; ++i) s += p.S[i * p.split_stride + o];
+    if (p.rule == 1) {
+      s = bb * p.Mm[o] + s;
+      p.Mm[o] = s;
     }
-    on = warp_sum(on);
-    nn = warp_sum(nn);
-    const float sc = nn > 0.f ? sqrtf(on) / sqrtf(nn) : 0.f;
-    __syncwarp();
-    for (int c = lane; c < p.d; c += 32) {
-      const float w = p.Wm[base + c] * sc;
-      p.Wm[base + c] = w;
-      store_shadow(p.Ws, p.Ws_lo, base + c, w);
-    }
-  } else {
-    __shared__ float red_o[8][32], red_n[8][32], scale[32];
-    const int cb = blockIdx.x - p.row_blocks;
-    const int groups = (p.d + 31) / 32;
-    const int bh = cb / groups, c = (cb % groups) * 32 + (threadIdx.x & 31);
-    const int wrp = threadIdx.x >> 5;
-    const bool cv = c < p.d;
-    const float bb = p.rule == 1 ? p.beta_bar[bh * p.nch + p.chunk_idx] : 0.f;
-    const int64_t base = (static_cast<int64_t>(1) * p.BH + bh) * plane;
-    float on = 0.f, nn = 0.f;
-    if (cv) {
-      for (int r = wrp; r < p.dh; r += 8) {
-        const int64_t o = base + static_cast<int64_t>(r) * p.d + c;
-        const float w = p.Wm[o];
-        const float wn = w + rule_dir(p, o, bb);
-        p.Wm[o] = wn;
-        on += w * w;
-        nn += wn * wn;
-      }
-    }
-    red_o[wrp][threadIdx.x & 31] = on;
-    red_n[wrp][threadIdx.x & 31] = nn;
-    __syncthreads();
-    if (wrp == 0) {
-      float so = 0.f, sn = 0.f;
-      for (int i = 0; i < 8; ++i) {
-        so += red_o[i][threadIdx.x];
-        sn += red_n[i][threadIdx.x];
-      }
-      scale[threadIdx.x] = sn > 0.f ? sqrtf(so) / sqrtf(sn) : 0.f;
-    }
-    __syncthreads();
-    if (cv) {
-      const float sc = scale[threadIdx.x & 31];
-      for (int r = wrp; r < p.dh; r += 8) {
-        const int64_t o = base + static_cast<int64_t>(r) * p.d + c;
-        const float w = p.Wm[o] * sc;
-        p.Wm[o] = w;
-        store_shadow(p.Ws, p.Ws_lo, o, w);
-      }
-    }
+    const float w = p.Wm[o];
+    const float wn = w + s;
+    p.Wm[o] = wn;
+    on += w * w;
+    nn += wn * wn;
+  }
+  on = warp_sum(on);
+  nn = warp_sum(nn);
+  const float sc = nn > 0.f ? sqrtf(on) / sqrtf(nn) : 0.f;
+  for (int c = lane; c < len; c += 32) {
+    const int64_t o = base + c;
+    const float w = p.Wm[o] * sc;
+    p.Wm[o] = w;
+    store_shadow(p.Ws, p.Ws_lo, o, w);
   }
 }
 

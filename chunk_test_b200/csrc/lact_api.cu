@@ -14,6 +14,7 @@
 // The fp32 path runs the same sequence with CUDA-core kernels.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -182,8 +183,21 @@ static bool map3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows
 }
 
 // ------------------------------------------------------------------ launches
+// SMs of the current device (the persistent kernels launch one CTA per SM).
+static int sm_count() {
+  static int sms[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    sms[dev] = n;
+  }
+  return sms[dev];
+}
+
 template <class Op>
-static cudaError_t launch_umma(dim3 grid, const typename Op::Params& p, cudaStream_t st) {
+static cudaError_t launch_umma(int64_t ntiles, const typename Op::Params& p, cudaStream_t st) {
   constexpr int smem = umma_smem_bytes<Op>();
   static bool attr_set[64] = {};
   int dev = 0;
@@ -194,17 +208,24 @@ static cudaError_t launch_umma(dim3 grid, const typename Op::Params& p, cudaStre
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  if (ntiles <= 0 || ntiles > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sm_count()));
   umma_kernel<Op><<<grid, kThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
+// grid = (tiles along N, tiles along M, splits * items), as a tile list.
 template <bool A_MN, bool B_MN, bool SPLIT = false>
-static cudaError_t launch_gemm(int bn, dim3 grid, const GemmParams& p, cudaStream_t st) {
+static cudaError_t launch_gemm(int bn, dim3 grid, GemmParams p, cudaStream_t st) {
+  p.nt_n = static_cast<int>(grid.x);
+  p.nt_m = static_cast<int>(grid.y);
+  const int64_t ntiles = int64_t(grid.x) * grid.y * grid.z;
+  p.n_tiles = static_cast<int>(ntiles);
   switch (bn) {
-    case 64: return launch_umma<GemmOp<A_MN, B_MN, 64, SPLIT>>(grid, p, st);
-    case 128: return launch_umma<GemmOp<A_MN, B_MN, 128, SPLIT>>(grid, p, st);
-    case 192: return launch_umma<GemmOp<A_MN, B_MN, 192, SPLIT>>(grid, p, st);
-    case 256: return launch_umma<GemmOp<A_MN, B_MN, 256, SPLIT>>(grid, p, st);
+    case 64: return launch_umma<GemmOp<A_MN, B_MN, 64, SPLIT>>(ntiles, p, st);
+    case 128: return launch_umma<GemmOp<A_MN, B_MN, 128, SPLIT>>(ntiles, p, st);
+    case 192: return launch_umma<GemmOp<A_MN, B_MN, 192, SPLIT>>(ntiles, p, st);
+    case 256: return launch_umma<GemmOp<A_MN, B_MN, 256, SPLIT>>(ntiles, p, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -274,10 +295,36 @@ struct Inputs {
   float *w1o, *w2o, *w3o;
 };
 
+template <typename T, int VEC, int S, int MAXV>
+static cudaError_t prologue_as(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st) {
+  const int64_t rows = D.BH * D.Tq + D.BH * D.T;
+  const unsigned blocks = static_cast<unsigned>(cdiv(rows * S, 256));
+  k_qk_prologue<T, VEC, S, MAXV><<<blocks, 256, 0, st>>>(
+      static_cast<const T*>(in.q), static_cast<T*>(b.qh), D.BH * D.Tq, static_cast<const T*>(in.k),
+      static_cast<T*>(b.kh), D.BH * D.T, static_cast<int>(D.d), reinterpret_cast<T*>(b.kh_lo));
+  return cudaGetLastError();
+}
+
+// Rows of d elements: 16-byte vectors, S = the power of two >= vectors per
+// row (at most a warp), MAXV vectors per thread.
+static cudaError_t launch_prologue(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st) {
+  if (D.dtype == LACT_BF16) {
+    const int nv = static_cast<int>(D.d / 8);  // d is a multiple of 64
+    if (nv <= 8) return prologue_as<__nv_bfloat16, 8, 8, 1>(D, b, in, st);
+    if (nv <= 16) return prologue_as<__nv_bfloat16, 8, 16, 1>(D, b, in, st);
+    if (nv <= 32) return prologue_as<__nv_bfloat16, 8, 32, 1>(D, b, in, st);
+    return prologue_as<__nv_bfloat16, 8, 32, 2>(D, b, in, st);
+  }
+  if (D.d % 4 == 0) return prologue_as<float, 4, 32, 4>(D, b, in, st);
+  return prologue_as<float, 1, 32, 16>(D, b, in, st);
+}
+
 static GemmParams gemm_params() {
   GemmParams g;
   std::memset(&g, 0, sizeof(g));
   g.alt_group = -1;
+  g.tr_group = -1;
+  g.tr_mod = 1;
   g.alpha = 1.0f;
   return g;
 }
@@ -289,6 +336,8 @@ static SimtGemmParams simt_params() {
   s.alt_b = -1;
   s.za_mod = 1 << 30;
   s.zb_mod = 1 << 30;
+  s.tr_group = -1;
+  s.tr_mod = 1;
   s.alpha = 1.0f;
   return s;
 }
@@ -302,29 +351,16 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
   const bool bf = D.dtype == LACT_BF16;
   const int BH = static_cast<int>(D.BH), d = static_cast<int>(D.d), dh = static_cast<int>(D.dh);
   const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane;
-  const dim3 tile_grid(cdiv(d, 32), cdiv(dh, 32), 3 * BH), tile_block(32, 8);
+  const unsigned state_blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(planes, 256), 4096));
 
   // Fast-weight masters (+ bf16 shadows), momentum = 0.
   L(K_INIT, [&] {
-    k_init_state<<<tile_grid, tile_block, 0, st>>>(in.w1, in.w2, in.w3, static_cast<int>(D.H),
+    k_init_state<<<state_blocks, 256, 0, st>>>(in.w1, in.w2, in.w3, static_cast<int>(D.H),
                                                    D.w_shared, BH, d, dh, b.Wm, b.Ws, b.Ws_lo, b.Mm);
     return cudaGetLastError();
   });
   // q^, k^ = silu + L2 norm rows.
-  L(K_PROLOGUE, [&] {
-    const int64_t rows = D.BH * D.Tq + D.BH * D.T;
-    const unsigned blocks = static_cast<unsigned>(cdiv(rows * 32, 256));
-    if (bf)
-      k_qk_prologue<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(in.q), static_cast<__nv_bfloat16*>(b.qh), D.BH * D.Tq,
-          static_cast<const __nv_bfloat16*>(in.k), static_cast<__nv_bfloat16*>(b.kh), D.BH * D.T, d,
-          b.kh_lo);
-    else
-      k_qk_prologue<float><<<blocks, 256, 0, st>>>(
-          static_cast<const float*>(in.q), static_cast<float*>(b.qh), D.BH * D.Tq,
-          static_cast<const float*>(in.k), static_cast<float*>(b.kh), D.BH * D.T, d, nullptr);
-    return cudaGetLastError();
-  });
+  L(K_PROLOGUE, [&] { return launch_prologue(D, b, in, st); });
   if (D.rule == LACT_RULE_MOMENTUM) {
     L(K_BETA_MEAN, [&] {
       const int64_t w = D.BH * D.nch;
@@ -350,17 +386,19 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           f.bh_count = BH; f.x_row0 = static_cast<int>(qr0); f.rows_valid = nq; f.kb_count = d / 64;
           f.dh = dh; f.T = static_cast<int>(D.T); f.hq = static_cast<__nv_bfloat16*>(b.Hq);
           f.buf_rows = D.q_rows; f.lr = in.lr;
-          return launch_umma<FwdOp<false>>(dim3(dh / 64, cdiv(nq, 128), BH), f, st);
+          f.n_slices = dh / 64; f.n_row_tiles = static_cast<int>(cdiv(nq, 128));
+          return launch_umma<FwdOp<false>>(int64_t(f.n_slices) * f.n_row_tiles * BH, f, st);
         });
         L(K_APPLY_OUT, [&] {
           GemmParams g = gemm_params();
-          if (!map3d(&g.tmA, b.Hq, dh, D.q_rows, BH, 64, 128) || !map3d(&g.tmB, b.Ws, d, dh, 3 * BH, 64, 64))
+          if (!map3d(&g.tmA, b.Hq, dh, D.q_rows, BH, 64, 128) ||
+              !map3d(&g.tmB, b.Ws + D.BH * plane, dh, d, BH, 64, D.bn))
             return cudaErrorInvalidValue;
           g.items = BH; g.kb_count = dh / 64; g.kb_total = g.kb_count;
-          g.zb_mod = BH; g.zb_add = BH; g.m_valid = nq;
+          g.zb_mod = BH; g.zb_add = 0; g.m_valid = nq;
           g.outb = static_cast<__nv_bfloat16*>(in.out) + qr0 * d;
           g.item_stride = D.Tq * D.d; g.ld = d;
-          return launch_gemm<false, true>(D.bn, dim3(d / D.bn, cdiv(nq, 128), BH), g, st);
+          return launch_gemm<false, false>(D.bn, dim3(d / D.bn, cdiv(nq, 128), BH), g, st);
         });
       } else {
         float* Z = b.Z;
@@ -384,7 +422,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
         L(K_SIMT_GEMM, [&] {
           SimtGemmParams s = simt_params();
           s.A = static_cast<const float*>(b.Hq); s.a_item = D.q_rows * D.dh; s.a_m = dh; s.a_k = 1;
-          s.B = b.Wm + D.BH * plane; s.b_item = plane; s.b_n = 1; s.b_k = d;
+          s.B = b.Wm + D.BH * plane; s.b_item = plane; s.b_n = dh; s.b_k = 1;   // W2[i][r]
           s.M = nq; s.N = d; s.K = dh;
           s.outf = static_cast<float*>(in.out) + qr0 * d; s.item_stride = D.Tq * D.d; s.ld = d;
           return simt(s, BH, st);
@@ -401,15 +439,18 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           if (!map3d(&f.tmX, b.kh, d, D.T, BH, 64, 128) || !map3d(&f.tmV, in.v, d, D.T, BH, 64, 128) ||
               !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 64))
             return cudaErrorInvalidValue;
+          if (!map3d(&f.tmW2, b.Ws + D.BH * plane, dh, d, BH, 64, 64)) return cudaErrorInvalidValue;
           if (D.split && (!map3d(&f.tmXlo, b.kh_lo, d, D.T, BH, 64, 128) ||
-                          !map3d(&f.tmWlo, b.Ws_lo, d, dh, 3 * BH, 64, 64)))
+                          !map3d(&f.tmWlo, b.Ws_lo, d, dh, 3 * BH, 64, 64) ||
+                          !map3d(&f.tmW2lo, b.Ws_lo + D.BH * plane, dh, d, BH, 64, 64)))
             return cudaErrorInvalidValue;
           f.bh_count = BH; f.x_row0 = static_cast<int>(c0); f.rows_valid = nc; f.kb_count = d / 64;
           f.dh = dh; f.T = static_cast<int>(D.T); f.e = static_cast<__nv_bfloat16*>(b.E);
           f.e_lo = static_cast<__nv_bfloat16*>(b.E_lo);
           f.buf_rows = D.key_rows; f.lr = in.lr;
-          const dim3 grid(dh / 64, cdiv(nc, 128), BH);
-          return D.split ? launch_umma<FwdOp<true, true>>(grid, f, st) : launch_umma<FwdOp<true>>(grid, f, st);
+          f.n_slices = dh / 64; f.n_row_tiles = static_cast<int>(cdiv(nc, 128));
+          const int64_t tiles = int64_t(f.n_slices) * f.n_row_tiles * BH;
+          return D.split ? launch_umma<FwdOp<true, true>>(tiles, f, st) : launch_umma<FwdOp<true>>(tiles, f, st);
         });
         const int kbt = static_cast<int>(cdiv(nc, 64));
         const int kbp = static_cast<int>(cdiv(kbt, D.splits));
@@ -426,6 +467,9 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           g.a_k0 = 0; g.b_k0 = static_cast<int>(c0);
           g.zb_mod = BH; g.zb_add = 0; g.alt_group = 1; g.m_valid = dh;
           g.outf = b.P; g.item_stride = plane; g.ld = d;
+          if (D.rule != LACT_RULE_MUON) {  // W2's gradient straight into its [d, dh] layout
+            g.tr_group = 1; g.tr_mod = BH; g.ld_t = dh;
+          }
           return launch_gemm_any<true, true>(D.split, D.bn, dim3(d / D.bn, cdiv(dh, 128), splits * 3 * BH), g, st);
         });
       } else {
@@ -435,7 +479,8 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
             SimtGemmParams s = simt_params();
             s.A = (j == 1 ? static_cast<const float*>(in.v) : static_cast<const float*>(b.kh)) + c0 * d;
             s.a_item = D.T * D.d; s.a_m = d; s.a_k = 1;
-            s.B = b.Wm + j * D.BH * plane; s.b_item = plane; s.b_n = d; s.b_k = 1;
+            s.B = b.Wm + j * D.BH * plane; s.b_item = plane;
+            s.b_n = j == 1 ? 1 : d; s.b_k = j == 1 ? dh : 1;   // W2[a][r] for DH = V W2
             s.M = nc; s.N = dh; s.K = d;
             s.outf = b.Z + j * zpl; s.item_stride = D.key_rows * D.dh; s.ld = dh;
             return simt(s, BH, st);
@@ -453,6 +498,9 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           s.b_item = D.T * D.d; s.b_n = 1; s.b_k = d; s.zb_mod = BH; s.alt_b = 1;
           s.M = dh; s.N = d; s.K = nc;
           s.outf = b.P; s.item_stride = plane; s.ld = d;
+          if (D.rule != LACT_RULE_MUON) {
+            s.tr_group = 1; s.tr_mod = BH; s.ld_t = dh;
+          }
           return simt(s, 3 * BH, st);
         });
       }
@@ -510,6 +558,9 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
               g.zb_mod = 3 * BH; g.m_valid = dh;
               g.alpha = 1.0f; g.beta = kNsA; g.cin = b.Yf[cur];
               g.outf = b.Yf[nxt]; g.outb = b.Yb[nxt]; g.outb_lo = b.Yb_lo[nxt]; g.item_stride = plane; g.ld = d;
+              if (it == kNsSteps - 1) {  // W2's update back in its [d, dh] layout
+                g.tr_group = 1; g.tr_mod = BH; g.ld_t = dh;
+              }
               return launch_gemm_any<false, false>(D.split, D.bn, dim3(d / D.bn, cdiv(dh, 128), 3 * BH), g, st);
             });
           } else {
@@ -537,6 +588,9 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
               s.M = dh; s.N = d; s.K = d;
               s.alpha = 1.0f; s.beta = kNsA; s.cin = b.Yf[cur];
               s.outf = b.Yf[nxt]; s.item_stride = plane; s.ld = d;
+              if (it == kNsSteps - 1) {
+                s.tr_group = 1; s.tr_mod = BH; s.ld_t = dh;
+              }
               return simt(s, 3 * BH, st);
             });
           }
@@ -550,8 +604,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
         r.Wm = b.Wm; r.Ws = b.Ws; r.Ws_lo = b.Ws_lo; r.S = dir; r.splits = dir_splits; r.split_stride = planes;
         r.Mm = b.Mm; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c);
         r.rule = D.rule; r.BH = BH; r.dh = dh; r.d = d;
-        r.row_blocks = static_cast<int>(cdiv(2 * D.BH * D.dh * 32, 256));
-        const unsigned grid = static_cast<unsigned>(r.row_blocks + D.BH * cdiv(d, 32));
+        const unsigned grid = static_cast<unsigned>(cdiv((2 * D.BH * D.dh + D.BH * D.d) * 32, 256));
         k_rule_renorm<<<grid, 256, 0, st>>>(r);
         return cudaGetLastError();
       });
@@ -567,7 +620,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
   }
 
   L(K_FINALIZE, [&] {
-    k_finalize_state<<<tile_grid, tile_block, 0, st>>>(b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o);
+    k_finalize_state<<<state_blocks, 256, 0, st>>>(b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o);
     return cudaGetLastError();
   });
 }

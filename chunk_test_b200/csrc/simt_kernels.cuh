@@ -26,6 +26,8 @@ struct SimtGemmParams {
   const float* cin;
   float* outf;
   int64_t item_stride, ld;
+  int tr_group, tr_mod;   // items with item / tr_mod == tr_group store C^T
+  int64_t ld_t;           //   at n * ld_t + m
 };
 
 __global__ void __launch_bounds__(256) k_simt_gemm(const SimtGemmParams p) {
@@ -80,7 +82,10 @@ __global__ void __launch_bounds__(256) k_simt_gemm(const SimtGemmParams p) {
       const int64_t o = static_cast<int64_t>(item) * p.item_stride + static_cast<int64_t>(m) * p.ld + n;
       float v = p.alpha * acc[i][j];
       if (p.cin) v += p.beta * p.cin[o];
-      p.outf[o] = v;
+      if (p.tr_group >= 0 && item / p.tr_mod == p.tr_group)
+        p.outf[static_cast<int64_t>(item) * p.item_stride + static_cast<int64_t>(n) * p.ld_t + m] = v;
+      else
+        p.outf[o] = v;
     }
   }
 }

@@ -1,10 +1,15 @@
 // umma_kernels.cuh -- tcgen05 (sm_100a) tensor-core kernels of the bf16 path.
 //
-// Every kernel here is one output tile of 128 rows per CTA, 192 threads:
-//   warp 0      TMA producer (one elected lane), STAGES-deep smem ring
-//   warp 1      TMEM allocator + MMA issuer (one elected lane)
+// Every kernel here is a persistent, warp-specialized tile loop (one CTA per
+// SM, 192 threads) over output tiles of 128 rows:
+//   warp 0      TMA producer (one elected lane): a STAGES-deep smem ring that
+//               runs on across tiles
+//   warp 1      TMEM allocator + MMA issuer (one elected lane), accumulating
+//               tile i into TMEM buffer (i & 1)
 //   warps 2..5  epilogue: tcgen05.ld of one 32-lane TMEM quarter each, fused
-//               elementwise math, stores to global memory
+//               elementwise math, stores to global memory; the buffer is
+//               handed back to the MMA warp when read, so tile i's epilogue
+//               overlaps tile i+1's loads and MMAs
 // Operands are bf16 in 128-byte-swizzled smem tiles fed by TMA, accumulators
 // fp32 in TMEM.  K is consumed in blocks of 64 (one 128-byte swizzle row).
 #pragma once
@@ -16,24 +21,29 @@ namespace lact {
 constexpr int kBM = 128;  // rows of every output tile (one TMEM lane per row)
 constexpr int kBK = 64;   // K elements per stage (128 bytes of bf16)
 constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
 
 template <int N>
 struct TmemCols {
   static constexpr int value = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : N <= 256 ? 256 : 512;
 };
 
-// The shared pipeline: Op supplies kStages, kStageBytes, kTmemCols, Tile,
-// map_tile(), num_kb(), load(), mma(), epilogue().
+// The shared pipeline: Op supplies kStages, kStageBytes, kAccCols (TMEM
+// columns of one accumulator buffer; two are allocated), Tile, num_tiles(),
+// map_tile(), num_kb(), stage_bytes(), prefetch(), load(), mma(), epilogue().
 template <class Op>
 __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant__ typename Op::Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int S = Op::kStages;
+  constexpr uint32_t kCols = 2 * Op::kAccCols;
+  static_assert(kCols <= 512, "two accumulator buffers must fit in TMEM");
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Op::kStageBytes);
   uint64_t* empty = full + S;
-  uint64_t* tmem_full = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  uint64_t* acc_full = empty + S;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   // Once a bounded wait anywhere has given up, later CTAs do no work (the
   // results are already invalid and flagged); decided once per CTA.
@@ -43,20 +53,22 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
   if (abort_cta) return;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const typename Op::Tile tile = Op::map_tile(p);
-  const int nkb = Op::num_kb(p, tile);
+  const int ntiles = Op::num_tiles(p);
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tmem_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
     fence_barrier_init();
     Op::prefetch(p);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Op::kTmemCols);
+    tmem_alloc(tmem_slot, kCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -66,35 +78,59 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % S;
-        if (kb >= S && !mbar_wait(&empty[s], ((kb / S) - 1) & 1)) break;
-        mbar_arrive_expect_tx(&full[s], Op::stage_bytes(p, tile));
-        Op::load(p, tile, kb, smem + s * Op::kStageBytes, &full[s]);
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        const typename Op::Tile t = Op::map_tile(p, tile);
+        const int nkb = Op::num_kb(p, t);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % S;
+          if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], Op::stage_bytes(p, t));
+          Op::load(p, t, kb, smem + s * Op::kStageBytes, &full[s]);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % S;
-        if (!mbar_wait(&full[s], (kb / S) & 1)) break;
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++local) {
+        const typename Op::Tile t = Op::map_tile(p, tile);
+        const int nkb = Op::num_kb(p, t);
+        const int buf = local & 1, use = local >> 1;
+        if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) break;
         tc_fence_after();
-        Op::mma(p, tile, smem_u32(smem + s * Op::kStageBytes), tmem, kb);
-        umma_commit(&empty[s]);
+        const uint32_t acc = tmem + buf * Op::kAccCols;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&full[s], (it / S) & 1)) { ok = false; break; }
+          tc_fence_after();
+          Op::mma(p, t, smem_u32(smem + s * Op::kStageBytes), acc, kb);
+          umma_commit(&empty[s]);
+        }
+        umma_commit(&acc_full[buf]);
       }
-      umma_commit(tmem_full);
     }
   } else {
-    const bool ok = mbar_wait(tmem_full, 0);
-    tc_fence_after();
-    if (ok) Op::epilogue(p, tile, tmem, warp & 3, lane);
+    int local = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
+      const typename Op::Tile t = Op::map_tile(p, tile);
+      const int buf = local & 1, use = local >> 1;
+      if (!mbar_wait(&acc_full[buf], use & 1)) break;
+      tc_fence_after();
+      Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, Op::kTmemCols);
+    tmem_dealloc(tmem, kCols);
   }
 }
 
@@ -129,7 +165,7 @@ __device__ __forceinline__ uint32_t pack_lo_bf16x2(float a, float b, uint32_t hi
 // ---------------------------------------------------------------------------
 // Fast-net forward on one chunk, one (128-token x 64-hidden-unit) tile.
 //   Z1 = X W1^T, Z3 = X W3^T   (X = q^ or k^ rows, K = d)      -> TMEM [0,128)
-//   KMODE also: DH = V (W2^T)^T = V W2                           -> TMEM [128,192)
+//   KMODE also: DH = V W2[:, slice] (W2 [d, dh], an MN-major tile) -> TMEM [128,192)
 // Epilogue, per token t and hidden unit r (s1 = sigmoid(z1)):
 //   query tile: Hq = silu(z1) z3                                  (bf16)
 //   key tile:   E1 = lr1 dh z3 s1 (1 + z1 (1 - s1))               (d<f,v>/dz1)
@@ -146,9 +182,13 @@ struct FwdParams {
   CUtensorMap tmX;   // q^ or k^ [BH, rows, d] bf16, box {64, 128, 1}
   CUtensorMap tmXlo; // k^ lo part (split)
   CUtensorMap tmV;   // v [BH, T, d] bf16, box {64, 128, 1}          (key tiles)
-  CUtensorMap tmW;   // bf16 shadows [3*BH, dh, d] (W1, W2^T, W3), box {64, 64, 1}
+  CUtensorMap tmW;   // bf16 shadows as [3*BH, dh, d] (W1, -, W3 planes), box {64, 64, 1}
   CUtensorMap tmWlo; // shadow lo parts (split)
+  CUtensorMap tmW2;  // W2 shadow plane [BH, d, dh], box {64 (dh), 64 (d), 1}
+  CUtensorMap tmW2lo;
   int bh_count;      // B*H
+  int n_slices;      // dh / 64 hidden slices
+  int n_row_tiles;   // 128-token tiles of the chunk
   int x_row0;        // first token of the chunk in tmX / tmV
   int rows_valid;    // tokens in this chunk
   int kb_count;      // d / 64
@@ -167,7 +207,7 @@ struct FwdOp {
   using Params = FwdParams;
   static constexpr int kXBytes = kBM * kBK * 2;           // 16 KB
   static constexpr int kWBytes = 64 * kBK * 2;            // 8 KB per 64-row slice
-  // stage layout: X [X_lo] [V] W1 W3 [W1_lo W3_lo] [W2^T [W2^T_lo]]
+  // stage layout: X [X_lo] [V] W1 W3 [W1_lo W3_lo] [W2 [W2_lo]]
   static constexpr int kOffXlo = kXBytes;
   static constexpr int kOffV = kXBytes * (SPLIT ? 2 : 1);
   static constexpr int kOffW = kOffV + (KMODE ? kXBytes : 0);
@@ -175,12 +215,17 @@ struct FwdOp {
   static constexpr int kOffW2 = kOffW + (SPLIT ? 4 : 2) * kWBytes;
   static constexpr int kStageBytes = kOffW2 + (KMODE ? (SPLIT ? 2 : 1) * kWBytes : 0);
   static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
-  static constexpr int kTmemCols = KMODE ? 256 : 128;
+  static constexpr int kAccCols = KMODE ? 256 : 128;
   struct Tile { int slice, row0, bh; };
 
-  __device__ static Tile map_tile(const Params&) {
-    return Tile{static_cast<int>(blockIdx.x), static_cast<int>(blockIdx.y) * kBM,
-                static_cast<int>(blockIdx.z)};
+  // Tile order: hidden slice fastest, so CTAs running together share the
+  // same token tile of q^ / k^ / v in L2.
+  __device__ static int num_tiles(const Params& p) { return p.n_slices * p.n_row_tiles * p.bh_count; }
+  __device__ static Tile map_tile(const Params& p, int idx) {
+    const int sl = idx % p.n_slices;
+    const int rt = (idx / p.n_slices) % p.n_row_tiles;
+    const int bh = idx / (p.n_slices * p.n_row_tiles);
+    return Tile{sl, rt * kBM, bh};
   }
   __device__ static int num_kb(const Params& p, const Tile&) { return p.kb_count; }
   __device__ static uint32_t stage_bytes(const Params&, const Tile&) { return kStageBytes; }
@@ -188,14 +233,16 @@ struct FwdOp {
     tma_prefetch_map(&p.tmX);
     tma_prefetch_map(&p.tmW);
     if (KMODE) tma_prefetch_map(&p.tmV);
+    if (KMODE) tma_prefetch_map(&p.tmW2);
     if (SPLIT) {
       tma_prefetch_map(&p.tmXlo);
       tma_prefetch_map(&p.tmWlo);
+      tma_prefetch_map(&p.tmW2lo);
     }
   }
   __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
     const int k = kb * kBK, row = p.x_row0 + t.row0, hs = t.slice * 64;
-    const int z1 = t.bh, z2 = p.bh_count + t.bh, z3 = 2 * p.bh_count + t.bh;
+    const int z1 = t.bh, z3 = 2 * p.bh_count + t.bh;
     tma_load_3d(st, &p.tmX, bar, k, row, t.bh);
     tma_load_3d(st + kOffW, &p.tmW, bar, k, hs, z1);                 // W1
     tma_load_3d(st + kOffW + kWBytes, &p.tmW, bar, k, hs, z3);       // W3
@@ -206,8 +253,8 @@ struct FwdOp {
     }
     if (KMODE) {
       tma_load_3d(st + kOffV, &p.tmV, bar, k, row, t.bh);
-      tma_load_3d(st + kOffW2, &p.tmW, bar, k, hs, z2);              // W2^T
-      if (SPLIT) tma_load_3d(st + kOffW2 + kWBytes, &p.tmWlo, bar, k, hs, z2);
+      tma_load_3d(st + kOffW2, &p.tmW2, bar, hs, k, t.bh);           // W2[k.., hs..]
+      if (SPLIT) tma_load_3d(st + kOffW2 + kWBytes, &p.tmW2lo, bar, hs, k, t.bh);
     }
   }
   __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {
@@ -219,9 +266,9 @@ struct FwdOp {
       mma_kblock<false, false>(tmem, st + kOffXlo, 0, st + kOffW, 0, id0, false);
     }
     if (KMODE) {
-      constexpr uint32_t id1 = idesc_bf16(kBM, 64, false, false);
-      mma_kblock<false, false>(tmem + 128, st + kOffV, 0, st + kOffW2, 0, id1, f);
-      if (SPLIT) mma_kblock<false, false>(tmem + 128, st + kOffV, 0, st + kOffW2 + kWBytes, 0, id1, false);
+      constexpr uint32_t id1 = idesc_bf16(kBM, 64, false, true);
+      mma_kblock<false, true>(tmem + 128, st + kOffV, 0, st + kOffW2, 8192u, id1, f);
+      if (SPLIT) mma_kblock<false, true>(tmem + 128, st + kOffV, 0, st + kOffW2 + kWBytes, 8192u, id1, false);
     }
   }
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
@@ -312,13 +359,16 @@ struct FwdOp {
 // [s*kb_count, (s+1)*kb_count) and writes output item (s*items + item).
 // B's batch coordinate is (item % zb_mod) + zb_add, read from tmB2 instead of
 // tmB when item / zb_mod == alt_group (tmB2 is an exact bf16 input in split
-// mode: no lo part).
+// mode: no lo part).  Items with item / tr_mod == tr_group store their fp32
+// output transposed, at n * ld_t + m (coalesced: lanes hold consecutive m).
 // Used for: the apply output (Hq W2), the chunk gradients (E^T X), and the
 // three Newton-Schulz products.
 // ---------------------------------------------------------------------------
 struct GemmParams {
   CUtensorMap tmA, tmB, tmB2;
   CUtensorMap tmAlo, tmBlo;  // split mode
+  int nt_n, nt_m;            // tiles along N and M; the z extent is splits * items
+  int n_tiles;               // nt_n * nt_m * splits * items
   int items;
   int kb_count;           // K blocks per split
   int kb_total;           // K blocks in all (the last split may hold fewer)
@@ -331,6 +381,8 @@ struct GemmParams {
   __nv_bfloat16* outb;
   __nv_bfloat16* outb_lo;  // split mode
   int64_t item_stride, ld;
+  int tr_group, tr_mod;
+  int64_t ld_t;
 };
 
 template <bool A_MN, bool B_MN, int BN, bool SPLIT = false>
@@ -343,16 +395,18 @@ struct GemmOp {
   static constexpr int kOffB = kABytes * (SPLIT ? 2 : 1);
   static constexpr int kStageBytes = kOffB + kBBytes * (SPLIT ? 2 : 1);
   static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
-  static constexpr int kTmemCols = TmemCols<BN>::value;
+  static constexpr int kAccCols = TmemCols<BN>::value;
   struct Tile { int m0, n0, item, out_item, split, zb; bool alt; };
 
-  __device__ static Tile map_tile(const Params& p) {
+  __device__ static int num_tiles(const Params& p) { return p.n_tiles; }
+  __device__ static Tile map_tile(const Params& p, int idx) {
     Tile t;
-    t.n0 = blockIdx.x * BN;
-    t.m0 = blockIdx.y * kBM;
-    t.item = blockIdx.z % p.items;
-    t.split = blockIdx.z / p.items;
-    t.out_item = blockIdx.z;
+    const int z = idx / (p.nt_n * p.nt_m);
+    t.n0 = (idx % p.nt_n) * BN;
+    t.m0 = ((idx / p.nt_n) % p.nt_m) * kBM;
+    t.item = z % p.items;
+    t.split = z / p.items;
+    t.out_item = z;
     t.zb = (t.item % p.zb_mod) + p.zb_add;
     t.alt = p.alt_group >= 0 && (t.item / p.zb_mod) == p.alt_group;
     return t;
@@ -415,6 +469,7 @@ struct GemmOp {
     const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const int64_t off = static_cast<int64_t>(t.out_item) * p.item_stride +
                         static_cast<int64_t>(grow) * p.ld + t.n0;
+    const bool tr = p.tr_group >= 0 && (t.item / p.tr_mod) == p.tr_group;
 #pragma unroll 1
     for (int j = 0; j < BN; j += 16) {
       float v[16];
@@ -436,7 +491,12 @@ struct GemmOp {
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] *= p.alpha;
         }
-        if (p.outf) {
+        if (p.outf && tr) {
+          float* o = p.outf + static_cast<int64_t>(t.out_item) * p.item_stride +
+                     static_cast<int64_t>(t.n0 + j) * p.ld_t + grow;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i * p.ld_t] = v[i];
+        } else if (p.outf) {
           float* o = p.outf + off + j;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -466,7 +526,7 @@ struct GemmOp {
 
 template <class Op>
 constexpr int umma_smem_bytes() {
-  return Op::kStages * Op::kStageBytes + (2 * Op::kStages + 1) * 8 + 16 + 1024;
+  return Op::kStages * Op::kStageBytes + (2 * Op::kStages + 4) * 8 + 16 + 1024;
 }
 
 }  // namespace lact
