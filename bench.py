@@ -66,6 +66,7 @@ def kernel_work(w: Workload):
     return {
         "fwd_query_umma": ("tensor", 4.0 * Tq * d * dh * BH, "FLOP"),
         "apply_out_umma": ("tensor", 2.0 * Tq * d * dh * BH, "FLOP"),
+        "apply_fused_umma": ("tensor", 6.0 * Tq * d * dh * BH, "FLOP"),
         "fwd_key_umma": ("tensor", 6.0 * T * d * dh * BH, "FLOP"),
         "grad_umma": ("tensor", 6.0 * T * d * dh * BH, "FLOP"),
         "ns_gram_umma": ("tensor", 2.0 * d * d * dh * ns, "FLOP"),
@@ -288,6 +289,7 @@ def main():
             roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                     "frac": achieved / hbm}
         roof.update({"kernel": name, "launches": n_launch, "avg_launch_us": 1e3 * ms_kind / n_launch,
+                     "concurrent": bool(w.order == 0 and w.dtype == BF16),
                      "traffic": traffic_for(name, w), "peak_source": f"{pk_src} sustained bf16"
                      if bound == "tensor" else f"{pk_src} copy bandwidth"})
     kernels = {k: {"launches": v[0], "ms": round(v[1], 4),

@@ -206,24 +206,35 @@ struct RuleParams {
   int BH, dh, d;
 };
 
+struct RuleRow {
+  int j, bh, len;
+  int64_t base;
+};
+
+__device__ __forceinline__ bool rule_row(const RuleParams& p, int64_t row, RuleRow& r) {
+  const int64_t r13 = static_cast<int64_t>(p.BH) * p.dh, r2 = static_cast<int64_t>(p.BH) * p.d;
+  if (row >= 2 * r13 + r2) return false;
+  const int64_t plane = static_cast<int64_t>(p.dh) * p.d;
+  int64_t rr;
+  if (row < r13) { r.j = 0; rr = row; }
+  else if (row < r13 + r2) { r.j = 1; rr = row - r13; }
+  else { r.j = 2; rr = row - r13 - r2; }
+  r.len = r.j == 1 ? p.dh : p.d;
+  r.bh = static_cast<int>(rr / (r.j == 1 ? p.d : p.dh));
+  r.base = static_cast<int64_t>(r.j) * p.BH * plane + rr * r.len;
+  return true;
+}
+
+// Generic form (any row length): two passes over the row in global memory.
 __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t r13 = static_cast<int64_t>(p.BH) * p.dh, r2 = static_cast<int64_t>(p.BH) * p.d;
-  if (row >= 2 * r13 + r2) return;
-  const int64_t plane = static_cast<int64_t>(p.dh) * p.d;
-  int j;
-  int64_t rr;
-  if (row < r13) { j = 0; rr = row; }
-  else if (row < r13 + r2) { j = 1; rr = row - r13; }
-  else { j = 2; rr = row - r13 - r2; }
-  const int len = j == 1 ? p.dh : p.d;
-  const int bh = static_cast<int>(rr / (j == 1 ? p.d : p.dh));
-  const int64_t base = static_cast<int64_t>(j) * p.BH * plane + rr * len;
-  const float bb = p.rule == 1 ? p.beta_bar[bh * p.nch + p.chunk_idx] : 0.f;
+  RuleRow r;
+  if (!rule_row(p, row, r)) return;
+  const float bb = p.rule == 1 ? p.beta_bar[r.bh * p.nch + p.chunk_idx] : 0.f;
   float on = 0.f, nn = 0.f;
-  for (int c = lane; c < len; c += 32) {
-    const int64_t o = base + c;
+  for (int c = lane; c < r.len; c += 32) {
+    const int64_t o = r.base + c;
     float s = 0.f;
     for (int i = 0; i < p.splits; ++i) s += p.S[i * p.split_stride + o];
     if (p.rule == 1) {
@@ -239,11 +250,72 @@ __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
   on = warp_sum(on);
   nn = warp_sum(nn);
   const float sc = nn > 0.f ? sqrtf(on) / sqrtf(nn) : 0.f;
-  for (int c = lane; c < len; c += 32) {
-    const int64_t o = base + c;
+  for (int c = lane; c < r.len; c += 32) {
+    const int64_t o = r.base + c;
     const float w = p.Wm[o] * sc;
     p.Wm[o] = w;
     store_shadow(p.Ws, p.Ws_lo, o, w);
+  }
+}
+
+// Rows whose length is a multiple of 4 and at most 128 * MAXV: one pass,
+// 16-byte accesses, the updated row kept in registers until it is scaled.
+template <int MAXV>
+__global__ void __launch_bounds__(256) k_rule_renorm_v4(const RuleParams p) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  RuleRow r;
+  if (!rule_row(p, row, r)) return;
+  const float bb = p.rule == 1 ? p.beta_bar[r.bh * p.nch + p.chunk_idx] : 0.f;
+  const int nv = r.len >> 2;
+  float4 wn[MAXV];
+  float on = 0.f, nn = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = lane + 32 * i;
+    if (v < nv) {
+      const int64_t o = r.base + 4 * v;
+      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < p.splits; ++k) {
+        const float4 x = *reinterpret_cast<const float4*>(p.S + k * p.split_stride + o);
+        s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
+      }
+      if (p.rule == 1) {
+        const float4 m = *reinterpret_cast<const float4*>(p.Mm + o);
+        s.x += bb * m.x; s.y += bb * m.y; s.z += bb * m.z; s.w += bb * m.w;
+        *reinterpret_cast<float4*>(p.Mm + o) = s;
+      }
+      const float4 w = *reinterpret_cast<const float4*>(p.Wm + o);
+      on += w.x * w.x + w.y * w.y + w.z * w.z + w.w * w.w;
+      wn[i] = make_float4(w.x + s.x, w.y + s.y, w.z + s.z, w.w + s.w);
+      nn += wn[i].x * wn[i].x + wn[i].y * wn[i].y + wn[i].z * wn[i].z + wn[i].w * wn[i].w;
+    }
+  }
+  on = warp_sum(on);
+  nn = warp_sum(nn);
+  const float sc = nn > 0.f ? sqrtf(on) / sqrtf(nn) : 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = lane + 32 * i;
+    if (v < nv) {
+      const int64_t o = r.base + 4 * v;
+      const float4 w = make_float4(wn[i].x * sc, wn[i].y * sc, wn[i].z * sc, wn[i].w * sc);
+      *reinterpret_cast<float4*>(p.Wm + o) = w;
+      if (p.Ws) {
+        uint2 hi;
+        hi.x = pack_bf16x2(w.x, w.y);
+        hi.y = pack_bf16x2(w.z, w.w);
+        *reinterpret_cast<uint2*>(p.Ws + o) = hi;
+        if (p.Ws_lo) {
+          const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&hi.x);
+          const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&hi.y);
+          uint2 lo;
+          lo.x = pack_bf16x2(w.x - __low2float(h0), w.y - __high2float(h0));
+          lo.y = pack_bf16x2(w.z - __low2float(h1), w.w - __high2float(h1));
+          *reinterpret_cast<uint2*>(p.Ws_lo + o) = lo;
+        }
+      }
+    }
   }
 }
 

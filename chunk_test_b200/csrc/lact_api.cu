@@ -24,6 +24,7 @@
 #include "simt_kernels.cuh"
 #include "sm100.cuh"
 #include "umma_kernels.cuh"
+#include "apply_kernel.cuh"
 
 namespace lact {
 
@@ -214,6 +215,24 @@ static cudaError_t launch_umma(int64_t ntiles, const typename Op::Params& p, cud
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_apply(int64_t ntiles, const ApplyParams& p, cudaStream_t st) {
+  constexpr int smem = ApplyCfg<D>::kSmem;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(k_apply<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  if (ntiles <= 0 || ntiles > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sm_count()));
+  k_apply<D><<<grid, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 // grid = (tiles along N, tiles along M, splits * items), as a tile list.
 template <bool A_MN, bool B_MN, bool SPLIT = false>
 static cudaError_t launch_gemm(int bn, dim3 grid, GemmParams p, cudaStream_t st) {
@@ -239,12 +258,12 @@ static cudaError_t launch_gemm_any(bool split, int bn, dim3 grid, const GemmPara
 enum Kind {
   K_INIT, K_PROLOGUE, K_BETA_MEAN, K_FWD_QUERY, K_APPLY_OUT, K_FWD_KEY, K_GRAD, K_NS_SUMSQ,
   K_NS_SCALE, K_NS_GRAM, K_NS_POLY, K_NS_UPDATE, K_RULE, K_FINALIZE, K_SIMT_GEMM, K_FWD_ELEM_F32,
-  K_COUNT
+  K_APPLY_FUSED, K_COUNT
 };
 static const char* const kKindNames[K_COUNT] = {
     "init_state", "qk_prologue", "beta_mean", "fwd_query_umma", "apply_out_umma", "fwd_key_umma",
     "grad_umma", "ns_sumsq", "ns_scale", "ns_gram_umma", "ns_poly_umma", "ns_update_umma",
-    "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32"};
+    "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32", "apply_fused_umma"};
 
 // Optional per-launch CUDA-event pairs on the launching stream.
 struct ProfRec { int kind; cudaEvent_t a, b; };
@@ -287,6 +306,30 @@ struct Launcher {
     }
   }
 };
+
+// Per device: a library-owned side stream and two events, used to run a
+// chunk's apply concurrently with its key forward + gradient (both read only
+// the previous state) in apply-then-update order.
+struct SideRes {
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static SideRes g_side[64];
+static std::mutex g_side_mu;
+
+static const SideRes* side_resources() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  SideRes& r = g_side[dev];
+  if (!r.side) {
+    if (cudaStreamCreateWithFlags(&r.side, cudaStreamNonBlocking) != cudaSuccess) return r.side = nullptr, nullptr;
+    if (cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+  }
+  return &r;
+}
 
 struct Inputs {
   const void *q, *k, *v;
@@ -347,7 +390,10 @@ static cudaError_t simt(const SimtGemmParams& p, int items, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st, Launcher& L) {
+static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t main_st, Launcher& L,
+                const SideRes* side) {
+  cudaStream_t st = main_st;  // the stream the next launch goes to
+  L.st = st;
   const bool bf = D.dtype == LACT_BF16;
   const int BH = static_cast<int>(D.BH), d = static_cast<int>(D.d), dh = static_cast<int>(D.dh);
   const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane;
@@ -370,6 +416,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
     });
   }
 
+  bool join_before_rule = false;
   for (int64_t c = 0; c < D.nch; ++c) {
     const int64_t c0 = c * D.chunk;
     const int nc = static_cast<int>((c0 + D.chunk < D.T ? c0 + D.chunk : D.T) - c0);
@@ -377,7 +424,25 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
     const int nq = static_cast<int>(D.nch == 1 ? D.Tq : nc);
 
     auto apply = [&] {
-      if (bf) {
+      if (bf && d <= 256) {
+        L(K_APPLY_FUSED, [&] {
+          ApplyParams a;
+          std::memset(&a, 0, sizeof(a));
+          if (!map3d(&a.tmQ, b.qh, d, D.Tq, BH, 64, 128) || !map3d(&a.tmW, b.Ws, d, dh, 3 * BH, 64, 64) ||
+              !map3d(&a.tmW2, b.Ws + D.BH * plane, dh, d, BH, 64, d))
+            return cudaErrorInvalidValue;
+          a.bh_count = BH; a.dh = dh; a.n_row_tiles = static_cast<int>(cdiv(nq, 128));
+          a.q_row0 = static_cast<int>(qr0); a.rows_valid = nq;
+          a.out = static_cast<__nv_bfloat16*>(in.out); a.Tq = D.Tq;
+          const int64_t tiles = int64_t(a.n_row_tiles) * BH;
+          switch (d) {
+            case 64: return launch_apply<64>(tiles, a, st);
+            case 128: return launch_apply<128>(tiles, a, st);
+            case 192: return launch_apply<192>(tiles, a, st);
+            default: return launch_apply<256>(tiles, a, st);
+          }
+        });
+      } else if (bf) {
         L(K_FWD_QUERY, [&] {
           FwdParams f;
           std::memset(&f, 0, sizeof(f));
@@ -386,8 +451,12 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           f.bh_count = BH; f.x_row0 = static_cast<int>(qr0); f.rows_valid = nq; f.kb_count = d / 64;
           f.dh = dh; f.T = static_cast<int>(D.T); f.hq = static_cast<__nv_bfloat16*>(b.Hq);
           f.buf_rows = D.q_rows; f.lr = in.lr;
-          f.n_slices = dh / 64; f.n_row_tiles = static_cast<int>(cdiv(nq, 128));
-          return launch_umma<FwdOp<false>>(int64_t(f.n_slices) * f.n_row_tiles * BH, f, st);
+          const bool wide = dh % 128 == 0;                    // 128-wide hidden slices
+          f.n_slices = dh / (wide ? 128 : 64); f.n_row_tiles = static_cast<int>(cdiv(nq, 128));
+          if (wide && !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 128)) return cudaErrorInvalidValue;
+          const int64_t tiles = int64_t(f.n_slices) * f.n_row_tiles * BH;
+          return wide ? launch_umma<FwdOp<false, false, 128>>(tiles, f, st)
+                      : launch_umma<FwdOp<false>>(tiles, f, st);
         });
         L(K_APPLY_OUT, [&] {
           GemmParams g = gemm_params();
@@ -448,10 +517,16 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
           f.dh = dh; f.T = static_cast<int>(D.T); f.e = static_cast<__nv_bfloat16*>(b.E);
           f.e_lo = static_cast<__nv_bfloat16*>(b.E_lo);
           f.buf_rows = D.key_rows; f.lr = in.lr;
-          f.n_slices = dh / 64; f.n_row_tiles = static_cast<int>(cdiv(nc, 128));
+          // 128-wide hidden slices (Z MMAs of N = 256) unless split mode needs the smem.
+          const bool wide = !D.split && dh % 128 == 0;
+          f.n_slices = dh / (wide ? 128 : 64); f.n_row_tiles = static_cast<int>(cdiv(nc, 128));
+          if (wide && !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 128)) return cudaErrorInvalidValue;
           const int64_t tiles = int64_t(f.n_slices) * f.n_row_tiles * BH;
-          return D.split ? launch_umma<FwdOp<true, true>>(tiles, f, st) : launch_umma<FwdOp<true>>(tiles, f, st);
+          if (D.split) return launch_umma<FwdOp<true, true>>(tiles, f, st);
+          return wide ? launch_umma<FwdOp<true, false, 128>>(tiles, f, st) : launch_umma<FwdOp<true>>(tiles, f, st);
         });
+      }
+      if (bf) {
         const int kbt = static_cast<int>(cdiv(nc, 64));
         const int kbp = static_cast<int>(cdiv(kbt, D.splits));
         splits = static_cast<int>(cdiv(kbt, kbp));
@@ -598,6 +673,10 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
         dir = b.Yf[kNsSteps & 1];
         dir_splits = 1;
       }
+      if (join_before_rule) {
+        if (L.err == LACT_OK && cudaStreamWaitEvent(main_st, side->join, 0) != cudaSuccess) L.err = LACT_ECUDA;
+        join_before_rule = false;
+      }
       L(K_RULE, [&] {
         RuleParams r;
         std::memset(&r, 0, sizeof(r));
@@ -605,12 +684,34 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st,
         r.Mm = b.Mm; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c);
         r.rule = D.rule; r.BH = BH; r.dh = dh; r.d = d;
         const unsigned grid = static_cast<unsigned>(cdiv((2 * D.BH * D.dh + D.BH * D.d) * 32, 256));
-        k_rule_renorm<<<grid, 256, 0, st>>>(r);
+        const int64_t longest = std::max(D.d, D.dh);
+        if (D.d % 4 != 0 || D.dh % 4 != 0 || longest > 128 * 8)
+          k_rule_renorm<<<grid, 256, 0, st>>>(r);
+        else if (longest <= 128 * 2)
+          k_rule_renorm_v4<2><<<grid, 256, 0, st>>>(r);
+        else if (longest <= 128 * 4)
+          k_rule_renorm_v4<4><<<grid, 256, 0, st>>>(r);
+        else
+          k_rule_renorm_v4<8><<<grid, 256, 0, st>>>(r);
         return cudaGetLastError();
       });
     };
 
-    if (D.order == LACT_APPLY_THEN_UPDATE) {
+    if (D.order == LACT_APPLY_THEN_UPDATE && side && bf && !L.dry) {
+      // apply on the side stream, concurrently with the key forward and the
+      // gradient; joined before the rule rewrites the state.
+      if (L.err == LACT_OK && (cudaEventRecord(side->fork, main_st) != cudaSuccess ||
+                               cudaStreamWaitEvent(side->side, side->fork, 0) != cudaSuccess))
+        L.err = LACT_ECUDA;
+      st = side->side;
+      L.st = st;
+      apply();
+      if (L.err == LACT_OK && cudaEventRecord(side->join, side->side) != cudaSuccess) L.err = LACT_ECUDA;
+      st = main_st;
+      L.st = st;
+      join_before_rule = true;
+      update();
+    } else if (D.order == LACT_APPLY_THEN_UPDATE) {
       apply();
       update();
     } else {
@@ -725,14 +826,14 @@ int64_t lact_ttt_launch_count(const lact_problem* p) {
   Inputs in;
   std::memset(&in, 0, sizeof(in));
   Launcher L{true, nullptr};
-  run(D, b, in, nullptr, L);
+  run(D, b, in, nullptr, L, nullptr);
   return L.count;
 }
 
-int lact_ttt_fwd(const lact_problem* p, const void* q, const void* k, const void* v, const float* lr,
-                 const float* beta, const float* w1, const float* w2, const float* w3, void* out,
-                 float* w1_out, float* w2_out, float* w3_out, void* workspace, size_t workspace_bytes_,
-                 void* stream) {
+static int ttt_fwd_impl(const lact_problem* p, const void* q, const void* k, const void* v,
+                        const float* lr, const float* beta, const float* w1, const float* w2,
+                        const float* w3, void* out, float* w1_out, float* w2_out, float* w3_out,
+                        void* workspace, size_t workspace_bytes_, void* stream, bool allow_side) {
   Dims D;
   int rc = validate(p, D);
   if (rc != LACT_OK) return rc;
@@ -746,8 +847,17 @@ int lact_ttt_fwd(const lact_problem* p, const void* q, const void* k, const void
   Bufs b;
   plan(D, bp, b);
   Launcher L{false, static_cast<cudaStream_t>(stream)};
-  run(D, b, in, static_cast<cudaStream_t>(stream), L);
+  const SideRes* side = allow_side ? side_resources() : nullptr;
+  run(D, b, in, static_cast<cudaStream_t>(stream), L, side);
   return L.err;
+}
+
+int lact_ttt_fwd(const lact_problem* p, const void* q, const void* k, const void* v, const float* lr,
+                 const float* beta, const float* w1, const float* w2, const float* w3, void* out,
+                 float* w1_out, float* w2_out, float* w3_out, void* workspace, size_t workspace_bytes_,
+                 void* stream) {
+  return ttt_fwd_impl(p, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, workspace,
+                      workspace_bytes_, stream, true);
 }
 
 int lact_ttt_fwd_noalloc(const lact_problem* p, const void* q, const void* k, const void* v,
@@ -761,8 +871,8 @@ int lact_ttt_fwd_noalloc(const lact_problem* p, const void* q, const void* k, co
   void* scratch = nullptr;
   rc = noalloc_scratch(&scratch);
   if (rc != LACT_OK) return rc;
-  return lact_ttt_fwd(p, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, scratch,
-                      LACT_NOALLOC_SCRATCH_BYTES, stream);
+  return ttt_fwd_impl(p, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, scratch,
+                      LACT_NOALLOC_SCRATCH_BYTES, stream, false);
 }
 
 size_t lact_ttt_host_workspace_bytes(const lact_problem* p) {

@@ -29,16 +29,18 @@ struct TmemCols {
 };
 
 // The shared pipeline: Op supplies kStages, kStageBytes, kAccCols (TMEM
-// columns of one accumulator buffer; two are allocated), Tile, num_tiles(),
-// map_tile(), num_kb(), stage_bytes(), prefetch(), load(), mma(), epilogue().
+// column stride of one accumulator buffer), kAccBufs (1 or 2 buffers), Tile,
+// num_tiles(), map_tile(), num_kb(), stage_bytes(), prefetch(), load(),
+// mma(), epilogue().
 template <class Op>
 __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant__ typename Op::Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int S = Op::kStages;
-  constexpr uint32_t kCols = 2 * Op::kAccCols;
-  static_assert(kCols <= 512, "two accumulator buffers must fit in TMEM");
+  constexpr int NB = Op::kAccBufs;
+  constexpr uint32_t kCols = TmemCols<NB * Op::kAccCols>::value;
+  static_assert(NB * Op::kAccCols <= 512, "accumulator buffers must fit in TMEM");
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Op::kStageBytes);
   uint64_t* empty = full + S;
   uint64_t* acc_full = empty + S;   // [2]
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
       for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++local) {
         const typename Op::Tile t = Op::map_tile(p, tile);
         const int nkb = Op::num_kb(p, t);
-        const int buf = local & 1, use = local >> 1;
+        const int buf = local % NB, use = local / NB;
         if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) break;
         tc_fence_after();
         const uint32_t acc = tmem + buf * Op::kAccCols;
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
     int local = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
       const typename Op::Tile t = Op::map_tile(p, tile);
-      const int buf = local & 1, use = local >> 1;
+      const int buf = local % NB, use = local / NB;
       if (!mbar_wait(&acc_full[buf], use & 1)) break;
       tc_fence_after();
       Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane);
@@ -201,12 +203,13 @@ struct FwdParams {
   const float* lr;   // [BH, T, 3]
 };
 
-template <bool KMODE, bool SPLIT = false>
+template <bool KMODE, bool SPLIT = false, int NSL = 64>
 struct FwdOp {
   static_assert(KMODE || !SPLIT, "split mode is for key tiles");
+  static_assert(NSL == 64 || NSL == 128, "hidden slice width");
   using Params = FwdParams;
   static constexpr int kXBytes = kBM * kBK * 2;           // 16 KB
-  static constexpr int kWBytes = 64 * kBK * 2;            // 8 KB per 64-row slice
+  static constexpr int kWBytes = NSL * kBK * 2;           // one NSL-row weight slice of a K block
   // stage layout: X [X_lo] [V] W1 W3 [W1_lo W3_lo] [W2 [W2_lo]]
   static constexpr int kOffXlo = kXBytes;
   static constexpr int kOffV = kXBytes * (SPLIT ? 2 : 1);
@@ -215,7 +218,9 @@ struct FwdOp {
   static constexpr int kOffW2 = kOffW + (SPLIT ? 4 : 2) * kWBytes;
   static constexpr int kStageBytes = kOffW2 + (KMODE ? (SPLIT ? 2 : 1) * kWBytes : 0);
   static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
-  static constexpr int kAccCols = KMODE ? 256 : 128;
+  // TMEM per tile: Z1 | Z3 (2 * NSL) [| DH (NSL)]
+  static constexpr int kAccCols = KMODE ? (NSL == 64 ? 256 : 384) : 2 * NSL;
+  static constexpr int kAccBufs = (2 * kAccCols <= 512) ? 2 : 1;
   struct Tile { int slice, row0, bh; };
 
   // Tile order: hidden slice fastest, so CTAs running together share the
@@ -241,11 +246,11 @@ struct FwdOp {
     }
   }
   __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
-    const int k = kb * kBK, row = p.x_row0 + t.row0, hs = t.slice * 64;
+    const int k = kb * kBK, row = p.x_row0 + t.row0, hs = t.slice * NSL;
     const int z1 = t.bh, z3 = 2 * p.bh_count + t.bh;
     tma_load_3d(st, &p.tmX, bar, k, row, t.bh);
-    tma_load_3d(st + kOffW, &p.tmW, bar, k, hs, z1);                 // W1
-    tma_load_3d(st + kOffW + kWBytes, &p.tmW, bar, k, hs, z3);       // W3
+    tma_load_3d(st + kOffW, &p.tmW, bar, k, hs, z1);                 // W1 rows of the slice
+    tma_load_3d(st + kOffW + kWBytes, &p.tmW, bar, k, hs, z3);       // W3 rows of the slice
     if (SPLIT) {
       tma_load_3d(st + kOffXlo, &p.tmXlo, bar, k, row, t.bh);
       tma_load_3d(st + kOffWlo, &p.tmWlo, bar, k, hs, z1);
@@ -253,12 +258,15 @@ struct FwdOp {
     }
     if (KMODE) {
       tma_load_3d(st + kOffV, &p.tmV, bar, k, row, t.bh);
-      tma_load_3d(st + kOffW2, &p.tmW2, bar, hs, k, t.bh);           // W2[k.., hs..]
-      if (SPLIT) tma_load_3d(st + kOffW2 + kWBytes, &p.tmW2lo, bar, hs, k, t.bh);
+#pragma unroll
+      for (int b = 0; b < NSL / 64; ++b) {                           // W2[k.., hs..]: MN blocks of 64
+        tma_load_3d(st + kOffW2 + b * 8192, &p.tmW2, bar, hs + 64 * b, k, t.bh);
+        if (SPLIT) tma_load_3d(st + kOffW2 + kWBytes + b * 8192, &p.tmW2lo, bar, hs + 64 * b, k, t.bh);
+      }
     }
   }
   __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {
-    constexpr uint32_t id0 = idesc_bf16(kBM, 128, false, false);
+    constexpr uint32_t id0 = idesc_bf16(kBM, 2 * NSL, false, false);
     const bool f = kb == 0;
     mma_kblock<false, false>(tmem, st, 0, st + kOffW, 0, id0, f);
     if (SPLIT) {
@@ -266,9 +274,9 @@ struct FwdOp {
       mma_kblock<false, false>(tmem, st + kOffXlo, 0, st + kOffW, 0, id0, false);
     }
     if (KMODE) {
-      constexpr uint32_t id1 = idesc_bf16(kBM, 64, false, true);
-      mma_kblock<false, true>(tmem + 128, st + kOffV, 0, st + kOffW2, 8192u, id1, f);
-      if (SPLIT) mma_kblock<false, true>(tmem + 128, st + kOffV, 0, st + kOffW2 + kWBytes, 8192u, id1, false);
+      constexpr uint32_t id1 = idesc_bf16(kBM, NSL, false, true);
+      mma_kblock<false, true>(tmem + 2 * NSL, st + kOffV, 0, st + kOffW2, 8192u, id1, f);
+      if (SPLIT) mma_kblock<false, true>(tmem + 2 * NSL, st + kOffV, 0, st + kOffW2 + kWBytes, 8192u, id1, false);
     }
   }
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
@@ -277,15 +285,15 @@ struct FwdOp {
     const int grow = t.row0 + r;
     const bool valid = grow < p.rows_valid;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const int64_t col0 = static_cast<int64_t>(t.slice) * 64;
+    const int64_t col0 = static_cast<int64_t>(t.slice) * NSL;
     if (!KMODE) {
       __nv_bfloat16* dst = p.hq + (static_cast<int64_t>(t.bh) * p.buf_rows + grow) * p.dh + col0;
 #pragma unroll 1
-      for (int j = 0; j < 64; j += 16) {
+      for (int j = 0; j < NSL; j += 16) {
         float z1[16], z3[16];
         __syncwarp();
         tmem_ld16(tq + j, z1);
-        tmem_ld16(tq + 64 + j, z3);
+        tmem_ld16(tq + NSL + j, z3);
         tmem_ld_wait();
         uint32_t w[8];
 #pragma unroll
@@ -310,12 +318,12 @@ struct FwdOp {
       const int64_t plane = static_cast<int64_t>(p.bh_count) * p.buf_rows * p.dh;
       const int64_t off = (static_cast<int64_t>(t.bh) * p.buf_rows + grow) * p.dh + col0;
 #pragma unroll 1
-      for (int j = 0; j < 64; j += 16) {
+      for (int j = 0; j < NSL; j += 16) {
         float z1[16], z3[16], u[16];
         __syncwarp();
         tmem_ld16(tq + j, z1);
-        tmem_ld16(tq + 64 + j, z3);
-        tmem_ld16(tq + 128 + j, u);
+        tmem_ld16(tq + NSL + j, z3);
+        tmem_ld16(tq + 2 * NSL + j, u);
         tmem_ld_wait();
         float e[3][16];
 #pragma unroll
@@ -396,6 +404,7 @@ struct GemmOp {
   static constexpr int kStageBytes = kOffB + kBBytes * (SPLIT ? 2 : 1);
   static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
   static constexpr int kAccCols = TmemCols<BN>::value;
+  static constexpr int kAccBufs = 2;
   struct Tile { int m0, n0, item, out_item, split, zb; bool alt; };
 
   __device__ static int num_tiles(const Params& p) { return p.n_tiles; }

@@ -51,7 +51,9 @@ def test_workspace_and_launch_count_for_each_workload(idx):
     assert ws > 0 and ws % 256 == 0
     assert _abi.host_workspace_bytes(p) > ws
     n = _abi.launch_count(p)
-    per_chunk = {0: 5, 1: 5, 2: 22}[w.rule] if w.dtype == BF16 else None
+    per_chunk = None
+    if w.dtype == BF16:  # fused apply for d <= 256, else forward + output GEMM
+        per_chunk = (20 if w.rule == 2 else 3) + (1 if w.d <= 256 else 2)
     if per_chunk is not None:
         fixed = 3 + (1 if w.rule == 1 else 0)
         assert n == fixed + per_chunk * w.n_chunks
