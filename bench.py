@@ -69,6 +69,7 @@ def kernel_work(w: Workload):
         "apply_fused_umma": ("tensor", 6.0 * Tq * d * dh * BH, "FLOP"),
         "fwd_key_umma": ("tensor", 6.0 * T * d * dh * BH, "FLOP"),
         "grad_umma": ("tensor", 6.0 * T * d * dh * BH, "FLOP"),
+        "key_grad_umma": ("tensor", 12.0 * T * d * dh * BH, "FLOP"),
         "ns_gram_umma": ("tensor", 2.0 * d * d * dh * ns, "FLOP"),
         "ns_poly_umma": ("tensor", 2.0 * d ** 3 * ns, "FLOP"),
         "ns_update_umma": ("tensor", 2.0 * dh * d * d * ns, "FLOP"),

@@ -25,6 +25,7 @@
 #include "sm100.cuh"
 #include "umma_kernels.cuh"
 #include "apply_kernel.cuh"
+#include "key_grad_kernel.cuh"
 
 namespace lact {
 
@@ -44,7 +45,13 @@ struct Dims {
   int splits;        // token splits of the gradient contraction (bf16)
   int bn;            // N tile over d (bf16 GEMMs)
   bool split;        // split-bf16 update path (bf16 + Muon)
+  bool fused_kg;     // fused key forward + gradient (bf16, d = 64, dh = 128, not split)
+  int kg_splits;     // its token splits per head
 };
+
+// Planning constant for the fused key + gradient kernel: work items are
+// (head, token split) with about one item per SM of a B200.
+constexpr int kPlanSMs = 148;
 
 static int choose_bn(int64_t d) {
   if (d <= 256) return static_cast<int>(d);
@@ -75,6 +82,8 @@ static int validate(const lact_problem* p, Dims& D) {
   if (D.key_rows / 128 > 65535 || D.q_rows / 128 > 65535) return LACT_EINVAL;
   D.bn = choose_bn(D.d);
   D.split = D.dtype == LACT_BF16 && D.rule == LACT_RULE_MUON;
+  D.fused_kg = D.dtype == LACT_BF16 && !D.split && D.d == 64 && D.dh == 128;
+  D.kg_splits = 1;
   // Token splits of the gradient contraction: fill ~2 waves of 148 SMs when
   // the output tiles alone do not.
   const int64_t tiles = (D.d / D.bn) * cdiv(D.dh, 128) * 3 * D.BH;
@@ -83,6 +92,16 @@ static int validate(const lact_problem* p, Dims& D) {
   if (s > kbt) s = kbt;
   if (s * 3 * D.BH > 65535) s = 65535 / (3 * D.BH);
   D.splits = static_cast<int>(s < 1 ? 1 : s);
+  if (D.fused_kg) {
+    // (head, token split) items, about one per SM; no split left empty.
+    const int64_t tiles = cdiv(D.chunk, 128);
+    int64_t ks = std::max<int64_t>(1, kPlanSMs / D.BH);
+    if (ks > tiles) ks = tiles;
+    const int64_t tps = cdiv(tiles, ks);
+    ks = cdiv(tiles, tps);
+    D.kg_splits = static_cast<int>(ks);
+    D.splits = std::max(D.splits, D.kg_splits);
+  }
   if (3 * D.BH * D.splits > 65535) return LACT_EINVAL;
   return LACT_OK;
 }
@@ -233,6 +252,23 @@ static cudaError_t launch_apply(int64_t ntiles, const ApplyParams& p, cudaStream
   return cudaGetLastError();
 }
 
+static cudaError_t launch_key_grad(int64_t items, const KeyGradParams& p, cudaStream_t st) {
+  constexpr int smem = KGCfg::kSmem;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(k_key_grad64, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  if (items <= 0 || items > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, sm_count()));
+  k_key_grad64<<<grid, kKGThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 // grid = (tiles along N, tiles along M, splits * items), as a tile list.
 template <bool A_MN, bool B_MN, bool SPLIT = false>
 static cudaError_t launch_gemm(int bn, dim3 grid, GemmParams p, cudaStream_t st) {
@@ -258,12 +294,13 @@ static cudaError_t launch_gemm_any(bool split, int bn, dim3 grid, const GemmPara
 enum Kind {
   K_INIT, K_PROLOGUE, K_BETA_MEAN, K_FWD_QUERY, K_APPLY_OUT, K_FWD_KEY, K_GRAD, K_NS_SUMSQ,
   K_NS_SCALE, K_NS_GRAM, K_NS_POLY, K_NS_UPDATE, K_RULE, K_FINALIZE, K_SIMT_GEMM, K_FWD_ELEM_F32,
-  K_APPLY_FUSED, K_COUNT
+  K_APPLY_FUSED, K_KEY_GRAD, K_COUNT
 };
 static const char* const kKindNames[K_COUNT] = {
     "init_state", "qk_prologue", "beta_mean", "fwd_query_umma", "apply_out_umma", "fwd_key_umma",
     "grad_umma", "ns_sumsq", "ns_scale", "ns_gram_umma", "ns_poly_umma", "ns_update_umma",
-    "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32", "apply_fused_umma"};
+    "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32", "apply_fused_umma",
+    "key_grad_umma"};
 
 // Optional per-launch CUDA-event pairs on the launching stream.
 struct ProfRec { int kind; cudaEvent_t a, b; };
@@ -501,7 +538,24 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
 
     auto update = [&] {
       int splits = 1;
-      if (bf) {
+      if (bf && D.fused_kg) {
+        const int tiles = static_cast<int>(cdiv(nc, 128));
+        int ks = std::min(D.kg_splits, tiles);
+        const int tps = static_cast<int>(cdiv(tiles, ks));
+        ks = static_cast<int>(cdiv(tiles, tps));
+        splits = ks;
+        L(K_KEY_GRAD, [&] {
+          KeyGradParams k;
+          std::memset(&k, 0, sizeof(k));
+          if (!map3d(&k.tmK, b.kh, d, D.T, BH, 64, 128) || !map3d(&k.tmV, in.v, d, D.T, BH, 64, 128) ||
+              !map3d(&k.tmW, b.Ws, d, dh, 3 * BH, 64, 64) ||
+              !map3d(&k.tmW2, b.Ws + D.BH * plane, dh, d, BH, 64, 64))
+            return cudaErrorInvalidValue;
+          k.bh_count = BH; k.splits = ks; k.n_tiles = tiles; k.x_row0 = static_cast<int>(c0);
+          k.rows_valid = nc; k.T = static_cast<int>(D.T); k.lr = in.lr; k.P = b.P;
+          return launch_key_grad(int64_t(BH) * ks, k, st);
+        });
+      } else if (bf) {
         L(K_FWD_KEY, [&] {
           FwdParams f;
           std::memset(&f, 0, sizeof(f));
@@ -526,7 +580,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           return wide ? launch_umma<FwdOp<true, false, 128>>(tiles, f, st) : launch_umma<FwdOp<true>>(tiles, f, st);
         });
       }
-      if (bf) {
+      if (bf && !D.fused_kg) {
         const int kbt = static_cast<int>(cdiv(nc, 64));
         const int kbp = static_cast<int>(cdiv(kbt, D.splits));
         splits = static_cast<int>(cdiv(kbt, kbp));
@@ -547,7 +601,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           }
           return launch_gemm_any<true, true>(D.split, D.bn, dim3(d / D.bn, cdiv(dh, 128), splits * 3 * BH), g, st);
         });
-      } else {
+      } else if (!bf) {
         const int64_t zpl = D.BH * D.key_rows * D.dh;
         for (int j = 0; j < 3; ++j) {
           L(K_SIMT_GEMM, [&] {

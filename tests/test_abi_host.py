@@ -53,7 +53,8 @@ def test_workspace_and_launch_count_for_each_workload(idx):
     n = _abi.launch_count(p)
     per_chunk = None
     if w.dtype == BF16:  # fused apply for d <= 256, else forward + output GEMM
-        per_chunk = (20 if w.rule == 2 else 3) + (1 if w.d <= 256 else 2)
+        fused_kg = w.rule != 2 and w.d == 64 and w.dh == 128   # key forward + gradient in one
+        per_chunk = (20 if w.rule == 2 else 3) + (1 if w.d <= 256 else 2) - (1 if fused_kg else 0)
     if per_chunk is not None:
         fixed = 3 + (1 if w.rule == 1 else 0)
         assert n == fixed + per_chunk * w.n_chunks
