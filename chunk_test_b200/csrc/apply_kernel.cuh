@@ -31,17 +31,6 @@ struct ApplyParams {
   int64_t Tq;
 };
 
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-
 template <int D>
 struct ApplyCfg {
   static_assert(D % 64 == 0 && D >= 64 && D <= 256, "apply kernel head dim");
@@ -219,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_apply(const __grid_constant__ A
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float a0 = z1[2 * i], a1 = z1[2 * i + 1];
-            hw[j / 2 + i] = pack_bf16x2(a0 * sigmoidf_(a0) * z3[2 * i], a1 * sigmoidf_(a1) * z3[2 * i + 1]);
+            hw[j / 2 + i] = pack_bf16x2(a0 * sigmoid_fast(a0) * z3[2 * i], a1 * sigmoid_fast(a1) * z3[2 * i + 1]);
           }
         }
         tc_fence_before();

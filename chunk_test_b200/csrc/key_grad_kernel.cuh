@@ -14,8 +14,13 @@
 // The k^ / v tiles serve twice: as the K-major A operand of the forward and,
 // viewed MN-major (d contiguous), as the B operand of the gradients.
 //
-// Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..9 epilogue (two
-// warps per 32-lane TMEM quarter, each taking half of the columns).
+// Warps: 0 TMA producer, 1 TMEM allocator, 2..17 epilogue (four warps per
+// 32-lane TMEM quarter, each taking 16 of every 64 columns).  The epilogue
+// group issues the MMAs itself: after a named barrier that follows its TMEM
+// reads (or its shared-memory writes), one elected thread issues exactly the
+// MMAs those reads or writes unblocked (Z_1 after Z_0 is read; the next
+// tile's DH and Z_0 after Z_1 and DH are read; the gradients after E is
+// written), so no hand-off to another warp sits on the per-tile chain.
 #pragma once
 
 #include "apply_kernel.cuh"
@@ -37,8 +42,8 @@ struct KeyGradParams {
   float* P;           // partial gradients [splits][3][BH][plane], W2's in [d, dh]
 };
 
-constexpr int kKGThreads = 320;   // 10 warps
-constexpr int kKGEpiWarps = 8;
+constexpr int kKGThreads = 576;   // 18 warps
+constexpr int kKGEpiWarps = 16;
 
 struct KGCfg {
   static constexpr int kOffW13 = 0;          // [W1 rows 0-63 | W3 rows 0-63 | W1 64-127 | W3 64-127]
@@ -147,41 +152,117 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idf = idesc_bf16(kBM, 128, false, false);   // Z_h
-      constexpr uint32_t idd = idesc_bf16(kBM, 128, false, true);    // DH (W2 MN-major)
-      constexpr uint32_t idg = idesc_bf16(kBM, 64, true, true);      // gradients
-      const uint32_t sb = smem_u32(smem);
-      int it = 0, ic = 0, zc = 0, ze = 0, g = 0;
-      bool ok = true;
-      for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
-        int bh, s, t0, t1;
-        item_range(item, bh, s, t0, t1);
-        if (t0 >= t1) continue;
-        if (!mbar_wait(wfull, ic & 1)) break;
-        tc_fence_after();
-        for (int t = t0; t < t1; ++t, ++it, ++g) {
-          const int slot = it & 1;
-          const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
-          if (!mbar_wait(&tfull[slot], (it >> 1) & 1)) { ok = false; break; }
-          if (g > 0 && !mbar_wait(dhempty, (g - 1) & 1)) { ok = false; break; }
-          if (zc > 0 && !mbar_wait(zempty, ze++ & 1)) { ok = false; break; }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue + MMA issue
+    constexpr uint32_t idf = idesc_bf16(kBM, 128, false, false);   // Z_h
+    constexpr uint32_t idd = idesc_bf16(kBM, 128, false, true);    // DH (W2 MN-major)
+    constexpr uint32_t idg = idesc_bf16(kBM, 64, true, true);      // gradients
+    const uint32_t sb = smem_u32(smem);
+    const bool leader = warp == 2 && lane == 0;
+    const int ew = warp - 2;                 // 0..15
+    const int quarter = warp & 3;
+    const int cg = ew >> 2;                  // which 16 of every 64 columns
+    const int r = quarter * 32 + lane;       // token row (TMEM lane) of the tile
+    const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int64_t plane = 128 * 64;
+    const uint32_t erow = sb + C::kOffE + r * 128;
+    const uint32_t sw0 = ((2 * cg) ^ (r & 7)) << 4, sw1 = ((2 * cg + 1) ^ (r & 7)) << 4;
+    // Named barrier over the epilogue group that also ANDs everyone's `ok`:
+    // a bounded wait that gave up in any thread makes the whole group leave
+    // together, so no thread is left at a barrier the others skipped.
+    auto group_and = [](bool v) -> bool {
+      int out;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+          "bar.red.and.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+          : "=r"(out)
+          : "r"(static_cast<int>(v)), "n"(kKGEpiWarps * 32)
+          : "memory");
+      return out != 0;
+    };
+    // Leader: the forward MMAs of one token tile's first half (DH and Z_0).
+    auto issue_first_half = [&](int it) -> bool {
+      const int slot = it & 1;
+      if (!mbar_wait(&tfull[slot], (it >> 1) & 1)) return false;
+      tc_fence_after();
+      const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
+      mma_kblock<false, true>(tmem + C::kColD, vx, 0, sb + C::kOffW2, 8192u, idd, true);
+      mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13, 0, idf, true);
+      umma_commit(zfull);
+      return true;
+    };
+    int it = 0, ic = 0, zc = 0, g = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+      int bh, s, t0, t1;
+      item_range(item, bh, s, t0, t1);
+      if (t0 >= t1) continue;
+      if (leader) ok = mbar_wait(wfull, ic & 1) && issue_first_half(it);
+      for (int t = t0; t < t1; ++t, ++it, ++g) {
+        const int slot = it & 1;
+        const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
+        const int grow = t * kBM + r;
+        float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
+        if (grow < p.rows_valid) {
+          const float* l = p.lr + (static_cast<int64_t>(bh) * p.T + p.x_row0 + grow) * 3;
+          eta0 = l[0];
+          eta1 = l[1];
+          eta2 = l[2];
+        }
+        for (int h = 0; h < 2; ++h, ++zc) {
+          ok = mbar_wait(zfull, zc & 1) && ok;
           tc_fence_after();
-          // DH = V W2 (K = 64), Z_0 = K^ [W1_0; W3_0]^T
-          mma_kblock<false, true>(tmem + C::kColD, vx, 0, sb + C::kOffW2, 8192u, idd, true);
-          mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13, 0, idf, true);
-          umma_commit(zfull);
-          ++zc;
-          if (!mbar_wait(zempty, ze++ & 1)) { ok = false; break; }
-          tc_fence_after();
-          mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13 + 16384, 0, idf, true);
-          umma_commit(zfull);
-          ++zc;
-          // gradients: M = 128 hidden (E MN-major, 2 blocks of 16 KB), K = 128 tokens
-          if (!mbar_wait(efull, g & 1)) { ok = false; break; }
-          if (t == t0 && ic > 0 && !mbar_wait(gempty, (ic - 1) & 1)) { ok = false; break; }
+          float z1[16], z3[16], u[16];
+          const int c = cg * 16;
+          __syncwarp();
+          tmem_ld16(tq + C::kColZ + c, z1);
+          tmem_ld16(tq + C::kColZ + 64 + c, z3);
+          tmem_ld16(tq + C::kColD + h * 64 + c, u);
+          tmem_ld_wait();
+          tc_fence_before();
+          ok = group_and(ok);  // every read of Z_h (and, for h = 1, of DH) is done
+          if (!ok) break;
+          if (leader) {
+            tc_fence_after();
+            if (h == 0) {  // Z_1 into the freed Z buffer
+              mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13 + 16384, 0, idf, true);
+              umma_commit(zfull);
+            } else if (t + 1 < t1) {  // the next tile's DH and Z_0
+              if (!issue_first_half(it + 1)) ok = false;
+            }
+          }
+          uint32_t e1w[8], ehw[8], e3w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float v1[2], vh[2], v3[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float a = z1[2 * i + q], bz = z3[2 * i + q], gd = u[2 * i + q];
+              const float sg = sigmoid_fast(a);
+              const float sa = a * sg;
+              const float ds = fmaf(sa, 1.0f - sg, sg);       // silu'(a) = s + a s (1 - s)
+              v1[q] = (eta0 * gd) * (bz * ds);
+              vh[q] = eta1 * (sa * bz);
+              v3[q] = (eta2 * gd) * sa;
+            }
+            e1w[i] = pack_bf16x2(v1[0], v1[1]);
+            ehw[i] = pack_bf16x2(vh[0], vh[1]);
+            e3w[i] = pack_bf16x2(v3[0], v3[1]);
+          }
+          if (h == 0 && g > 0) ok = mbar_wait(eempty, (g - 1) & 1) && ok;
+          // Row r of MN block h of each factor; 16-byte chunk c sits at c ^ (r % 8).
+          const uint32_t rb = erow + h * 16384;
+          st_shared_v4(rb + sw0, e1w[0], e1w[1], e1w[2], e1w[3]);
+          st_shared_v4(rb + sw1, e1w[4], e1w[5], e1w[6], e1w[7]);
+          st_shared_v4(rb + C::kEBytes + sw0, ehw[0], ehw[1], ehw[2], ehw[3]);
+          st_shared_v4(rb + C::kEBytes + sw1, ehw[4], ehw[5], ehw[6], ehw[7]);
+          st_shared_v4(rb + 2 * C::kEBytes + sw0, e3w[0], e3w[1], e3w[2], e3w[3]);
+          st_shared_v4(rb + 2 * C::kEBytes + sw1, e3w[4], e3w[5], e3w[6], e3w[7]);
+        }
+        fence_async_smem();
+        ok = group_and(ok);  // every factor of this tile is in shared memory
+        if (!ok) break;
+        if (leader) {
           tc_fence_after();
           const bool first = t == t0;
 #pragma unroll
@@ -201,98 +282,16 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
             umma_commit(wempty);
           }
         }
-        ++ic;
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;                 // 0..7
-    const int quarter = warp & 3;
-    const int colh = ew >> 2;                // which 32 of each 64 columns
-    const int r = quarter * 32 + lane;       // token row (TMEM lane) of the tile
-    const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const int64_t plane = 128 * 64;
-    int ic = 0, zc = 0, g = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
-      int bh, s, t0, t1;
-      item_range(item, bh, s, t0, t1);
-      if (t0 >= t1) continue;
-      for (int t = t0; t < t1; ++t, ++g) {
-        const int grow = t * kBM + r;
-        float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
-        if (grow < p.rows_valid) {
-          const float* l = p.lr + (static_cast<int64_t>(bh) * p.T + p.x_row0 + grow) * 3;
-          eta0 = l[0];
-          eta1 = l[1];
-          eta2 = l[2];
-        }
-        for (int h = 0; h < 2; ++h, ++zc) {
-          if (!mbar_wait(zfull, zc & 1)) { ok = false; break; }
-          tc_fence_after();
-          uint32_t e1w[16], ehw[16], e3w[16];   // 32 bf16 of each factor
-#pragma unroll
-          for (int j = 0; j < 32; j += 16) {
-            float z1[16], z3[16], u[16];
-            const int c = colh * 32 + j;
-            __syncwarp();
-            tmem_ld16(tq + C::kColZ + c, z1);
-            tmem_ld16(tq + C::kColZ + 64 + c, z3);
-            tmem_ld16(tq + C::kColD + h * 64 + c, u);
-            tmem_ld_wait();
-            if (j == 16) {   // all TMEM reads of this half done
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) {
-                mbar_arrive(zempty);
-                if (h == 1) mbar_arrive(dhempty);
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float v1[2], vh[2], v3[2];
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const float a = z1[2 * i + q], bz = z3[2 * i + q], gd = u[2 * i + q];
-                const float sg = sigmoidf_(a);
-                const float sa = a * sg;
-                v1[q] = eta0 * gd * bz * (sg * (1.0f + a * (1.0f - sg)));
-                vh[q] = eta1 * sa * bz;
-                v3[q] = eta2 * gd * sa;
-              }
-              e1w[j / 2 + i] = pack_bf16x2(v1[0], v1[1]);
-              ehw[j / 2 + i] = pack_bf16x2(vh[0], vh[1]);
-              e3w[j / 2 + i] = pack_bf16x2(v3[0], v3[1]);
-            }
-          }
-          if (h == 0 && g > 0 && !mbar_wait(eempty, (g - 1) & 1)) { ok = false; break; }
-          // Row r of MN block h (hidden 64h..64h+63) of each factor: the
-          // 16-byte chunk c of the 128-byte row sits at c ^ (r % 8).
-          const uint32_t rowb = smem_u32(smem + C::kOffE) + h * 16384 + r * 128;
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int c = colh * 4 + c4;
-            const uint32_t o = ((c ^ (r & 7)) << 4);
-            st_shared_v4(rowb + o, e1w[4 * c4], e1w[4 * c4 + 1], e1w[4 * c4 + 2], e1w[4 * c4 + 3]);
-            st_shared_v4(rowb + C::kEBytes + o, ehw[4 * c4], ehw[4 * c4 + 1], ehw[4 * c4 + 2], ehw[4 * c4 + 3]);
-            st_shared_v4(rowb + 2 * C::kEBytes + o, e3w[4 * c4], e3w[4 * c4 + 1], e3w[4 * c4 + 2],
-                         e3w[4 * c4 + 3]);
-          }
-        }
-        if (!ok) break;
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(efull);
       }
       if (!ok) break;
       // this item's partial gradients: TMEM lane = hidden unit
-      if (!mbar_wait(gfull, ic & 1)) break;
+      ok = mbar_wait(gfull, ic & 1);
       tc_fence_after();
       const int hr = r;  // hidden row of the gradient tile
       float* base = p.P + static_cast<int64_t>(s) * 3 * p.bh_count * plane;
 #pragma unroll 1
-      for (int cc = 0; cc < 96; cc += 16) {
-        const int col = colh * 96 + cc;        // of the 192 gradient columns
+      for (int cc = 0; cc < 48; cc += 16) {
+        const int col = cg * 48 + cc;          // of the 192 gradient columns
         float v[16];
         __syncwarp();
         tmem_ld16(tq + C::kColG + col, v);
@@ -311,8 +310,7 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
         }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(gempty);
+      ok = group_and(ok);  // the gradient accumulator may be overwritten by the next item
       ++ic;
     }
   }

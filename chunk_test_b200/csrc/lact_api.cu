@@ -141,9 +141,9 @@ static void plan(const Dims& D, Bump& bp, Bufs& b) {
     b.Mm = bp.take<float>(planes);
     b.bbar = bp.take<float>(D.BH * D.nch);
   }
-  b.E = bp.take<uint8_t>(3 * D.BH * D.key_rows * D.dh * esz);
+  if (!D.fused_kg) b.E = bp.take<uint8_t>(3 * D.BH * D.key_rows * D.dh * esz);
   if (D.split) b.E_lo = bp.take<uint8_t>(3 * D.BH * D.key_rows * D.dh * esz);
-  b.Hq = bp.take<uint8_t>(D.BH * D.q_rows * D.dh * esz);
+  if (!bf || D.d > 256) b.Hq = bp.take<uint8_t>(D.BH * D.q_rows * D.dh * esz);  // unfused apply only
   if (!bf) b.Z = bp.take<float>(3 * D.BH * (D.key_rows > D.q_rows ? D.key_rows : D.q_rows) * D.dh);
   if (D.rule == LACT_RULE_MUON) {
     for (int i = 0; i < 2; ++i) {
@@ -572,7 +572,10 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           f.e_lo = static_cast<__nv_bfloat16*>(b.E_lo);
           f.buf_rows = D.key_rows; f.lr = in.lr;
           // 128-wide hidden slices (Z MMAs of N = 256) unless split mode needs the smem.
-          const bool wide = !D.split && dh % 128 == 0;
+          // 64-wide hidden slices: double-buffered TMEM and TMA-stored E measured
+          // faster than 128-wide ones (N = 256 MMAs, single-buffered).
+          const bool wide = false;
+          if (!D.split && !map3d(&f.tmE, b.E, dh, D.key_rows, 3 * BH, 64, 32)) return cudaErrorInvalidValue;
           f.n_slices = dh / (wide ? 128 : 64); f.n_row_tiles = static_cast<int>(cdiv(nc, 128));
           if (wide && !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 128)) return cudaErrorInvalidValue;
           const int64_t tiles = int64_t(f.n_slices) * f.n_row_tiles * BH;

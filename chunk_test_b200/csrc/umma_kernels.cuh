@@ -28,10 +28,11 @@ struct TmemCols {
   static constexpr int value = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : N <= 256 ? 256 : 512;
 };
 
-// The shared pipeline: Op supplies kStages, kStageBytes, kAccCols (TMEM
-// column stride of one accumulator buffer), kAccBufs (1 or 2 buffers), Tile,
-// num_tiles(), map_tile(), num_kb(), stage_bytes(), prefetch(), load(),
-// mma(), epilogue().
+// The shared pipeline: Op supplies kStages, kStageBytes, kExtraBytes (shared
+// memory for the epilogue, after the ring), kAccCols (TMEM column stride of
+// one accumulator buffer), kAccBufs (1 or 2 buffers), Tile, num_tiles(),
+// map_tile(), num_kb(), stage_bytes(), prefetch(), load(), mma(),
+// epilogue(), epilogue_done().
 template <class Op>
 __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant__ typename Op::Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -41,7 +42,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
   constexpr int NB = Op::kAccBufs;
   constexpr uint32_t kCols = TmemCols<NB * Op::kAccCols>::value;
   static_assert(NB * Op::kAccCols <= 512, "accumulator buffers must fit in TMEM");
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Op::kStageBytes);
+  uint8_t* extra = smem + S * Op::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(extra + Op::kExtraBytes);
   uint64_t* empty = full + S;
   uint64_t* acc_full = empty + S;   // [2]
   uint64_t* acc_empty = acc_full + 2;  // [2]
@@ -121,11 +123,12 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
       const int buf = local % NB, use = local / NB;
       if (!mbar_wait(&acc_full[buf], use & 1)) break;
       tc_fence_after();
-      Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane);
+      Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane, extra);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
+    Op::epilogue_done(lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -188,6 +191,7 @@ struct FwdParams {
   CUtensorMap tmWlo; // shadow lo parts (split)
   CUtensorMap tmW2;  // W2 shadow plane [BH, d, dh], box {64 (dh), 64 (d), 1}
   CUtensorMap tmW2lo;
+  CUtensorMap tmE;   // E as [3*BH, buf_rows, dh], box {64, 32, 1}: the epilogue's TMA stores
   int bh_count;      // B*H
   int n_slices;      // dh / 64 hidden slices
   int n_row_tiles;   // 128-token tiles of the chunk
@@ -218,6 +222,10 @@ struct FwdOp {
   static constexpr int kOffW2 = kOffW + (SPLIT ? 4 : 2) * kWBytes;
   static constexpr int kStageBytes = kOffW2 + (KMODE ? (SPLIT ? 2 : 1) * kWBytes : 0);
   static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
+  // Plain key tiles stage E in shared memory (per epilogue warp: 3 swizzled
+  // 32-row x 64-column tiles) and write it with TMA bulk stores.
+  static constexpr bool kTmaStore = KMODE && !SPLIT && NSL == 64;
+  static constexpr int kExtraBytes = kTmaStore ? 4 * 3 * 4096 : 0;
   // TMEM per tile: Z1 | Z3 (2 * NSL) [| DH (NSL)]
   static constexpr int kAccCols = KMODE ? (NSL == 64 ? 256 : 384) : 2 * NSL;
   static constexpr int kAccBufs = (2 * kAccCols <= 512) ? 2 : 1;
@@ -279,13 +287,74 @@ struct FwdOp {
       if (SPLIT) mma_kblock<false, true>(tmem + 2 * NSL, st + kOffV, 0, st + kOffW2 + kWBytes, 8192u, id1, false);
     }
   }
+  __device__ static void epilogue_done(int lane) {
+    if (kTmaStore && lane == 0) bulk_wait_all();
+  }
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
-                                  int lane) {
+                                  int lane, uint8_t* extra) {
     const int r = quarter * 32 + lane;
     const int grow = t.row0 + r;
     const bool valid = grow < p.rows_valid;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const int64_t col0 = static_cast<int64_t>(t.slice) * NSL;
+    if constexpr (kTmaStore) {
+      // This warp's 32 rows of E1, Eh, E3 -> swizzled staging -> TMA stores.
+      float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
+      if (valid) {
+        const float* l = p.lr + (static_cast<int64_t>(t.bh) * p.T + p.x_row0 + grow) * 3;
+        eta0 = l[0];
+        eta1 = l[1];
+        eta2 = l[2];
+      }
+      const uint32_t stg = smem_u32(extra) + quarter * 3 * 4096 + lane * 128;
+      if (lane == 0) bulk_wait_read_all();  // the previous tile's stores have read the staging
+      __syncwarp();
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float z1[16], z3[16], u[16];
+        __syncwarp();
+        tmem_ld16(tq + j, z1);
+        tmem_ld16(tq + 64 + j, z3);
+        tmem_ld16(tq + 128 + j, u);
+        tmem_ld_wait();
+        uint32_t w[3][8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float e1[2], eh[2], e3[2];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const float a = z1[2 * i + c], b = z3[2 * i + c], g = u[2 * i + c];
+            const float s = sigmoid_fast(a);
+            const float sa = a * s;
+            const float ds = fmaf(sa, 1.0f - s, s);
+            e1[c] = (eta0 * g) * (b * ds);
+            eh[c] = eta1 * (sa * b);
+            e3[c] = (eta2 * g) * sa;
+          }
+          w[0][i] = pack_bf16x2(e1[0], e1[1]);
+          w[1][i] = pack_bf16x2(eh[0], eh[1]);
+          w[2][i] = pack_bf16x2(e3[0], e3[1]);
+        }
+        // row `lane` of each staging tile; 16-byte chunk c at c ^ (lane % 8)
+        const uint32_t c0 = ((j / 8) ^ (lane & 7)) << 4, c1 = ((j / 8 + 1) ^ (lane & 7)) << 4;
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          st_shared_v4(stg + m * 4096 + c0, w[m][0], w[m][1], w[m][2], w[m][3]);
+          st_shared_v4(stg + m * 4096 + c1, w[m][4], w[m][5], w[m][6], w[m][7]);
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint8_t* src = extra + quarter * 3 * 4096;
+        const int row = t.row0 + quarter * 32;
+#pragma unroll
+        for (int m = 0; m < 3; ++m)
+          tma_store_3d(&p.tmE, src + m * 4096, static_cast<int>(col0), row, m * p.bh_count + t.bh);
+        bulk_commit_group();
+      }
+      return;
+    }
     if (!KMODE) {
       __nv_bfloat16* dst = p.hq + (static_cast<int64_t>(t.bh) * p.buf_rows + grow) * p.dh + col0;
 #pragma unroll 1
@@ -298,8 +367,8 @@ struct FwdOp {
         uint32_t w[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float h0 = z1[2 * i] * sigmoidf_(z1[2 * i]) * z3[2 * i];
-          const float h1 = z1[2 * i + 1] * sigmoidf_(z1[2 * i + 1]) * z3[2 * i + 1];
+          const float h0 = z1[2 * i] * sigmoid_fast(z1[2 * i]) * z3[2 * i];
+          const float h1 = z1[2 * i + 1] * sigmoid_fast(z1[2 * i + 1]) * z3[2 * i + 1];
           w[i] = pack_bf16x2(h0, h1);
         }
         if (valid) {
@@ -329,7 +398,7 @@ struct FwdOp {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float a = z1[i], b = z3[i], g = u[i];
-          const float s = sigmoidf_(a);
+          const float s = SPLIT ? sigmoidf_(a) : sigmoid_fast(a);
           const float sa = a * s;
           e[0][i] = eta0 * g * b * (s * (1.0f + a * (1.0f - s)));
           e[1][i] = eta1 * sa * b;
@@ -405,6 +474,7 @@ struct GemmOp {
   static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
   static constexpr int kAccCols = TmemCols<BN>::value;
   static constexpr int kAccBufs = 2;
+  static constexpr int kExtraBytes = 0;
   struct Tile { int m0, n0, item, out_item, split, zb; bool alt; };
 
   __device__ static int num_tiles(const Params& p) { return p.n_tiles; }
@@ -470,8 +540,9 @@ struct GemmOp {
       mma_kblock<A_MN, B_MN>(tmem, st + kABytes, 8192u, st + kOffB, 8192u, id, false);
     }
   }
+  __device__ static void epilogue_done(int) {}
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
-                                  int lane) {
+                                  int lane, uint8_t*) {
     const int r = quarter * 32 + lane;
     const int grow = t.m0 + r;
     const bool valid = grow < p.m_valid;
@@ -535,7 +606,7 @@ struct GemmOp {
 
 template <class Op>
 constexpr int umma_smem_bytes() {
-  return Op::kStages * Op::kStageBytes + (2 * Op::kStages + 4) * 8 + 16 + 1024;
+  return Op::kStages * Op::kStageBytes + Op::kExtraBytes + (2 * Op::kStages + 4) * 8 + 16 + 1024;
 }
 
 }  // namespace lact
