@@ -197,8 +197,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload at this sequence length instead (a scaled case "
+                         "for profiling; named in config.workload)")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        T = args.tokens
+        single = w.Tq != w.T
+        w = w.scaled(name=f"{w.name}@T{T}", T=T, Tq=w.Tq if single else T,
+                     chunk=T if single else min(w.chunk, T))
     if args.impl == "reference":
         return run_reference(args, w)
 

@@ -58,57 +58,74 @@ template <> struct Vec<float, 1> {
   __device__ void set(int, float x) { u = x; }
 };
 
-template <typename T, int VEC, int S, int MAXV>
+template <typename T, int VEC, int S, int MAXV, int ROWS>
 __global__ void __launch_bounds__(256) k_qk_prologue(const T* __restrict__ q, T* __restrict__ qh,
                                                      int64_t q_rows, const T* __restrict__ k,
                                                      T* __restrict__ kh, int64_t k_rows, int d,
                                                      T* __restrict__ kh_lo) {
+  // Each group of S threads handles ROWS rows, all loads issued before any
+  // reduction, so every thread keeps ROWS * MAXV 16-byte loads in flight.
   using V = Vec<T, VEC>;
   using U = decltype(V::u);
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t row = gtid / S;
+  const int64_t group = gtid / S;
   const int sl = static_cast<int>(gtid % S);
-  const bool active = row < q_rows + k_rows;
-  const bool is_q = row < q_rows;
+  const int64_t total = q_rows + k_rows;
   const int nv = d / VEC;
-  const T* src = is_q ? q + row * d : k + (row - q_rows) * d;
-  float y[MAXV][VEC];
-  float ss = 0.f;
+  V in[ROWS][MAXV];
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int v = sl + i * S;
-    V in;
-    if (active && v < nv) in.u = reinterpret_cast<const U*>(src)[v];
+  for (int rr = 0; rr < ROWS; ++rr) {
+    const int64_t row = group * ROWS + rr;
+    const T* src = row < q_rows ? q + row * d : k + (row - q_rows) * d;
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      float t = 0.f;
-      if (active && v < nv) {
-        const float a = in.get(e);
-        t = __fdividef(a, 1.0f + __expf(-a));
-      }
-      y[i][e] = t;
-      ss += t * t;
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = sl + i * S;
+      if (row < total && v < nv) in[rr][i].u = reinterpret_cast<const U*>(src)[v];
     }
   }
 #pragma unroll
-  for (int o = S / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (!active) return;
-  const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
-  T* dst = is_q ? qh + row * d : kh + (row - q_rows) * d;
-  T* dst_lo = (kh_lo && !is_q) ? kh_lo + (row - q_rows) * d : nullptr;
+  for (int rr = 0; rr < ROWS; ++rr) {
+    const int64_t row = group * ROWS + rr;
+    const bool active = row < total;
+    float y[MAXV][VEC];
+    float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int v = sl + i * S;
-    if (v < nv) {
-      V hi, lo;
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = sl + i * S;
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
-        const float val = y[i][e] * inv;
-        hi.set(e, val);
-        lo.set(e, val - hi.get(e));
+        float t = 0.f;
+        if (active && v < nv) {
+          const float a = in[rr][i].get(e);
+          // Split-bf16 keys (kh_lo) need the accurate sigmoid; plain bf16
+          // rounding hides the one-op approximation.
+          t = (kh_lo || VEC != 8) ? __fdividef(a, 1.0f + __expf(-a)) : a * sigmoid_fast(a);
+        }
+        y[i][e] = t;
+        ss += t * t;
       }
-      reinterpret_cast<U*>(dst)[v] = hi.u;
-      if (dst_lo) reinterpret_cast<U*>(dst_lo)[v] = lo.u;
+    }
+#pragma unroll
+    for (int o = S / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (!active) continue;
+    const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+    const bool is_q = row < q_rows;
+    T* dst = is_q ? qh + row * d : kh + (row - q_rows) * d;
+    T* dst_lo = (kh_lo && !is_q) ? kh_lo + (row - q_rows) * d : nullptr;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = sl + i * S;
+      if (v < nv) {
+        V hi, lo;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          const float val = y[i][e] * inv;
+          hi.set(e, val);
+          lo.set(e, val - hi.get(e));
+        }
+        reinterpret_cast<U*>(dst)[v] = hi.u;
+        if (dst_lo) reinterpret_cast<U*>(dst_lo)[v] = lo.u;
+      }
     }
   }
 }
@@ -136,8 +153,27 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
                                                     float* __restrict__ Mm) {
   const int64_t plane = static_cast<int64_t>(dh) * d;
   const int64_t total = 3 * BH * plane;
-  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < total;
-       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  if (plane % 4 == 0) {  // 16-byte steps
+    for (int64_t o = 4 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); o < total;
+         o += 4 * stride) {
+      const int64_t jb = o / plane, e = o % plane;
+      const int j = static_cast<int>(jb / BH), bh = static_cast<int>(jb % BH);
+      const int src_h = w_shared ? bh % H : bh;
+      const float* src = j == 0 ? w1 : (j == 1 ? w2 : w3);
+      const float4 x = *reinterpret_cast<const float4*>(src + static_cast<int64_t>(src_h) * plane + e);
+      *reinterpret_cast<float4*>(Wm + o) = x;
+      if (Ws) {
+        store_shadow(Ws, Ws_lo, o, x.x);
+        store_shadow(Ws, Ws_lo, o + 1, x.y);
+        store_shadow(Ws, Ws_lo, o + 2, x.z);
+        store_shadow(Ws, Ws_lo, o + 3, x.w);
+      }
+      if (Mm) *reinterpret_cast<float4*>(Mm + o) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
+  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < total; o += stride) {
     const int64_t jb = o / plane, e = o % plane;
     const int j = static_cast<int>(jb / BH), bh = static_cast<int>(jb % BH);
     const int src_h = w_shared ? bh % H : bh;
@@ -156,8 +192,17 @@ __global__ void __launch_bounds__(256) k_finalize_state(const float* __restrict_
                                                         float* __restrict__ w3o) {
   const int64_t plane = static_cast<int64_t>(dh) * d;
   const int64_t per = BH * plane;
-  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < 3 * per;
-       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  if (per % 4 == 0) {
+    for (int64_t o = 4 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); o < 3 * per;
+         o += 4 * stride) {
+      const int j = static_cast<int>(o / per);
+      float* dst = j == 0 ? w1o : (j == 1 ? w2o : w3o);
+      *reinterpret_cast<float4*>(dst + (o - j * per)) = *reinterpret_cast<const float4*>(Wm + o);
+    }
+    return;
+  }
+  for (int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; o < 3 * per; o += stride) {
     const int j = static_cast<int>(o / per);
     float* dst = j == 0 ? w1o : (j == 1 ? w2o : w3o);
     dst[o - j * per] = Wm[o];
@@ -259,60 +304,78 @@ __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
 }
 
 // Rows whose length is a multiple of 4 and at most 128 * MAXV: one pass,
-// 16-byte accesses, the updated row kept in registers until it is scaled.
-template <int MAXV>
+// 16-byte accesses, the updated rows kept in registers until they are
+// scaled.  Each warp takes ROWS consecutive rows and issues all their loads
+// before the first reduction.
+template <int MAXV, int ROWS>
 __global__ void __launch_bounds__(256) k_rule_renorm_v4(const RuleParams p) {
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  const int64_t row0 = ((static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5) * ROWS;
   const int lane = threadIdx.x & 31;
-  RuleRow r;
-  if (!rule_row(p, row, r)) return;
-  const float bb = p.rule == 1 ? p.beta_bar[r.bh * p.nch + p.chunk_idx] : 0.f;
-  const int nv = r.len >> 2;
-  float4 wn[MAXV];
-  float on = 0.f, nn = 0.f;
+  RuleRow r[ROWS];
+  bool have[ROWS];
+  float4 wn[ROWS][MAXV];
+  float on[ROWS], nn[ROWS];
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int v = lane + 32 * i;
-    if (v < nv) {
-      const int64_t o = r.base + 4 * v;
-      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int k = 0; k < p.splits; ++k) {
-        const float4 x = *reinterpret_cast<const float4*>(p.S + k * p.split_stride + o);
-        s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
+  for (int k = 0; k < ROWS; ++k) {
+    have[k] = rule_row(p, row0 + k, r[k]);
+    on[k] = 0.f;
+    nn[k] = 0.f;
+    if (!have[k]) continue;
+    const float bb = p.rule == 1 ? p.beta_bar[r[k].bh * p.nch + p.chunk_idx] : 0.f;
+    const int nv = r[k].len >> 2;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = lane + 32 * i;
+      if (v < nv) {
+        const int64_t o = r[k].base + 4 * v;
+        float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int t = 0; t < p.splits; ++t) {
+          const float4 x = *reinterpret_cast<const float4*>(p.S + t * p.split_stride + o);
+          s4.x += x.x; s4.y += x.y; s4.z += x.z; s4.w += x.w;
+        }
+        if (p.rule == 1) {
+          const float4 m = *reinterpret_cast<const float4*>(p.Mm + o);
+          s4.x += bb * m.x; s4.y += bb * m.y; s4.z += bb * m.z; s4.w += bb * m.w;
+          *reinterpret_cast<float4*>(p.Mm + o) = s4;
+        }
+        const float4 w = *reinterpret_cast<const float4*>(p.Wm + o);
+        on[k] += w.x * w.x + w.y * w.y + w.z * w.z + w.w * w.w;
+        wn[k][i] = make_float4(w.x + s4.x, w.y + s4.y, w.z + s4.z, w.w + s4.w);
+        nn[k] += wn[k][i].x * wn[k][i].x + wn[k][i].y * wn[k][i].y + wn[k][i].z * wn[k][i].z +
+                 wn[k][i].w * wn[k][i].w;
       }
-      if (p.rule == 1) {
-        const float4 m = *reinterpret_cast<const float4*>(p.Mm + o);
-        s.x += bb * m.x; s.y += bb * m.y; s.z += bb * m.z; s.w += bb * m.w;
-        *reinterpret_cast<float4*>(p.Mm + o) = s;
-      }
-      const float4 w = *reinterpret_cast<const float4*>(p.Wm + o);
-      on += w.x * w.x + w.y * w.y + w.z * w.z + w.w * w.w;
-      wn[i] = make_float4(w.x + s.x, w.y + s.y, w.z + s.z, w.w + s.w);
-      nn += wn[i].x * wn[i].x + wn[i].y * wn[i].y + wn[i].z * wn[i].z + wn[i].w * wn[i].w;
     }
   }
-  on = warp_sum(on);
-  nn = warp_sum(nn);
-  const float sc = nn > 0.f ? sqrtf(on) / sqrtf(nn) : 0.f;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int v = lane + 32 * i;
-    if (v < nv) {
-      const int64_t o = r.base + 4 * v;
-      const float4 w = make_float4(wn[i].x * sc, wn[i].y * sc, wn[i].z * sc, wn[i].w * sc);
-      *reinterpret_cast<float4*>(p.Wm + o) = w;
-      if (p.Ws) {
-        uint2 hi;
-        hi.x = pack_bf16x2(w.x, w.y);
-        hi.y = pack_bf16x2(w.z, w.w);
-        *reinterpret_cast<uint2*>(p.Ws + o) = hi;
-        if (p.Ws_lo) {
-          const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&hi.x);
-          const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&hi.y);
-          uint2 lo;
-          lo.x = pack_bf16x2(w.x - __low2float(h0), w.y - __high2float(h0));
-          lo.y = pack_bf16x2(w.z - __low2float(h1), w.w - __high2float(h1));
-          *reinterpret_cast<uint2*>(p.Ws_lo + o) = lo;
+  for (int k = 0; k < ROWS; ++k) {
+    on[k] = warp_sum(on[k]);
+    nn[k] = warp_sum(nn[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < ROWS; ++k) {
+    if (!have[k]) continue;
+    const float sc = nn[k] > 0.f ? sqrtf(on[k]) / sqrtf(nn[k]) : 0.f;
+    const int nv = r[k].len >> 2;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = lane + 32 * i;
+      if (v < nv) {
+        const int64_t o = r[k].base + 4 * v;
+        const float4 w = make_float4(wn[k][i].x * sc, wn[k][i].y * sc, wn[k][i].z * sc, wn[k][i].w * sc);
+        *reinterpret_cast<float4*>(p.Wm + o) = w;
+        if (p.Ws) {
+          uint2 hi;
+          hi.x = pack_bf16x2(w.x, w.y);
+          hi.y = pack_bf16x2(w.z, w.w);
+          *reinterpret_cast<uint2*>(p.Ws + o) = hi;
+          if (p.Ws_lo) {
+            const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&hi.x);
+            const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&hi.y);
+            uint2 lo;
+            lo.x = pack_bf16x2(w.x - __low2float(h0), w.y - __high2float(h0));
+            lo.y = pack_bf16x2(w.z - __low2float(h1), w.w - __high2float(h1));
+            *reinterpret_cast<uint2*>(p.Ws_lo + o) = lo;
+          }
         }
       }
     }

@@ -377,9 +377,10 @@ struct Inputs {
 
 template <typename T, int VEC, int S, int MAXV>
 static cudaError_t prologue_as(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st) {
+  constexpr int ROWS = 4;  // rows per thread group, loads issued together
   const int64_t rows = D.BH * D.Tq + D.BH * D.T;
-  const unsigned blocks = static_cast<unsigned>(cdiv(rows * S, 256));
-  k_qk_prologue<T, VEC, S, MAXV><<<blocks, 256, 0, st>>>(
+  const unsigned blocks = static_cast<unsigned>(cdiv(cdiv(rows, ROWS) * S, 256));
+  k_qk_prologue<T, VEC, S, MAXV, ROWS><<<blocks, 256, 0, st>>>(
       static_cast<const T*>(in.q), static_cast<T*>(b.qh), D.BH * D.Tq, static_cast<const T*>(in.k),
       static_cast<T*>(b.kh), D.BH * D.T, static_cast<int>(D.d), reinterpret_cast<T*>(b.kh_lo));
   return cudaGetLastError();
@@ -434,7 +435,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
   const bool bf = D.dtype == LACT_BF16;
   const int BH = static_cast<int>(D.BH), d = static_cast<int>(D.d), dh = static_cast<int>(D.dh);
   const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane;
-  const unsigned state_blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(planes, 256), 4096));
+  const unsigned state_blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(planes, 1024), 148 * 16));
 
   // Fast-weight masters (+ bf16 shadows), momentum = 0.
   L(K_INIT, [&] {
@@ -740,16 +741,17 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
         r.Wm = b.Wm; r.Ws = b.Ws; r.Ws_lo = b.Ws_lo; r.S = dir; r.splits = dir_splits; r.split_stride = planes;
         r.Mm = b.Mm; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c);
         r.rule = D.rule; r.BH = BH; r.dh = dh; r.d = d;
-        const unsigned grid = static_cast<unsigned>(cdiv((2 * D.BH * D.dh + D.BH * D.d) * 32, 256));
+        const int64_t rows = 2 * D.BH * D.dh + D.BH * D.d;
+        const unsigned grid = static_cast<unsigned>(cdiv(rows * 32, 256));
         const int64_t longest = std::max(D.d, D.dh);
         if (D.d % 4 != 0 || D.dh % 4 != 0 || longest > 128 * 8)
           k_rule_renorm<<<grid, 256, 0, st>>>(r);
         else if (longest <= 128 * 2)
-          k_rule_renorm_v4<2><<<grid, 256, 0, st>>>(r);
+          k_rule_renorm_v4<2, 1><<<grid, 256, 0, st>>>(r);
         else if (longest <= 128 * 4)
-          k_rule_renorm_v4<4><<<grid, 256, 0, st>>>(r);
+          k_rule_renorm_v4<4, 1><<<grid, 256, 0, st>>>(r);
         else
-          k_rule_renorm_v4<8><<<grid, 256, 0, st>>>(r);
+          k_rule_renorm_v4<8, 1><<<grid, 256, 0, st>>>(r);
         return cudaGetLastError();
       });
     };
