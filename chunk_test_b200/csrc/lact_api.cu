@@ -26,6 +26,7 @@
 #include "umma_kernels.cuh"
 #include "apply_kernel.cuh"
 #include "key_grad_kernel.cuh"
+#include "pair_kernels.cuh"
 
 namespace lact {
 
@@ -267,6 +268,55 @@ static cudaError_t launch_key_grad(int64_t items, const KeyGradParams& p, cudaSt
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, sm_count()));
   k_key_grad64<<<grid, kKGThreads, smem, st>>>(p);
   return cudaGetLastError();
+}
+
+// CTA-pair kernels: one 2-CTA cluster per pair tile, up to one CTA per SM.
+template <class Op>
+static cudaError_t launch_pair(int64_t ntiles, const typename Op::Params& p, cudaStream_t st) {
+  constexpr int smem = umma_pair_smem_bytes<Op>();
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(umma_pair_kernel<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  // Pairs that fit at once (a cluster's two CTAs share a GPC, so an SM can
+  // be left without a partner).
+  static int max_pairs[64] = {};
+  if (dev < 64 && !max_pairs[dev]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sm_count() / 2));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, umma_pair_kernel<Op>, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = sm_count() / 2;
+    }
+    max_pairs[dev] = std::min(n, sm_count() / 2);
+  }
+  const int cap = dev < 64 ? max_pairs[dev] : sm_count() / 2;
+  if (ntiles <= 0 || ntiles > (int64_t(1) << 30)) return cudaErrorInvalidValue;
+  const unsigned pairs = static_cast<unsigned>(std::min<int64_t>(ntiles, cap));
+  umma_pair_kernel<Op><<<2 * pairs, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+// Pair GEMM: grid.y counts 256-row tiles.
+template <bool A_MN, bool B_MN>
+static cudaError_t launch_gemm_pair(int bn, dim3 grid, GemmParams p, cudaStream_t st) {
+  p.nt_n = static_cast<int>(grid.x);
+  p.nt_m = static_cast<int>(grid.y);
+  const int64_t ntiles = int64_t(grid.x) * grid.y * grid.z;
+  p.n_tiles = static_cast<int>(ntiles);
+  switch (bn) {
+    case 128: return launch_pair<GemmPairOp<A_MN, B_MN, 128>>(ntiles, p, st);
+    case 256: return launch_pair<GemmPairOp<A_MN, B_MN, 256>>(ntiles, p, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 // grid = (tiles along N, tiles along M, splits * items), as a tile list.
@@ -603,6 +653,8 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           if (D.rule != LACT_RULE_MUON) {  // W2's gradient straight into its [d, dh] layout
             g.tr_group = 1; g.tr_mod = BH; g.ld_t = dh;
           }
+          if (!D.split && (D.bn == 128 || D.bn == 256))   // 256-row pair tiles over dh
+            return launch_gemm_pair<true, true>(D.bn, dim3(d / D.bn, cdiv(dh, 256), splits * 3 * BH), g, st);
           return launch_gemm_any<true, true>(D.split, D.bn, dim3(d / D.bn, cdiv(dh, 128), splits * 3 * BH), g, st);
         });
       } else if (!bf) {
