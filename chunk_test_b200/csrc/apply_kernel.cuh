@@ -7,11 +7,17 @@
 //   Z_s = Q^ [W1_s; W3_s]^T          tcgen05, fp32 in TMEM (2 buffers)
 //   H_s = silu(Z1_s) * Z3_s          epilogue warps, bf16 into shared memory
 //   O  += H_s W2[:, s]^T             tcgen05, fp32 in TMEM
-// so the gated hidden activations never leave the SM.  The MMA warp issues
-// Z_{s+1} before O_s, so the tensor core computes the next slice while the
-// epilogue warps gate the current one.
+// so the gated hidden activations never leave the SM.
 //
-// Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue.
+// Two warps issue the MMAs: warp 1 the Z MMAs and warp 6 the O MMAs, each
+// from one lane.  An MMA issue holds its thread until the tensor core takes
+// it, so every barrier wait or commit between two MMAs of one issuer leaves
+// the tensor core idle for tens of cycles; with the Z and O streams on
+// separate warps, one issuer's waits overlap the other's MMAs (and the
+// tensor core computes Z_{s+1} while the epilogue warps gate slice s).
+//
+// Warps: 0 TMA producer, 1 TMEM allocator + Z issuer, 2..5 epilogue,
+// 6 O issuer.
 // Head dims D = 64, 128, 192 or 256 (TMEM: D columns of O + 2 x 128 of Z).
 #pragma once
 
@@ -30,6 +36,9 @@ struct ApplyParams {
   __nv_bfloat16* out; // [BH, Tq, d]
   int64_t Tq;
 };
+
+constexpr int kApplyThreads = 224;   // 7 warps
+constexpr int kApplyOWarp = 6;
 
 template <int D>
 struct ApplyCfg {
@@ -51,7 +60,7 @@ struct ApplyCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) k_apply(const __grid_constant__ ApplyParams p) {
+__global__ void __launch_bounds__(kApplyThreads, 1) k_apply(const __grid_constant__ ApplyParams p) {
   using C = ApplyCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
@@ -137,48 +146,53 @@ __global__ void __launch_bounds__(kThreads, 1) k_apply(const __grid_constant__ A
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ Z issuer
     if (lane == 0) {
       constexpr uint32_t idz = idesc_bf16(kBM, 128, false, false);
-      constexpr uint32_t ido = idesc_bf16(kBM, D, false, false);
       const uint32_t sbase = smem_u32(smem);
-      int ia = 0, ib = 0, tc = 0, zc = 0, hc = 0;
+      int ia = 0, tc = 0, zc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
         if (!mbar_wait(qfull, tc & 1)) break;
-        tc_fence_after();
-        for (int step = 0; ok && step <= S; ++step) {
-          if (step < S) {  // Z_step = Q^ [W1; W3]_step^T
-            const int zb = zc & 1;
-            if (zc >= 2 && !mbar_wait(&zempty[zb], ((zc >> 1) - 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t zd = tmem + C::kColZ + zb * 128;
-            for (int kb = 0; kb < C::kKb; ++kb, ++ia) {
-              const int st = ia % C::kAStages;
-              if (!mbar_wait(&afull[st], (ia / C::kAStages) & 1)) { ok = false; break; }
-              tc_fence_after();
-              mma_kblock<false, false>(zd, sbase + kb * 16384, 0, sbase + C::kOffA + st * C::kABytes, 0,
-                                       idz, kb == 0);
-              umma_commit(&aempty[st]);
-            }
-            if (!ok) break;
-            umma_commit(&zfull[zb]);
-            ++zc;
-            if (step == S - 1) umma_commit(qempty);  // every read of this tile's q^ issued
+        for (int s = 0; ok && s < S; ++s) {  // Z_s = Q^ [W1; W3]_s^T
+          const int zb = zc & 1;
+          if (zc >= 2 && !mbar_wait(&zempty[zb], ((zc >> 1) - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t zd = tmem + C::kColZ + zb * 128;
+          for (int kb = 0; kb < C::kKb; ++kb, ++ia) {
+            const int st = ia % C::kAStages;
+            if (!mbar_wait(&afull[st], (ia / C::kAStages) & 1)) { ok = false; break; }
+            mma_kblock<false, false>(zd, sbase + kb * 16384, 0, sbase + C::kOffA + st * C::kABytes, 0,
+                                     idz, kb == 0);
+            umma_commit(&aempty[st]);
           }
-          if (step >= 1) {  // O += H_{step-1} W2[:, step-1]^T
-            const int s = step - 1, hb = hc & 1, st = ib % C::kBStages;
-            if (s == 0 && tc > 0 && !mbar_wait(oempty, (tc - 1) & 1)) { ok = false; break; }
-            if (!mbar_wait(&hfull[hb], (hc >> 1) & 1)) { ok = false; break; }
-            if (!mbar_wait(&bfull[st], (ib / C::kBStages) & 1)) { ok = false; break; }
-            tc_fence_after();
-            mma_kblock<false, false>(tmem + C::kColO, sbase + C::kOffH + hb * C::kHBytes, 0,
-                                     sbase + C::kOffB + st * C::kBBytes, 0, ido, s == 0);
-            umma_commit(&bempty[st]);
-            umma_commit(&hempty[hb]);
-            ++ib;
-            ++hc;
-          }
+          if (!ok) break;
+          umma_commit(&zfull[zb]);
+          ++zc;
+        }
+        if (ok) umma_commit(qempty);  // every read of this tile's q^ issued
+      }
+    }
+  } else if (warp == kApplyOWarp) {
+    // ------------------------------------------------------------ O issuer
+    if (lane == 0) {
+      constexpr uint32_t ido = idesc_bf16(kBM, D, false, false);
+      const uint32_t sbase = smem_u32(smem);
+      int ib = 0, tc = 0, hc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
+        for (int s = 0; ok && s < S; ++s) {  // O += H_s W2[:, s]^T
+          const int hb = hc & 1, st = ib % C::kBStages;
+          if (s == 0 && tc > 0 && !mbar_wait(oempty, (tc - 1) & 1)) { ok = false; break; }
+          if (!mbar_wait(&hfull[hb], (hc >> 1) & 1)) { ok = false; break; }
+          if (!mbar_wait(&bfull[st], (ib / C::kBStages) & 1)) { ok = false; break; }
+          tc_fence_after();
+          mma_kblock<false, false>(tmem + C::kColO, sbase + C::kOffH + hb * C::kHBytes, 0,
+                                   sbase + C::kOffB + st * C::kBBytes, 0, ido, s == 0);
+          umma_commit(&bempty[st]);
+          umma_commit(&hempty[hb]);
+          ++ib;
+          ++hc;
         }
         if (ok) umma_commit(ofull);
       }

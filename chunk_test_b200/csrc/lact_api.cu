@@ -249,7 +249,7 @@ static cudaError_t launch_apply(int64_t ntiles, const ApplyParams& p, cudaStream
   }
   if (ntiles <= 0 || ntiles > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sm_count()));
-  k_apply<D><<<grid, kThreads, smem, st>>>(p);
+  k_apply<D><<<grid, kApplyThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
