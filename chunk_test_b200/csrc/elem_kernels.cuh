@@ -305,8 +305,10 @@ __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
 
 // Rows whose length is a multiple of 4 and at most 128 * MAXV: one pass,
 // 16-byte accesses, the updated rows kept in registers until they are
-// scaled.  Each warp takes ROWS consecutive rows and issues all their loads
-// before the first reduction.
+// scaled.  Each warp takes ROWS consecutive rows.  Every load of a row (all
+// gradient splits, the momentum buffer, the master weights) is issued before
+// the first arithmetic or store, so the row costs one memory latency rather
+// than one per 16-byte chunk.
 template <int MAXV, int ROWS>
 __global__ void __launch_bounds__(256) k_rule_renorm_v4(const RuleParams p) {
   const int64_t row0 = ((static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5) * ROWS;
@@ -315,32 +317,52 @@ __global__ void __launch_bounds__(256) k_rule_renorm_v4(const RuleParams p) {
   bool have[ROWS];
   float4 wn[ROWS][MAXV];
   float on[ROWS], nn[ROWS];
+  const float* __restrict__ S = p.S;
+  const float* __restrict__ W = p.Wm;
+  const bool mom = p.rule == 1;
 #pragma unroll
   for (int k = 0; k < ROWS; ++k) {
     have[k] = rule_row(p, row0 + k, r[k]);
     on[k] = 0.f;
     nn[k] = 0.f;
     if (!have[k]) continue;
-    const float bb = p.rule == 1 ? p.beta_bar[r[k].bh * p.nch + p.chunk_idx] : 0.f;
     const int nv = r[k].len >> 2;
+    float4 g[MAXV], w[MAXV], m[MAXV];
+    // loads
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = lane + 32 * i;
+      g[i] = w[i] = m[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (v < nv) {
+        const int64_t o = r[k].base + 4 * v;
+        g[i] = __ldcs(reinterpret_cast<const float4*>(S + o));
+        w[i] = *reinterpret_cast<const float4*>(W + o);
+        if (mom) m[i] = *reinterpret_cast<const float4*>(p.Mm + o);
+      }
+    }
+    for (int t = 1; t < p.splits; ++t) {
+#pragma unroll
+      for (int i = 0; i < MAXV; ++i) {
+        const int v = lane + 32 * i;
+        if (v < nv) {
+          const float4 x = __ldcs(reinterpret_cast<const float4*>(S + t * p.split_stride + r[k].base + 4 * v));
+          g[i].x += x.x; g[i].y += x.y; g[i].z += x.z; g[i].w += x.w;
+        }
+      }
+    }
+    // update (momentum: S <- beta_bar S + G) and the new row
+    const float bb = mom ? p.beta_bar[r[k].bh * p.nch + p.chunk_idx] : 0.f;
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
       const int v = lane + 32 * i;
       if (v < nv) {
-        const int64_t o = r[k].base + 4 * v;
-        float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int t = 0; t < p.splits; ++t) {
-          const float4 x = *reinterpret_cast<const float4*>(p.S + t * p.split_stride + o);
-          s4.x += x.x; s4.y += x.y; s4.z += x.z; s4.w += x.w;
+        float4 s4 = g[i];
+        if (mom) {
+          s4.x += bb * m[i].x; s4.y += bb * m[i].y; s4.z += bb * m[i].z; s4.w += bb * m[i].w;
+          *reinterpret_cast<float4*>(p.Mm + r[k].base + 4 * v) = s4;
         }
-        if (p.rule == 1) {
-          const float4 m = *reinterpret_cast<const float4*>(p.Mm + o);
-          s4.x += bb * m.x; s4.y += bb * m.y; s4.z += bb * m.z; s4.w += bb * m.w;
-          *reinterpret_cast<float4*>(p.Mm + o) = s4;
-        }
-        const float4 w = *reinterpret_cast<const float4*>(p.Wm + o);
-        on[k] += w.x * w.x + w.y * w.y + w.z * w.z + w.w * w.w;
-        wn[k][i] = make_float4(w.x + s4.x, w.y + s4.y, w.z + s4.z, w.w + s4.w);
+        on[k] += w[i].x * w[i].x + w[i].y * w[i].y + w[i].z * w[i].z + w[i].w * w[i].w;
+        wn[k][i] = make_float4(w[i].x + s4.x, w[i].y + s4.y, w[i].z + s4.z, w[i].w + s4.w);
         nn[k] += wn[k][i].x * wn[k][i].x + wn[k][i].y * wn[k][i].y + wn[k][i].z * wn[k][i].z +
                  wn[k][i].w * wn[k][i].w;
       }
