@@ -231,7 +231,7 @@ static cudaError_t launch_umma(int64_t ntiles, const typename Op::Params& p, cud
   }
   if (ntiles <= 0 || ntiles > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sm_count()));
-  umma_kernel<Op><<<grid, kThreads, smem, st>>>(p);
+  umma_kernel<Op><<<grid, umma_threads<Op>(), smem, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -6,6 +6,11 @@
 //               runs on across tiles
 //   warp 1      TMEM allocator + MMA issuer (one elected lane), accumulating
 //               tile i into TMEM buffer (i & 1)
+//   warp 6      (Ops with kIssuers = 2) a second MMA issuer for an
+//               independent part of the tile's MMAs: an MMA issue holds its
+//               thread until the tensor core takes it, so the barrier waits
+//               and commits of one issuer idle the tensor core unless another
+//               issuer has MMAs to give it
 //   warps 2..5  epilogue: tcgen05.ld of one 32-lane TMEM quarter each, fused
 //               elementwise math, stores to global memory; the buffer is
 //               handed back to the MMA warp when read, so tile i's epilogue
@@ -22,6 +27,11 @@ constexpr int kBM = 128;  // rows of every output tile (one TMEM lane per row)
 constexpr int kBK = 64;   // K elements per stage (128 bytes of bf16)
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
+constexpr int kIssuer2Warp = 6;
+
+// Block size of a kernel whose Op has kIssuers MMA issuers.
+template <class Op>
+constexpr int umma_threads() { return Op::kIssuers == 2 ? kThreads + 32 : kThreads; }
 
 template <int N>
 struct TmemCols {
@@ -30,11 +40,12 @@ struct TmemCols {
 
 // The shared pipeline: Op supplies kStages, kStageBytes, kExtraBytes (shared
 // memory for the epilogue, after the ring), kAccCols (TMEM column stride of
-// one accumulator buffer), kAccBufs (1 or 2 buffers), Tile, num_tiles(),
-// map_tile(), num_kb(), stage_bytes(), prefetch(), load(), mma(),
-// epilogue(), epilogue_done().
+// one accumulator buffer), kAccBufs (1 or 2 buffers), kIssuers (1 or 2),
+// Tile, num_tiles(), map_tile(), num_kb(), stage_bytes(), prefetch(),
+// load(), mma(p, t, stage, tmem, kb, issuer), epilogue(), epilogue_done().
 template <class Op>
-__global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant__ typename Op::Params p) {
+__global__ void __launch_bounds__(umma_threads<Op>(), 1)
+    umma_kernel(const __grid_constant__ typename Op::Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -62,10 +73,10 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], Op::kIssuers);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_full[b], Op::kIssuers);
       mbar_init(&acc_empty[b], kEpiWarps);
     }
     fence_barrier_init();
@@ -95,8 +106,9 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || (Op::kIssuers == 2 && warp == kIssuer2Warp)) {
     if (lane == 0) {
+      const int issuer = warp == 1 ? 0 : 1;
       int it = 0, local = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++local) {
@@ -109,14 +121,13 @@ __global__ void __launch_bounds__(kThreads, 1) umma_kernel(const __grid_constant
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % S;
           if (!mbar_wait(&full[s], (it / S) & 1)) { ok = false; break; }
-          tc_fence_after();
-          Op::mma(p, t, smem_u32(smem + s * Op::kStageBytes), acc, kb);
+          Op::mma(p, t, smem_u32(smem + s * Op::kStageBytes), acc, kb, issuer);
           umma_commit(&empty[s]);
         }
         umma_commit(&acc_full[buf]);
       }
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     int local = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
       const typename Op::Tile t = Op::map_tile(p, tile);
@@ -229,6 +240,9 @@ struct FwdOp {
   // TMEM per tile: Z1 | Z3 (2 * NSL) [| DH (NSL)]
   static constexpr int kAccCols = KMODE ? (NSL == 64 ? 256 : 384) : 2 * NSL;
   static constexpr int kAccBufs = (2 * kAccCols <= 512) ? 2 : 1;
+  // Key tiles: issuer 0 the Z MMAs, issuer 1 the DH MMAs (independent
+  // accumulators and A operands).
+  static constexpr int kIssuers = KMODE ? 2 : 1;
   struct Tile { int slice, row0, bh; };
 
   // Tile order: hidden slice fastest, so CTAs running together share the
@@ -273,15 +287,17 @@ struct FwdOp {
       }
     }
   }
-  __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {
-    constexpr uint32_t id0 = idesc_bf16(kBM, 2 * NSL, false, false);
+  __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb, int issuer) {
     const bool f = kb == 0;
-    mma_kblock<false, false>(tmem, st, 0, st + kOffW, 0, id0, f);
-    if (SPLIT) {
-      mma_kblock<false, false>(tmem, st, 0, st + kOffWlo, 0, id0, false);
-      mma_kblock<false, false>(tmem, st + kOffXlo, 0, st + kOffW, 0, id0, false);
+    if (issuer == 0) {
+      constexpr uint32_t id0 = idesc_bf16(kBM, 2 * NSL, false, false);
+      mma_kblock<false, false>(tmem, st, 0, st + kOffW, 0, id0, f);
+      if (SPLIT) {
+        mma_kblock<false, false>(tmem, st, 0, st + kOffWlo, 0, id0, false);
+        mma_kblock<false, false>(tmem, st + kOffXlo, 0, st + kOffW, 0, id0, false);
+      }
     }
-    if (KMODE) {
+    if (KMODE && issuer == 1) {
       constexpr uint32_t id1 = idesc_bf16(kBM, NSL, false, true);
       mma_kblock<false, true>(tmem + 2 * NSL, st + kOffV, 0, st + kOffW2, 8192u, id1, f);
       if (SPLIT) mma_kblock<false, true>(tmem + 2 * NSL, st + kOffV, 0, st + kOffW2 + kWBytes, 8192u, id1, false);
@@ -475,6 +491,7 @@ struct GemmOp {
   static constexpr int kAccCols = TmemCols<BN>::value;
   static constexpr int kAccBufs = 2;
   static constexpr int kExtraBytes = 0;
+  static constexpr int kIssuers = 1;
   struct Tile { int m0, n0, item, out_item, split, zb; bool alt; };
 
   __device__ static int num_tiles(const Params& p) { return p.n_tiles; }
@@ -532,7 +549,7 @@ struct GemmOp {
       if (!t.alt) load_b(&p.tmBlo, st + kOffB + kBBytes, bar, t.n0, bk, t.zb);
     }
   }
-  __device__ static void mma(const Params&, const Tile& t, uint32_t st, uint32_t tmem, int kb) {
+  __device__ static void mma(const Params&, const Tile& t, uint32_t st, uint32_t tmem, int kb, int) {
     constexpr uint32_t id = idesc_bf16(kBM, BN, A_MN, B_MN);
     mma_kblock<A_MN, B_MN>(tmem, st, 8192u, st + kOffB, 8192u, id, kb == 0);
     if (SPLIT) {
