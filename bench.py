@@ -151,6 +151,23 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of x over all ranks (x itself on one rank); `device` is
+    where the reduction tensor lives (cuda for NCCL, cpu for gloo)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, tokens_per_rank_step: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput (tokens/s): every rank processes its own batch of
+    tokens_per_rank_step per step; the job takes the slowest rank's time."""
+    return world * tokens_per_rank_step * steps / (ms_max / 1e3)
+
+
 def workload_config(w: Workload, n_gpus: int) -> dict:
     in_bytes = (w.B * w.H * (w.Tq + 2 * w.T) * w.d) * (2 if w.dtype == BF16 else 4)
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "Tq": w.Tq, "d": w.d, "dh": w.dh,
@@ -221,12 +238,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     def barrier_max(x: float) -> float:
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(x, dev)
 
     def barrier():
         if world > 1:
@@ -275,7 +287,7 @@ def main():
 
     ms_step = ms_total / args.steps
     tok_step = w.tokens
-    value = world * tok_step * args.steps / (ms_total / 1e3)
+    value = job_value(world, tok_step, args.steps, ms_total)
     hbm, pk_burst, pk_sust, pk_src = peaks()
     flops = step_flops(w)
     launches_per_step = ct.launch_count(inp["q"], inp["k"], inp["w1"], w.chunk, w.order, w.rule)
@@ -346,7 +358,7 @@ def main():
         "roofline": roof,
         "kernels": kernels,
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": world * tok_step * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": job_value(world, tok_step, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk,
     }
