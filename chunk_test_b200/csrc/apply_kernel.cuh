@@ -61,6 +61,7 @@ struct ApplyCfg {
 
 template <int D>
 __global__ void __launch_bounds__(kApplyThreads, 1) k_apply(const __grid_constant__ ApplyParams p) {
+  griddep_launch();
   using C = ApplyCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
@@ -115,6 +116,7 @@ __global__ void __launch_bounds__(kApplyThreads, 1) k_apply(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // after the local setup, before any global access
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

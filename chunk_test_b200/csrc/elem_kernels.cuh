@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const T* __restrict__ q, T*
                                                      int64_t q_rows, const T* __restrict__ k,
                                                      T* __restrict__ kh, int64_t k_rows, int d,
                                                      T* __restrict__ kh_lo) {
+  griddep_launch();
+  griddep_wait();
   // Each group of S threads handles ROWS rows, all loads issued before any
   // reduction, so every thread keeps ROWS * MAXV 16-byte loads in flight.
   using V = Vec<T, VEC>;
@@ -151,6 +153,8 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
                                                     __nv_bfloat16* __restrict__ Ws,
                                                     __nv_bfloat16* __restrict__ Ws_lo,
                                                     float* __restrict__ Mm) {
+  griddep_launch();
+  griddep_wait();
   const int64_t plane = static_cast<int64_t>(dh) * d;
   const int64_t total = 3 * BH * plane;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -190,6 +194,8 @@ __global__ void __launch_bounds__(256) k_finalize_state(const float* __restrict_
                                                         int dh, float* __restrict__ w1o,
                                                         float* __restrict__ w2o,
                                                         float* __restrict__ w3o) {
+  griddep_launch();
+  griddep_wait();
   const int64_t plane = static_cast<int64_t>(dh) * d;
   const int64_t per = BH * plane;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -213,6 +219,8 @@ __global__ void __launch_bounds__(256) k_finalize_state(const float* __restrict_
 __global__ void __launch_bounds__(256) k_beta_mean(const float* __restrict__ beta, int BH, int64_t T,
                                                    int64_t chunk, int nch,
                                                    float* __restrict__ beta_bar) {
+  griddep_launch();
+  griddep_wait();
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= static_cast<int64_t>(BH) * nch) return;
@@ -272,6 +280,8 @@ __device__ __forceinline__ bool rule_row(const RuleParams& p, int64_t row, RuleR
 
 // Generic form (any row length): two passes over the row in global memory.
 __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
+  griddep_launch();
+  griddep_wait();
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   RuleRow r;
@@ -311,6 +321,8 @@ __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
 // than one per 16-byte chunk.
 template <int MAXV, int ROWS>
 __global__ void __launch_bounds__(256) k_rule_renorm_v4(const RuleParams p) {
+  griddep_launch();
+  griddep_wait();
   const int64_t row0 = ((static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5) * ROWS;
   const int lane = threadIdx.x & 31;
   RuleRow r[ROWS];
@@ -430,6 +442,8 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
 __global__ void __launch_bounds__(256) k_ns_sumsq(const float* __restrict__ S, int splits,
                                                   int64_t split_stride, int64_t plane,
                                                   float* __restrict__ Y, float* __restrict__ part) {
+  griddep_launch();
+  griddep_wait();
   __shared__ float red[9];
   const int item = blockIdx.y;
   const int64_t per = (plane + gridDim.x - 1) / gridDim.x;
@@ -451,6 +465,8 @@ __global__ void __launch_bounds__(256) k_ns_scale(float* __restrict__ Y,
                                                   __nv_bfloat16* __restrict__ Yb_lo, int64_t plane,
                                                   const float* __restrict__ part, int nblk,
                                                   float eps) {
+  griddep_launch();
+  griddep_wait();
   __shared__ float sc;
   const int item = blockIdx.y;
   if (threadIdx.x == 0) {

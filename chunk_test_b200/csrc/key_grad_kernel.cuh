@@ -62,6 +62,7 @@ struct KGCfg {
 };
 
 __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_constant__ KeyGradParams p) {
+  griddep_launch();
   using C = KGCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // after the local setup, before any global access
 
   // item -> (head, split); its tiles [t0, t1)
   auto item_range = [&](int item, int& bh, int& s, int& t0, int& t1) {

@@ -17,6 +17,7 @@
 #include <algorithm>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/lact.h"
@@ -204,6 +205,26 @@ static bool map3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows
 }
 
 // ------------------------------------------------------------------ launches
+// Every kernel is launched with programmatic stream serialization: the
+// next kernel of the stream may start while this one drains, does its local
+// setup (barrier init, TMEM allocation, tensor-map prefetch), and waits in
+// griddep_wait() for this one to finish before touching global memory.
+template <class... KArgs, class... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // SMs of the current device (the persistent kernels launch one CTA per SM).
 static int sm_count() {
   static int sms[64] = {};
@@ -231,7 +252,7 @@ static cudaError_t launch_umma(int64_t ntiles, const typename Op::Params& p, cud
   }
   if (ntiles <= 0 || ntiles > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sm_count()));
-  umma_kernel<Op><<<grid, umma_threads<Op>(), smem, st>>>(p);
+  (void)launch_pdl(umma_kernel<Op>, grid, umma_threads<Op>(), smem, st, p);
   return cudaGetLastError();
 }
 
@@ -249,7 +270,7 @@ static cudaError_t launch_apply(int64_t ntiles, const ApplyParams& p, cudaStream
   }
   if (ntiles <= 0 || ntiles > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sm_count()));
-  k_apply<D><<<grid, kApplyThreads, smem, st>>>(p);
+  (void)launch_pdl(k_apply<D>, grid, kApplyThreads, smem, st, p);
   return cudaGetLastError();
 }
 
@@ -266,7 +287,7 @@ static cudaError_t launch_key_grad(int64_t items, const KeyGradParams& p, cudaSt
   }
   if (items <= 0 || items > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, sm_count()));
-  k_key_grad64<<<grid, kKGThreads, smem, st>>>(p);
+  (void)launch_pdl(k_key_grad64, grid, kKGThreads, smem, st, p);
   return cudaGetLastError();
 }
 
@@ -301,7 +322,7 @@ static cudaError_t launch_pair(int64_t ntiles, const typename Op::Params& p, cud
   const int cap = dev < 64 ? max_pairs[dev] : sm_count() / 2;
   if (ntiles <= 0 || ntiles > (int64_t(1) << 30)) return cudaErrorInvalidValue;
   const unsigned pairs = static_cast<unsigned>(std::min<int64_t>(ntiles, cap));
-  umma_pair_kernel<Op><<<2 * pairs, kThreads, smem, st>>>(p);
+  (void)launch_pdl(umma_pair_kernel<Op>, 2 * pairs, kThreads, smem, st, p);
   return cudaGetLastError();
 }
 
@@ -430,7 +451,7 @@ static cudaError_t prologue_as(const Dims& D, const Bufs& b, const Inputs& in, c
   constexpr int ROWS = 4;  // rows per thread group, loads issued together
   const int64_t rows = D.BH * D.Tq + D.BH * D.T;
   const unsigned blocks = static_cast<unsigned>(cdiv(cdiv(rows, ROWS) * S, 256));
-  k_qk_prologue<T, VEC, S, MAXV, ROWS><<<blocks, 256, 0, st>>>(
+  (void)launch_pdl(k_qk_prologue<T, VEC, S, MAXV, ROWS>, blocks, 256, 0, st, 
       static_cast<const T*>(in.q), static_cast<T*>(b.qh), D.BH * D.Tq, static_cast<const T*>(in.k),
       static_cast<T*>(b.kh), D.BH * D.T, static_cast<int>(D.d), reinterpret_cast<T*>(b.kh_lo));
   return cudaGetLastError();
@@ -474,7 +495,7 @@ static SimtGemmParams simt_params() {
 }
 
 static cudaError_t simt(const SimtGemmParams& p, int items, cudaStream_t st) {
-  k_simt_gemm<<<dim3(cdiv(p.N, 64), cdiv(p.M, 64), items), 256, 0, st>>>(p);
+  (void)launch_pdl(k_simt_gemm, dim3(cdiv(p.N, 64), cdiv(p.M, 64), items), 256, 0, st, p);
   return cudaGetLastError();
 }
 
@@ -489,7 +510,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
 
   // Fast-weight masters (+ bf16 shadows), momentum = 0.
   L(K_INIT, [&] {
-    k_init_state<<<state_blocks, 256, 0, st>>>(in.w1, in.w2, in.w3, static_cast<int>(D.H),
+    (void)launch_pdl(k_init_state, state_blocks, 256, 0, st, in.w1, in.w2, in.w3, static_cast<int>(D.H),
                                                    D.w_shared, BH, d, dh, b.Wm, b.Ws, b.Ws_lo, b.Mm);
     return cudaGetLastError();
   });
@@ -498,7 +519,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
   if (D.rule == LACT_RULE_MOMENTUM) {
     L(K_BETA_MEAN, [&] {
       const int64_t w = D.BH * D.nch;
-      k_beta_mean<<<static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st>>>(in.beta, BH, D.T, D.chunk,
+      (void)launch_pdl(k_beta_mean, static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st, in.beta, BH, D.T, D.chunk,
                                                                             static_cast<int>(D.nch), b.bbar);
       return cudaGetLastError();
     });
@@ -572,7 +593,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
         }
         L(K_FWD_ELEM_F32, [&] {
           const int64_t n = zpl;
-          k_fwd_elem_f32<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, st>>>(
+          (void)launch_pdl(k_fwd_elem_f32, static_cast<unsigned>(cdiv(n, 256)), 256, 0, st, 
               Z, BH, D.q_rows, dh, nq, 0, nullptr, D.T, 0, static_cast<float*>(b.Hq));
           return cudaGetLastError();
         });
@@ -672,7 +693,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           });
         }
         L(K_FWD_ELEM_F32, [&] {
-          k_fwd_elem_f32<<<static_cast<unsigned>(cdiv(zpl, 256)), 256, 0, st>>>(
+          (void)launch_pdl(k_fwd_elem_f32, static_cast<unsigned>(cdiv(zpl, 256)), 256, 0, st, 
               b.Z, BH, D.key_rows, dh, nc, 1, in.lr, D.T, c0, static_cast<float*>(b.E));
           return cudaGetLastError();
         });
@@ -694,11 +715,11 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
       int dir_splits = splits;
       if (D.rule == LACT_RULE_MUON) {
         L(K_NS_SUMSQ, [&] {
-          k_ns_sumsq<<<dim3(kNsBlocks, 3 * BH), 256, 0, st>>>(b.P, splits, planes, plane, b.Yf[0], b.part);
+          (void)launch_pdl(k_ns_sumsq, dim3(kNsBlocks, 3 * BH), 256, 0, st, b.P, splits, planes, plane, b.Yf[0], b.part);
           return cudaGetLastError();
         });
         L(K_NS_SCALE, [&] {
-          k_ns_scale<<<dim3(kNsBlocks, 3 * BH), 256, 0, st>>>(b.Yf[0], b.Yb[0], b.Yb_lo[0], plane, b.part,
+          (void)launch_pdl(k_ns_scale, dim3(kNsBlocks, 3 * BH), 256, 0, st, b.Yf[0], b.Yb[0], b.Yb_lo[0], plane, b.part,
                                                               kNsBlocks, kNsEps);
           return cudaGetLastError();
         });
@@ -797,13 +818,13 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
         const unsigned grid = static_cast<unsigned>(cdiv(rows * 32, 256));
         const int64_t longest = std::max(D.d, D.dh);
         if (D.d % 4 != 0 || D.dh % 4 != 0 || longest > 128 * 8)
-          k_rule_renorm<<<grid, 256, 0, st>>>(r);
+          (void)launch_pdl(k_rule_renorm, grid, 256, 0, st, r);
         else if (longest <= 128 * 2)
-          k_rule_renorm_v4<2, 1><<<grid, 256, 0, st>>>(r);
+          (void)launch_pdl(k_rule_renorm_v4<2, 1>, grid, 256, 0, st, r);
         else if (longest <= 128 * 4)
-          k_rule_renorm_v4<4, 1><<<grid, 256, 0, st>>>(r);
+          (void)launch_pdl(k_rule_renorm_v4<4, 1>, grid, 256, 0, st, r);
         else
-          k_rule_renorm_v4<8, 1><<<grid, 256, 0, st>>>(r);
+          (void)launch_pdl(k_rule_renorm_v4<8, 1>, grid, 256, 0, st, r);
         return cudaGetLastError();
       });
     };
@@ -832,7 +853,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
   }
 
   L(K_FINALIZE, [&] {
-    k_finalize_state<<<state_blocks, 256, 0, st>>>(b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o);
+    (void)launch_pdl(k_finalize_state, state_blocks, 256, 0, st, b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o);
     return cudaGetLastError();
   });
 }

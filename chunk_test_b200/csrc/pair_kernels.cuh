@@ -111,6 +111,7 @@ __device__ __forceinline__ void mma_kblock_pair(uint32_t d_tmem, uint32_t a_base
 template <class Op>
 __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
     umma_pair_kernel(const __grid_constant__ typename Op::Params p) {
+  griddep_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
   cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // after the local setup, before any global access
 
   if (warp == 0) {
     if (lane == 0) {

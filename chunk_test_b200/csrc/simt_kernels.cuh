@@ -31,6 +31,8 @@ struct SimtGemmParams {
 };
 
 __global__ void __launch_bounds__(256) k_simt_gemm(const SimtGemmParams p) {
+  griddep_launch();
+  griddep_wait();
   __shared__ float As[16][68], Bs[16][68];
   const int item = blockIdx.z;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
@@ -100,6 +102,8 @@ __global__ void __launch_bounds__(256) k_fwd_elem_f32(const float* __restrict__ 
                                                       int kmode, const float* __restrict__ lr,
                                                       int64_t T, int64_t row0,
                                                       float* __restrict__ out) {
+  griddep_launch();
+  griddep_wait();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t plane = static_cast<int64_t>(BH) * rows * dh;
   if (i >= plane) return;

@@ -30,6 +30,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ------------------------------------------------------------------ launch chaining
+// Programmatic dependent launch: a kernel lets the next kernel of its stream
+// launch as soon as all of its own CTAs are running (griddep_launch), and a
+// kernel waits for the previous kernel of its stream to finish and flush its
+// memory (griddep_wait) before its first global access, after its local
+// setup.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -46,6 +46,7 @@ struct TmemCols {
 template <class Op>
 __global__ void __launch_bounds__(umma_threads<Op>(), 1)
     umma_kernel(const __grid_constant__ typename Op::Params p) {
+  griddep_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -90,6 +91,7 @@ __global__ void __launch_bounds__(umma_threads<Op>(), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // after the local setup, before any global access
 
   if (warp == 0) {
     if (lane == 0) {
