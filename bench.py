@@ -208,7 +208,7 @@ def run_reference(args, w: Workload):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -265,10 +265,11 @@ def main():
     if ct.status(stream) != ct.LACT_OK:
         raise SystemExit("device status not OK after warm-up")
 
-    # ---- timed region (device time, CUDA events on the launching stream)
+    # ---- timed region (device time, CUDA events on the launching stream).
+    # The K steps run exactly as a caller runs them: no events between the
+    # kernels, whose launches overlap (programmatic dependent launch).
     clocks = ClockSampler(local)
     time.sleep(0.3)
-    ct.profile_enable(True)
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -278,12 +279,30 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    ct.profile_enable(False)
     clk = clocks.stop()
     ms_total = barrier_max(e0.elapsed_time(e1))
-    prof = ct.profile_read()
     if ct.status(stream) != ct.LACT_OK:
         raise SystemExit("device status not OK after the timed region")
+
+    # ---- per-kernel pass: the same K steps again with a CUDA event pair around
+    # every launch (the library's launch profiler).  Events between launches
+    # stop the overlap of consecutive launches, so this pass gives the
+    # per-kernel durations (kernel shares, roofline) but not the headline time.
+    ct.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(args.steps):
+        step()
+    p1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ct.profile_enable(False)
+    ms_profiled = barrier_max(p0.elapsed_time(p1))
+    prof = ct.profile_read()
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after the per-kernel pass")
 
     ms_step = ms_total / args.steps
     tok_step = w.tokens
@@ -357,6 +376,11 @@ def main():
                              "peak_source": pk_src},
         "roofline": roof,
         "kernels": kernels,
+        "kernel_pass": {"ms_per_step": ms_profiled / args.steps,
+                        "method": "the same K steps again with a CUDA event pair around every launch "
+                                  "(kernel shares, roofline durations); per-launch events stop the "
+                                  "overlap of consecutive launches, so the headline time is the "
+                                  "first pass, without them"},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": job_value(world, tok_step, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
