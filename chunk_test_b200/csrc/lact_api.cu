@@ -48,6 +48,7 @@ struct Dims {
   int bn;            // N tile over d (bf16 GEMMs)
   bool split;        // split-bf16 update path (bf16 + Muon)
   bool fused_kg;     // fused key forward + gradient (bf16, d = 64, dh = 128, not split)
+  bool dbuf;         // two bf16 shadow sets (bf16, apply-then-update): chunk c reads set c % 2
   int kg_splits;     // its token splits per head
 };
 
@@ -85,6 +86,7 @@ static int validate(const lact_problem* p, Dims& D) {
   D.bn = choose_bn(D.d);
   D.split = D.dtype == LACT_BF16 && D.rule == LACT_RULE_MUON;
   D.fused_kg = D.dtype == LACT_BF16 && !D.split && D.d == 64 && D.dh == 128;
+  D.dbuf = D.dtype == LACT_BF16 && D.order == LACT_APPLY_THEN_UPDATE && D.nch > 1;
   D.kg_splits = 1;
   // Token splits of the gradient contraction: fill ~2 waves of 148 SMs when
   // the output tiles alone do not.
@@ -136,8 +138,8 @@ static void plan(const Dims& D, Bump& bp, Bufs& b) {
   b.kh = bp.take<uint8_t>(D.BH * D.T * D.d * esz);
   if (D.split) b.kh_lo = bp.take<__nv_bfloat16>(D.BH * D.T * D.d);
   b.Wm = bp.take<float>(planes);
-  if (bf) b.Ws = bp.take<__nv_bfloat16>(planes);
-  if (D.split) b.Ws_lo = bp.take<__nv_bfloat16>(planes);
+  if (bf) b.Ws = bp.take<__nv_bfloat16>((D.dbuf ? 2 : 1) * planes);
+  if (D.split) b.Ws_lo = bp.take<__nv_bfloat16>((D.dbuf ? 2 : 1) * planes);
   b.P = bp.take<float>((bf ? D.splits : 1) * planes);
   if (D.rule == LACT_RULE_MOMENTUM) {
     b.Mm = bp.take<float>(planes);
@@ -420,7 +422,7 @@ struct Launcher {
 // the previous state) in apply-then-update order.
 struct SideRes {
   cudaStream_t side = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, join[2] = {nullptr, nullptr};
 };
 static SideRes g_side[64];
 static std::mutex g_side_mu;
@@ -433,7 +435,8 @@ static const SideRes* side_resources() {
   if (!r.side) {
     if (cudaStreamCreateWithFlags(&r.side, cudaStreamNonBlocking) != cudaSuccess) return r.side = nullptr, nullptr;
     if (cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&r.join[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&r.join[1], cudaEventDisableTiming) != cudaSuccess)
       return nullptr;
   }
   return &r;
@@ -525,20 +528,28 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
     });
   }
 
-  bool join_before_rule = false;
+  bool join_before_rule = false, side_used = false;
   for (int64_t c = 0; c < D.nch; ++c) {
     const int64_t c0 = c * D.chunk;
     const int nc = static_cast<int>((c0 + D.chunk < D.T ? c0 + D.chunk : D.T) - c0);
     const int64_t qr0 = D.nch == 1 ? 0 : c0;
     const int nq = static_cast<int>(D.nch == 1 ? D.Tq : nc);
+    // bf16 shadows of W_c (read by this chunk's kernels) and of W_{c+1}
+    // (written by its rule): with two sets, chunk c's apply may still run
+    // while chunk c's rule writes the other set.
+    const int64_t cur = D.dbuf ? (c & 1) : 0, nxt = D.dbuf ? 1 - cur : 0;
+    __nv_bfloat16* const Wsc = b.Ws ? b.Ws + cur * planes : nullptr;
+    __nv_bfloat16* const Wsc_lo = b.Ws_lo ? b.Ws_lo + cur * planes : nullptr;
+    __nv_bfloat16* const Wsn = b.Ws ? b.Ws + nxt * planes : nullptr;
+    __nv_bfloat16* const Wsn_lo = b.Ws_lo ? b.Ws_lo + nxt * planes : nullptr;
 
     auto apply = [&] {
       if (bf && d <= 256) {
         L(K_APPLY_FUSED, [&] {
           ApplyParams a;
           std::memset(&a, 0, sizeof(a));
-          if (!map3d(&a.tmQ, b.qh, d, D.Tq, BH, 64, 128) || !map3d(&a.tmW, b.Ws, d, dh, 3 * BH, 64, 64) ||
-              !map3d(&a.tmW2, b.Ws + D.BH * plane, dh, d, BH, 64, d))
+          if (!map3d(&a.tmQ, b.qh, d, D.Tq, BH, 64, 128) || !map3d(&a.tmW, Wsc, d, dh, 3 * BH, 64, 64) ||
+              !map3d(&a.tmW2, Wsc + D.BH * plane, dh, d, BH, 64, d))
             return cudaErrorInvalidValue;
           a.bh_count = BH; a.dh = dh; a.n_row_tiles = static_cast<int>(cdiv(nq, 128));
           a.q_row0 = static_cast<int>(qr0); a.rows_valid = nq;
@@ -555,14 +566,14 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
         L(K_FWD_QUERY, [&] {
           FwdParams f;
           std::memset(&f, 0, sizeof(f));
-          if (!map3d(&f.tmX, b.qh, d, D.Tq, BH, 64, 128) || !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 64))
+          if (!map3d(&f.tmX, b.qh, d, D.Tq, BH, 64, 128) || !map3d(&f.tmW, Wsc, d, dh, 3 * BH, 64, 64))
             return cudaErrorInvalidValue;
           f.bh_count = BH; f.x_row0 = static_cast<int>(qr0); f.rows_valid = nq; f.kb_count = d / 64;
           f.dh = dh; f.T = static_cast<int>(D.T); f.hq = static_cast<__nv_bfloat16*>(b.Hq);
           f.buf_rows = D.q_rows; f.lr = in.lr;
           const bool wide = dh % 128 == 0;                    // 128-wide hidden slices
           f.n_slices = dh / (wide ? 128 : 64); f.n_row_tiles = static_cast<int>(cdiv(nq, 128));
-          if (wide && !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 128)) return cudaErrorInvalidValue;
+          if (wide && !map3d(&f.tmW, Wsc, d, dh, 3 * BH, 64, 128)) return cudaErrorInvalidValue;
           const int64_t tiles = int64_t(f.n_slices) * f.n_row_tiles * BH;
           return wide ? launch_umma<FwdOp<false, false, 128>>(tiles, f, st)
                       : launch_umma<FwdOp<false>>(tiles, f, st);
@@ -570,7 +581,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
         L(K_APPLY_OUT, [&] {
           GemmParams g = gemm_params();
           if (!map3d(&g.tmA, b.Hq, dh, D.q_rows, BH, 64, 128) ||
-              !map3d(&g.tmB, b.Ws + D.BH * plane, dh, d, BH, 64, D.bn))
+              !map3d(&g.tmB, Wsc + D.BH * plane, dh, d, BH, 64, D.bn))
             return cudaErrorInvalidValue;
           g.items = BH; g.kb_count = dh / 64; g.kb_total = g.kb_count;
           g.zb_mod = BH; g.zb_add = 0; g.m_valid = nq;
@@ -620,8 +631,8 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           KeyGradParams k;
           std::memset(&k, 0, sizeof(k));
           if (!map3d(&k.tmK, b.kh, d, D.T, BH, 64, 128) || !map3d(&k.tmV, in.v, d, D.T, BH, 64, 128) ||
-              !map3d(&k.tmW, b.Ws, d, dh, 3 * BH, 64, 64) ||
-              !map3d(&k.tmW2, b.Ws + D.BH * plane, dh, d, BH, 64, 64))
+              !map3d(&k.tmW, Wsc, d, dh, 3 * BH, 64, 64) ||
+              !map3d(&k.tmW2, Wsc + D.BH * plane, dh, d, BH, 64, 64))
             return cudaErrorInvalidValue;
           k.bh_count = BH; k.splits = ks; k.n_tiles = tiles; k.x_row0 = static_cast<int>(c0);
           k.rows_valid = nc; k.T = static_cast<int>(D.T); k.lr = in.lr; k.P = b.P;
@@ -632,12 +643,12 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           FwdParams f;
           std::memset(&f, 0, sizeof(f));
           if (!map3d(&f.tmX, b.kh, d, D.T, BH, 64, 128) || !map3d(&f.tmV, in.v, d, D.T, BH, 64, 128) ||
-              !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 64))
+              !map3d(&f.tmW, Wsc, d, dh, 3 * BH, 64, 64))
             return cudaErrorInvalidValue;
-          if (!map3d(&f.tmW2, b.Ws + D.BH * plane, dh, d, BH, 64, 64)) return cudaErrorInvalidValue;
+          if (!map3d(&f.tmW2, Wsc + D.BH * plane, dh, d, BH, 64, 64)) return cudaErrorInvalidValue;
           if (D.split && (!map3d(&f.tmXlo, b.kh_lo, d, D.T, BH, 64, 128) ||
-                          !map3d(&f.tmWlo, b.Ws_lo, d, dh, 3 * BH, 64, 64) ||
-                          !map3d(&f.tmW2lo, b.Ws_lo + D.BH * plane, dh, d, BH, 64, 64)))
+                          !map3d(&f.tmWlo, Wsc_lo, d, dh, 3 * BH, 64, 64) ||
+                          !map3d(&f.tmW2lo, Wsc_lo + D.BH * plane, dh, d, BH, 64, 64)))
             return cudaErrorInvalidValue;
           f.bh_count = BH; f.x_row0 = static_cast<int>(c0); f.rows_valid = nc; f.kb_count = d / 64;
           f.dh = dh; f.T = static_cast<int>(D.T); f.e = static_cast<__nv_bfloat16*>(b.E);
@@ -649,7 +660,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           const bool wide = false;
           if (!D.split && !map3d(&f.tmE, b.E, dh, D.key_rows, 3 * BH, 64, 32)) return cudaErrorInvalidValue;
           f.n_slices = dh / (wide ? 128 : 64); f.n_row_tiles = static_cast<int>(cdiv(nc, 128));
-          if (wide && !map3d(&f.tmW, b.Ws, d, dh, 3 * BH, 64, 128)) return cudaErrorInvalidValue;
+          if (wide && !map3d(&f.tmW, Wsc, d, dh, 3 * BH, 64, 128)) return cudaErrorInvalidValue;
           const int64_t tiles = int64_t(f.n_slices) * f.n_row_tiles * BH;
           if (D.split) return launch_umma<FwdOp<true, true>>(tiles, f, st);
           return wide ? launch_umma<FwdOp<true, false, 128>>(tiles, f, st) : launch_umma<FwdOp<true>>(tiles, f, st);
@@ -805,13 +816,17 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
         dir_splits = 1;
       }
       if (join_before_rule) {
-        if (L.err == LACT_OK && cudaStreamWaitEvent(main_st, side->join, 0) != cudaSuccess) L.err = LACT_ECUDA;
+        // the rule rewrites the shadow set that the apply launched one chunk
+        // earlier (two sets) or in this chunk (one set) reads
+        const int64_t jc = D.dbuf ? c - 1 : c;
+        if (jc >= 0 && L.err == LACT_OK && cudaStreamWaitEvent(main_st, side->join[jc & 1], 0) != cudaSuccess)
+          L.err = LACT_ECUDA;
         join_before_rule = false;
       }
       L(K_RULE, [&] {
         RuleParams r;
         std::memset(&r, 0, sizeof(r));
-        r.Wm = b.Wm; r.Ws = b.Ws; r.Ws_lo = b.Ws_lo; r.S = dir; r.splits = dir_splits; r.split_stride = planes;
+        r.Wm = b.Wm; r.Ws = Wsn; r.Ws_lo = Wsn_lo; r.S = dir; r.splits = dir_splits; r.split_stride = planes;
         r.Mm = b.Mm; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c);
         r.rule = D.rule; r.BH = BH; r.dh = dh; r.d = d;
         const int64_t rows = 2 * D.BH * D.dh + D.BH * D.d;
@@ -830,6 +845,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
     };
 
     if (D.order == LACT_APPLY_THEN_UPDATE && side && bf && !L.dry) {
+      side_used = true;
       // apply on the side stream, concurrently with the key forward and the
       // gradient; joined before the rule rewrites the state.
       if (L.err == LACT_OK && (cudaEventRecord(side->fork, main_st) != cudaSuccess ||
@@ -838,7 +854,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
       st = side->side;
       L.st = st;
       apply();
-      if (L.err == LACT_OK && cudaEventRecord(side->join, side->side) != cudaSuccess) L.err = LACT_ECUDA;
+      if (L.err == LACT_OK && cudaEventRecord(side->join[c & 1], side->side) != cudaSuccess) L.err = LACT_ECUDA;
       st = main_st;
       L.st = st;
       join_before_rule = true;
@@ -852,6 +868,8 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
     }
   }
 
+  if (side_used && L.err == LACT_OK && cudaStreamWaitEvent(main_st, side->join[(D.nch - 1) & 1], 0) != cudaSuccess)
+    L.err = LACT_ECUDA;   // the last chunks' applies are done before the call's work ends
   L(K_FINALIZE, [&] {
     (void)launch_pdl(k_finalize_state, state_blocks, 256, 0, st, b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o);
     return cudaGetLastError();
