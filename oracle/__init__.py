@@ -44,10 +44,24 @@ design notes):
   R9  a final chunk shorter than `chunk` is processed as it is.
   R10 with a single chunk the queries may have their own length Tq (the target
       views of a posed image set); with several chunks Tq must equal T.
+  R11 the update mask has one flag per chunk, shared by every (batch, head)
+      (the clean/noisy pattern is a property of the sequence).  A chunk whose
+      flag is 0 is still applied in its place in the order, but skips the
+      whole update -- gradient, rule, momentum and renorm -- so the state
+      passes through unchanged (video: only clean-frame chunks update the
+      memory, noisy chunks read what the earlier chunks wrote; [P3]
+      「更新顺序必须遵守信息可见范围」, [P1 §3.2]).
+  R12 the per-head output scale [P1 §2.1] is given as its values s (after
+      the silu of the page's linear map), one per (batch, head, query
+      token); the output row is s_t * f_W(q_t).
+  R13 resuming a sequence across calls: the momentum may start from a given
+      M_0 (zeros otherwise) and the final M is returned, so two calls split
+      at a chunk boundary equal one call.
 """
 from .lact_oracle import (  # noqa: F401
     APPLY_THEN_UPDATE, UPDATE_THEN_APPLY, RULE_GD, RULE_MOMENTUM, RULE_MUON,
     NS_COEFFS, NS_STEPS, NS_EPS,
     sigmoid, silu, silu_prime, qk_prologue, fast_net, chunk_gradient,
-    newton_schulz5, renorm_rows, rule_step, ttt_head, ttt_layer, blas_threads,
+    newton_schulz5, renorm_rows, rule_step, ttt_head, ttt_head_state, ttt_layer, ttt_layer_ex,
+    blas_threads,
 )

@@ -123,7 +123,8 @@ def rule_step(rule, G, M, beta_chunk):
     raise ValueError(f"unknown rule {rule}")
 
 
-def ttt_head(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule):
+def ttt_head_state(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule,
+                   update_mask=None, out_scale=None, M0=None):
     """The layer for one (batch, head): q [Tq, d], k, v [T, d], lr [T, 3],
     beta [T] (momentum only), W1, W3 [dh, d], W2 [d, dh].
 
@@ -132,27 +133,52 @@ def ttt_head(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule):
       order 0 (apply-then-update, causal): o_c = f_{W_{c-1}}(q_c), then
               W_c = renorm(W_{c-1} - U(grad of chunk c on W_{c-1}));
       order 1 (update-then-apply, sets):  W_c first, then o_c = f_{W_c}(q_c).
-    Returns out [Tq, d] and the final (W1, W2, W3)."""
+    Options (R11-R13):
+      update_mask  one flag per chunk; a chunk whose flag is 0 is applied in
+                   its place in the order but skips the whole update
+                   (gradient, rule, momentum, renorm), so W_c = W_{c-1}
+                   (noisy video chunks read the memory, clean ones write
+                   it: [P3] 「更新顺序…」, [P1 §3.2]).
+      out_scale    [Tq] per-query factor s_t: o_t = s_t * f_W(q_t)
+                   ([P1 §2.1] per-head output scale).
+      M0           initial momentum (M1, M2, M3) instead of zeros.
+    Returns out [Tq, d], the final (W1, W2, W3) and the final momentum."""
     T, Tq = k.shape[0], q.shape[0]
     starts = list(range(0, T, chunk))
     if len(starts) > 1 and Tq != T:
         raise ValueError("Tq != T needs a single chunk (R10)")
+    if update_mask is not None and len(update_mask) != len(starts):
+        raise ValueError("update_mask needs one flag per chunk")
     qh = qk_prologue(q)
     kh = qk_prologue(k)
     W = (np.array(W1, dtype=np.float64), np.array(W2, dtype=np.float64),
          np.array(W3, dtype=np.float64))
-    M = tuple(np.zeros_like(w) for w in W)
+    if M0 is None:
+        M = tuple(np.zeros_like(w) for w in W)
+    else:
+        M = tuple(np.array(m, dtype=np.float64) for m in M0)
     out = np.zeros_like(qh)
-    for c0 in starts:
+    for ci, c0 in enumerate(starts):
         c1 = min(c0 + chunk, T)                       # R9: ragged last chunk
         rows = slice(0, Tq) if len(starts) == 1 else slice(c0, c1)
+        updates = update_mask is None or bool(update_mask[ci])
         if order == APPLY_THEN_UPDATE:
             out[rows] = fast_net(*W, qh[rows])
-        G = chunk_gradient(*W, kh[c0:c1], v[c0:c1], lr[c0:c1])
-        U, M = rule_step(rule, G, M, None if beta is None else beta[c0:c1])
-        W = tuple(renorm_rows(w - u, w) for w, u in zip(W, U))
+        if updates:
+            G = chunk_gradient(*W, kh[c0:c1], v[c0:c1], lr[c0:c1])
+            U, M = rule_step(rule, G, M, None if beta is None else beta[c0:c1])
+            W = tuple(renorm_rows(w - u, w) for w, u in zip(W, U))
         if order == UPDATE_THEN_APPLY:
             out[rows] = fast_net(*W, qh[rows])
+    if out_scale is not None:
+        out = np.asarray(out_scale, dtype=np.float64)[:, None] * out
+    return out, W, M
+
+
+def ttt_head(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule):
+    """ttt_head_state without options; returns out [Tq, d] and the final
+    (W1, W2, W3)."""
+    out, W, _ = ttt_head_state(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule)
     return out, W
 
 
@@ -164,7 +190,8 @@ def _f64(t):
     return np.asarray(t, dtype=np.float64)
 
 
-def ttt_layer(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, heads=None):
+def ttt_layer_ex(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, heads=None,
+                 update_mask=None, out_scale=None, m_in=None):
     """The whole layer on the ABI layout: q [B,H,Tq,d], k, v [B,H,T,d],
     lr [B,H,T,3], beta [B,H,T] or None, w1, w3 [Hw,dh,d], w2 [Hw,d,dh] with
     Hw = H (initial state shared across the batch) or B*H.  Inputs may be
@@ -172,7 +199,11 @@ def ttt_layer(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, heads=None):
 
     heads: optional list of (b, h) pairs to compute (the heads are
     independent); the others are left as NaN.
-    Returns out [B,H,Tq,d], w1o [B*H,dh,d], w2o [B*H,d,dh], w3o [B*H,dh,d]."""
+    update_mask: one flag per chunk, shared by every (b, h) (R11).
+    out_scale: [B,H,Tq] per-query output factors (R12).
+    m_in: (m1 [B*H,dh,d], m2 [B*H,d,dh], m3 [B*H,dh,d]) initial momentum (R13).
+    Returns out [B,H,Tq,d], w1o [B*H,dh,d], w2o [B*H,d,dh], w3o [B*H,dh,d],
+    m1o, m2o, m3o (the final momentum, zeros unless the rule is momentum)."""
     B, H, Tq, d = q.shape
     dh = w1.shape[1]
     if w1.shape[0] not in (H, B * H):
@@ -181,15 +212,29 @@ def ttt_layer(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, heads=None):
     w1o = np.full((B * H, dh, d), np.nan)
     w2o = np.full((B * H, d, dh), np.nan)
     w3o = np.full((B * H, dh, d), np.nan)
+    m1o, m2o, m3o = np.full_like(w1o, np.nan), np.full_like(w2o, np.nan), np.full_like(w3o, np.nan)
     todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    mask = None if update_mask is None else [int(x) for x in update_mask]
     for b, h in todo:
         wi = b * H + h if w1.shape[0] == B * H else h
-        o, W = ttt_head(_f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h]), _f64(lr[b, h]),
-                        None if beta is None else _f64(beta[b, h]),
-                        _f64(w1[wi]), _f64(w2[wi]), _f64(w3[wi]), chunk, order, rule)
+        bh = b * H + h
+        M0 = None if m_in is None else tuple(_f64(m[bh]) for m in m_in)
+        o, W, M = ttt_head_state(
+            _f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h]), _f64(lr[b, h]),
+            None if beta is None else _f64(beta[b, h]),
+            _f64(w1[wi]), _f64(w2[wi]), _f64(w3[wi]), chunk, order, rule,
+            update_mask=mask, out_scale=None if out_scale is None else _f64(out_scale[b, h]),
+            M0=M0)
         out[b, h] = o
-        w1o[b * H + h], w2o[b * H + h], w3o[b * H + h] = W
-    return out, w1o, w2o, w3o
+        w1o[bh], w2o[bh], w3o[bh] = W
+        m1o[bh], m2o[bh], m3o[bh] = M
+    return out, w1o, w2o, w3o, m1o, m2o, m3o
+
+
+def ttt_layer(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, heads=None):
+    """ttt_layer_ex without options.  Returns out [B,H,Tq,d], w1o [B*H,dh,d],
+    w2o [B*H,d,dh], w3o [B*H,dh,d]."""
+    return ttt_layer_ex(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, heads=heads)[:4]
 
 
 def blas_threads() -> int:

@@ -389,3 +389,158 @@ def test_ragged_last_chunk_is_processed_as_a_short_chunk(order):
     for x, y in zip(full[1:], b[1:]):
         np.testing.assert_allclose(x, y, rtol=1e-13, atol=1e-15)
     assert not np.allclose(full[1], a[1])
+
+
+# ---------------------------------------------------------------- options
+def _state_after(k, v, lr, beta, w1, w2, w3, ch, rule, n_tokens):
+    """(W1, W2, W3) of every (b, h) after the first n_tokens keys, from a run
+    without options (the initial weights when n_tokens is 0)."""
+    if n_tokens == 0:
+        return w1, w2, w3
+    t = slice(0, n_tokens)
+    q = k[:, :, t]                      # the queries do not touch the state
+    _, a1, a2, a3 = _layer(q, k[:, :, t], v[:, :, t], lr[:, :, t],
+                           None if beta is None else beta[:, :, t], w1, w2, w3, ch,
+                           APPLY_THEN_UPDATE, rule)
+    return a1, a2, a3
+
+
+@pytest.mark.parametrize("rule", [RULE_GD, RULE_MOMENTUM, RULE_MUON])
+@pytest.mark.parametrize("order", [APPLY_THEN_UPDATE, UPDATE_THEN_APPLY])
+def test_masked_chunks_act_as_if_their_keys_were_absent(rule, order):
+    """A chunk whose update flag is 0 is read but writes nothing ("LaCT：以大
+    分块更新人工智能的临时记忆" 「更新顺序必须遵守信息可见范围」: video chunks
+    with noise read the memory, only clean chunks update it; "LaCT架构核心思想
+    解析" §3.2).  So the final weights and momentum equal a run over the
+    unmasked chunks alone, and each chunk's output is f of the state that the
+    unmasked chunks before it (order 0) or up to and including it (order 1)
+    leave, checked through library modules."""
+    ch, mask = 5, [1, 0, 0, 1, 0, 1]
+    T = ch * len(mask)
+    q, k, v, lr, beta, w1, w2, w3 = _problem(T=T, H=2, beta=True, lr_scale=5.0)
+    res = oracle.ttt_layer_ex(q, k, v, lr, beta, w1, w2, w3, ch, order, rule, update_mask=mask)
+    keep = np.concatenate([np.arange(c * ch, (c + 1) * ch) for c, m in enumerate(mask) if m])
+    sub = lambda x: x[:, :, keep]
+    red = oracle.ttt_layer_ex(sub(q), sub(k), sub(v), sub(lr), sub(beta), w1, w2, w3, ch, order,
+                              rule)
+    for x, y in zip(res[1:], red[1:]):
+        np.testing.assert_allclose(x, y, rtol=1e-13, atol=1e-15)
+    for c in range(len(mask)):
+        n_upd = sum(mask[:c]) + (mask[c] if order == UPDATE_THEN_APPLY else 0)
+        W = _state_after(sub(k), sub(v), sub(lr), sub(beta), w1, w2, w3, ch, rule, n_upd * ch)
+        rows = slice(c * ch, (c + 1) * ch)
+        for h in range(2):
+            want = _torch_swiglu(W[0][h], W[1][h], W[2][h], oracle.qk_prologue(q[0, h, rows]))
+            np.testing.assert_allclose(res[0][0, h, rows], want, rtol=1e-11, atol=1e-13)
+    assert not np.allclose(res[1], w1)
+
+
+@pytest.mark.parametrize("order", [APPLY_THEN_UPDATE, UPDATE_THEN_APPLY])
+def test_all_chunks_masked_reads_only_the_initial_state(order):
+    """With every flag 0 nothing updates: out = f_{W0}(q^) for every query
+    (library modules), the weights and the given momentum come back as they
+    went in."""
+    q, k, v, lr, beta, w1, w2, w3 = _problem(B=2, H=2, T=12, beta=True)
+    m_in = tuple(_rand(4, *w.shape[1:]) for w in (w1, w2, w3))
+    out, o1, o2, o3, m1, m2, m3 = oracle.ttt_layer_ex(
+        q, k, v, lr, beta, w1, w2, w3, 4, order, RULE_MOMENTUM, update_mask=[0, 0, 0], m_in=m_in)
+    for b in range(2):
+        for h in range(2):
+            np.testing.assert_allclose(out[b, h], _torch_swiglu(w1[h], w2[h], w3[h],
+                                                                oracle.qk_prologue(q[b, h])),
+                                       rtol=1e-12, atol=1e-14)
+            np.testing.assert_array_equal(o1[b * 2 + h], w1[h])
+            np.testing.assert_array_equal(o2[b * 2 + h], w2[h])
+            np.testing.assert_array_equal(o3[b * 2 + h], w3[h])
+    for got, want in zip((m1, m2, m3), m_in):
+        np.testing.assert_array_equal(got, want)
+
+
+def test_all_ones_mask_is_the_plain_layer():
+    q, k, v, lr, beta, w1, w2, w3 = _problem(T=18, beta=True)
+    a = _layer(q, k, v, lr, beta, w1, w2, w3, 6, APPLY_THEN_UPDATE, RULE_MOMENTUM)
+    b = oracle.ttt_layer_ex(q, k, v, lr, beta, w1, w2, w3, 6, APPLY_THEN_UPDATE, RULE_MOMENTUM,
+                            update_mask=[1, 1, 1])
+    for x, y in zip(a, b[:4]):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_momentum_resume_in_two_calls():
+    """Momentum carried across calls ("LaCT架构核心思想解析" §1.2 momentum,
+    resumed): one call over T equals two calls over the halves with the first
+    call's weights AND momentum passed in.  Without the momentum the second
+    half differs.  A masked chunk on each side of the split too."""
+    q, k, v, lr, beta, w1, w2, w3 = _problem(B=2, H=2, T=24, beta=True, lr_scale=5.0)
+    mask = [1, 0, 1, 1, 0, 1]
+    full = oracle.ttt_layer_ex(q, k, v, lr, beta, w1, w2, w3, 4, APPLY_THEN_UPDATE,
+                               RULE_MOMENTUM, update_mask=mask)
+    h1, h2 = slice(0, 12), slice(12, 24)
+    cut = lambda x, s: x[:, :, s]
+    a = oracle.ttt_layer_ex(cut(q, h1), cut(k, h1), cut(v, h1), cut(lr, h1), cut(beta, h1),
+                            w1, w2, w3, 4, APPLY_THEN_UPDATE, RULE_MOMENTUM, update_mask=mask[:3])
+    b = oracle.ttt_layer_ex(cut(q, h2), cut(k, h2), cut(v, h2), cut(lr, h2), cut(beta, h2),
+                            a[1], a[2], a[3], 4, APPLY_THEN_UPDATE, RULE_MOMENTUM,
+                            update_mask=mask[3:], m_in=a[4:])
+    np.testing.assert_allclose(full[0][:, :, h1], a[0], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(full[0][:, :, h2], b[0], rtol=1e-13, atol=1e-15)
+    for x, y in zip(full[1:], b[1:]):
+        np.testing.assert_allclose(x, y, rtol=1e-13, atol=1e-15)
+    c = oracle.ttt_layer_ex(cut(q, h2), cut(k, h2), cut(v, h2), cut(lr, h2), cut(beta, h2),
+                            a[1], a[2], a[3], 4, APPLY_THEN_UPDATE, RULE_MOMENTUM,
+                            update_mask=mask[3:])
+    assert not np.allclose(c[1], b[1])
+
+
+def test_given_momentum_is_the_first_decayed_term():
+    """One chunk from M_0: U = mean(beta) M_0 + G ("LaCT架构核心思想解析"
+    §1.2), built from the oracle's gradient; beta = 0 makes M_0 irrelevant."""
+    d, dh, n = 6, 8, 5
+    W = _weights(d, dh)
+    M0 = tuple(_rand(*w.shape) * 0.05 for w in W)
+    k, v, q = _rand(n, d), _rand(n, d), _rand(n, d)
+    lr = np.abs(_rand(n, 3)) * 0.3
+    beta = RNG.uniform(0.2, 0.9, n)
+    G = oracle.chunk_gradient(*W, oracle.qk_prologue(k), v, lr)
+    M1 = tuple(beta.mean() * m + g for m, g in zip(M0, G))
+    want = tuple(oracle.renorm_rows(w - m, w) for w, m in zip(W, M1))
+    one = lambda x: x[None, None]
+    res = oracle.ttt_layer_ex(one(q), one(k), one(v), one(lr), one(beta), W[0][None], W[1][None],
+                              W[2][None], n, APPLY_THEN_UPDATE, RULE_MOMENTUM,
+                              m_in=tuple(m[None] for m in M0))
+    for got, w in zip(res[1:4], want):
+        np.testing.assert_allclose(got[0], w, rtol=1e-12)
+    for got, m in zip(res[4:], M1):
+        np.testing.assert_allclose(got[0], m, rtol=1e-12)
+    zero = oracle.ttt_layer_ex(one(q), one(k), one(v), one(lr), one(0 * beta), W[0][None],
+                               W[1][None], W[2][None], n, APPLY_THEN_UPDATE, RULE_MOMENTUM,
+                               m_in=tuple(m[None] for m in M0))
+    plain = _layer(one(q), one(k), one(v), one(lr), one(0 * beta), W[0][None], W[1][None],
+                   W[2][None], n, APPLY_THEN_UPDATE, RULE_GD)
+    for x, y in zip(zero[:4], plain):
+        np.testing.assert_allclose(x, y, rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("order", [APPLY_THEN_UPDATE, UPDATE_THEN_APPLY])
+def test_output_scale_multiplies_each_query_row(order):
+    """The per-head output scale ("LaCT架构核心思想解析" §2.1) multiplies the
+    output row of its own (batch, head, query) and nothing else: a scale of 1
+    changes no bit, other scales (negative and zero included) scale exactly
+    that row, and the state is untouched."""
+    B, H, T = 2, 3, 12
+    q, k, v, lr, beta, w1, w2, w3 = _problem(B=B, H=H, T=T)
+    base = _layer(q, k, v, lr, beta, w1, w2, w3, 4, order, RULE_GD)
+    ones = oracle.ttt_layer_ex(q, k, v, lr, beta, w1, w2, w3, 4, order, RULE_GD,
+                               out_scale=np.ones((B, H, T)))
+    for x, y in zip(base, ones[:4]):
+        np.testing.assert_array_equal(x, y)
+    s = _rand(B, H, T)
+    s[0, 1, 3] = 0.0
+    s[1, 2, 5] = -2.0
+    res = oracle.ttt_layer_ex(q, k, v, lr, beta, w1, w2, w3, 4, order, RULE_GD, out_scale=s)
+    for b in range(B):
+        for h in range(H):
+            for t in range(T):
+                np.testing.assert_allclose(res[0][b, h, t], s[b, h, t] * base[0][b, h, t],
+                                           rtol=1e-15, atol=0)
+    for x, y in zip(base[1:], res[1:4]):
+        np.testing.assert_array_equal(x, y)
