@@ -26,6 +26,15 @@ class LactProblem(ctypes.Structure):
     ]
 
 
+class LactFwdOpts(ctypes.Structure):
+    """lact_fwd_opts: update_mask is a HOST byte array (one per chunk);
+    out_scale, m1, m2, m3 are device pointers (0 = off)."""
+    _fields_ = [
+        ("update_mask", ctypes.c_void_p), ("out_scale", ctypes.c_void_p),
+        ("m1", ctypes.c_void_p), ("m2", ctypes.c_void_p), ("m3", ctypes.c_void_p),
+    ]
+
+
 class LactError(RuntimeError):
     def __init__(self, code: int, what: str = ""):
         self.code = code
@@ -38,12 +47,15 @@ _vp = ctypes.c_void_p
 SIGNATURES = {
     "lact_ttt_workspace_bytes": (ctypes.c_size_t, [_P]),
     "lact_ttt_fwd": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]),
+    "lact_ttt_fwd_ex": (ctypes.c_int, [_P, ctypes.POINTER(LactFwdOpts)] + [_vp] * 12
+                        + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_fwd_noalloc": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp]),
     "lact_ttt_host_workspace_bytes": (ctypes.c_size_t, [_P]),
     "lact_ttt_fwd_host": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_status": (ctypes.c_int, [_vp]),
     "lact_device_check": (ctypes.c_int, []),
     "lact_ttt_launch_count": (ctypes.c_int64, [_P]),
+    "lact_ttt_launch_count_ex": (ctypes.c_int64, [_P, ctypes.POINTER(LactFwdOpts)]),
     "lact_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, _vp]),
     "lact_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "lact_profile_enable": (ctypes.c_int, [ctypes.c_int]),

@@ -35,6 +35,7 @@ struct ApplyParams {
   int rows_valid;     // queries in this chunk
   __nv_bfloat16* out; // [BH, Tq, d]
   int64_t Tq;
+  const float* scale; // [BH, Tq] per-query output factor, or null
 };
 
 constexpr int kApplyThreads = 224;   // 7 warps
@@ -246,7 +247,9 @@ __global__ void __launch_bounds__(kApplyThreads, 1) k_apply(const __grid_constan
       tc_fence_after();
       const int grow = rt * kBM + r;
       const bool valid = grow < p.rows_valid;
-      __nv_bfloat16* dst = p.out + (static_cast<int64_t>(bh) * p.Tq + p.q_row0 + grow) * D;
+      const int64_t orow = static_cast<int64_t>(bh) * p.Tq + p.q_row0 + grow;
+      __nv_bfloat16* dst = p.out + orow * D;
+      const float s = (p.scale && valid) ? __ldg(p.scale + orow) : 1.0f;
 #pragma unroll 1
       for (int j = 0; j < D; j += 16) {
         float v[16];
@@ -254,6 +257,10 @@ __global__ void __launch_bounds__(kApplyThreads, 1) k_apply(const __grid_constan
         tmem_ld16(tq + C::kColO + j, v);
         tmem_ld_wait();
         if (valid) {
+          if (p.scale) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= s;
+          }
           st_global_v4(dst + j, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                        pack_bf16x2(v[6], v[7]));
           st_global_v4(dst + j + 8, pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),

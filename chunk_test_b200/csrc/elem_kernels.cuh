@@ -143,7 +143,9 @@ __device__ __forceinline__ void store_shadow(__nv_bfloat16* hi, __nv_bfloat16* l
 // ---------------------------------------------------------------------------
 // State set-up: Wm[j][bh] = the caller's initial weights (state h of the H
 // shared ones, or state bh), plus the bf16 shadow (and its split lo part);
-// momentum zeroed.  Grid-stride over 3 * BH * dh * d elements.
+// momentum = the caller's m1/m2/m3 ([BH] states each) or zero, held negated
+// like the rule's M' = -M (an exact sign flip).  Grid-stride over
+// 3 * BH * dh * d elements.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1,
                                                     const float* __restrict__ w2,
@@ -152,11 +154,15 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
                                                     float* __restrict__ Wm,
                                                     __nv_bfloat16* __restrict__ Ws,
                                                     __nv_bfloat16* __restrict__ Ws_lo,
-                                                    float* __restrict__ Mm) {
+                                                    float* __restrict__ Mm,
+                                                    const float* __restrict__ m1,
+                                                    const float* __restrict__ m2,
+                                                    const float* __restrict__ m3) {
   griddep_launch();
   griddep_wait();
   const int64_t plane = static_cast<int64_t>(dh) * d;
   const int64_t total = 3 * BH * plane;
+  const int64_t per = BH * plane;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   if (plane % 4 == 0) {  // 16-byte steps
     for (int64_t o = 4 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); o < total;
@@ -173,7 +179,15 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
         store_shadow(Ws, Ws_lo, o + 2, x.z);
         store_shadow(Ws, Ws_lo, o + 3, x.w);
       }
-      if (Mm) *reinterpret_cast<float4*>(Mm + o) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (Mm) {
+        const float* m = j == 0 ? m1 : (j == 1 ? m2 : m3);
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (m) {
+          x = *reinterpret_cast<const float4*>(m + (o - j * per));
+          x = make_float4(-x.x, -x.y, -x.z, -x.w);
+        }
+        *reinterpret_cast<float4*>(Mm + o) = x;
+      }
     }
     return;
   }
@@ -185,26 +199,40 @@ __global__ void __launch_bounds__(256) k_init_state(const float* __restrict__ w1
     const float x = src[static_cast<int64_t>(src_h) * plane + e];
     Wm[o] = x;
     store_shadow(Ws, Ws_lo, o, x);
-    if (Mm) Mm[o] = 0.f;
+    if (Mm) {
+      const float* m = j == 0 ? m1 : (j == 1 ? m2 : m3);
+      Mm[o] = m ? -m[o - j * per] : 0.f;
+    }
   }
 }
 
-// Write-back of the final state into w1_out, w2_out, w3_out.
+// Write-back of the final state into w1_out, w2_out, w3_out, and of the
+// final momentum M = -M' into m1o, m2o, m3o when they are given.
 __global__ void __launch_bounds__(256) k_finalize_state(const float* __restrict__ Wm, int BH, int d,
                                                         int dh, float* __restrict__ w1o,
                                                         float* __restrict__ w2o,
-                                                        float* __restrict__ w3o) {
+                                                        float* __restrict__ w3o,
+                                                        const float* __restrict__ Mm,
+                                                        float* __restrict__ m1o,
+                                                        float* __restrict__ m2o,
+                                                        float* __restrict__ m3o) {
   griddep_launch();
   griddep_wait();
   const int64_t plane = static_cast<int64_t>(dh) * d;
   const int64_t per = BH * plane;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const bool mom = Mm && m1o;
   if (per % 4 == 0) {
     for (int64_t o = 4 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); o < 3 * per;
          o += 4 * stride) {
       const int j = static_cast<int>(o / per);
       float* dst = j == 0 ? w1o : (j == 1 ? w2o : w3o);
       *reinterpret_cast<float4*>(dst + (o - j * per)) = *reinterpret_cast<const float4*>(Wm + o);
+      if (mom) {
+        float* mdst = j == 0 ? m1o : (j == 1 ? m2o : m3o);
+        const float4 x = *reinterpret_cast<const float4*>(Mm + o);
+        *reinterpret_cast<float4*>(mdst + (o - j * per)) = make_float4(-x.x, -x.y, -x.z, -x.w);
+      }
     }
     return;
   }
@@ -212,6 +240,7 @@ __global__ void __launch_bounds__(256) k_finalize_state(const float* __restrict_
     const int j = static_cast<int>(o / per);
     float* dst = j == 0 ? w1o : (j == 1 ? w2o : w3o);
     dst[o - j * per] = Wm[o];
+    if (mom) (j == 0 ? m1o : (j == 1 ? m2o : m3o))[o - j * per] = -Mm[o];
   }
 }
 

@@ -447,6 +447,10 @@ struct Inputs {
   const float *lr, *beta, *w1, *w2, *w3;
   void* out;
   float *w1o, *w2o, *w3o;
+  // options (null = off)
+  const uint8_t* mask;     // host, one byte per chunk: 0 = the chunk does not update
+  const float* scale;      // [BH, Tq] output factors
+  float *m1, *m2, *m3;     // momentum in/out
 };
 
 template <typename T, int VEC, int S, int MAXV>
@@ -511,10 +515,11 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
   const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane;
   const unsigned state_blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(planes, 1024), 148 * 16));
 
-  // Fast-weight masters (+ bf16 shadows), momentum = 0.
+  // Fast-weight masters (+ bf16 shadows), momentum = the caller's or 0.
   L(K_INIT, [&] {
     (void)launch_pdl(k_init_state, state_blocks, 256, 0, st, in.w1, in.w2, in.w3, static_cast<int>(D.H),
-                                                   D.w_shared, BH, d, dh, b.Wm, b.Ws, b.Ws_lo, b.Mm);
+                     D.w_shared, BH, d, dh, b.Wm, b.Ws, b.Ws_lo, b.Mm, static_cast<const float*>(in.m1),
+                     static_cast<const float*>(in.m2), static_cast<const float*>(in.m3));
     return cudaGetLastError();
   });
   // q^, k^ = silu + L2 norm rows.
@@ -529,15 +534,23 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
   }
 
   bool join_before_rule = false, side_used = false;
+  // Updates done so far.  With two bf16 shadow sets the state after `ver`
+  // updates is in set ver % 2; a chunk that does not update leaves it there.
+  int64_t ver = 0;
+  // Per shadow set: an apply that reads it was launched on the side stream
+  // and the set's join event was recorded after it.
+  bool set_joined[2] = {false, false};
+  int last_join = 0;
   for (int64_t c = 0; c < D.nch; ++c) {
     const int64_t c0 = c * D.chunk;
     const int nc = static_cast<int>((c0 + D.chunk < D.T ? c0 + D.chunk : D.T) - c0);
     const int64_t qr0 = D.nch == 1 ? 0 : c0;
     const int nq = static_cast<int>(D.nch == 1 ? D.Tq : nc);
-    // bf16 shadows of W_c (read by this chunk's kernels) and of W_{c+1}
-    // (written by its rule): with two sets, chunk c's apply may still run
-    // while chunk c's rule writes the other set.
-    const int64_t cur = D.dbuf ? (c & 1) : 0, nxt = D.dbuf ? 1 - cur : 0;
+    const bool upd = !in.mask || in.mask[c] != 0;
+    // bf16 shadows of the current state (read by this chunk's kernels) and
+    // of the next one (written by its rule): with two sets, chunk c's apply
+    // may still run while chunk c's rule writes the other set.
+    const int64_t cur = D.dbuf ? (ver & 1) : 0, nxt = D.dbuf ? 1 - cur : 0;
     __nv_bfloat16* const Wsc = b.Ws ? b.Ws + cur * planes : nullptr;
     __nv_bfloat16* const Wsc_lo = b.Ws_lo ? b.Ws_lo + cur * planes : nullptr;
     __nv_bfloat16* const Wsn = b.Ws ? b.Ws + nxt * planes : nullptr;
@@ -553,7 +566,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
             return cudaErrorInvalidValue;
           a.bh_count = BH; a.dh = dh; a.n_row_tiles = static_cast<int>(cdiv(nq, 128));
           a.q_row0 = static_cast<int>(qr0); a.rows_valid = nq;
-          a.out = static_cast<__nv_bfloat16*>(in.out); a.Tq = D.Tq;
+          a.out = static_cast<__nv_bfloat16*>(in.out); a.Tq = D.Tq; a.scale = in.scale;
           const int64_t tiles = int64_t(a.n_row_tiles) * BH;
           switch (d) {
             case 64: return launch_apply<64>(tiles, a, st);
@@ -587,6 +600,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           g.zb_mod = BH; g.zb_add = 0; g.m_valid = nq;
           g.outb = static_cast<__nv_bfloat16*>(in.out) + qr0 * d;
           g.item_stride = D.Tq * D.d; g.ld = d;
+          g.row_scale = in.scale ? in.scale + qr0 : nullptr; g.rs_item = D.Tq;
           return launch_gemm<false, false>(D.bn, dim3(d / D.bn, cdiv(nq, 128), BH), g, st);
         });
       } else {
@@ -614,6 +628,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           s.B = b.Wm + D.BH * plane; s.b_item = plane; s.b_n = dh; s.b_k = 1;   // W2[i][r]
           s.M = nq; s.N = d; s.K = dh;
           s.outf = static_cast<float*>(in.out) + qr0 * d; s.item_stride = D.Tq * D.d; s.ld = d;
+          s.row_scale = in.scale ? in.scale + qr0 : nullptr; s.rs_item = D.Tq;
           return simt(s, BH, st);
         });
       }
@@ -816,10 +831,10 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
         dir_splits = 1;
       }
       if (join_before_rule) {
-        // the rule rewrites the shadow set that the apply launched one chunk
-        // earlier (two sets) or in this chunk (one set) reads
-        const int64_t jc = D.dbuf ? c - 1 : c;
-        if (jc >= 0 && L.err == LACT_OK && cudaStreamWaitEvent(main_st, side->join[jc & 1], 0) != cudaSuccess)
+        // the rule rewrites the shadow set that the applies of the previous
+        // state (two sets) or of this chunk (one set) read
+        if (set_joined[nxt] && L.err == LACT_OK &&
+            cudaStreamWaitEvent(main_st, side->join[nxt], 0) != cudaSuccess)
           L.err = LACT_ECUDA;
         join_before_rule = false;
       }
@@ -854,24 +869,30 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
       st = side->side;
       L.st = st;
       apply();
-      if (L.err == LACT_OK && cudaEventRecord(side->join[c & 1], side->side) != cudaSuccess) L.err = LACT_ECUDA;
+      if (L.err == LACT_OK && cudaEventRecord(side->join[cur], side->side) != cudaSuccess) L.err = LACT_ECUDA;
+      set_joined[cur] = true;
+      last_join = static_cast<int>(cur);
       st = main_st;
       L.st = st;
-      join_before_rule = true;
-      update();
+      if (upd) {
+        join_before_rule = true;
+        update();
+      }
     } else if (D.order == LACT_APPLY_THEN_UPDATE) {
       apply();
-      update();
+      if (upd) update();
     } else {
-      update();
+      if (upd) update();
       apply();
     }
+    if (upd) ++ver;
   }
 
-  if (side_used && L.err == LACT_OK && cudaStreamWaitEvent(main_st, side->join[(D.nch - 1) & 1], 0) != cudaSuccess)
+  if (side_used && L.err == LACT_OK && cudaStreamWaitEvent(main_st, side->join[last_join], 0) != cudaSuccess)
     L.err = LACT_ECUDA;   // the last chunks' applies are done before the call's work ends
   L(K_FINALIZE, [&] {
-    (void)launch_pdl(k_finalize_state, state_blocks, 256, 0, st, b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o);
+    (void)launch_pdl(k_finalize_state, state_blocks, 256, 0, st, b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o,
+                     static_cast<const float*>(b.Mm), in.m1, in.m2, in.m3);
     return cudaGetLastError();
   });
 }
@@ -906,6 +927,49 @@ static int check_pointers(const Dims& D, const Inputs& in) {
   for (int i = 0; i < 3; ++i)
     if (overlaps(in.out, on, outs[i], won)) return LACT_EINVAL;
   return LACT_OK;
+}
+
+// Options of lact_ttt_fwd_ex: momentum buffers all or none, momentum rule
+// only, aligned, and no overlap of an option buffer with a buffer the call
+// writes (or, for the in-place momentum, with the initial weights).
+static int check_options(const Dims& D, const Inputs& in) {
+  const size_t won = static_cast<size_t>(D.BH * D.d * D.dh) * 4;
+  const size_t wn = static_cast<size_t>((D.w_shared ? D.H : D.BH) * D.d * D.dh) * 4;
+  const size_t on = static_cast<size_t>(D.BH * D.Tq * D.d) * (D.dtype == LACT_BF16 ? 2 : 4);
+  const void* wouts[4] = {in.out, in.w1o, in.w2o, in.w3o};
+  const size_t wout_n[4] = {on, won, won, won};
+  const bool any_m = in.m1 || in.m2 || in.m3;
+  const float* ms[3] = {in.m1, in.m2, in.m3};
+  if (any_m) {
+    if (!in.m1 || !in.m2 || !in.m3 || D.rule != LACT_RULE_MOMENTUM) return LACT_EINVAL;
+    const float* wins[3] = {in.w1, in.w2, in.w3};
+    for (int i = 0; i < 3; ++i) {
+      if (!aligned16(ms[i])) return LACT_EINVAL;
+      for (int j = i + 1; j < 3; ++j)
+        if (overlaps(ms[i], won, ms[j], won)) return LACT_EINVAL;
+      for (int j = 0; j < 4; ++j)
+        if (overlaps(ms[i], won, wouts[j], wout_n[j])) return LACT_EINVAL;
+      for (int j = 0; j < 3; ++j)
+        if (overlaps(ms[i], won, wins[j], wn)) return LACT_EINVAL;
+    }
+  }
+  if (in.scale) {
+    if ((reinterpret_cast<uintptr_t>(in.scale) & 3u) != 0) return LACT_EINVAL;
+    const size_t sn = static_cast<size_t>(D.BH * D.Tq) * 4;
+    for (int j = 0; j < 4; ++j)
+      if (overlaps(in.scale, sn, wouts[j], wout_n[j])) return LACT_EINVAL;
+    for (int i = 0; any_m && i < 3; ++i)
+      if (overlaps(in.scale, sn, ms[i], won)) return LACT_EINVAL;
+  }
+  return LACT_OK;
+}
+
+static void set_options(Inputs& in, const lact_fwd_opts* o) {
+  in.mask = o ? o->update_mask : nullptr;
+  in.scale = o ? o->out_scale : nullptr;
+  in.m1 = o ? o->m1 : nullptr;
+  in.m2 = o ? o->m2 : nullptr;
+  in.m3 = o ? o->m3 : nullptr;
 }
 
 static int input_bytes(const Dims& D, size_t sz[8]) {
@@ -967,7 +1031,7 @@ size_t lact_ttt_workspace_bytes(const lact_problem* p) {
   return workspace_bytes(D);
 }
 
-int64_t lact_ttt_launch_count(const lact_problem* p) {
+int64_t lact_ttt_launch_count_ex(const lact_problem* p, const lact_fwd_opts* opts) {
   Dims D;
   if (validate(p, D) != LACT_OK) return 0;
   Bump bp{0, 0};
@@ -975,20 +1039,30 @@ int64_t lact_ttt_launch_count(const lact_problem* p) {
   plan(D, bp, b);
   Inputs in;
   std::memset(&in, 0, sizeof(in));
+  in.mask = opts ? opts->update_mask : nullptr;   // the only option that changes the launches
   Launcher L{true, nullptr};
   run(D, b, in, nullptr, L, nullptr);
   return L.count;
 }
 
-static int ttt_fwd_impl(const lact_problem* p, const void* q, const void* k, const void* v,
-                        const float* lr, const float* beta, const float* w1, const float* w2,
-                        const float* w3, void* out, float* w1_out, float* w2_out, float* w3_out,
-                        void* workspace, size_t workspace_bytes_, void* stream, bool allow_side) {
+int64_t lact_ttt_launch_count(const lact_problem* p) { return lact_ttt_launch_count_ex(p, nullptr); }
+
+static int ttt_fwd_impl(const lact_problem* p, const lact_fwd_opts* opts, const void* q,
+                        const void* k, const void* v, const float* lr, const float* beta,
+                        const float* w1, const float* w2, const float* w3, void* out,
+                        float* w1_out, float* w2_out, float* w3_out, void* workspace,
+                        size_t workspace_bytes_, void* stream, bool allow_side) {
   Dims D;
   int rc = validate(p, D);
   if (rc != LACT_OK) return rc;
-  Inputs in{q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out};
+  Inputs in;
+  std::memset(&in, 0, sizeof(in));
+  in.q = q; in.k = k; in.v = v; in.lr = lr; in.beta = beta; in.w1 = w1; in.w2 = w2; in.w3 = w3;
+  in.out = out; in.w1o = w1_out; in.w2o = w2_out; in.w3o = w3_out;
+  set_options(in, opts);
   rc = check_pointers(D, in);
+  if (rc != LACT_OK) return rc;
+  rc = check_options(D, in);
   if (rc != LACT_OK) return rc;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LACT_EINVAL;
   if (workspace_bytes_ < workspace_bytes(D)) return LACT_ENOSPC;
@@ -1006,7 +1080,15 @@ int lact_ttt_fwd(const lact_problem* p, const void* q, const void* k, const void
                  const float* beta, const float* w1, const float* w2, const float* w3, void* out,
                  float* w1_out, float* w2_out, float* w3_out, void* workspace, size_t workspace_bytes_,
                  void* stream) {
-  return ttt_fwd_impl(p, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, workspace,
+  return ttt_fwd_impl(p, nullptr, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, workspace,
+                      workspace_bytes_, stream, true);
+}
+
+int lact_ttt_fwd_ex(const lact_problem* p, const lact_fwd_opts* opts, const void* q, const void* k,
+                    const void* v, const float* lr, const float* beta, const float* w1,
+                    const float* w2, const float* w3, void* out, float* w1_out, float* w2_out,
+                    float* w3_out, void* workspace, size_t workspace_bytes_, void* stream) {
+  return ttt_fwd_impl(p, opts, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, workspace,
                       workspace_bytes_, stream, true);
 }
 
@@ -1021,7 +1103,7 @@ int lact_ttt_fwd_noalloc(const lact_problem* p, const void* q, const void* k, co
   void* scratch = nullptr;
   rc = noalloc_scratch(&scratch);
   if (rc != LACT_OK) return rc;
-  return ttt_fwd_impl(p, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, scratch,
+  return ttt_fwd_impl(p, nullptr, q, k, v, lr, beta, w1, w2, w3, out, w1_out, w2_out, w3_out, scratch,
                       LACT_NOALLOC_SCRATCH_BYTES, stream, false);
 }
 

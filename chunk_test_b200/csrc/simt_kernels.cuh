@@ -28,6 +28,8 @@ struct SimtGemmParams {
   int64_t item_stride, ld;
   int tr_group, tr_mod;   // items with item / tr_mod == tr_group store C^T
   int64_t ld_t;           //   at n * ld_t + m
+  const float* row_scale; // or null: row m of item z scaled by row_scale[z * rs_item + m]
+  int64_t rs_item;
 };
 
 __global__ void __launch_bounds__(256) k_simt_gemm(const SimtGemmParams p) {
@@ -84,6 +86,7 @@ __global__ void __launch_bounds__(256) k_simt_gemm(const SimtGemmParams p) {
       const int64_t o = static_cast<int64_t>(item) * p.item_stride + static_cast<int64_t>(m) * p.ld + n;
       float v = p.alpha * acc[i][j];
       if (p.cin) v += p.beta * p.cin[o];
+      if (p.row_scale) v *= p.row_scale[static_cast<int64_t>(item) * p.rs_item + m];
       if (p.tr_group >= 0 && item / p.tr_mod == p.tr_group)
         p.outf[static_cast<int64_t>(item) * p.item_stride + static_cast<int64_t>(n) * p.ld_t + m] = v;
       else

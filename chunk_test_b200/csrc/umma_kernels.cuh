@@ -478,6 +478,8 @@ struct GemmParams {
   int64_t item_stride, ld;
   int tr_group, tr_mod;
   int64_t ld_t;
+  const float* row_scale;  // or null: row m of output item z scaled by row_scale[z * rs_item + m]
+  int64_t rs_item;
 };
 
 template <bool A_MN, bool B_MN, int BN, bool SPLIT = false>
@@ -569,6 +571,7 @@ struct GemmOp {
     const int64_t off = static_cast<int64_t>(t.out_item) * p.item_stride +
                         static_cast<int64_t>(grow) * p.ld + t.n0;
     const bool tr = p.tr_group >= 0 && (t.item / p.tr_mod) == p.tr_group;
+    const float rs = (p.row_scale && valid) ? __ldg(p.row_scale + t.out_item * p.rs_item + grow) : 1.0f;
 #pragma unroll 1
     for (int j = 0; j < BN; j += 16) {
       float v[16];
@@ -589,6 +592,10 @@ struct GemmOp {
         } else if (p.alpha != 1.0f) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] *= p.alpha;
+        }
+        if (p.row_scale) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] *= rs;
         }
         if (p.outf && tr) {
           float* o = p.outf + static_cast<int64_t>(t.out_item) * p.item_stride +

@@ -57,17 +57,56 @@ def workspace_bytes(q, k, w1, chunk, order, rule) -> int:
     return _abi.workspace_bytes(make_problem(q, k, w1, chunk, order, rule))
 
 
-def launch_count(q, k, w1, chunk, order, rule) -> int:
-    return _abi.launch_count(make_problem(q, k, w1, chunk, order, rule))
+def launch_count(q, k, w1, chunk, order, rule, update_mask=None) -> int:
+    p = make_problem(q, k, w1, chunk, order, rule)
+    if update_mask is None:
+        return _abi.launch_count(p)
+    opts, _keep = _options(p, update_mask, None, None, q)
+    return int(_abi.lib().lact_ttt_launch_count_ex(ctypes.byref(p), ctypes.byref(opts)))
+
+
+def _options(p, update_mask, out_scale, m_inout, q):
+    """lact_fwd_opts for the given options (None when none is given) and the
+    host mask buffer it points into (kept alive by the caller)."""
+    if update_mask is None and out_scale is None and m_inout is None:
+        return None, None
+    nch = -(-p.T // min(p.chunk, p.T))
+    mask_buf = None
+    if update_mask is not None:
+        flags = [1 if int(x) else 0 for x in update_mask]
+        if len(flags) != nch:
+            raise ValueError(f"update_mask needs {nch} flags (one per chunk), got {len(flags)}")
+        mask_buf = (ctypes.c_uint8 * nch)(*flags)
+    if out_scale is not None:
+        B, H, Tq, _ = q.shape
+        if (out_scale.device != q.device or out_scale.dtype != torch.float32
+                or not out_scale.is_contiguous() or tuple(out_scale.shape) != (B, H, Tq)):
+            raise ValueError("out_scale must be a contiguous float32 [B, H, Tq] tensor on q's device")
+    ms = (None, None, None)
+    if m_inout is not None:
+        ms = tuple(m_inout)
+        for m in ms:
+            if m.device != q.device or m.dtype != torch.float32 or not m.is_contiguous():
+                raise ValueError("m_inout must be contiguous float32 tensors on q's device")
+    o = _abi.LactFwdOpts(ctypes.addressof(mask_buf) if mask_buf is not None else None,
+                         None if out_scale is None else out_scale.data_ptr(),
+                         *(None if m is None else m.data_ptr() for m in ms))
+    return o, mask_buf
 
 
 def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_out=None,
-            workspace=None, stream=None):
+            workspace=None, stream=None, update_mask=None, out_scale=None, m_inout=None):
     """Runs the layer on the current CUDA device.  Returns (out, w1o, w2o, w3o).
     Optional `out`, `w_out` (a 3-tuple) and `workspace` (uint8 tensor) avoid
-    allocations; `stream` defaults to torch's current stream."""
+    allocations; `stream` defaults to torch's current stream.
+    Options (lact_fwd_opts in include/lact.h): `update_mask`, one flag per
+    chunk (0 = the chunk is applied but does not update the state);
+    `out_scale`, a [B, H, Tq] float32 tensor of per-query output factors;
+    `m_inout`, three float32 momentum tensors (shapes of the w_out) read as
+    the initial momentum and overwritten with the final one."""
     _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
     p = make_problem(q, k, w1, chunk, order, rule)
+    opts, _mask_keep = _options(p, update_mask, out_scale, m_inout, q)
     B, H, Tq, d = q.shape
     dh = w1.shape[1]
     if out is None:
@@ -83,12 +122,13 @@ def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_ou
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    rc = _abi.lib().lact_ttt_fwd(
-        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(beta), _ptr(w1), _ptr(w2),
-        _ptr(w3), _ptr(out), _ptr(w_out[0]), _ptr(w_out[1]), _ptr(w_out[2]), _ptr(workspace),
-        ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
+    rc = _abi.lib().lact_ttt_fwd_ex(
+        ctypes.byref(p), None if opts is None else ctypes.byref(opts), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(lr), _ptr(beta), _ptr(w1), _ptr(w2), _ptr(w3), _ptr(out), _ptr(w_out[0]),
+        _ptr(w_out[1]), _ptr(w_out[2]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+        ctypes.c_void_p(stream.cuda_stream))
     if rc != _abi.LACT_OK:
-        raise LactError(rc, "lact_ttt_fwd")
+        raise LactError(rc, "lact_ttt_fwd_ex")
     return out, w_out[0], w_out[1], w_out[2]
 
 

@@ -3,7 +3,7 @@
  *
  * The layer (Large-Chunk Test-Time Training).  Sources are cited by page
  * title and section:
- *   [P1] "LaCT架构核心思想解析" (gsyq.cn) §1.2, §2.1, §2.2
+ *   [P1] "LaCT架构核心思想解析" (gsyq.cn) §1.2, §2.1, §2.2, §3.2
  *   [P2] "大块测试时训练（LaCT）技术解析" (dpshk.com) §2.1, §2.2.1
  *   [P3] "LaCT：以大分块更新人工智能的临时记忆" (iplexlaw.co.kr), sections
  *        「局部注意力与非线性记忆相互补充」 and 「更新顺序必须遵守信息可见范围」
@@ -113,6 +113,51 @@ int lact_ttt_fwd(const lact_problem* p,
                  void* out, float* w1_out, float* w2_out, float* w3_out,
                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* Options of lact_ttt_fwd_ex.  Zero-initialise the struct and set what is
+ * used; a NULL field leaves its feature off, and a NULL options pointer is
+ * lact_ttt_fwd.
+ *
+ * update_mask  HOST array of ceil(T / chunk) bytes, one per chunk, shared by
+ *              every (b, h).  A chunk whose byte is 0 is applied in its
+ *              place in the order but skips the whole update (gradient,
+ *              rule, momentum, renorm), so the state passes through it
+ *              unchanged: in autoregressive video only the clean-frame
+ *              chunks write the memory and the noisy ones read it
+ *              ([P3] 「更新顺序必须遵守信息可见范围」; [P1 §3.2]).  Read
+ *              during the call only (the launches are planned from it).
+ * out_scale    DEVICE [B, H, Tq] float32, 4-byte aligned: the per-head,
+ *              per-token output factor of [P1 §2.1] (the values after the
+ *              page's silu of a linear map of x).  out[b,h,t,:] =
+ *              out_scale[b,h,t] * f_W(q_t), the product formed in fp32 before
+ *              the output's one rounding.  It may not overlap any output.
+ * m1, m2, m3   DEVICE momentum state, in place, rule LACT_RULE_MOMENTUM only,
+ *              all three or none: m1, m3 [B*H, dh, d], m2 [B*H, d, dh]
+ *              float32, 16-byte aligned, the layouts of w*_out.  Read as the
+ *              momentum before the first chunk (instead of zeros) and
+ *              overwritten with the momentum after the last chunk, so a
+ *              sequence split at chunk boundaries into several calls (w*_out
+ *              and m* handed from one call to the next) gives the results of
+ *              one call.  They may not overlap each other or any other
+ *              argument. */
+typedef struct lact_fwd_opts {
+  const uint8_t* update_mask;
+  const float* out_scale;
+  float* m1;
+  float* m2;
+  float* m3;
+} lact_fwd_opts;
+
+/* lact_ttt_fwd with options (see lact_fwd_opts); the same arguments,
+ * layouts, workspace and error behaviour otherwise.  LACT_EINVAL also for:
+ * momentum buffers with another rule, only some of m1/m2/m3, misaligned or
+ * overlapping option buffers. */
+int lact_ttt_fwd_ex(const lact_problem* p, const lact_fwd_opts* opts,
+                    const void* q, const void* k, const void* v,
+                    const float* lr, const float* beta,
+                    const float* w1, const float* w2, const float* w3,
+                    void* out, float* w1_out, float* w2_out, float* w3_out,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Size of the library's built-in device scratch buffer used by
  * lact_ttt_fwd_noalloc (32 MiB). */
 #define LACT_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
@@ -174,6 +219,10 @@ int lact_device_check(void);
 /* Kernel launches one lact_ttt_fwd call of problem *p enqueues (0 if *p is
  * invalid).  Pure host arithmetic. */
 int64_t lact_ttt_launch_count(const lact_problem* p);
+
+/* The same for lact_ttt_fwd_ex with options *opts (NULL = none): masked
+ * chunks launch no update kernels. */
+int64_t lact_ttt_launch_count_ex(const lact_problem* p, const lact_fwd_opts* opts);
 
 /* Failure-path self-test: launches one block whose thread waits on a shared
  * memory barrier that nothing ever completes, with a wait budget of

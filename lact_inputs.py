@@ -15,6 +15,15 @@ Recipe (one torch CPU generator, seeded, drawn in this order, all fp32):
 then q, k, v are cast to bf16 for the bf16 workloads.  The fast-weight
 initialisation is one per head, shared by every batch element (a learned
 initial state is a per-head parameter of the model).
+
+Option inputs (their own generator, so the layer inputs above do not move):
+  out_scale [B,H,Tq] = z * sigmoid(z), z ~ N(0,1): the per-head, per-token
+      output factor, drawn as the silu of a unit-variance linear map of x
+      (the multi-head fusion of "LaCT架构核心思想解析" §2.1);
+  update mask: the chunk pattern of an autoregressive video sequence whose
+      noisy chunks precede each clean one, [noisy x k, clean] repeated
+      ("LaCT架构核心思想解析" §3.2: one noisy copy per clean chunk, or two in
+      the teacher-forcing sequence).
 """
 from __future__ import annotations
 
@@ -102,3 +111,18 @@ def head_slice(inp: dict, b: int, h: int) -> dict:
     for name in ("w1", "w2", "w3"):
         out[name] = inp[name][h:h + 1]
     return out
+
+
+def make_out_scale(w: Workload, seed: int = 0) -> torch.Tensor:
+    """out_scale [B,H,Tq] fp32 = silu of N(0,1) draws."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(10_000 + seed)
+    z = torch.randn((w.B, w.H, w.Tq), generator=g, dtype=torch.float32)
+    return z * torch.sigmoid(z)
+
+
+def video_update_mask(n_chunks: int, noisy_per_clean: int = 1) -> list:
+    """One flag per chunk: 0 for the noisy chunks, 1 for the clean chunk
+    that follows them, in groups of noisy_per_clean + 1 chunks."""
+    period = noisy_per_clean + 1
+    return [1 if c % period == period - 1 else 0 for c in range(n_chunks)]

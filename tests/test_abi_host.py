@@ -104,3 +104,65 @@ def test_ragged_and_single_chunk_problems_are_accepted():
 def test_status_strings():
     for code in (0, -1, -2, -3, -4, -5):
         assert isinstance(ct.status_string(code), str) and ct.status_string(code)
+
+
+def _opts(mask=None, scale=0, m=(0, 0, 0)):
+    buf = None
+    if mask is not None:
+        buf = (ctypes.c_uint8 * len(mask))(*mask)
+    o = _abi.LactFwdOpts(ctypes.addressof(buf) if buf is not None else None, scale or None,
+                         *(x or None for x in m))
+    return o, buf
+
+
+@pytest.mark.parametrize("idx", [2, 3])
+def test_masked_chunks_launch_no_update_kernels(idx):
+    """lact_ttt_launch_count_ex: a chunk whose flag is 0 launches its apply
+    only; the fixed launches (state set-up, prologue, beta means, write-back)
+    stay."""
+    w = WORKLOADS[idx]
+    p = _prob(w)
+    full = _abi.launch_count(p)
+    o, keep = _opts(mask=[1] * w.n_chunks)
+    assert ct.lib().lact_ttt_launch_count_ex(ctypes.byref(p), ctypes.byref(o)) == full
+    mask = [1 if c % 3 == 0 else 0 for c in range(w.n_chunks)]
+    o, keep = _opts(mask=mask)
+    apply_per_chunk = 1 if w.d <= 256 else 2
+    per_chunk = (full - (3 + (1 if w.rule == 1 else 0))) // w.n_chunks
+    want = full - (per_chunk - apply_per_chunk) * mask.count(0)
+    assert ct.lib().lact_ttt_launch_count_ex(ctypes.byref(p), ctypes.byref(o)) == want
+    assert ct.lib().lact_ttt_launch_count_ex(ctypes.byref(p), None) == full
+
+
+def test_bad_options_are_rejected_without_a_gpu():
+    """Option checks of lact_ttt_fwd_ex run before anything is enqueued."""
+    fake = [ctypes.c_void_p((1 << 30) * (i + 1)) for i in range(12)]
+    ws = ctypes.c_void_p(1 << 40)
+    lib = ct.lib()
+    G = 1 << 30
+    m_ok = (13 * G, 14 * G, 15 * G)
+
+    def call(p, o):
+        return lib.lact_ttt_fwd_ex(ctypes.byref(p), ctypes.byref(o), *fake, ws,
+                                   ctypes.c_size_t(1 << 40), None)
+
+    mom = _prob(WORKLOADS[1], rule=1)
+    gd = _prob(WORKLOADS[1])
+    o, _ = _opts(m=m_ok)
+    assert call(gd, o) == ct.LACT_EINVAL                 # momentum buffers with GD
+    o, _ = _opts(m=(13 * G, 0, 15 * G))
+    assert call(mom, o) == ct.LACT_EINVAL                # only some of them
+    o, _ = _opts(m=(13 * G + 8, 14 * G, 15 * G))
+    assert call(mom, o) == ct.LACT_EINVAL                # not 16-byte aligned
+    o, _ = _opts(m=(13 * G, 13 * G, 15 * G))
+    assert call(mom, o) == ct.LACT_EINVAL                # m1 and m2 overlap
+    o, _ = _opts(m=(13 * G, 11 * G, 15 * G))
+    assert call(mom, o) == ct.LACT_EINVAL                # m2 on w2_out
+    o, _ = _opts(m=(6 * G, 14 * G, 15 * G))
+    assert call(mom, o) == ct.LACT_EINVAL                # m1 on the initial w1
+    o, _ = _opts(scale=16 * G + 2)
+    assert call(gd, o) == ct.LACT_EINVAL                 # scale not 4-byte aligned
+    o, _ = _opts(scale=9 * G)
+    assert call(gd, o) == ct.LACT_EINVAL                 # scale on out
+    o, _ = _opts(scale=14 * G, m=m_ok)
+    assert call(mom, o) == ct.LACT_EINVAL                # scale on m2
