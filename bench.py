@@ -79,7 +79,70 @@ def kernel_work(w: Workload):
 
 
 # ---------------------------------------------------------------- clocks
-class ClockSampler:
+_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+def _summary(sm, mx, reasons, source, power=None):
+    if not sm:
+        return None
+    out = {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": max(mx),
+           "reasons": sorted(reasons), "samples": len(sm), "source": source}
+    if power:
+        out["power_w_median"] = round(statistics.median(power), 1)
+    return out
+
+
+class NvmlClockSampler:
+    """Reads the SM clock, the power draw and the clock-event reasons of this
+    rank's GPU every `period_s` seconds on a background thread (NVML; reads
+    only, changes no setting).  Found by PCI bus id, so a restricted
+    CUDA_VISIBLE_DEVICES does not mislead it."""
+
+    def __init__(self, device: int, period_s: float = 0.002):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(device)
+        bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.mx = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.bits = {
+            "hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+            "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+            "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+            "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap,
+        }
+        self.sm, self.power, self.reasons = [], [], set()
+        self.period = period_s
+        self.stop_flag = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                self.power.append(nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.reasons.update(n for n, b in self.bits.items() if mask & b)
+            except Exception:
+                pass
+            self.stop_flag.wait(self.period)
+
+    def stop(self):
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        return _summary(self.sm, [self.mx], self.reasons, "nvml", self.power)
+
+
+class SmiClockSampler:
+    """nvidia-smi fallback (200 ms period) where NVML is not available."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -91,6 +154,7 @@ class ClockSampler:
                 ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)                     # its first row before the timed region
         except Exception:
             self.proc = None
 
@@ -105,20 +169,23 @@ class ClockSampler:
             out, _ = self.proc.communicate()
         rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
         sm, mx, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for r in rows:
             try:
                 sm.append(float(r[0]))
                 mx.append(float(r[1]))
             except (ValueError, IndexError):
                 continue
-            for name, val in zip(names, r[4:8]):
+            for name, val in zip(_REASONS, r[4:8]):
                 if val.strip().lower() == "active":
                     reasons.add(name)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return _summary(sm, mx, reasons, "nvidia-smi")
+
+
+def ClockSampler(device: int):
+    try:
+        return NvmlClockSampler(device)
+    except Exception:
+        return SmiClockSampler(device)
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -269,7 +336,6 @@ def main():
     # The K steps run exactly as a caller runs them: no events between the
     # kernels, whose launches overlap (programmatic dependent launch).
     clocks = ClockSampler(local)
-    time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
