@@ -351,9 +351,10 @@ def main():
         raise SystemExit("device status not OK after the timed region")
 
     # ---- per-kernel pass: the same K steps again with a CUDA event pair around
-    # every launch (the library's launch profiler).  Events between launches
-    # stop the overlap of consecutive launches, so this pass gives the
-    # per-kernel durations (kernel shares, roofline) but not the headline time.
+    # every launch (the library's launch profiler).  The profiler runs every
+    # launch alone on the caller's stream (no side-stream apply, no overlap of
+    # consecutive launches), so this pass gives each kernel's own duration
+    # (kernel shares, roofline) but not the headline time.
     ct.profile_enable(True)
     barrier()
     torch.cuda.synchronize(dev)
@@ -395,7 +396,7 @@ def main():
             roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                     "frac": achieved / hbm}
         roof.update({"kernel": name, "launches": n_launch, "avg_launch_us": 1e3 * ms_kind / n_launch,
-                     "concurrent": bool(w.order == 0 and w.dtype == BF16),
+                     "timed": "alone (per-kernel pass)",
                      "traffic": traffic_for(name, w), "peak_source": f"{pk_src} sustained bf16"
                      if bound == "tensor" else f"{pk_src} copy bandwidth"})
     kernels = {k: {"launches": v[0], "ms": round(v[1], 4),
@@ -443,10 +444,11 @@ def main():
         "roofline": roof,
         "kernels": kernels,
         "kernel_pass": {"ms_per_step": ms_profiled / args.steps,
-                        "method": "the same K steps again with a CUDA event pair around every launch "
-                                  "(kernel shares, roofline durations); per-launch events stop the "
-                                  "overlap of consecutive launches, so the headline time is the "
-                                  "first pass, without them"},
+                        "method": "the same K steps again, every launch alone on one stream "
+                                  "with a CUDA event pair around it (kernel shares, roofline "
+                                  "durations); this stops the side-stream apply and the overlap "
+                                  "of consecutive launches, so the headline time is the first "
+                                  "pass, without them"},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": job_value(world, tok_step, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -466,9 +468,22 @@ def main():
     return 0
 
 
+# The source files each timed kernel is built from: a traffic record holds
+# only while their hash is the one it was taken with.
+KERNEL_SOURCES = {
+    "apply_fused_umma": ("apply_kernel.cuh", "umma_kernels.cuh", "sm100.cuh"),
+    "key_grad_umma": ("key_grad_kernel.cuh", "apply_kernel.cuh", "umma_kernels.cuh", "sm100.cuh"),
+    "fwd_key_umma": ("umma_kernels.cuh", "sm100.cuh"),
+    "grad_umma": ("pair_kernels.cuh", "umma_kernels.cuh", "sm100.cuh"),
+    "rule_renorm": ("elem_kernels.cuh", "sm100.cuh"),
+    "qk_prologue": ("elem_kernels.cuh", "sm100.cuh"),
+}
+
+
 def traffic_for(kernel: str, w: Workload):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
-    was taken on this workload with the current kernel sources; else None."""
+    was taken on this workload with the current sources of that kernel; else
+    None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -476,16 +491,16 @@ def traffic_for(kernel: str, w: Workload):
     except Exception:
         return None
     r = rec.get(f"{kernel}@{w.name}")
-    if not r or r.get("source_hash") != source_hash():
+    if not r or kernel not in KERNEL_SOURCES or r.get("source_hash") != source_hash(kernel):
         return None
     return r.get("bytes_per_launch")
 
 
-def source_hash() -> str:
+def source_hash(kernel: str) -> str:
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "chunk_test_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

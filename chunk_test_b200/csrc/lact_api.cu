@@ -1071,7 +1071,14 @@ static int ttt_fwd_impl(const lact_problem* p, const lact_fwd_opts* opts, const 
   Bufs b;
   plan(D, bp, b);
   Launcher L{false, static_cast<cudaStream_t>(stream)};
-  const SideRes* side = allow_side ? side_resources() : nullptr;
+  bool profiling;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    profiling = g_prof_on;
+  }
+  // While the launch profiler is on, every launch goes to the caller's
+  // stream, one after another, so each event pair times one kernel alone.
+  const SideRes* side = (allow_side && !profiling) ? side_resources() : nullptr;
   run(D, b, in, static_cast<cudaStream_t>(stream), L, side);
   return L.err;
 }

@@ -234,7 +234,9 @@ int64_t lact_ttt_launch_count_ex(const lact_problem* p, const lact_fwd_opts* opt
 int lact_selftest_wait_timeout(int64_t budget_cycles, void* stream);
 
 /* Launch profiler.  While enabled, every kernel launch of lact_ttt_fwd is
- * bracketed by a pair of CUDA events recorded on the launching stream.
+ * bracketed by a pair of CUDA events recorded on the launching stream, and
+ * all launches of a call go to the caller's stream one after another (no
+ * side-stream overlap), so each pair times one kernel running alone.
  * lact_profile_read waits for those events, returns per kernel kind the
  * number of launches and the summed device milliseconds since the last read
  * (arrays of lact_kernel_kinds() entries), and forgets them.  Off by default;
