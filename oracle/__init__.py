@@ -44,17 +44,17 @@ design notes):
   R9  a final chunk shorter than `chunk` is processed as it is.
   R10 with a single chunk the queries may have their own length Tq (the target
       views of a posed image set); with several chunks Tq must equal T.
-  R11 the update mask has one flag per chunk, shared by every (batch, head)
+  R13 the update mask has one flag per chunk, shared by every (batch, head)
       (the clean/noisy pattern is a property of the sequence).  A chunk whose
       flag is 0 is still applied in its place in the order, but skips the
       whole update -- gradient, rule, momentum and renorm -- so the state
       passes through unchanged (video: only clean-frame chunks update the
       memory, noisy chunks read what the earlier chunks wrote; [P3]
       「更新顺序必须遵守信息可见范围」, [P1 §3.2]).
-  R12 the per-head output scale [P1 §2.1] is given as its values s (after
+  R14 the per-head output scale [P1 §2.1] is given as its values s (after
       the silu of the page's linear map), one per (batch, head, query
       token); the output row is s_t * f_W(q_t).
-  R13 resuming a sequence across calls: the momentum may start from a given
+  R15 resuming a sequence across calls: the momentum may start from a given
       M_0 (zeros otherwise) and the final M is returned, so two calls split
       at a chunk boundary equal one call.
 """

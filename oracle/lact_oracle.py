@@ -133,7 +133,7 @@ def ttt_head_state(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule,
       order 0 (apply-then-update, causal): o_c = f_{W_{c-1}}(q_c), then
               W_c = renorm(W_{c-1} - U(grad of chunk c on W_{c-1}));
       order 1 (update-then-apply, sets):  W_c first, then o_c = f_{W_c}(q_c).
-    Options (R11-R13):
+    Options (R13-R15):
       update_mask  one flag per chunk; a chunk whose flag is 0 is applied in
                    its place in the order but skips the whole update
                    (gradient, rule, momentum, renorm), so W_c = W_{c-1}
@@ -199,9 +199,9 @@ def ttt_layer_ex(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, heads=None,
 
     heads: optional list of (b, h) pairs to compute (the heads are
     independent); the others are left as NaN.
-    update_mask: one flag per chunk, shared by every (b, h) (R11).
-    out_scale: [B,H,Tq] per-query output factors (R12).
-    m_in: (m1 [B*H,dh,d], m2 [B*H,d,dh], m3 [B*H,dh,d]) initial momentum (R13).
+    update_mask: one flag per chunk, shared by every (b, h) (R13).
+    out_scale: [B,H,Tq] per-query output factors (R14).
+    m_in: (m1 [B*H,dh,d], m2 [B*H,d,dh], m3 [B*H,dh,d]) initial momentum (R15).
     Returns out [B,H,Tq,d], w1o [B*H,dh,d], w2o [B*H,d,dh], w3o [B*H,dh,d],
     m1o, m2o, m3o (the final momentum, zeros unless the rule is momentum)."""
     B, H, Tq, d = q.shape
