@@ -132,6 +132,90 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const T* __restrict__ q, T*
   }
 }
 
+// bf16 prologue.  Rows of d bf16 values, 8 per 16-byte vector: S lanes per
+// row (the power of two >= d / 8, at most 32), MAXV vectors per lane, ROWS
+// rows per lane group with every load issued before any arithmetic.  The bf16
+// pairs are widened with two integer ops, and silu(a) = h + h * tanh(h) with
+// h = a / 2 (the logistic written through tanh) costs one hardware tanh and
+// two FP ops per element.  SPLIT also writes the lo part x - bf16(x) of each
+// key value (split-bf16 operands) and then uses the exact-form logistic for
+// every row, since the lo part would carry the tanh approximation's error.
+template <int S, int MAXV, int ROWS, bool SPLIT>
+__global__ void __launch_bounds__(256) k_qk_prologue_bf16(const __nv_bfloat16* __restrict__ q,
+                                                          __nv_bfloat16* __restrict__ qh,
+                                                          int64_t q_rows,
+                                                          const __nv_bfloat16* __restrict__ k,
+                                                          __nv_bfloat16* __restrict__ kh,
+                                                          int64_t k_rows, int d,
+                                                          __nv_bfloat16* __restrict__ kh_lo) {
+  griddep_launch();
+  griddep_wait();
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t group = gtid / S;
+  const int sl = static_cast<int>(gtid % S);
+  const int64_t total = q_rows + k_rows;
+  const int nv = d >> 3;
+  uint4 in[ROWS][MAXV];
+#pragma unroll
+  for (int rr = 0; rr < ROWS; ++rr) {
+    const int64_t row = group * ROWS + rr;
+    const __nv_bfloat16* src = row < q_rows ? q + row * d : k + (row - q_rows) * d;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = sl + i * S;
+      in[rr][i] = (row < total && v < nv) ? reinterpret_cast<const uint4*>(src)[v]
+                                          : make_uint4(0u, 0u, 0u, 0u);   // silu(0) = 0
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < ROWS; ++rr) {
+    const int64_t row = group * ROWS + rr;
+    float y[MAXV][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const uint32_t w[4] = {in[rr][i].x, in[rr][i].y, in[rr][i].z, in[rr][i].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float a = __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+        float t;
+        if (SPLIT) {
+          t = __fdividef(a, 1.0f + __expf(-a));
+        } else {
+          const float h = 0.5f * a;
+          t = fmaf(h, tanh_approx(h), h);
+        }
+        y[i][e] = t;
+        ss = fmaf(t, t, ss);
+      }
+    }
+#pragma unroll
+    for (int o = S / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (row >= total) continue;
+    const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+    const bool is_q = row < q_rows;
+    __nv_bfloat16* dst = is_q ? qh + row * d : kh + (row - q_rows) * d;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = sl + i * S;
+      if (v >= nv) continue;
+      uint32_t hw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) hw[e] = pack_bf16x2(y[i][2 * e] * inv, y[i][2 * e + 1] * inv);
+      reinterpret_cast<uint4*>(dst)[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      if (SPLIT && !is_q) {
+        uint32_t lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = y[i][2 * e] * inv, x1 = y[i][2 * e + 1] * inv;
+          lw[e] = pack_bf16x2(x0 - __uint_as_float(hw[e] << 16), x1 - __uint_as_float(hw[e] & 0xffff0000u));
+        }
+        reinterpret_cast<uint4*>(kh_lo + (row - q_rows) * d)[v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    }
+  }
+}
+
 // bf16 shadow of an fp32 value, and its split-bf16 lo part when asked for.
 __device__ __forceinline__ void store_shadow(__nv_bfloat16* hi, __nv_bfloat16* lo, int64_t o, float x) {
   if (!hi) return;

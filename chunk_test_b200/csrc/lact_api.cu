@@ -464,15 +464,28 @@ static cudaError_t prologue_as(const Dims& D, const Bufs& b, const Inputs& in, c
   return cudaGetLastError();
 }
 
+template <int S, int MAXV>
+static cudaError_t prologue_bf16(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st) {
+  constexpr int ROWS = 4;  // rows per lane group, loads issued together
+  const int64_t rows = D.BH * D.Tq + D.BH * D.T;
+  const unsigned blocks = static_cast<unsigned>(cdiv(cdiv(rows, ROWS) * S, 256));
+  using B16 = __nv_bfloat16;
+  auto kern = b.kh_lo ? k_qk_prologue_bf16<S, MAXV, ROWS, true> : k_qk_prologue_bf16<S, MAXV, ROWS, false>;
+  (void)launch_pdl(kern, blocks, 256, 0, st, static_cast<const B16*>(in.q), static_cast<B16*>(b.qh),
+                   D.BH * D.Tq, static_cast<const B16*>(in.k), static_cast<B16*>(b.kh), D.BH * D.T,
+                   static_cast<int>(D.d), b.kh_lo);
+  return cudaGetLastError();
+}
+
 // Rows of d elements: 16-byte vectors, S = the power of two >= vectors per
 // row (at most a warp), MAXV vectors per thread.
 static cudaError_t launch_prologue(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t st) {
   if (D.dtype == LACT_BF16) {
     const int nv = static_cast<int>(D.d / 8);  // d is a multiple of 64
-    if (nv <= 8) return prologue_as<__nv_bfloat16, 8, 8, 1>(D, b, in, st);
-    if (nv <= 16) return prologue_as<__nv_bfloat16, 8, 16, 1>(D, b, in, st);
-    if (nv <= 32) return prologue_as<__nv_bfloat16, 8, 32, 1>(D, b, in, st);
-    return prologue_as<__nv_bfloat16, 8, 32, 2>(D, b, in, st);
+    if (nv <= 8) return prologue_bf16<8, 1>(D, b, in, st);
+    if (nv <= 16) return prologue_bf16<16, 1>(D, b, in, st);
+    if (nv <= 32) return prologue_bf16<32, 1>(D, b, in, st);
+    return prologue_bf16<32, 2>(D, b, in, st);
   }
   if (D.d % 4 == 0) return prologue_as<float, 4, 32, 4>(D, b, in, st);
   return prologue_as<float, 1, 32, 16>(D, b, in, st);
