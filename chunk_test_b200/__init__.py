@@ -8,10 +8,11 @@ torch CUDA tensors, `ttt_fwd_host` takes host tensors.
 from ._abi import (  # noqa: F401
     APPLY_THEN_UPDATE, UPDATE_THEN_APPLY, RULE_GD, RULE_MOMENTUM, RULE_MUON,
     LACT_OK, LACT_EINVAL, LACT_ENOSPC, LACT_ECUDA, LACT_ETIMEOUT, LACT_ENODEV, LACT_ETOOBIG,
+    LACT_ECOMM, REDUCE_SUM, REDUCE_MEAN,
     NOALLOC_SCRATCH_BYTES,
     LactError, LactProblem, LactFwdOpts, LIB_PATH, lib, status_string, profile_enable, profile_read,
 )
 from .layer import (  # noqa: F401
     ttt_fwd, ttt_fwd_host, ttt_fwd_noalloc, workspace_bytes, host_workspace_bytes, launch_count, status,
-    device_check, selftest_wait_timeout, make_problem,
+    device_check, selftest_wait_timeout, make_problem, torch_distributed_allreduce,
 )

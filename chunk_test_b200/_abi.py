@@ -11,6 +11,11 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblact_b20
 
 LACT_OK, LACT_EINVAL, LACT_ENOSPC, LACT_ECUDA, LACT_ETIMEOUT, LACT_ENODEV = 0, -1, -2, -3, -4, -5
 LACT_ETOOBIG = -6
+LACT_ECOMM = -7
+REDUCE_SUM, REDUCE_MEAN = 0, 1
+# int (*lact_allreduce_fn)(float* data, int64_t count, int op, void* stream, void* user)
+ALLREDUCE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                ctypes.c_void_p, ctypes.c_void_p)
 NOALLOC_SCRATCH_BYTES = 32 << 20  # LACT_NOALLOC_SCRATCH_BYTES
 LACT_F32, LACT_BF16 = 0, 1
 APPLY_THEN_UPDATE, UPDATE_THEN_APPLY = 0, 1
@@ -28,10 +33,12 @@ class LactProblem(ctypes.Structure):
 
 class LactFwdOpts(ctypes.Structure):
     """lact_fwd_opts: update_mask is a HOST byte array (one per chunk);
-    out_scale, m1, m2, m3 are device pointers (0 = off)."""
+    out_scale, m1, m2, m3 are device pointers (0 = off); allreduce is the
+    context-parallel hook (NULL = one rank)."""
     _fields_ = [
         ("update_mask", ctypes.c_void_p), ("out_scale", ctypes.c_void_p),
         ("m1", ctypes.c_void_p), ("m2", ctypes.c_void_p), ("m3", ctypes.c_void_p),
+        ("allreduce", ALLREDUCE_FN), ("allreduce_user", ctypes.c_void_p),
     ]
 
 

@@ -417,21 +417,21 @@ struct Launcher {
   }
 };
 
-// Per device: a library-owned side stream and two events, used to run a
-// chunk's apply concurrently with its key forward + gradient (both read only
-// the previous state) in apply-then-update order.
+// Per host thread and device: a library-owned side stream and three events,
+// used to run a chunk's apply concurrently with its key forward + gradient
+// (both read only the previous state) in apply-then-update order.  Each
+// thread has its own, so calls made at the same time from several threads
+// never record over each other's events.  They live until the process exits.
 struct SideRes {
   cudaStream_t side = nullptr;
   cudaEvent_t fork = nullptr, join[2] = {nullptr, nullptr};
 };
-static SideRes g_side[64];
-static std::mutex g_side_mu;
+static thread_local SideRes tl_side[64];
 
 static const SideRes* side_resources() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(g_side_mu);
-  SideRes& r = g_side[dev];
+  SideRes& r = tl_side[dev];
   if (!r.side) {
     if (cudaStreamCreateWithFlags(&r.side, cudaStreamNonBlocking) != cudaSuccess) return r.side = nullptr, nullptr;
     if (cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming) != cudaSuccess ||
@@ -451,6 +451,8 @@ struct Inputs {
   const uint8_t* mask;     // host, one byte per chunk: 0 = the chunk does not update
   const float* scale;      // [BH, Tq] output factors
   float *m1, *m2, *m3;     // momentum in/out
+  lact_allreduce_fn allreduce;   // context-parallel reduction hook
+  void* allreduce_user;
 };
 
 template <typename T, int VEC, int S, int MAXV>
@@ -527,6 +529,12 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
   const int BH = static_cast<int>(D.BH), d = static_cast<int>(D.d), dh = static_cast<int>(D.dh);
   const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane;
   const unsigned state_blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(planes, 1024), 148 * 16));
+  // Context parallelism: reduce a buffer over the ranks, in place, ordered on
+  // the main stream (the hook enqueues the collective there).
+  auto reduce = [&](float* data, int64_t count, int op) {
+    if (!in.allreduce || L.dry || L.err != LACT_OK) return;
+    if (in.allreduce(data, count, op, static_cast<void*>(main_st), in.allreduce_user) != 0) L.err = LACT_ECOMM;
+  };
 
   // Fast-weight masters (+ bf16 shadows), momentum = the caller's or 0.
   L(K_INIT, [&] {
@@ -544,6 +552,7 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
                                                                             static_cast<int>(D.nch), b.bbar);
       return cudaGetLastError();
     });
+    reduce(b.bbar, D.BH * D.nch, LACT_REDUCE_MEAN);   // equal shares: mean of the ranks' means
   }
 
   bool join_before_rule = false, side_used = false;
@@ -750,6 +759,8 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
         });
       }
 
+      // the chunk's gradient is the sum of every rank's partial planes
+      reduce(b.P, static_cast<int64_t>(splits) * planes, LACT_REDUCE_SUM);
       const float* dir = b.P;
       int dir_splits = splits;
       if (D.rule == LACT_RULE_MUON) {
@@ -983,6 +994,8 @@ static void set_options(Inputs& in, const lact_fwd_opts* o) {
   in.m1 = o ? o->m1 : nullptr;
   in.m2 = o ? o->m2 : nullptr;
   in.m3 = o ? o->m3 : nullptr;
+  in.allreduce = o ? o->allreduce : nullptr;
+  in.allreduce_user = o ? o->allreduce_user : nullptr;
 }
 
 static int input_bytes(const Dims& D, size_t sz[8]) {
@@ -1261,6 +1274,7 @@ const char* lact_status_string(int code) {
     case LACT_ETOOBIG:
       return "problem needs more scratch than lact_ttt_fwd_noalloc's built-in buffer "
              "(LACT_NOALLOC_SCRATCH_BYTES) holds; use lact_ttt_fwd with a caller workspace";
+    case LACT_ECOMM: return "the context-parallel all-reduce hook returned an error";
     default: return "unknown status";
   }
 }

@@ -65,10 +65,64 @@ def launch_count(q, k, w1, chunk, order, rule, update_mask=None) -> int:
     return int(_abi.lib().lact_ttt_launch_count_ex(ctypes.byref(p), ctypes.byref(opts)))
 
 
-def _options(p, update_mask, out_scale, m_inout, q):
+class _CudaBuf:
+    """A device buffer of fp32 values seen through __cuda_array_interface__,
+    so that torch can alias it without a copy."""
+
+    def __init__(self, ptr: int, n: int):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<f4", "data": (ptr, False),
+                                         "version": 2, "strides": None}
+
+
+def _hook(py_fn, device, errors: list):
+    """C hook (lact_allreduce_fn) around py_fn(buf, op, stream): buf is a
+    float32 tensor aliasing the library's buffer, op REDUCE_SUM or
+    REDUCE_MEAN, stream the torch stream of the call.  An exception is kept
+    in `errors` and reported to the library as a failure."""
+
+    def c_fn(ptr, count, op, stream_ptr, user):
+        try:
+            buf = torch.as_tensor(_CudaBuf(int(ptr), int(count)), device=device)
+            st = torch.cuda.ExternalStream(int(stream_ptr or 0), device=device)
+            py_fn(buf, int(op), st)
+            return 0
+        except BaseException as e:  # noqa: BLE001 - handed back to the caller
+            errors.append(e)
+            return 1
+
+    return _abi.ALLREDUCE_FN(c_fn)
+
+
+def torch_distributed_allreduce(group=None):
+    """A context-parallel hook for ttt_fwd(allreduce=...): all-reduce over the
+    torch.distributed process group `group` (NCCL for CUDA tensors), enqueued
+    on the layer's stream, so that the layer's later kernels see the sum (or
+    the mean, for REDUCE_MEAN)."""
+    import torch.distributed as dist
+
+    def fn(buf, op, stream=None):
+        ctx = torch.cuda.stream(stream) if (stream is not None and buf.is_cuda) else _nullctx()
+        with ctx:
+            dist.all_reduce(buf, op=dist.ReduceOp.SUM, group=group)
+            if op == _abi.REDUCE_MEAN:
+                buf.div_(dist.get_world_size(group))
+
+    return fn
+
+
+class _nullctx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def _options(p, update_mask, out_scale, m_inout, q, allreduce=None, errors=None):
     """lact_fwd_opts for the given options (None when none is given) and the
-    host mask buffer it points into (kept alive by the caller)."""
-    if update_mask is None and out_scale is None and m_inout is None:
+    objects it points into (the host mask buffer, the C hook), which the
+    caller keeps alive for the call."""
+    if update_mask is None and out_scale is None and m_inout is None and allreduce is None:
         return None, None
     nch = -(-p.T // min(p.chunk, p.T))
     mask_buf = None
@@ -88,14 +142,18 @@ def _options(p, update_mask, out_scale, m_inout, q):
         for m in ms:
             if m.device != q.device or m.dtype != torch.float32 or not m.is_contiguous():
                 raise ValueError("m_inout must be contiguous float32 tensors on q's device")
+    hook = None if allreduce is None else _hook(allreduce, q.device, errors if errors is not None else [])
     o = _abi.LactFwdOpts(ctypes.addressof(mask_buf) if mask_buf is not None else None,
                          None if out_scale is None else out_scale.data_ptr(),
                          *(None if m is None else m.data_ptr() for m in ms))
-    return o, mask_buf
+    if hook is not None:
+        o.allreduce = hook
+    return o, (mask_buf, hook)
 
 
 def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_out=None,
-            workspace=None, stream=None, update_mask=None, out_scale=None, m_inout=None):
+            workspace=None, stream=None, update_mask=None, out_scale=None, m_inout=None,
+            allreduce=None):
     """Runs the layer on the current CUDA device.  Returns (out, w1o, w2o, w3o).
     Optional `out`, `w_out` (a 3-tuple) and `workspace` (uint8 tensor) avoid
     allocations; `stream` defaults to torch's current stream.
@@ -103,10 +161,15 @@ def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_ou
     chunk (0 = the chunk is applied but does not update the state);
     `out_scale`, a [B, H, Tq] float32 tensor of per-query output factors;
     `m_inout`, three float32 momentum tensors (shapes of the w_out) read as
-    the initial momentum and overwritten with the final one."""
+    the initial momentum and overwritten with the final one;
+    `allreduce`, a context-parallel hook fn(buf, op, stream) that reduces
+    `buf` in place over the ranks (see torch_distributed_allreduce); each
+    rank then passes its own equal share of every chunk's tokens, with
+    `chunk` the local share's length."""
     _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
     p = make_problem(q, k, w1, chunk, order, rule)
-    opts, _mask_keep = _options(p, update_mask, out_scale, m_inout, q)
+    errors = []
+    opts, _keep = _options(p, update_mask, out_scale, m_inout, q, allreduce, errors)
     B, H, Tq, d = q.shape
     dh = w1.shape[1]
     if out is None:
@@ -127,6 +190,8 @@ def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_ou
         _ptr(lr), _ptr(beta), _ptr(w1), _ptr(w2), _ptr(w3), _ptr(out), _ptr(w_out[0]),
         _ptr(w_out[1]), _ptr(w_out[2]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
         ctypes.c_void_p(stream.cuda_stream))
+    if errors:
+        raise errors[0]
     if rc != _abi.LACT_OK:
         raise LactError(rc, "lact_ttt_fwd_ex")
     return out, w_out[0], w_out[1], w_out[2]

@@ -4,9 +4,10 @@
  * The layer (Large-Chunk Test-Time Training).  Sources are cited by page
  * title and section:
  *   [P1] "LaCT架构核心思想解析" (gsyq.cn) §1.2, §2.1, §2.2, §3.2
- *   [P2] "大块测试时训练（LaCT）技术解析" (dpshk.com) §2.1, §2.2.1
+ *   [P2] "大块测试时训练（LaCT）技术解析" (dpshk.com) §2.1, §2.2.1, §2.2.2
  *   [P3] "LaCT：以大分块更新人工智能的临时记忆" (iplexlaw.co.kr), sections
- *        「局部注意力与非线性记忆相互补充」 and 「更新顺序必须遵守信息可见范围」
+ *        「局部注意力与非线性记忆相互补充」, 「更新顺序必须遵守信息可见范围」 and
+ *        「视频实验和分布式计算」
  *
  * Per (batch b, head h) the layer keeps a SwiGLU fast-weight net
  *     f_W(x) = W2 (silu(W1 x) * (W3 x)),   W1, W3: [dh, d],  W2: [d, dh]
@@ -76,8 +77,9 @@ enum {
   LACT_ECUDA = -3,        /* a CUDA runtime call or kernel launch failed */
   LACT_ETIMEOUT = -4,     /* a bounded device wait gave up (see lact_ttt_status) */
   LACT_ENODEV = -5,       /* the current device is not an sm_100 GPU */
-  LACT_ETOOBIG = -6       /* the problem needs more scratch than the built-in
+  LACT_ETOOBIG = -6,      /* the problem needs more scratch than the built-in
                              buffer of lact_ttt_fwd_noalloc holds */
+  LACT_ECOMM = -7         /* the context-parallel all-reduce hook failed */
 };
 
 enum { LACT_F32 = 0, LACT_BF16 = 1 };
@@ -113,6 +115,29 @@ int lact_ttt_fwd(const lact_problem* p,
                  void* out, float* w1_out, float* w2_out, float* w3_out,
                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* Context parallelism ([P2 §2.2.2]: each device takes the gradient of its
+ * shard of the chunk, the gradients are summed across devices, then the
+ * update is applied; [P3] 「视频实验和分布式计算」).  G ranks each hold one equal share of every chunk's
+ * tokens and call lact_ttt_fwd_ex with their local q, k, v, lr, beta (local
+ * T = T / G, local chunk = chunk / G) and the same initial state.  The
+ * library calls the hook, on the calling thread while it enqueues the work,
+ * with a device buffer of `count` floats whose contents are produced by the
+ * work already enqueued on `stream`:
+ *   - after each chunk's gradient, on its partial gradient planes, op SUM
+ *     (the summed gradient is then the whole chunk's);
+ *   - once before the chunk loop (momentum rule), on the per-chunk means of
+ *     beta [B*H, nchunks], op MEAN (equal shares: the mean of the means).
+ * The hook must reduce the buffer in place over the ranks so that work
+ * enqueued on `stream` after it returns sees the result (for example NCCL on
+ * that stream), and return 0; any other value stops the call with
+ * LACT_ECOMM.  Every rank then applies the same rule to the same reduced
+ * gradient, so all ranks hold the same fast weights; each rank's `out` holds
+ * its own queries.  Every rank must make the same sequence of calls with
+ * the same problem shape and options (the hook is called the same number of
+ * times with the same counts on every rank). */
+enum { LACT_REDUCE_SUM = 0, LACT_REDUCE_MEAN = 1 };
+typedef int (*lact_allreduce_fn)(float* data, int64_t count, int op, void* stream, void* user);
+
 /* Options of lact_ttt_fwd_ex.  Zero-initialise the struct and set what is
  * used; a NULL field leaves its feature off, and a NULL options pointer is
  * lact_ttt_fwd.
@@ -138,13 +163,17 @@ int lact_ttt_fwd(const lact_problem* p,
  *              sequence split at chunk boundaries into several calls (w*_out
  *              and m* handed from one call to the next) gives the results of
  *              one call.  They may not overlap each other or any other
- *              argument. */
+ *              argument.
+ * allreduce    context-parallel hook (see lact_allreduce_fn above), called
+ *              with `allreduce_user` as its last argument; NULL: one rank. */
 typedef struct lact_fwd_opts {
   const uint8_t* update_mask;
   const float* out_scale;
   float* m1;
   float* m2;
   float* m3;
+  lact_allreduce_fn allreduce;
+  void* allreduce_user;
 } lact_fwd_opts;
 
 /* lact_ttt_fwd with options (see lact_fwd_opts); the same arguments,

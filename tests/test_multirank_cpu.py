@@ -119,3 +119,79 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+# ---------------------------------------------------------------- context parallelism
+def _cp_hook_worker(rank, world, port, outdir):
+    sys.path.insert(0, ROOT)
+    import chunk_test_b200 as ct
+    _init(rank, world, port)
+    try:
+        fn = ct.torch_distributed_allreduce()
+        a = torch.arange(6, dtype=torch.float32) + 10.0 * rank
+        fn(a, ct.REDUCE_SUM)
+        b = torch.full((4,), 1.0 + rank)
+        fn(b, ct.REDUCE_MEAN)
+        with open(os.path.join(outdir, f"cp{rank}.json"), "w") as f:
+            json.dump({"sum": a.tolist(), "mean": b.tolist()}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_hook_sums_and_averages_over_ranks():
+    """The torch.distributed hook that the layer calls between a chunk's
+    gradient and its rule: a sum over the ranks in place (gradients), or the
+    mean (the per-chunk beta means of equal shares)."""
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_cp_hook_worker, args=(2, _free_port(), d), nprocs=2, join=True,
+                           start_method="spawn")
+        res = [json.load(open(os.path.join(d, f"cp{r}.json"))) for r in range(2)]
+    for r in res:
+        assert r["sum"] == [10.0 + 2 * i for i in range(6)]
+        assert r["mean"] == [1.5] * 4
+
+
+@pytest.mark.parametrize("rule", [0, 1, 2])
+def test_context_parallel_shards_reproduce_the_layer(rule):
+    """Context parallelism ("大块测试时训练（LaCT）技术解析" §2.2.2): every
+    rank takes the gradient of its share of the chunk, the gradients are
+    summed over the ranks, and every rank applies the same update.  Emulated
+    here on the oracle's own steps for 2 ranks: the per-rank gradients of the
+    shares sum to the whole chunk's gradient (the chunk gradient is a sum
+    over tokens), and the beta mean of the chunk is the mean of the shares'
+    means, so the sharded loop gives the layer's weights and outputs."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    rng = np.random.default_rng(7)
+    H, T, d, dh, chunk, world = 2, 24, 6, 8, 8, 2
+    q, k, v = (rng.standard_normal((1, H, T, d)) for _ in range(3))
+    lr = np.log1p(np.exp(rng.standard_normal((1, H, T, 3)) - 1.0))
+    beta = 1 / (1 + np.exp(-(2 + 0.5 * rng.standard_normal((1, H, T)))))
+    w1 = rng.standard_normal((H, dh, d)) / d ** 0.5
+    w2 = rng.standard_normal((H, d, dh)) / dh ** 0.5
+    w3 = rng.standard_normal((H, dh, d)) / d ** 0.5
+    want = oracle.ttt_layer(q, k, v, lr, beta if rule == 1 else None, w1, w2, w3, chunk, 0, rule)
+    for h in range(H):
+        W = (w1[h].copy(), w2[h].copy(), w3[h].copy())
+        M = tuple(np.zeros_like(x) for x in W)
+        out = np.zeros((T, d))
+        kh, qh = oracle.qk_prologue(k[0, h]), oracle.qk_prologue(q[0, h])
+        for c0 in range(0, T, chunk):
+            rows = slice(c0, c0 + chunk)
+            out[rows] = oracle.fast_net(*W, qh[rows])
+            parts, means = [], []
+            for r in range(world):
+                sl = slice(c0 + r * chunk // world, c0 + (r + 1) * chunk // world)
+                parts.append(oracle.chunk_gradient(*W, kh[sl], v[0, h, sl], lr[0, h, sl]))
+                means.append(beta[0, h, sl].mean())
+            G = tuple(sum(p[j] for p in parts) for j in range(3))
+            if rule == 1:
+                bbar = float(np.mean(means))
+                M = tuple(bbar * m + g for m, g in zip(M, G))
+                U = M
+            else:
+                U, _ = oracle.rule_step(rule, G, M, None)
+            W = tuple(oracle.renorm_rows(w - u, w) for w, u in zip(W, U))
+        np.testing.assert_allclose(out, want[0][0, h], rtol=1e-10, atol=1e-12)
+        for j in range(3):
+            np.testing.assert_allclose(W[j], want[1 + j][h], rtol=1e-10, atol=1e-12)
