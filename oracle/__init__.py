@@ -65,3 +65,4 @@ from .lact_oracle import (  # noqa: F401
     newton_schulz5, renorm_rows, rule_step, ttt_head, ttt_head_state, ttt_layer, ttt_layer_ex,
     blas_threads,
 )
+from . import lact_oracle_bwd  # noqa: F401,E402
