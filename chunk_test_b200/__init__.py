@@ -13,6 +13,7 @@ from ._abi import (  # noqa: F401
     LactError, LactProblem, LactFwdOpts, LIB_PATH, lib, status_string, profile_enable, profile_read,
 )
 from .layer import (  # noqa: F401
-    ttt_fwd, ttt_fwd_host, ttt_fwd_noalloc, workspace_bytes, host_workspace_bytes, launch_count, status,
+    ttt_fwd, ttt_fwd_host, ttt_fwd_noalloc, ttt_bwd, workspace_bytes, bwd_workspace_bytes,
+    host_workspace_bytes, launch_count, status,
     device_check, selftest_wait_timeout, make_problem, torch_distributed_allreduce,
 )

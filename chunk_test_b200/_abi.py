@@ -57,6 +57,9 @@ SIGNATURES = {
     "lact_ttt_fwd_ex": (ctypes.c_int, [_P, ctypes.POINTER(LactFwdOpts)] + [_vp] * 12
                         + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_fwd_noalloc": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp]),
+    "lact_ttt_bwd_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "lact_ttt_bwd": (ctypes.c_int, [_P, ctypes.POINTER(LactFwdOpts)] + [_vp] * 21
+                     + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_host_workspace_bytes": (ctypes.c_size_t, [_P]),
     "lact_ttt_fwd_host": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_status": (ctypes.c_int, [_vp]),
@@ -102,6 +105,10 @@ def problem(B, H, T, Tq, d, dh, chunk, order, rule, dtype, w_shared) -> LactProb
 
 def workspace_bytes(p: LactProblem) -> int:
     return int(lib().lact_ttt_workspace_bytes(ctypes.byref(p)))
+
+
+def bwd_workspace_bytes(p: LactProblem) -> int:
+    return int(lib().lact_ttt_bwd_workspace_bytes(ctypes.byref(p)))
 
 
 def host_workspace_bytes(p: LactProblem) -> int:

@@ -370,6 +370,7 @@ struct RuleParams {
   int nch, chunk_idx;
   int rule;
   int BH, dh, d;
+  float* nrm_out;         // or null: per row, the norm of W - U before the renorm
 };
 
 struct RuleRow {
@@ -418,6 +419,7 @@ __global__ void __launch_bounds__(256) k_rule_renorm(const RuleParams p) {
   on = warp_sum(on);
   nn = warp_sum(nn);
   const float sc = nn > 0.f ? sqrtf(on) / sqrtf(nn) : 0.f;
+  if (p.nrm_out && lane == 0) p.nrm_out[row] = sqrtf(nn);
   for (int c = lane; c < r.len; c += 32) {
     const int64_t o = r.base + c;
     const float w = p.Wm[o] * sc;

@@ -367,13 +367,13 @@ static cudaError_t launch_gemm_any(bool split, int bn, dim3 grid, const GemmPara
 enum Kind {
   K_INIT, K_PROLOGUE, K_BETA_MEAN, K_FWD_QUERY, K_APPLY_OUT, K_FWD_KEY, K_GRAD, K_NS_SUMSQ,
   K_NS_SCALE, K_NS_GRAM, K_NS_POLY, K_NS_UPDATE, K_RULE, K_FINALIZE, K_SIMT_GEMM, K_FWD_ELEM_F32,
-  K_APPLY_FUSED, K_KEY_GRAD, K_COUNT
+  K_APPLY_FUSED, K_KEY_GRAD, K_BWD_ELEM, K_COUNT
 };
 static const char* const kKindNames[K_COUNT] = {
     "init_state", "qk_prologue", "beta_mean", "fwd_query_umma", "apply_out_umma", "fwd_key_umma",
     "grad_umma", "ns_sumsq", "ns_scale", "ns_gram_umma", "ns_poly_umma", "ns_update_umma",
     "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32", "apply_fused_umma",
-    "key_grad_umma"};
+    "key_grad_umma", "bwd_elem"};
 
 // Optional per-launch CUDA-event pairs on the launching stream.
 struct ProfRec { int kind; cudaEvent_t a, b; };
@@ -1047,6 +1047,8 @@ __global__ void k_selftest_wait() {
 
 }  // namespace lact
 
+#include "lact_bwd.cuh"
+
 using namespace lact;
 
 extern "C" {
@@ -1193,6 +1195,65 @@ int lact_ttt_fwd_host(const lact_problem* p, const void* q, const void* k, const
     return LACT_ECUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return LACT_ECUDA;
   return LACT_OK;
+}
+
+size_t lact_ttt_bwd_workspace_bytes(const lact_problem* p) {
+  Dims D;
+  if (validate(p, D) != LACT_OK || D.rule == LACT_RULE_MUON) return 0;
+  return bwd_workspace_bytes(D);
+}
+
+int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts, const void* q, const void* k,
+                 const void* v, const float* lr, const float* beta, const float* w1, const float* w2,
+                 const float* w3, const void* dout, const float* dw1_out, const float* dw2_out,
+                 const float* dw3_out, float* dq, float* dk, float* dv, float* dlr, float* dbeta,
+                 float* dw1, float* dw2, float* dw3, float* dout_scale, void* workspace,
+                 size_t workspace_bytes_, void* stream) {
+  Dims D;
+  int rc = validate(p, D);
+  if (rc != LACT_OK) return rc;
+  if (D.rule == LACT_RULE_MUON) return LACT_EINVAL;
+  if (opts && (opts->m1 || opts->m2 || opts->m3 || opts->allreduce)) return LACT_EINVAL;
+  const float* scale = opts ? opts->out_scale : nullptr;
+  const bool mom = D.rule == LACT_RULE_MOMENTUM;
+  const size_t e = D.dtype == LACT_BF16 ? 2 : 4;
+  const size_t nq = static_cast<size_t>(D.BH * D.Tq * D.d), nk = static_cast<size_t>(D.BH * D.T * D.d);
+  const size_t hw = static_cast<size_t>(D.w_shared ? D.H : D.BH) * D.d * D.dh * 4;
+  const size_t wo = static_cast<size_t>(D.BH * D.d * D.dh) * 4;
+  struct Buf { const void* p; size_t n; bool need; };
+  const Buf ins[] = {{q, nq * e, true}, {k, nk * e, true}, {v, nk * e, true},
+                     {lr, static_cast<size_t>(D.BH * D.T) * 12, true}, {beta, static_cast<size_t>(D.BH * D.T) * 4, mom},
+                     {w1, hw, true}, {w2, hw, true}, {w3, hw, true}, {dout, nq * e, true},
+                     {dw1_out, wo, false}, {dw2_out, wo, false}, {dw3_out, wo, false},
+                     {scale, static_cast<size_t>(D.BH * D.Tq) * 4, false}};
+  const Buf outs[] = {{dq, nq * 4, true}, {dk, nk * 4, true}, {dv, nk * 4, true},
+                      {dlr, static_cast<size_t>(D.BH * D.T) * 12, true},
+                      {dbeta, static_cast<size_t>(D.BH * D.T) * 4, mom}, {dw1, hw, true}, {dw2, hw, true},
+                      {dw3, hw, true}, {dout_scale, static_cast<size_t>(D.BH * D.Tq) * 4, scale != nullptr}};
+  for (const Buf& b : ins)
+    if ((b.need && !b.p) || (b.p && !aligned16(b.p) && b.p != scale)) return LACT_EINVAL;
+  for (const Buf& b : outs)
+    if (b.need && (!b.p || (b.p != dout_scale && !aligned16(b.p)))) return LACT_EINVAL;
+  if (scale && (reinterpret_cast<uintptr_t>(scale) & 3u)) return LACT_EINVAL;
+  if (dout_scale && (reinterpret_cast<uintptr_t>(dout_scale) & 3u)) return LACT_EINVAL;
+  if ((dw1_out || dw2_out || dw3_out) && !(dw1_out && dw2_out && dw3_out)) return LACT_EINVAL;
+  for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+    if (!outs[i].need) continue;
+    for (const Buf& b : ins)
+      if (b.p && overlaps(outs[i].p, outs[i].n, b.p, b.n)) return LACT_EINVAL;
+    for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+      if (outs[j].need && overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return LACT_EINVAL;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LACT_EINVAL;
+  if (workspace_bytes_ < bwd_workspace_bytes(D)) return LACT_ENOSPC;
+  Bump bp{reinterpret_cast<uintptr_t>(workspace), 0};
+  BwdBufs b;
+  plan_bwd(D, bp, b);
+  BwdInputs in{q, k, v, lr, beta, w1, w2, w3, dout, dw1_out, dw2_out, dw3_out,
+               opts ? opts->update_mask : nullptr, scale, dq, dk, dv, dlr, dbeta, dw1, dw2, dw3, dout_scale};
+  Launcher L{false, static_cast<cudaStream_t>(stream)};
+  run_bwd(D, b, in, static_cast<cudaStream_t>(stream), L);
+  return L.err;
 }
 
 int lact_ttt_status(void* stream) {

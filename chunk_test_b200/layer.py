@@ -197,6 +197,49 @@ def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_ou
     return out, w_out[0], w_out[1], w_out[2]
 
 
+def bwd_workspace_bytes(q, k, w1, chunk, order, rule) -> int:
+    return _abi.bwd_workspace_bytes(make_problem(q, k, w1, chunk, order, rule))
+
+
+def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=None,
+            update_mask=None, out_scale=None, workspace=None, stream=None):
+    """The layer's backward on the current CUDA device (lact_ttt_bwd): the
+    gradients of a loss given dL/d out (`dout`, like q) and optionally
+    dL/d w_out (`dw_out`, three tensors like the forward's w_out).  Returns a
+    dict of float32 tensors: dq, dk, dv, dlr, dbeta (momentum, else None),
+    dw1, dw2, dw3 (shaped like w1, w2, w3) and dout_scale (when out_scale is
+    given, else None)."""
+    _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
+    if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_contiguous():
+        raise ValueError("dout must be a contiguous tensor shaped like q, in q's dtype")
+    p = make_problem(q, k, w1, chunk, order, rule)
+    opts, _keep = _options(p, update_mask, out_scale, None, q)
+    f32 = dict(device=q.device, dtype=torch.float32)
+    res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
+           "dv": torch.empty(v.shape, **f32), "dlr": torch.empty(lr.shape, **f32),
+           "dbeta": None if beta is None else torch.empty(beta.shape, **f32),
+           "dw1": torch.empty(w1.shape, **f32), "dw2": torch.empty(w2.shape, **f32),
+           "dw3": torch.empty(w3.shape, **f32),
+           "dout_scale": None if out_scale is None else torch.empty(out_scale.shape, **f32)}
+    need = _abi.bwd_workspace_bytes(p)
+    if need == 0:
+        raise LactError(_abi.LACT_EINVAL, "lact_ttt_bwd_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    dw = (None, None, None) if dw_out is None else tuple(dw_out)
+    rc = _abi.lib().lact_ttt_bwd(
+        ctypes.byref(p), None if opts is None else ctypes.byref(opts), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(lr), _ptr(beta), _ptr(w1), _ptr(w2), _ptr(w3), _ptr(dout), *(_ptr(x) for x in dw),
+        _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dlr"]), _ptr(res["dbeta"]),
+        _ptr(res["dw1"]), _ptr(res["dw2"]), _ptr(res["dw3"]), _ptr(res["dout_scale"]),
+        _ptr(workspace), ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
+    if rc != _abi.LACT_OK:
+        raise LactError(rc, "lact_ttt_bwd")
+    return res
+
+
 def ttt_fwd_noalloc(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out, w_out,
                     stream=None):
     """The forward for callers that cannot allocate device memory: no

@@ -1,5 +1,6 @@
 /*
- * lact.h -- C ABI of the B200 (sm_100a) LaCT fast-weight TTT layer forward.
+ * lact.h -- C ABI of the B200 (sm_100a) LaCT fast-weight TTT layer (forward
+ * and backward).
  *
  * The layer (Large-Chunk Test-Time Training).  Sources are cited by page
  * title and section:
@@ -234,6 +235,40 @@ int lact_ttt_fwd_host(const lact_problem* p,
                       const float* w1, const float* w2, const float* w3,
                       void* out, float* w1_out, float* w2_out, float* w3_out,
                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Device scratch bytes lact_ttt_bwd needs for problem *p (0 if *p is invalid
+ * or uses the Muon rule).  Pure host arithmetic. */
+size_t lact_ttt_bwd_workspace_bytes(const lact_problem* p);
+
+/* The layer's backward: the gradients of a scalar loss L with respect to
+ * every input, given dL/d out (`dout`) and, optionally, dL/d w*_out
+ * (`dw*_out`, all three or none).  It is the vector-Jacobian product of
+ * lact_ttt_fwd_ex with the same problem, inputs and options, computed in
+ * fp32: the forward's updates are recomputed (the states before each chunk
+ * are kept in the workspace), then a reverse chunk loop takes, per chunk,
+ * the apply's backward, the renorm and rule backward, and the backward of
+ * the chunk gradient (its second-order terms: [P2 §2.1] eqs. 4-5 written as
+ * functions of W, k, v and lr).  Rules: GD and momentum (LACT_EINVAL for
+ * Muon).  Options: update_mask and out_scale; the momentum buffers and the
+ * all-reduce hook are not supported (LACT_EINVAL).
+ * Layouts: the inputs as in lact_ttt_fwd; dout [B,H,Tq,d] in the problem's
+ * dtype; dw*_out in the layouts of w*_out, or NULL (zero).  Outputs, all
+ * float32 device buffers: dq [B,H,Tq,d], dk, dv [B,H,T,d], dlr [B,H,T,3],
+ * dbeta [B,H,T] (momentum; else may be NULL), dw1, dw3 [Hw,dh,d], dw2
+ * [Hw,d,dh] (Hw as the initial weights: summed over the batch when the
+ * batch shares them), dout_scale [B,H,Tq] (required when out_scale is
+ * given, else ignored).  No output may overlap an input or another output.
+ * `workspace` is device scratch of lact_ttt_bwd_workspace_bytes(p) bytes,
+ * 256-byte aligned.  Asynchronous on `stream`, like the forward. */
+int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts,
+                 const void* q, const void* k, const void* v,
+                 const float* lr, const float* beta,
+                 const float* w1, const float* w2, const float* w3,
+                 const void* dout, const float* dw1_out, const float* dw2_out,
+                 const float* dw3_out,
+                 float* dq, float* dk, float* dv, float* dlr, float* dbeta,
+                 float* dw1, float* dw2, float* dw3, float* dout_scale,
+                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* Waits for `stream`, then returns and clears the device status word of the
  * current device: LACT_OK, or LACT_ETIMEOUT if a bounded wait inside one of

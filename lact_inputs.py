@@ -126,3 +126,21 @@ def video_update_mask(n_chunks: int, noisy_per_clean: int = 1) -> list:
     that follows them, in groups of noisy_per_clean + 1 chunks."""
     period = noisy_per_clean + 1
     return [1 if c % period == period - 1 else 0 for c in range(n_chunks)]
+
+
+def make_output_grads(w: Workload, seed: int = 0, with_weights: bool = False):
+    """Seeded gradients of a loss with respect to the layer's outputs, for
+    the backward: dout [B,H,Tq,d] ~ N(0,1) in the workload dtype and, when
+    asked, (dw1, dw2, dw3) ~ N(0,1) fp32 in the layouts of the final weights
+    [B*H, dh, d], [B*H, d, dh], [B*H, dh, d]."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(20_000 + seed)
+    dout = torch.randn((w.B, w.H, w.Tq, w.d), generator=g, dtype=torch.float32)
+    if w.dtype == BF16:
+        dout = dout.bfloat16()
+    dws = None
+    if with_weights:
+        BH = w.B * w.H
+        dws = (torch.randn((BH, w.dh, w.d), generator=g), torch.randn((BH, w.d, w.dh), generator=g),
+               torch.randn((BH, w.dh, w.d), generator=g))
+    return dout, dws
