@@ -281,6 +281,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
+                    help="time the layer forward (default) or its backward (lact_ttt_bwd)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload at this sequence length instead (a scaled case "
                          "for profiling; named in config.workload)")
@@ -293,6 +295,8 @@ def main():
                      chunk=T if single else min(w.chunk, T))
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.which == "bwd":
+        return run_backward(args, w)
 
     import chunk_test_b200 as ct
 
@@ -465,6 +469,155 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------- backward
+# fp32 FFMA peak of a B200: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz.
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_flops(w: Workload) -> float:
+    """Algorithmic FLOPs of lact_ttt_bwd, all in its contractions: per key
+    token per head 12 d dh to recompute the forward's updates (keys' forward
+    6, gradient 6) and 30 d dh in the reverse loop (keys' forward again 6,
+    (p, q, r) 6, the weight gradients 6, dk 8, dv 4); per query token per head
+    16 d dh for the apply's backward (its forward 6, the weight gradients 6,
+    dq 4)."""
+    return w.B * w.H * w.d * w.dh * (42.0 * w.T + 16.0 * w.Tq)
+
+
+def run_backward(args, w: Workload):
+    import chunk_test_b200 as ct
+    from lact_inputs import make_output_grads
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--pass bwd runs on one GPU")
+    if w.rule == RULE_MUON:
+        raise SystemExit("the backward covers GD and momentum")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    inp_cpu = make_inputs(w, seed=0)
+    dout_cpu, _ = make_output_grads(w, seed=0)
+    inp = {k: (None if v is None else v.to(dev)) for k, v in inp_cpu.items()}
+    dout = dout_cpu.to(dev)
+    ws = torch.empty(ct.bwd_workspace_bytes(inp["q"], inp["k"], inp["w1"], w.chunk, w.order, w.rule),
+                     device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ct.ttt_bwd(inp["q"], inp["k"], inp["v"], inp["lr"], inp["beta"], inp["w1"], inp["w2"],
+                          inp["w3"], w.chunk, w.order, w.rule, dout, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after warm-up")
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after the timed region")
+    # per-kernel pass (launch profiler on)
+    ct.profile_enable(True)
+    ct.profile_read()
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize(dev)
+    prof = ct.profile_read()
+    ct.profile_enable(False)
+    launches_per_step = sum(v[0] for v in prof.values()) // args.steps
+    dom_name, (n_launch, ms_kind) = max(prof.items(), key=lambda kv: kv[1][1])
+    flops = bwd_flops(w)
+    roof = None
+    _, _, pk_sust, pk_src = peaks()
+    if dom_name in ("simt_gemm_f32", "bwd_gemm_umma"):
+        # every FLOP of bwd_flops() is in these contractions
+        achieved = flops * args.steps / (ms_kind / 1e3) / 1e12
+        tensor = dom_name == "bwd_gemm_umma"
+        peak = pk_sust if tensor else FP32_FMA_TFLOPS
+        roof = {"bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "kernel": dom_name, "launches": n_launch,
+                "avg_launch_us": 1e3 * ms_kind / n_launch, "timed": "alone (per-kernel pass)",
+                "traffic": None,
+                "peak_source": f"{pk_src} sustained bf16" if tensor else
+                               "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz"}
+    kernels = {k: {"launches": v[0], "ms": round(v[1], 4),
+                   "share": round(v[1] / sum(x[1] for x in prof.values()), 4)}
+               for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    # end to end: inputs from pinned host memory, gradients back to it
+    pin = {k: (None if v is None else v.pin_memory()) for k, v in inp_cpu.items()}
+    pdout = dout_cpu.pin_memory()
+    grads0 = step()
+    hgrad = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype).pin_memory())
+             for k, v in grads0.items()}
+
+    def host_step():
+        for k, v in pin.items():
+            if v is not None:
+                inp[k].copy_(v, non_blocking=True)
+        dout.copy_(pdout, non_blocking=True)
+        g = step()
+        for k, v in g.items():
+            if v is not None:
+                hgrad[k].copy_(v, non_blocking=True)
+
+    for _ in range(args.warmup):
+        host_step()
+    torch.cuda.synchronize(dev)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for _ in range(args.steps):
+        host_step()
+    h1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = h0.elapsed_time(h1) / args.steps
+    h2d = sum(t.numel() * t.element_size() for t in pin.values() if t is not None) + \
+        pdout.numel() * pdout.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in hgrad.values() if t is not None)
+    tok = w.tokens
+    line = {
+        "metric": "TTT-layer backward tokens/s at 1 B200", "value": tok / (ms_step / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == BF16 else "f32",
+        "data": "synthetic (seeded normal q/k/v/dout, softplus lr, random-init fast weights)",
+        "config": dict(workload_config(w, 1), **{"pass": "backward (lact_ttt_bwd)"}),
+        "peak_frac": {"algorithmic_tflops": flops / (ms_step / 1e3) / 1e12,
+                      "frac_of_sustained_bf16": flops / (ms_step / 1e3) / 1e12 / pk_sust,
+                      "frac_of_fp32_fma": flops / (ms_step / 1e3) / 1e12 / FP32_FMA_TFLOPS},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": tok / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clk,
+    }
+    # the autograd oracle on whole (batch, head) sequences, until the budget
+    from oracle import lact_oracle_bwd as ob
+    heads, t0, done = [(b, h) for b in range(w.B) for h in range(w.H)], time.perf_counter(), 0
+    while done < len(heads) and (done == 0 or time.perf_counter() - t0 < args.cpu_budget):
+        b, h = heads[done]
+        sl = {k: (None if v is None else v[b:b + 1, h:h + 1]) for k, v in inp_cpu.items()
+              if k in ("q", "k", "v", "lr", "beta")}
+        ob.ttt_layer_bwd(sl["q"], sl["k"], sl["v"], sl["lr"], sl["beta"], inp_cpu["w1"][h:h + 1],
+                         inp_cpu["w2"][h:h + 1], inp_cpu["w3"][h:h + 1], w.chunk, w.order, w.rule,
+                         dout_cpu[b:b + 1, h:h + 1])
+        done += 1
+    sec = time.perf_counter() - t0
+    tok_done = done * (w.T if w.Tq == w.T else w.T + w.Tq)
+    line["cpu_baseline"] = {"value": tok_done / sec, "unit": "tokens/s", "cores": torch.get_num_threads(),
+                            "kind": "oracle",
+                            "sample": f"autograd backward oracle on {done} of {len(heads)} "
+                                      f"(batch, head) sequences, {tok_done} tokens, {sec:.1f} s"}
+    print(json.dumps(line), flush=True)
     return 0
 
 

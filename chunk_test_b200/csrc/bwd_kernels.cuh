@@ -60,7 +60,8 @@ struct RenormBwdParams {
   const float* Wc;      // W^c (after renorm)
   const float* Wp;      // W^{c-1}
   const float* mnorm;   // |W'_r| per row (rule row order)
-  float* Gam;           // out: dL/dG
+  float* Gam;           // out: dL/dG (fp32), or null
+  __nv_bfloat16* Gam16; // out: dL/dG (bf16), or null
   float* Ap;            // out: dL/dW^{c-1}, the renorm and direct parts
   int rule;             // 0 GD, 1 momentum
   float* Bm;            // momentum: dL/dM^c in, dL/dM^{c-1} out
@@ -106,14 +107,17 @@ __global__ void __launch_bounds__(256) k_renorm_bwd(const RenormBwdParams p) {
     const float u = p.Wc[o] * inv_n;
     const float D = g * (p.A[o] - u * dot);
     p.Ap[o] = D + dot * p.Wp[o] * inv_n;
+    float gam;
     if (p.rule == 1) {
       const float E = p.Bm[o] - D;
-      p.Gam[o] = E;
+      gam = E;
       pe -= E * p.Mprev[o];   // <E, M^{c-1}>, Mprev holding -M^{c-1}
       p.Bm[o] = bb * E;
     } else {
-      p.Gam[o] = -D;
+      gam = -D;
     }
+    if (p.Gam) p.Gam[o] = gam;
+    if (p.Gam16) p.Gam16[o] = __float2bfloat16_rn(gam);
   }
   if (p.rule == 1) {
     pe = warp_sum(pe);
@@ -151,6 +155,29 @@ __global__ void __launch_bounds__(256) k_head_dbeta(const float* __restrict__ pa
 
 __device__ __forceinline__ float sigm(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// The second-order factors of one element: the partials of phi with respect
+// to (z1, u, z3, p, q, r), and the element's terms of dphi/dlr.
+struct HvpOut { float fz1, fu, fz3, fp, fq, fr, g1, g2, g3; };
+__device__ __forceinline__ HvpOut hvp_factors(float z1, float u, float z3, float pp, float qq, float rr,
+                                              float e1, float e2, float e3) {
+  const float sg = 1.0f / (1.0f + expf(-z1));
+  const float s = z1 * sg;
+  const float sp = sg * (1.0f + z1 * (1.0f - sg));
+  const float spp = sg * (1.0f - sg) * (2.0f + z1 * (1.0f - 2.0f * sg));
+  const float a1 = u * z3 * sp, a3 = u * s, h = s * z3;
+  HvpOut o;
+  o.fz1 = -(e1 * u * z3 * spp * pp + e3 * u * sp * rr + e2 * qq * z3 * sp);
+  o.fu = -(e1 * z3 * sp * pp + e3 * s * rr);
+  o.fz3 = -(e1 * u * sp * pp + e2 * qq * s);
+  o.fp = -e1 * a1;
+  o.fq = -e2 * h;
+  o.fr = -e3 * a3;
+  o.g1 = -a1 * pp;
+  o.g2 = -qq * h;
+  o.g3 = -a3 * rr;
+  return o;
+}
+
 // Second-order factors of the gradient step, one warp per (head, token row).
 // In: Z = (z1, u, z3), Pz = (p, q, r) as [3][BH][rows][dh] planes.  Out, in
 // place: Z = (dphi/dz1, dphi/du, dphi/dz3), Pz = (dphi/dp, dphi/dq,
@@ -172,22 +199,17 @@ __global__ void __launch_bounds__(256) k_hvp_elem(float* __restrict__ Z, float* 
   float g1 = 0.f, g2 = 0.f, g3 = 0.f;
   for (int c = lane; c < dh; c += 32) {
     const int64_t o = base + c;
-    const float z1 = Z[o], u = Z[plane + o], z3 = Z[2 * plane + o];
-    const float pp = Pz[o], qq = Pz[plane + o], rr = Pz[2 * plane + o];
-    const float sg = sigm(z1);
-    const float s = z1 * sg;
-    const float sp = sg * (1.0f + z1 * (1.0f - sg));
-    const float spp = sg * (1.0f - sg) * (2.0f + z1 * (1.0f - 2.0f * sg));
-    const float a1 = u * z3 * sp, a3 = u * s, h = s * z3;
-    Z[o] = -(e1 * u * z3 * spp * pp + e3 * u * sp * rr + e2 * qq * z3 * sp);
-    Z[plane + o] = -(e1 * z3 * sp * pp + e3 * s * rr);
-    Z[2 * plane + o] = -(e1 * u * sp * pp + e2 * qq * s);
-    Pz[o] = -e1 * a1;
-    Pz[plane + o] = -e2 * h;
-    Pz[2 * plane + o] = -e3 * a3;
-    g1 -= a1 * pp;
-    g2 -= qq * h;
-    g3 -= a3 * rr;
+    const HvpOut f = hvp_factors(Z[o], Z[plane + o], Z[2 * plane + o], Pz[o], Pz[plane + o],
+                                 Pz[2 * plane + o], e1, e2, e3);
+    Z[o] = f.fz1;
+    Z[plane + o] = f.fu;
+    Z[2 * plane + o] = f.fz3;
+    Pz[o] = f.fp;
+    Pz[plane + o] = f.fq;
+    Pz[2 * plane + o] = f.fr;
+    g1 += f.g1;
+    g2 += f.g2;
+    g3 += f.g3;
   }
   g1 = warp_sum(g1);
   g2 = warp_sum(g2);
@@ -197,6 +219,124 @@ __global__ void __launch_bounds__(256) k_hvp_elem(float* __restrict__ Z, float* 
     o[0] = g1;
     o[1] = g2;
     o[2] = g3;
+  }
+}
+
+// The same factors as bf16 operands for the tensor-core contractions: Phi =
+// (dz1, du, dz3, dp, dq, dr) as [6][BH][rows][dh]; rows n..rows-1 of every
+// head are written as zeros (the contractions over tokens run in 64-row
+// blocks).  One warp per (head, row).
+__global__ void __launch_bounds__(256) k_hvp_elem_bf16(const float* __restrict__ Z,
+                                                       const float* __restrict__ Pz, int BH, int64_t rows,
+                                                       int dh, int n, const float* __restrict__ lr,
+                                                       int64_t T, int64_t row0, float* __restrict__ dlr,
+                                                       __nv_bfloat16* __restrict__ Phi) {
+  griddep_launch();
+  griddep_wait();
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<int64_t>(BH) * rows) return;
+  const int64_t bh = w / rows, i = w % rows;
+  const int64_t plane = static_cast<int64_t>(BH) * rows * dh;
+  const int64_t base = (bh * rows + i) * dh;
+  if (i >= n) {
+    for (int c = lane; c < dh; c += 32)
+      for (int j = 0; j < 6; ++j) Phi[j * plane + base + c] = __float2bfloat16_rn(0.f);
+    return;
+  }
+  const float* l = lr + (bh * T + row0 + i) * 3;
+  const float e1 = l[0], e2 = l[1], e3 = l[2];
+  float g1 = 0.f, g2 = 0.f, g3 = 0.f;
+  for (int c = lane; c < dh; c += 32) {
+    const int64_t o = base + c;
+    const HvpOut f = hvp_factors(Z[o], Z[plane + o], Z[2 * plane + o], Pz[o], Pz[plane + o],
+                                 Pz[2 * plane + o], e1, e2, e3);
+    Phi[o] = __float2bfloat16_rn(f.fz1);
+    Phi[plane + o] = __float2bfloat16_rn(f.fu);
+    Phi[2 * plane + o] = __float2bfloat16_rn(f.fz3);
+    Phi[3 * plane + o] = __float2bfloat16_rn(f.fp);
+    Phi[4 * plane + o] = __float2bfloat16_rn(f.fq);
+    Phi[5 * plane + o] = __float2bfloat16_rn(f.fr);
+    g1 += f.g1;
+    g2 += f.g2;
+    g3 += f.g3;
+  }
+  g1 = warp_sum(g1);
+  g2 = warp_sum(g2);
+  g3 = warp_sum(g3);
+  if (lane == 0) {
+    float* o = dlr + (bh * T + row0 + i) * 3;
+    o[0] = g1;
+    o[1] = g2;
+    o[2] = g3;
+  }
+}
+
+// The keys' gradient factors of the forward recompute as bf16 operands:
+// E = (lr1 u z3 silu'(z1), lr2 silu(z1) z3, lr3 u silu(z1)) from Z = (z1, u,
+// z3), [3][BH][rows][dh]; rows n..rows-1 written as zeros.
+__global__ void __launch_bounds__(256) k_key_factors_bf16(const float* __restrict__ Z, int BH, int64_t rows,
+                                                          int dh, int n, const float* __restrict__ lr,
+                                                          int64_t T, int64_t row0,
+                                                          __nv_bfloat16* __restrict__ E) {
+  griddep_launch();
+  griddep_wait();
+  const int64_t plane = static_cast<int64_t>(BH) * rows * dh;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < plane; i += stride) {
+    const int64_t r = (i / dh) % rows, bh = i / (rows * dh);
+    float e1 = 0.f, eh = 0.f, e3 = 0.f;
+    if (r < n) {
+      const float z1 = Z[i], u = Z[plane + i], z3 = Z[2 * plane + i];
+      const float sg = 1.0f / (1.0f + expf(-z1));
+      const float s = z1 * sg;
+      const float* l = lr + (bh * T + row0 + r) * 3;
+      e1 = l[0] * u * z3 * sg * (1.0f + z1 * (1.0f - sg));
+      eh = l[1] * s * z3;
+      e3 = l[2] * u * s;
+    }
+    E[i] = __float2bfloat16_rn(e1);
+    E[plane + i] = __float2bfloat16_rn(eh);
+    E[2 * plane + i] = __float2bfloat16_rn(e3);
+  }
+}
+
+// bf16 copy of y = s[r] * x[r][:] (the scaled output gradient).
+__global__ void __launch_bounds__(256) k_scale_rows_bf16(const __nv_bfloat16* __restrict__ x,
+                                                         const float* __restrict__ s,
+                                                         __nv_bfloat16* __restrict__ y, int64_t rows, int d) {
+  griddep_launch();
+  griddep_wait();
+  const int64_t n = rows * d;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
+    y[i] = __float2bfloat16_rn(s[i / d] * __bfloat162float(x[i]));
+}
+
+// Apply backward as bf16 operands: from Zq = (z1, g, z3) fp32 planes
+// [3][BH][rows][dh] (g = dO W2, dO already scaled) write out = (dz1, hq, dz3)
+// bf16, rows n..rows-1 of every head as zeros.
+__global__ void __launch_bounds__(256) k_apply_bwd_elem_bf16(const float* __restrict__ Zq, int BH,
+                                                             int64_t rows, int dh, int n,
+                                                             __nv_bfloat16* __restrict__ out) {
+  griddep_launch();
+  griddep_wait();
+  const int64_t plane = static_cast<int64_t>(BH) * rows * dh;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < plane; i += stride) {
+    const int64_t r = (i / dh) % rows;
+    float dz1 = 0.f, hq = 0.f, dz3 = 0.f;
+    if (r < n) {
+      const float z1 = Zq[i], g = Zq[plane + i], z3 = Zq[2 * plane + i];
+      const float sg = 1.0f / (1.0f + expf(-z1));
+      const float s = z1 * sg;
+      dz1 = g * z3 * sg * (1.0f + z1 * (1.0f - sg));
+      hq = s * z3;
+      dz3 = g * s;
+    }
+    out[i] = __float2bfloat16_rn(dz1);
+    out[plane + i] = __float2bfloat16_rn(hq);
+    out[2 * plane + i] = __float2bfloat16_rn(dz3);
   }
 }
 

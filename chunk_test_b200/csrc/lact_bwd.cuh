@@ -1,7 +1,7 @@
 // lact_bwd.cuh -- host side of the layer's backward (lact_ttt_bwd), included
 // by lact_api.cu after the forward's planning and launch helpers.
 //
-// The backward is the vector-Jacobian product of the forward, in fp32:
+// The backward is the vector-Jacobian product of the forward:
 //   1. the prologue and the updates of the forward are recomputed (the
 //      outputs are not needed), keeping every state W^c, the momentum before
 //      each update and the row norms |W'_r| before each renorm;
@@ -13,7 +13,11 @@
 //      contractions;
 //   3. the prologue's backward gives dq and dk; the initial weights'
 //      gradient is summed over the batch when the batch shares it.
-// Every contraction is a batched k_simt_gemm over the B*H heads.
+// fp32 problems run every contraction as a batched k_simt_gemm over the B*H
+// heads in fp32.  bf16 problems run them on the tensor cores (GemmOp, bf16
+// operands through TMA, fp32 accumulation); the elementwise kernels write
+// their results as bf16 operands, and the states, the gradients being
+// accumulated (dL/dW, dk^, dq^, dv) and all reductions stay fp32.
 #pragma once
 
 #include "bwd_kernels.cuh"
@@ -36,6 +40,8 @@ struct BwdBufs {
   float *Z, *Pz, *E, *P;
   float *A, *Ap, *Gam, *Bm;
   float *dqh, *dkh, *ofull, *part;
+  // bf16 problems (tensor-core contractions): bf16 operands
+  __nv_bfloat16 *qh16, *kh16, *dos16, *hist16, *op16, *Gam16;
   int64_t zr;   // rows per head of the per-chunk [rows][dh] planes
 };
 
@@ -48,15 +54,24 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
   const bool bf = D.dtype == LACT_BF16;
   const bool mom = D.rule == LACT_RULE_MOMENTUM;
   b.zr = std::max<int64_t>(D.chunk, D.nch == 1 ? D.Tq : D.chunk);
+  const int64_t zpl = D.BH * b.zr * D.dh;
   if (bf) {
-    b.q32 = bp.take<float>(nq);
+    b.q32 = bp.take<float>(nq);          // raw q, k for the prologue's backward
     b.k32 = bp.take<float>(nk);
-    b.v32 = bp.take<float>(nk);
-    b.do32 = bp.take<float>(nq);
+    b.do32 = bp.take<float>(nq);         // dout, for the scale's gradient
+    b.qh16 = bp.take<__nv_bfloat16>(nq);
+    b.kh16 = bp.take<__nv_bfloat16>(nk);
+    b.dos16 = bp.take<__nv_bfloat16>(nq);
+    b.hist16 = bp.take<__nv_bfloat16>((D.nch + 1) * planes);
+    b.op16 = bp.take<__nv_bfloat16>(6 * zpl);
+    b.Gam16 = bp.take<__nv_bfloat16>(planes);
+  } else {
+    b.dos32 = bp.take<float>(nq);
+    b.qh = bp.take<float>(nq);
+    b.kh = bp.take<float>(nk);
+    b.E = bp.take<float>(3 * zpl);
+    b.Gam = bp.take<float>(planes);
   }
-  b.dos32 = bp.take<float>(nq);
-  b.qh = bp.take<float>(nq);
-  b.kh = bp.take<float>(nk);
   b.hist = bp.take<float>((D.nch + 1) * planes);
   if (mom) {
     b.mh = bp.take<float>(D.nch * planes);
@@ -66,14 +81,11 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
     b.part = bp.take<float>(rule_rows(D));
   }
   b.mnorm = bp.take<float>(D.nch * rule_rows(D));
-  const int64_t zpl = D.BH * b.zr * D.dh;
   b.Z = bp.take<float>(3 * zpl);
   b.Pz = bp.take<float>(3 * zpl);
-  b.E = bp.take<float>(3 * zpl);
   b.P = bp.take<float>(planes);
   b.A = bp.take<float>(planes);
   b.Ap = bp.take<float>(planes);
-  b.Gam = bp.take<float>(planes);
   b.dqh = bp.take<float>(nq);
   b.dkh = bp.take<float>(nk);
   b.ofull = bp.take<float>(nq);
@@ -90,9 +102,10 @@ static unsigned grid_for(int64_t n, int per_thread = 1) {
   return static_cast<unsigned>(std::min<int64_t>(std::max<int64_t>(cdiv(n, 256LL * per_thread), 1), 148 * 32));
 }
 
-static void run_bwd(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaStream_t st, Launcher& L) {
+// fp32 problems: every contraction on the CUDA cores in fp32.
+static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaStream_t st, Launcher& L) {
   L.st = st;
-  const bool bf = D.dtype == LACT_BF16, mom = D.rule == LACT_RULE_MOMENTUM;
+  const bool mom = D.rule == LACT_RULE_MOMENTUM;
   const int BH = static_cast<int>(D.BH), d = static_cast<int>(D.d), dh = static_cast<int>(D.dh);
   const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane, jst = D.BH * plane;
   const int64_t nq = D.BH * D.Tq * D.d, nk = D.BH * D.T * D.d;
@@ -121,22 +134,11 @@ static void run_bwd(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaSt
     });
   };
 
-  // ---- fp32 inputs, the scaled output gradient, zeroed accumulators
-  const float* q32 = bf ? b.q32 : static_cast<const float*>(in.q);
-  const float* k32 = bf ? b.k32 : static_cast<const float*>(in.k);
-  const float* v32 = bf ? b.v32 : static_cast<const float*>(in.v);
-  const float* do32 = bf ? b.do32 : static_cast<const float*>(in.dout);
-  if (bf) {
-    const void* src[4] = {in.q, in.k, in.v, in.dout};
-    float* dst[4] = {b.q32, b.k32, b.v32, b.do32};
-    const int64_t n[4] = {nq, nk, nk, nq};
-    for (int i = 0; i < 4; ++i)
-      L(K_BWD_ELEM, [&] {
-        (void)launch_pdl(k_bf16_to_f32, grid_for(n[i], 4), 256, 0, st,
-                         static_cast<const __nv_bfloat16*>(src[i]), dst[i], n[i]);
-        return cudaGetLastError();
-      });
-  }
+  // ---- the scaled output gradient, zeroed accumulators
+  const float* q32 = static_cast<const float*>(in.q);
+  const float* k32 = static_cast<const float*>(in.k);
+  const float* v32 = static_cast<const float*>(in.v);
+  const float* do32 = static_cast<const float*>(in.dout);
   const float* dos = do32;
   if (in.scale) {
     L(K_BWD_ELEM, [&] {
@@ -331,6 +333,281 @@ static void run_bwd(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaSt
                      static_cast<int>(D.B), static_cast<int>(D.H), plane, D.w_shared, in.dw1, in.dw2, in.dw3);
     return cudaGetLastError();
   });
+}
+
+// One bf16 operand: a dense [batch][rows][inner] tensor.
+struct Opnd {
+  const void* p;
+  int64_t inner, rows, batch;
+};
+
+static int pick_bn(int64_t n) {
+  if (n <= 256) return static_cast<int>(n);
+  if (n % 256 == 0) return 256;
+  if (n % 192 == 0) return 192;
+  if (n % 128 == 0) return 128;
+  return 64;
+}
+
+// bf16 problems: the contractions on the tensor cores.
+static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaStream_t st, Launcher& L) {
+  L.st = st;
+  const bool mom = D.rule == LACT_RULE_MOMENTUM;
+  const int BH = static_cast<int>(D.BH), d = static_cast<int>(D.d), dh = static_cast<int>(D.dh);
+  const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane, jst = D.BH * plane;
+  const int64_t nq = D.BH * D.Tq * D.d, nk = D.BH * D.T * D.d;
+  const int64_t zr = b.zr, zpl = D.BH * zr * D.dh, rows_all = rule_rows(D);
+  using B16 = __nv_bfloat16;
+  auto memop = [&](cudaError_t e) {
+    if (!L.dry && L.err == LACT_OK && e != cudaSuccess) L.err = LACT_ECUDA;
+  };
+  auto zero = [&](void* p, int64_t bytes) {
+    if (!L.dry && p) memop(cudaMemsetAsync(p, 0, static_cast<size_t>(bytes), st));
+  };
+  auto copy = [&](void* dst, const void* src, int64_t bytes) {
+    if (!L.dry) memop(cudaMemcpyAsync(dst, src, static_cast<size_t>(bytes), cudaMemcpyDeviceToDevice, st));
+  };
+  // out[item] (+)= A(item) B(item)^T with A [M x K], B [N x K] per head, both
+  // bf16 through TMA: K-major A read from row a_m0, MN-major operands from K
+  // coordinate a_k0 / b_k0; rows of out past M are not written.
+  auto tcg = [&](auto a_mn, auto b_mn, Opnd a, int a_m0, int a_k0, Opnd bo, int b_k0, int M, int N, int K,
+                 float* out, int64_t out_item, int64_t ld, bool acc) {
+    constexpr bool AMN = decltype(a_mn)::value, BMN = decltype(b_mn)::value;
+    L(K_BWD_GEMM, [&] {
+      GemmParams g = gemm_params();
+      const int bn = pick_bn(N);
+      if (!map3d(&g.tmA, a.p, a.inner, a.rows, a.batch, 64, AMN ? 64 : 128) ||
+          !map3d(&g.tmB, bo.p, bo.inner, bo.rows, bo.batch, 64, BMN ? 64 : bn))
+        return cudaErrorInvalidValue;
+      g.items = BH; g.kb_count = g.kb_total = static_cast<int>(cdiv(K, 64));
+      g.a_m0 = a_m0; g.a_k0 = a_k0; g.b_k0 = b_k0;
+      g.zb_mod = BH; g.m_valid = M;
+      g.outf = out; g.item_stride = out_item; g.ld = ld;
+      if (acc) { g.beta = 1.0f; g.cin = out; }
+      return launch_gemm<AMN, BMN>(bn, dim3(N / bn, cdiv(M, 128), BH), g, st);
+    });
+  };
+  const std::false_type KM;   // K-major operand
+  const std::true_type MN;    // MN-major operand
+  const Opnd qh{b.qh16, D.d, D.Tq, D.BH}, kh{b.kh16, D.d, D.T, D.BH}, vv{in.v, D.d, D.T, D.BH};
+  auto Wop = [&](const B16* W, int j) {   // plane j of a state: W1, W3 [dh][d]; W2 [d][dh]
+    return j == 1 ? Opnd{W + jst, D.dh, D.d, D.BH} : Opnd{W + j * jst, D.d, D.dh, D.BH};
+  };
+  auto op = [&](int j) { return Opnd{b.op16 + j * zpl, D.dh, zr, D.BH}; };
+
+  // ---- raw fp32 q, k (prologue backward), dout (scale gradient), bf16 q^, k^
+  {
+    const void* src[3] = {in.q, in.k, in.dout};
+    float* dst[3] = {b.q32, b.k32, b.do32};
+    const int64_t n[3] = {nq, nk, nq};
+    for (int i = 0; i < 3; ++i) {
+      if (i == 2 && !in.scale) continue;
+      L(K_BWD_ELEM, [&] {
+        (void)launch_pdl(k_bf16_to_f32, grid_for(n[i], 4), 256, 0, st, static_cast<const B16*>(src[i]), dst[i],
+                         n[i]);
+        return cudaGetLastError();
+      });
+    }
+  }
+  const B16* dos16 = static_cast<const B16*>(in.dout);
+  if (in.scale) {
+    L(K_BWD_ELEM, [&] {
+      (void)launch_pdl(k_scale_rows_bf16, grid_for(nq, 4), 256, 0, st, static_cast<const B16*>(in.dout),
+                       in.scale, b.dos16, D.BH * D.Tq, d);
+      return cudaGetLastError();
+    });
+    dos16 = b.dos16;
+  }
+  const Opnd dos{dos16, D.d, D.Tq, D.BH};
+  zero(in.dlr, D.BH * D.T * 3 * 4);
+  if (mom) zero(in.dbeta, D.BH * D.T * 4);
+  zero(in.dv, nk * 4);
+  zero(b.dqh, nq * 4);
+  zero(b.dkh, nk * 4);
+  if (mom) zero(b.Bm, planes * 4);
+  const float* dwf[3] = {in.dw1f, in.dw2f, in.dw3f};
+  for (int j = 0; j < 3; ++j) {
+    if (dwf[j]) copy(b.A + j * jst, dwf[j], jst * 4);
+    else zero(b.A + j * jst, jst * 4);
+  }
+  L(K_PROLOGUE, [&] {
+    constexpr int ROWS = 4;
+    const int64_t rows = D.BH * D.Tq + D.BH * D.T;
+    const int nv = d / 8;
+    auto launch = [&](auto kern, int S) {
+      (void)launch_pdl(kern, static_cast<unsigned>(cdiv(cdiv(rows, ROWS) * S, 256)), 256, 0, st,
+                       static_cast<const B16*>(in.q), b.qh16, D.BH * D.Tq, static_cast<const B16*>(in.k), b.kh16,
+                       D.BH * D.T, d, static_cast<B16*>(nullptr));
+    };
+    if (nv <= 8) launch(k_qk_prologue_bf16<8, 1, ROWS, false>, 8);
+    else if (nv <= 16) launch(k_qk_prologue_bf16<16, 1, ROWS, false>, 16);
+    else if (nv <= 32) launch(k_qk_prologue_bf16<32, 1, ROWS, false>, 32);
+    else launch(k_qk_prologue_bf16<32, 2, ROWS, false>, 32);
+    return cudaGetLastError();
+  });
+  L(K_INIT, [&] {
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(planes, 1024), 148 * 16));
+    (void)launch_pdl(k_init_state, blocks, 256, 0, st, in.w1, in.w2, in.w3, static_cast<int>(D.H), D.w_shared,
+                     BH, d, dh, b.hist, b.hist16, static_cast<B16*>(nullptr), mom ? b.Mm : nullptr,
+                     static_cast<const float*>(nullptr), static_cast<const float*>(nullptr),
+                     static_cast<const float*>(nullptr));
+    return cudaGetLastError();
+  });
+  if (mom) {
+    L(K_BETA_MEAN, [&] {
+      const int64_t w = D.BH * D.nch;
+      (void)launch_pdl(k_beta_mean, static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st, in.beta, BH, D.T,
+                       D.chunk, static_cast<int>(D.nch), b.bbar);
+      return cudaGetLastError();
+    });
+  }
+  // the keys' forward at a state W (bf16): out = (k^ W1^T, v W2, k^ W3^T), rows of chunk c
+  auto key_forward = [&](const B16* W, int64_t c0, int nc, float* out) {
+    tcg(KM, KM, kh, static_cast<int>(c0), 0, Wop(W, 0), 0, nc, dh, d, out, zr * D.dh, dh, false);
+    tcg(KM, MN, vv, static_cast<int>(c0), 0, Wop(W, 1), 0, nc, dh, d, out + zpl, zr * D.dh, dh, false);
+    tcg(KM, KM, kh, static_cast<int>(c0), 0, Wop(W, 2), 0, nc, dh, d, out + 2 * zpl, zr * D.dh, dh, false);
+  };
+
+  // ---- forward recompute: the states, momenta and pre-renorm row norms
+  for (int64_t c = 0; c < D.nch; ++c) {
+    const int64_t c0 = c * D.chunk;
+    const int nc = static_cast<int>(std::min(c0 + D.chunk, D.T) - c0);
+    copy(b.hist + (c + 1) * planes, b.hist + c * planes, planes * 4);
+    copy(b.hist16 + (c + 1) * planes, b.hist16 + c * planes, planes * 2);
+    if (in.mask && in.mask[c] == 0) continue;
+    if (mom) copy(b.mh + c * planes, b.Mm, planes * 4);
+    key_forward(b.hist16 + c * planes, c0, nc, b.Z);
+    L(K_BWD_ELEM, [&] {
+      (void)launch_pdl(k_key_factors_bf16, grid_for(zpl, 4), 256, 0, st, b.Z, BH, zr, dh, nc, in.lr, D.T, c0,
+                       b.op16);
+      return cudaGetLastError();
+    });
+    L(K_BWD_GEMM, [&] {   // -G = E^T [k^, v, k^] over the chunk, W2's plane stored transposed
+      GemmParams g = gemm_params();
+      if (!map3d(&g.tmA, b.op16, dh, zr, 3 * BH, 64, 64) || !map3d(&g.tmB, b.kh16, d, D.T, BH, 64, 64) ||
+          !map3d(&g.tmB2, in.v, d, D.T, BH, 64, 64))
+        return cudaErrorInvalidValue;
+      const int bn = pick_bn(D.d);
+      g.items = 3 * BH; g.kb_count = g.kb_total = static_cast<int>(cdiv(nc, 64));
+      g.a_k0 = 0; g.b_k0 = static_cast<int>(c0);
+      g.zb_mod = BH; g.alt_group = 1; g.m_valid = dh;
+      g.outf = b.P; g.item_stride = plane; g.ld = d;
+      g.tr_group = 1; g.tr_mod = BH; g.ld_t = dh;
+      return launch_gemm<true, true>(bn, dim3(d / bn, cdiv(dh, 128), 3 * BH), g, st);
+    });
+    L(K_RULE, [&] {
+      RuleParams r;
+      std::memset(&r, 0, sizeof(r));
+      r.Wm = b.hist + (c + 1) * planes; r.Ws = b.hist16 + (c + 1) * planes; r.S = b.P; r.splits = 1;
+      r.split_stride = planes; r.Mm = mom ? b.Mm : nullptr; r.beta_bar = b.bbar;
+      r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c); r.rule = D.rule;
+      r.BH = BH; r.dh = dh; r.d = d; r.nrm_out = b.mnorm + c * rows_all;
+      (void)launch_pdl(k_rule_renorm, static_cast<unsigned>(cdiv(rows_all * 32, 256)), 256, 0, st, r);
+      return cudaGetLastError();
+    });
+  }
+
+  // ---- reverse chunk loop
+  float* A = b.A;
+  float* Ap = b.Ap;
+  auto apply_bwd = [&](const B16* W, int64_t qr0, int nq_c) {
+    const int r0 = static_cast<int>(qr0);
+    tcg(KM, KM, qh, r0, 0, Wop(W, 0), 0, nq_c, dh, d, b.Z, zr * D.dh, dh, false);
+    tcg(KM, MN, dos, r0, 0, Wop(W, 1), 0, nq_c, dh, d, b.Z + zpl, zr * D.dh, dh, false);
+    tcg(KM, KM, qh, r0, 0, Wop(W, 2), 0, nq_c, dh, d, b.Z + 2 * zpl, zr * D.dh, dh, false);
+    L(K_BWD_ELEM, [&] {   // -> op16 planes (dz1, hq, dz3)
+      (void)launch_pdl(k_apply_bwd_elem_bf16, grid_for(zpl, 4), 256, 0, st, b.Z, BH, zr, dh, nq_c, b.op16);
+      return cudaGetLastError();
+    });
+    // dW1 += dz1^T q^, dW3 += dz3^T q^, dW2 += dO^T hq
+    tcg(MN, MN, op(0), 0, 0, qh, r0, dh, d, nq_c, A, plane, d, true);
+    tcg(MN, MN, op(2), 0, 0, qh, r0, dh, d, nq_c, A + 2 * jst, plane, d, true);
+    tcg(MN, MN, dos, 0, r0, op(1), 0, d, dh, nq_c, A + jst, plane, dh, true);
+    // dq^ += dz1 W1 + dz3 W3
+    tcg(KM, MN, op(0), 0, 0, Wop(W, 0), 0, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
+    tcg(KM, MN, op(2), 0, 0, Wop(W, 2), 0, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
+    if (in.scale)   // the unscaled output hq W2^T, for the scale's gradient
+      tcg(KM, KM, op(1), 0, 0, Wop(W, 1), 0, nq_c, d, dh, b.ofull + qr0 * d, D.Tq * D.d, d, false);
+  };
+  for (int64_t c = D.nch - 1; c >= 0; --c) {
+    const int64_t c0 = c * D.chunk;
+    const int nc = static_cast<int>(std::min(c0 + D.chunk, D.T) - c0);
+    const int64_t qr0 = D.nch == 1 ? 0 : c0;
+    const int nq_c = static_cast<int>(D.nch == 1 ? D.Tq : nc);
+    const B16* Wp16 = b.hist16 + c * planes;
+    const B16* Wc16 = b.hist16 + (c + 1) * planes;
+    const bool upd = !in.mask || in.mask[c] != 0;
+    if (D.order == LACT_UPDATE_THEN_APPLY) apply_bwd(Wc16, qr0, nq_c);
+    if (upd) {
+      L(K_BWD_ELEM, [&] {
+        RenormBwdParams r;
+        std::memset(&r, 0, sizeof(r));
+        r.A = A; r.Wc = b.hist + (c + 1) * planes; r.Wp = b.hist + c * planes; r.mnorm = b.mnorm + c * rows_all;
+        r.Gam16 = b.Gam16; r.Ap = Ap; r.rule = D.rule; r.Bm = b.Bm;
+        r.Mprev = mom ? b.mh + c * planes : nullptr; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch);
+        r.chunk_idx = static_cast<int>(c); r.part = b.part; r.BH = BH; r.dh = dh; r.d = d;
+        (void)launch_pdl(k_renorm_bwd, static_cast<unsigned>(cdiv(rows_all * 32, 256)), 256, 0, st, r);
+        return cudaGetLastError();
+      });
+      if (mom)
+        L(K_BWD_ELEM, [&] {
+          (void)launch_pdl(k_head_dbeta, static_cast<unsigned>(BH), 256, 0, st, b.part, BH, dh, d, D.T, c0, nc,
+                           in.dbeta);
+          return cudaGetLastError();
+        });
+      key_forward(Wp16, c0, nc, b.Z);       // (z1, u, z3)
+      key_forward(b.Gam16, c0, nc, b.Pz);   // (p, q, r)
+      L(K_BWD_ELEM, [&] {   // -> op16 planes (dz1, du, dz3, dp, dq, dr)
+        (void)launch_pdl(k_hvp_elem_bf16, static_cast<unsigned>(cdiv(D.BH * zr * 32, 256)), 256, 0, st, b.Z,
+                         b.Pz, BH, zr, dh, nc, in.lr, D.T, c0, in.dlr, b.op16);
+        return cudaGetLastError();
+      });
+      const int k0 = static_cast<int>(c0);
+      // dW1 += dz1^T k^, dW3 += dz3^T k^, dW2 += v^T du
+      tcg(MN, MN, op(0), 0, 0, kh, k0, dh, d, nc, Ap, plane, d, true);
+      tcg(MN, MN, op(2), 0, 0, kh, k0, dh, d, nc, Ap + 2 * jst, plane, d, true);
+      tcg(MN, MN, vv, 0, k0, op(1), 0, d, dh, nc, Ap + jst, plane, dh, true);
+      // dk^ += dz1 W1 + dz3 W3 + dp Gam1 + dr Gam3
+      tcg(KM, MN, op(0), 0, 0, Wop(Wp16, 0), 0, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d, true);
+      tcg(KM, MN, op(2), 0, 0, Wop(Wp16, 2), 0, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d, true);
+      tcg(KM, MN, op(3), 0, 0, Wop(b.Gam16, 0), 0, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d, true);
+      tcg(KM, MN, op(5), 0, 0, Wop(b.Gam16, 2), 0, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d, true);
+      // dv += du W2^T + dq Gam2^T
+      tcg(KM, KM, op(1), 0, 0, Wop(Wp16, 1), 0, nc, d, dh, in.dv + c0 * d, D.T * D.d, d, true);
+      tcg(KM, KM, op(4), 0, 0, Wop(b.Gam16, 1), 0, nc, d, dh, in.dv + c0 * d, D.T * D.d, d, true);
+      std::swap(A, Ap);
+    }
+    if (D.order == LACT_APPLY_THEN_UPDATE) apply_bwd(Wp16, qr0, nq_c);
+  }
+
+  // ---- prologue backward, the scale's gradient, the initial weights' gradient
+  L(K_BWD_ELEM, [&] {
+    (void)launch_pdl(k_prologue_bwd, static_cast<unsigned>(cdiv(D.BH * D.Tq * 32, 256)), 256, 0, st,
+                     static_cast<const float*>(b.q32), static_cast<const float*>(b.dqh), in.dq, D.BH * D.Tq, d);
+    return cudaGetLastError();
+  });
+  L(K_BWD_ELEM, [&] {
+    (void)launch_pdl(k_prologue_bwd, static_cast<unsigned>(cdiv(D.BH * D.T * 32, 256)), 256, 0, st,
+                     static_cast<const float*>(b.k32), static_cast<const float*>(b.dkh), in.dk, D.BH * D.T, d);
+    return cudaGetLastError();
+  });
+  if (in.scale)
+    L(K_BWD_ELEM, [&] {
+      (void)launch_pdl(k_rowdot, static_cast<unsigned>(cdiv(D.BH * D.Tq * 32, 256)), 256, 0, st,
+                       static_cast<const float*>(b.do32), static_cast<const float*>(b.ofull), in.dscale,
+                       D.BH * D.Tq, d);
+      return cudaGetLastError();
+    });
+  L(K_BWD_ELEM, [&] {
+    (void)launch_pdl(k_sum_batch, grid_for(planes, 4), 256, 0, st, static_cast<const float*>(A),
+                     static_cast<int>(D.B), static_cast<int>(D.H), plane, D.w_shared, in.dw1, in.dw2, in.dw3);
+    return cudaGetLastError();
+  });
+}
+
+static void run_bwd(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaStream_t st, Launcher& L) {
+  if (D.dtype == LACT_BF16) run_bwd_tc(D, b, in, st, L);
+  else run_bwd_f32(D, b, in, st, L);
 }
 
 }  // namespace lact

@@ -480,6 +480,7 @@ struct GemmParams {
   int64_t ld_t;
   const float* row_scale;  // or null: row m of output item z scaled by row_scale[z * rs_item + m]
   int64_t rs_item;
+  int a_m0;                // K-major A: first row of A's map that tile row 0 reads
 };
 
 template <bool A_MN, bool B_MN, int BN, bool SPLIT = false>
@@ -546,10 +547,11 @@ struct GemmOp {
   __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
     const int kk = (t.split * p.kb_count + kb) * kBK;
     const int ak = p.a_k0 + kk, bk = p.b_k0 + kk;
-    load_a(&p.tmA, st, bar, t.m0, ak, t.item);
+    const int am = A_MN ? t.m0 : t.m0 + p.a_m0;
+    load_a(&p.tmA, st, bar, am, ak, t.item);
     load_b(t.alt ? &p.tmB2 : &p.tmB, st + kOffB, bar, t.n0, bk, t.zb);
     if (SPLIT) {
-      load_a(&p.tmAlo, st + kABytes, bar, t.m0, ak, t.item);
+      load_a(&p.tmAlo, st + kABytes, bar, am, ak, t.item);
       if (!t.alt) load_b(&p.tmBlo, st + kOffB + kBBytes, bar, t.n0, bk, t.zb);
     }
   }
