@@ -42,6 +42,7 @@ struct BwdBufs {
   float *dqh, *dkh, *ofull, *part;
   // bf16 problems (tensor-core contractions): bf16 operands
   __nv_bfloat16 *qh16, *kh16, *dos16, *hist16, *op16, *Gam16;
+  __nv_bfloat16 *Bk, *Bv, *Ba;   // stacked operands of the merged contractions
   int64_t zr;   // rows per head of the per-chunk [rows][dh] planes
 };
 
@@ -65,6 +66,9 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
     b.hist16 = bp.take<__nv_bfloat16>((D.nch + 1) * planes);
     b.op16 = bp.take<__nv_bfloat16>(6 * zpl);
     b.Gam16 = bp.take<__nv_bfloat16>(planes);
+    b.Bk = bp.take<__nv_bfloat16>(4 * D.BH * D.dh * D.d);
+    b.Bv = bp.take<__nv_bfloat16>(2 * D.BH * D.dh * D.d);
+    b.Ba = bp.take<__nv_bfloat16>(2 * D.BH * D.dh * D.d);
   } else {
     b.dos32 = bp.take<float>(nq);
     b.qh = bp.take<float>(nq);
@@ -81,8 +85,8 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
     b.part = bp.take<float>(rule_rows(D));
   }
   b.mnorm = bp.take<float>(D.nch * rule_rows(D));
-  b.Z = bp.take<float>(3 * zpl);
-  b.Pz = bp.take<float>(3 * zpl);
+  b.Z = bp.take<float>((bf ? 6 : 3) * zpl);     // bf16 problems: the merged blocks [z1|z3|p|r], [u|q]
+  if (!bf) b.Pz = bp.take<float>(3 * zpl);
   b.P = bp.take<float>(planes);
   b.A = bp.take<float>(planes);
   b.Ap = bp.take<float>(planes);
@@ -375,7 +379,11 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     constexpr bool AMN = decltype(a_mn)::value, BMN = decltype(b_mn)::value;
     L(K_BWD_GEMM, [&] {
       GemmParams g = gemm_params();
-      const int bn = pick_bn(N);
+      // halve the N tile while the launch has too few tiles to fill the SMs
+      int bn = pick_bn(N);
+      while (bn >= 128 && (bn / 2) % 64 == 0 && N % (bn / 2) == 0 &&
+             static_cast<int64_t>(N / bn) * cdiv(M, 128) * BH < 100)
+        bn /= 2;
       if (!map3d(&g.tmA, a.p, a.inner, a.rows, a.batch, 64, AMN ? 64 : 128) ||
           !map3d(&g.tmB, bo.p, bo.inner, bo.rows, bo.batch, 64, BMN ? 64 : bn))
         return cudaErrorInvalidValue;
@@ -393,7 +401,6 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
   auto Wop = [&](const B16* W, int j) {   // plane j of a state: W1, W3 [dh][d]; W2 [d][dh]
     return j == 1 ? Opnd{W + jst, D.dh, D.d, D.BH} : Opnd{W + j * jst, D.d, D.dh, D.BH};
   };
-  auto op = [&](int j) { return Opnd{b.op16 + j * zpl, D.dh, zr, D.BH}; };
 
   // ---- raw fp32 q, k (prologue backward), dout (scale gradient), bf16 q^, k^
   {
@@ -507,27 +514,54 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     });
   }
 
-  // ---- reverse chunk loop
+  // ---- reverse chunk loop, on merged contractions:
+  //   [z1|z3|p|r] = k^ [W1; W3; Gam1; Gam3]^T,  [u|q] = v [W2 | Gam2]
+  //   dk^ += [dz1|dz3|dp|dr] [W1; W3; Gam1; Gam3],  dv += [du|dq] [W2 | Gam2]^T
+  //   apply: [zq1|zq3] = q^ [W1; W3]^T,  dq^ += [dz1|dz3] [W1; W3]
   float* A = b.A;
   float* Ap = b.Ap;
+  const int64_t pb = plane * 2;   // bytes of one bf16 plane
+  auto copy2d = [&](void* dst, int64_t dpitch, const void* src, int64_t spitch, int64_t width, int64_t height) {
+    if (!L.dry)
+      memop(cudaMemcpy2DAsync(dst, static_cast<size_t>(dpitch), src, static_cast<size_t>(spitch),
+                              static_cast<size_t>(width), static_cast<size_t>(height), cudaMemcpyDeviceToDevice,
+                              st));
+  };
+  // stack per head: dst [BH][n_slots * dh][d] from [dh][d] planes
+  auto stack_rows = [&](B16* dst, int n_slots, int slot, const B16* src_plane) {
+    copy2d(dst + slot * plane, n_slots * pb, src_plane, pb, pb, D.BH);
+  };
+  const int64_t dh4 = 4 * D.dh, dh2 = 2 * D.dh;
+  float* Zk = b.Z;                    // [BH][zr][4 dh]
+  float* Zv = b.Z + 4 * zpl;          // [BH][zr][2 dh]
+  B16* Phik = b.op16;                 // [BH][zr][4 dh]
+  B16* Phiv = b.op16 + 4 * zpl;       // [BH][zr][2 dh]
+  const Opnd Zk_op{Phik, dh4, zr, D.BH}, Zv_op{Phiv, dh2, zr, D.BH};
   auto apply_bwd = [&](const B16* W, int64_t qr0, int nq_c) {
     const int r0 = static_cast<int>(qr0);
-    tcg(KM, KM, qh, r0, 0, Wop(W, 0), 0, nq_c, dh, d, b.Z, zr * D.dh, dh, false);
-    tcg(KM, MN, dos, r0, 0, Wop(W, 1), 0, nq_c, dh, d, b.Z + zpl, zr * D.dh, dh, false);
-    tcg(KM, KM, qh, r0, 0, Wop(W, 2), 0, nq_c, dh, d, b.Z + 2 * zpl, zr * D.dh, dh, false);
-    L(K_BWD_ELEM, [&] {   // -> op16 planes (dz1, hq, dz3)
-      (void)launch_pdl(k_apply_bwd_elem_bf16, grid_for(zpl, 4), 256, 0, st, b.Z, BH, zr, dh, nq_c, b.op16);
+    stack_rows(b.Ba, 2, 0, W);               // [W1; W3]
+    stack_rows(b.Ba, 2, 1, W + 2 * jst);
+    const Opnd Ba_op{b.Ba, D.d, dh2, D.BH};
+    float* Za = b.Z;                          // [BH][zr][2 dh]
+    float* G = b.Z + 2 * zpl;                 // [BH][zr][dh]
+    B16* Phia = b.op16;                       // [BH][zr][2 dh]
+    B16* Hq = b.op16 + 2 * zpl;               // [BH][zr][dh]
+    tcg(KM, KM, qh, r0, 0, Ba_op, 0, nq_c, 2 * dh, d, Za, zr * dh2, dh2, false);
+    tcg(KM, MN, dos, r0, 0, Wop(W, 1), 0, nq_c, dh, d, G, zr * D.dh, dh, false);
+    L(K_BWD_ELEM, [&] {
+      (void)launch_pdl(k_apply_bwd_cat, grid_for(zpl, 4), 256, 0, st, static_cast<const float*>(Za),
+                       static_cast<const float*>(G), BH, zr, dh, nq_c, Phia, Hq);
       return cudaGetLastError();
     });
+    const Opnd Pa{Phia, dh2, zr, D.BH}, Hq_op{Hq, D.dh, zr, D.BH};
     // dW1 += dz1^T q^, dW3 += dz3^T q^, dW2 += dO^T hq
-    tcg(MN, MN, op(0), 0, 0, qh, r0, dh, d, nq_c, A, plane, d, true);
-    tcg(MN, MN, op(2), 0, 0, qh, r0, dh, d, nq_c, A + 2 * jst, plane, d, true);
-    tcg(MN, MN, dos, 0, r0, op(1), 0, d, dh, nq_c, A + jst, plane, dh, true);
-    // dq^ += dz1 W1 + dz3 W3
-    tcg(KM, MN, op(0), 0, 0, Wop(W, 0), 0, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
-    tcg(KM, MN, op(2), 0, 0, Wop(W, 2), 0, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
+    tcg(MN, MN, Pa, 0, 0, qh, r0, dh, d, nq_c, A, plane, d, true);
+    tcg(MN, MN, Pa, dh, 0, qh, r0, dh, d, nq_c, A + 2 * jst, plane, d, true);
+    tcg(MN, MN, dos, 0, r0, Hq_op, 0, d, dh, nq_c, A + jst, plane, dh, true);
+    // dq^ += [dz1|dz3] [W1; W3]
+    tcg(KM, MN, Pa, 0, 0, Ba_op, 0, nq_c, d, 2 * dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
     if (in.scale)   // the unscaled output hq W2^T, for the scale's gradient
-      tcg(KM, KM, op(1), 0, 0, Wop(W, 1), 0, nq_c, d, dh, b.ofull + qr0 * d, D.Tq * D.d, d, false);
+      tcg(KM, KM, Hq_op, 0, 0, Wop(W, 1), 0, nq_c, d, dh, b.ofull + qr0 * d, D.Tq * D.d, d, false);
   };
   for (int64_t c = D.nch - 1; c >= 0; --c) {
     const int64_t c0 = c * D.chunk;
@@ -555,26 +589,30 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
                            in.dbeta);
           return cudaGetLastError();
         });
-      key_forward(Wp16, c0, nc, b.Z);       // (z1, u, z3)
-      key_forward(b.Gam16, c0, nc, b.Pz);   // (p, q, r)
-      L(K_BWD_ELEM, [&] {   // -> op16 planes (dz1, du, dz3, dp, dq, dr)
-        (void)launch_pdl(k_hvp_elem_bf16, static_cast<unsigned>(cdiv(D.BH * zr * 32, 256)), 256, 0, st, b.Z,
-                         b.Pz, BH, zr, dh, nc, in.lr, D.T, c0, in.dlr, b.op16);
+      // stacked operands: Bk = [W1; W3; Gam1; Gam3] [BH][4 dh][d], Bv = [W2 | Gam2] [BH][d][2 dh]
+      stack_rows(b.Bk, 4, 0, Wp16);
+      stack_rows(b.Bk, 4, 1, Wp16 + 2 * jst);
+      stack_rows(b.Bk, 4, 2, b.Gam16);
+      stack_rows(b.Bk, 4, 3, b.Gam16 + 2 * jst);
+      copy2d(b.Bv, dh2 * 2, Wp16 + jst, D.dh * 2, D.dh * 2, D.BH * D.d);
+      copy2d(b.Bv + D.dh, dh2 * 2, b.Gam16 + jst, D.dh * 2, D.dh * 2, D.BH * D.d);
+      const Opnd Bk_op{b.Bk, D.d, dh4, D.BH}, Bv_op{b.Bv, dh2, D.d, D.BH};
+      const int k0 = static_cast<int>(c0);
+      tcg(KM, KM, kh, k0, 0, Bk_op, 0, nc, 4 * dh, d, Zk, zr * dh4, dh4, false);   // [z1|z3|p|r]
+      tcg(KM, MN, vv, k0, 0, Bv_op, 0, nc, 2 * dh, d, Zv, zr * dh2, dh2, false);   // [u|q]
+      L(K_BWD_ELEM, [&] {
+        (void)launch_pdl(k_hvp_elem_cat, static_cast<unsigned>(cdiv(D.BH * zr * 32, 256)), 256, 0, st,
+                         static_cast<const float*>(Zk), static_cast<const float*>(Zv), BH, zr, dh, nc, in.lr, D.T,
+                         c0, in.dlr, Phik, Phiv);
         return cudaGetLastError();
       });
-      const int k0 = static_cast<int>(c0);
       // dW1 += dz1^T k^, dW3 += dz3^T k^, dW2 += v^T du
-      tcg(MN, MN, op(0), 0, 0, kh, k0, dh, d, nc, Ap, plane, d, true);
-      tcg(MN, MN, op(2), 0, 0, kh, k0, dh, d, nc, Ap + 2 * jst, plane, d, true);
-      tcg(MN, MN, vv, 0, k0, op(1), 0, d, dh, nc, Ap + jst, plane, dh, true);
-      // dk^ += dz1 W1 + dz3 W3 + dp Gam1 + dr Gam3
-      tcg(KM, MN, op(0), 0, 0, Wop(Wp16, 0), 0, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d, true);
-      tcg(KM, MN, op(2), 0, 0, Wop(Wp16, 2), 0, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d, true);
-      tcg(KM, MN, op(3), 0, 0, Wop(b.Gam16, 0), 0, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d, true);
-      tcg(KM, MN, op(5), 0, 0, Wop(b.Gam16, 2), 0, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d, true);
-      // dv += du W2^T + dq Gam2^T
-      tcg(KM, KM, op(1), 0, 0, Wop(Wp16, 1), 0, nc, d, dh, in.dv + c0 * d, D.T * D.d, d, true);
-      tcg(KM, KM, op(4), 0, 0, Wop(b.Gam16, 1), 0, nc, d, dh, in.dv + c0 * d, D.T * D.d, d, true);
+      tcg(MN, MN, Zk_op, 0, 0, kh, k0, dh, d, nc, Ap, plane, d, true);
+      tcg(MN, MN, Zk_op, dh, 0, kh, k0, dh, d, nc, Ap + 2 * jst, plane, d, true);
+      tcg(MN, MN, vv, 0, k0, Zv_op, 0, d, dh, nc, Ap + jst, plane, dh, true);
+      // dk^ += [dz1|dz3|dp|dr] [W1; W3; Gam1; Gam3],  dv += [du|dq] [W2 | Gam2]^T
+      tcg(KM, MN, Zk_op, 0, 0, Bk_op, 0, nc, d, 4 * dh, b.dkh + c0 * d, D.T * D.d, d, true);
+      tcg(KM, KM, Zv_op, 0, 0, Opnd{b.Bv, dh2, D.d, D.BH}, 0, nc, d, 2 * dh, in.dv + c0 * d, D.T * D.d, d, true);
       std::swap(A, Ap);
     }
     if (D.order == LACT_APPLY_THEN_UPDATE) apply_bwd(Wp16, qr0, nq_c);

@@ -480,7 +480,8 @@ struct GemmParams {
   int64_t ld_t;
   const float* row_scale;  // or null: row m of output item z scaled by row_scale[z * rs_item + m]
   int64_t rs_item;
-  int a_m0;                // K-major A: first row of A's map that tile row 0 reads
+  int a_m0;                // first M coordinate of A's map that tile row 0 reads (MN-major A:
+                           // a multiple of 8, the map's inner coordinate)
 };
 
 template <bool A_MN, bool B_MN, int BN, bool SPLIT = false>
@@ -547,7 +548,7 @@ struct GemmOp {
   __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
     const int kk = (t.split * p.kb_count + kb) * kBK;
     const int ak = p.a_k0 + kk, bk = p.b_k0 + kk;
-    const int am = A_MN ? t.m0 : t.m0 + p.a_m0;
+    const int am = t.m0 + p.a_m0;
     load_a(&p.tmA, st, bar, am, ak, t.item);
     load_b(t.alt ? &p.tmB2 : &p.tmB, st + kOffB, bar, t.n0, bk, t.zb);
     if (SPLIT) {
