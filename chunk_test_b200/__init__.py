@@ -15,5 +15,6 @@ from ._abi import (  # noqa: F401
 from .layer import (  # noqa: F401
     ttt_fwd, ttt_fwd_host, ttt_fwd_noalloc, ttt_bwd, workspace_bytes, bwd_workspace_bytes,
     host_workspace_bytes, launch_count, status,
-    device_check, selftest_wait_timeout, make_problem, torch_distributed_allreduce,
+    device_check, selftest_wait_timeout, make_problem, torch_distributed_allreduce, swa_fwd,
+    swa_workspace_bytes,
 )

@@ -42,6 +42,12 @@ class LactFwdOpts(ctypes.Structure):
     ]
 
 
+class LactSwaProblem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("T", ctypes.c_int64),
+                ("d", ctypes.c_int64), ("window", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
 class LactError(RuntimeError):
     def __init__(self, code: int, what: str = ""):
         self.code = code
@@ -62,6 +68,8 @@ SIGNATURES = {
                      + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_host_workspace_bytes": (ctypes.c_size_t, [_P]),
     "lact_ttt_fwd_host": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]),
+    "lact_swa_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(LactSwaProblem)]),
+    "lact_swa_fwd": (ctypes.c_int, [ctypes.POINTER(LactSwaProblem)] + [_vp] * 8 + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_status": (ctypes.c_int, [_vp]),
     "lact_device_check": (ctypes.c_int, []),
     "lact_ttt_launch_count": (ctypes.c_int64, [_P]),

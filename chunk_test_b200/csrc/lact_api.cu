@@ -367,13 +367,13 @@ static cudaError_t launch_gemm_any(bool split, int bn, dim3 grid, const GemmPara
 enum Kind {
   K_INIT, K_PROLOGUE, K_BETA_MEAN, K_FWD_QUERY, K_APPLY_OUT, K_FWD_KEY, K_GRAD, K_NS_SUMSQ,
   K_NS_SCALE, K_NS_GRAM, K_NS_POLY, K_NS_UPDATE, K_RULE, K_FINALIZE, K_SIMT_GEMM, K_FWD_ELEM_F32,
-  K_APPLY_FUSED, K_KEY_GRAD, K_BWD_ELEM, K_BWD_GEMM, K_COUNT
+  K_APPLY_FUSED, K_KEY_GRAD, K_BWD_ELEM, K_BWD_GEMM, K_SWA, K_SWA_GEMM, K_COUNT
 };
 static const char* const kKindNames[K_COUNT] = {
     "init_state", "qk_prologue", "beta_mean", "fwd_query_umma", "apply_out_umma", "fwd_key_umma",
     "grad_umma", "ns_sumsq", "ns_scale", "ns_gram_umma", "ns_poly_umma", "ns_update_umma",
     "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32", "apply_fused_umma",
-    "key_grad_umma", "bwd_elem", "bwd_gemm_umma"};
+    "key_grad_umma", "bwd_elem", "bwd_gemm_umma", "swa_elem", "swa_gemm_umma"};
 
 // Optional per-launch CUDA-event pairs on the launching stream.
 struct ProfRec { int kind; cudaEvent_t a, b; };
@@ -1048,6 +1048,7 @@ __global__ void k_selftest_wait() {
 }  // namespace lact
 
 #include "lact_bwd.cuh"
+#include "lact_swa.cuh"
 
 using namespace lact;
 
@@ -1253,6 +1254,36 @@ int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts, const void* q
                opts ? opts->update_mask : nullptr, scale, dq, dk, dv, dlr, dbeta, dw1, dw2, dw3, dout_scale};
   Launcher L{false, static_cast<cudaStream_t>(stream)};
   run_bwd(D, b, in, static_cast<cudaStream_t>(stream), L);
+  return L.err;
+}
+
+size_t lact_swa_workspace_bytes(const lact_swa_problem* p) {
+  SwaDims S;
+  if (swa_validate(p, S) != LACT_OK) return 0;
+  return swa_workspace_bytes(S);
+}
+
+int lact_swa_fwd(const lact_swa_problem* p, const void* q, const void* k, const void* v, const float* q_scale,
+                 const float* q_offset, const float* k_scale, const float* k_offset, void* out, void* workspace,
+                 size_t workspace_bytes_, void* stream) {
+  SwaDims S;
+  int rc = swa_validate(p, S);
+  if (rc != LACT_OK) return rc;
+  const void* need[] = {q, k, v, q_scale, q_offset, k_scale, k_offset, out};
+  for (const void* x : need)
+    if (!x || !aligned16(x)) return LACT_EINVAL;
+  const size_t n = static_cast<size_t>(S.BH * S.T * S.d) * 2;
+  const void* ins[] = {q, k, v};
+  for (const void* x : ins)
+    if (overlaps(out, n, x, n)) return LACT_EINVAL;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LACT_EINVAL;
+  if (workspace_bytes_ < swa_workspace_bytes(S)) return LACT_ENOSPC;
+  if (!encode_fn()) return LACT_ECUDA;
+  Bump bp{reinterpret_cast<uintptr_t>(workspace), 0};
+  SwaBufs b;
+  swa_plan(S, bp, b);
+  Launcher L{false, static_cast<cudaStream_t>(stream)};
+  swa_run(S, b, q, k, v, q_scale, q_offset, k_scale, k_offset, out, static_cast<cudaStream_t>(stream), L);
   return L.err;
 }
 

@@ -482,6 +482,7 @@ struct GemmParams {
   int64_t rs_item;
   int a_m0;                // first M coordinate of A's map that tile row 0 reads (MN-major A:
                            // a multiple of 8, the map's inner coordinate)
+  int zb_div, zb_mul;      // if zb_div > 0: B's batch = (item / zb_div) * zb_mul + item % zb_div
 };
 
 template <bool A_MN, bool B_MN, int BN, bool SPLIT = false>
@@ -509,7 +510,7 @@ struct GemmOp {
     t.item = z % p.items;
     t.split = z / p.items;
     t.out_item = z;
-    t.zb = (t.item % p.zb_mod) + p.zb_add;
+    t.zb = p.zb_div > 0 ? (t.item / p.zb_div) * p.zb_mul + t.item % p.zb_div : (t.item % p.zb_mod) + p.zb_add;
     t.alt = p.alt_group >= 0 && (t.item / p.zb_mod) == p.alt_group;
     return t;
   }

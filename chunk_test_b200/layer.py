@@ -240,6 +240,46 @@ def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=N
     return res
 
 
+def swa_problem(q, window) -> _abi.LactSwaProblem:
+    B, H, T, d = q.shape
+    return _abi.LactSwaProblem(int(B), int(H), int(T), int(d), int(window), _abi.LACT_BF16, 0)
+
+
+def swa_workspace_bytes(q, window) -> int:
+    return int(_abi.lib().lact_swa_workspace_bytes(ctypes.byref(swa_problem(q, window))))
+
+
+def swa_fwd(q, k, v, q_scale, q_offset, k_scale, k_offset, window, *, out=None, workspace=None,
+            stream=None):
+    """Sliding-window attention of the LaCT block (lact_swa_fwd): q, k, v
+    [B, H, T, d] bf16 CUDA tensors, scales and offsets [H, d] float32.
+    Returns out [B, H, T, d] bf16."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.device.type != "cuda" or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    for name, t in (("q_scale", q_scale), ("q_offset", q_offset), ("k_scale", k_scale),
+                    ("k_offset", k_offset)):
+        if t.device != q.device or not t.is_contiguous() or t.dtype != torch.float32:
+            raise ValueError(f"{name} must be a contiguous float32 tensor on q's device")
+    p = swa_problem(q, window)
+    need = int(_abi.lib().lact_swa_workspace_bytes(ctypes.byref(p)))
+    if need == 0:
+        raise LactError(_abi.LACT_EINVAL, "lact_swa_workspace_bytes")
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = _abi.lib().lact_swa_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_scale),
+                                 _ptr(q_offset), _ptr(k_scale), _ptr(k_offset), _ptr(out),
+                                 _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                 ctypes.c_void_p(stream.cuda_stream))
+    if rc != _abi.LACT_OK:
+        raise LactError(rc, "lact_swa_fwd")
+    return out
+
+
 def ttt_fwd_noalloc(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out, w_out,
                     stream=None):
     """The forward for callers that cannot allocate device memory: no

@@ -1,10 +1,10 @@
 /*
  * lact.h -- C ABI of the B200 (sm_100a) LaCT fast-weight TTT layer (forward
- * and backward).
+ * and backward) and of the block's sliding-window attention.
  *
  * The layer (Large-Chunk Test-Time Training).  Sources are cited by page
  * title and section:
- *   [P1] "LaCT架构核心思想解析" (gsyq.cn) §1.2, §2.1, §2.2, §3.2
+ *   [P1] "LaCT架构核心思想解析" (gsyq.cn) §1.1, §1.2, §2.1, §2.2, §3.2
  *   [P2] "大块测试时训练（LaCT）技术解析" (dpshk.com) §2.1, §2.2.1, §2.2.2
  *   [P3] "LaCT：以大分块更新人工智能的临时记忆" (iplexlaw.co.kr), sections
  *        「局部注意力与非线性记忆相互补充」, 「更新顺序必须遵守信息可见范围」 and
@@ -269,6 +269,31 @@ int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts,
                  float* dq, float* dk, float* dv, float* dlr, float* dbeta,
                  float* dw1, float* dw2, float* dw3, float* dout_scale,
                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Sliding-window attention, the other half of the LaCT block ([P1 §1.1]):
+ * per head and channel learnable scales and offsets on the queries and
+ * keys, q' = q * q_scale + q_offset, k' = k * k_scale + k_offset, then for
+ * every token t, out_t = sum_j softmax_j(q'_t . k'_j / sqrt(d)) v_j over the
+ * `window` most recent tokens, t - window < j <= t (causal; the window
+ * includes the token itself).  q, k, v, out [B, H, T, d] bf16 (device);
+ * q_scale, q_offset, k_scale, k_offset [H, d] float32 (device).  Limits: d
+ * a multiple of 64 up to 512, T and window multiples of 128, window <=
+ * 16384, B*H <= 4096.  The scores take a round trip through the workspace
+ * (fp32 scores, bf16 probabilities: B*H*T*(window+128)*6 bytes);
+ * lact_swa_workspace_bytes gives its size.  Asynchronous on `stream`; the
+ * error behaviour of lact_ttt_fwd. */
+typedef struct lact_swa_problem {
+  int64_t B, H, T, d, window;
+  int32_t dtype;   /* LACT_BF16 */
+  int32_t reserved;
+} lact_swa_problem;
+
+size_t lact_swa_workspace_bytes(const lact_swa_problem* p);
+
+int lact_swa_fwd(const lact_swa_problem* p, const void* q, const void* k, const void* v,
+                 const float* q_scale, const float* q_offset,
+                 const float* k_scale, const float* k_offset,
+                 void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Waits for `stream`, then returns and clears the device status word of the
  * current device: LACT_OK, or LACT_ETIMEOUT if a bounded wait inside one of

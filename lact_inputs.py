@@ -144,3 +144,18 @@ def make_output_grads(w: Workload, seed: int = 0, with_weights: bool = False):
         dws = (torch.randn((BH, w.dh, w.d), generator=g), torch.randn((BH, w.d, w.dh), generator=g),
                torch.randn((BH, w.dh, w.d), generator=g))
     return dout, dws
+
+
+def make_swa_inputs(B: int, H: int, T: int, d: int, seed: int = 0) -> dict:
+    """Seeded inputs of the sliding-window attention: q, k, v [B,H,T,d] ~ N(0,1)
+    in bf16, and per head and channel q/k scales 1 + 0.1 N(0,1) and offsets
+    0.1 N(0,1) [H,d] in fp32 (learnable parameters near their identity
+    initialisation)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(30_000 + seed)
+    q, k, v = (torch.randn((B, H, T, d), generator=g).bfloat16() for _ in range(3))
+    qs = 1.0 + 0.1 * torch.randn((H, d), generator=g)
+    qo = 0.1 * torch.randn((H, d), generator=g)
+    ks = 1.0 + 0.1 * torch.randn((H, d), generator=g)
+    ko = 0.1 * torch.randn((H, d), generator=g)
+    return dict(q=q, k=k, v=v, q_scale=qs, q_offset=qo, k_scale=ks, k_offset=ko)
