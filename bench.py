@@ -281,8 +281,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
-    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
-                    help="time the layer forward (default) or its backward (lact_ttt_bwd)")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "swa"],
+                    help="time the layer forward (default), its backward (lact_ttt_bwd) or the "
+                         "block's sliding-window attention (lact_swa_fwd, window = the chunk)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload at this sequence length instead (a scaled case "
                          "for profiling; named in config.workload)")
@@ -297,6 +298,8 @@ def main():
         return run_reference(args, w)
     if args.which == "bwd":
         return run_backward(args, w)
+    if args.which == "swa":
+        return run_swa(args, w)
 
     import chunk_test_b200 as ct
 
@@ -617,6 +620,138 @@ def run_backward(args, w: Workload):
                             "kind": "oracle",
                             "sample": f"autograd backward oracle on {done} of {len(heads)} "
                                       f"(batch, head) sequences, {tok_done} tokens, {sec:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- window attention
+def swa_flops(B: int, H: int, T: int, d: int, window: int) -> float:
+    """Algorithmic FLOPs of sliding-window attention: 4 d per (query, key)
+    pair in the window (q'.k and p v), min(t + 1, window) keys for token t."""
+    pairs = sum(min(t + 1, window) for t in range(min(T, window))) + max(0, T - window) * window
+    return 4.0 * d * B * H * pairs
+
+
+def run_swa(args, w: Workload):
+    import chunk_test_b200 as ct
+    from lact_inputs import make_swa_inputs
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--pass swa runs on one GPU")
+    window = w.chunk if w.Tq == w.T else 2048
+    B, H, T, d = w.B, w.H, w.T, w.d
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    inp_cpu = make_swa_inputs(B, H, T, d, seed=0)
+    inp = {k: v.to(dev) for k, v in inp_cpu.items()}
+    out = torch.empty_like(inp["q"])
+    ws = torch.empty(ct.swa_workspace_bytes(inp["q"], window), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ct.swa_fwd(inp["q"], inp["k"], inp["v"], inp["q_scale"], inp["q_offset"], inp["k_scale"],
+                   inp["k_offset"], window, out=out, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after the timed region")
+    ct.profile_enable(True)
+    ct.profile_read()
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize(dev)
+    prof = ct.profile_read()
+    ct.profile_enable(False)
+    _, _, pk_sust, pk_src = peaks()
+    hbm, *_ = peaks()
+    flops = swa_flops(B, H, T, d, window)
+    kernels = {k: {"launches": v[0], "ms": round(v[1], 4),
+                   "share": round(v[1] / sum(x[1] for x in prof.values()), 4)}
+               for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    dom, (n_launch, ms_kind) = max(prof.items(), key=lambda kv: kv[1][1])
+    roof = None
+    if dom == "swa_gemm_umma":
+        achieved = flops * args.steps / (ms_kind / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
+                "frac": achieved / pk_sust, "kernel": dom, "launches": n_launch,
+                "avg_launch_us": 1e3 * ms_kind / n_launch, "timed": "alone (per-kernel pass)",
+                "traffic": None, "peak_source": f"{pk_src} sustained bf16",
+                "work": "algorithmic: 4 d FLOPs per (query, key) pair in the window"}
+    elif dom == "swa_elem":
+        Lw = window + 128
+        bytes_step = B * H * T * (Lw * (4 + 4 + 2) + 3 * d * 2 * 2)
+        achieved = bytes_step * args.steps / (ms_kind / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "kernel": dom, "launches": n_launch, "avg_launch_us": 1e3 * ms_kind / n_launch,
+                "timed": "alone (per-kernel pass)", "traffic": None,
+                "peak_source": f"{pk_src} copy bandwidth",
+                "work": "scores read twice (fp32) and probabilities written (bf16), plus the prologue"}
+    # end to end from pinned host buffers
+    pin = {k: v.pin_memory() for k, v in inp_cpu.items()}
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def host_step():
+        for k, v in pin.items():
+            inp[k].copy_(v, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        host_step()
+    torch.cuda.synchronize(dev)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for _ in range(args.steps):
+        host_step()
+    h1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = h0.elapsed_time(h1) / args.steps
+    tok = B * T
+    line = {
+        "metric": "LaCT sliding-window attention tokens/s at 1 B200", "value": tok / (ms_step / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded normal q/k/v, near-identity q/k scales and offsets)",
+        "config": {"workload": f"swa-B{B}-H{H}-T{T}-d{d}-w{window}", "B": B, "H": H, "T": T, "d": d,
+                   "window": window, "pass": "sliding-window attention (lact_swa_fwd)",
+                   "l2": "inputs and scores larger than L2, no flush"},
+        "peak_frac": {"algorithmic_tflops": flops / (ms_step / 1e3) / 1e12,
+                      "frac_of_sustained_bf16": flops / (ms_step / 1e3) / 1e12 / pk_sust},
+        "roofline": roof, "kernels": kernels,
+        "gpu_launches": sum(v[0] for v in prof.values()),
+        "e2e": {"value": tok / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin.values()),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+        "clocks": clk,
+    }
+    # the oracle on a bounded sample: one head's first query rows
+    from oracle import swa_oracle as so
+    t0, n_rows = time.perf_counter(), 0
+    start = min(window, T - 1)      # rows with full windows (the steady state)
+    step_rows = 256
+    while start + n_rows < T and (n_rows == 0 or time.perf_counter() - t0 < args.cpu_budget):
+        rows = list(range(start + n_rows, min(T, start + n_rows + step_rows)))
+        so.swa_layer(inp_cpu["q"][:1, :1], inp_cpu["k"][:1, :1], inp_cpu["v"][:1, :1], inp_cpu["q_scale"][:1],
+                     inp_cpu["q_offset"][:1], inp_cpu["k_scale"][:1], inp_cpu["k_offset"][:1], window,
+                     rows=rows)
+        n_rows += len(rows)
+    sec = time.perf_counter() - t0
+    # per (batch, head) query rows per second -> tokens/s of the whole B x H problem
+    line["cpu_baseline"] = {"value": n_rows / sec / H, "unit": "tokens/s", "cores": blas_threads(),
+                            "kind": "oracle",
+                            "sample": f"{n_rows} query rows (full windows) of one (batch, head), "
+                                      f"{sec:.1f} s, scaled to {H} heads per token"}
     print(json.dumps(line), flush=True)
     return 0
 
