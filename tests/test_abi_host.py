@@ -166,3 +166,43 @@ def test_bad_options_are_rejected_without_a_gpu():
     assert call(gd, o) == ct.LACT_EINVAL                 # scale on out
     o, _ = _opts(scale=14 * G, m=m_ok)
     assert call(mom, o) == ct.LACT_EINVAL                # scale on m2
+
+
+def test_backward_and_attention_arguments_are_checked_without_a_gpu():
+    """lact_ttt_bwd and lact_swa_fwd reject bad problems, rules, options and
+    pointers before anything is enqueued."""
+    lib = ct.lib()
+    G = 1 << 30
+    ptrs = [ctypes.c_void_p(G * (i + 1)) for i in range(21)]
+    ws = ctypes.c_void_p(1 << 40)
+    big = ctypes.c_size_t(1 << 40)
+    gd = _prob(WORKLOADS[1])
+    assert _abi.bwd_workspace_bytes(gd) > 0
+    assert _abi.bwd_workspace_bytes(_prob(WORKLOADS[1], rule=2)) == 0          # no Muon backward
+    call = lambda p, o, a: lib.lact_ttt_bwd(ctypes.byref(p), o, *a, ws, big, None)
+    assert call(_prob(WORKLOADS[1], rule=2), None, ptrs) == ct.LACT_EINVAL
+    m_opts = _abi.LactFwdOpts(None, None, 13 * G, 14 * G, 15 * G)
+    assert call(_prob(WORKLOADS[1], rule=1), ctypes.byref(m_opts), ptrs) == ct.LACT_EINVAL
+    bad = list(ptrs)
+    bad[0] = ctypes.c_void_p(0)                                                # q missing
+    assert call(gd, None, bad) == ct.LACT_EINVAL
+    bad = list(ptrs)
+    bad[12] = ctypes.c_void_p(ptrs[0].value)                                   # dq on q
+    assert call(gd, None, bad) == ct.LACT_EINVAL
+    bad = list(ptrs)
+    bad[9] = ctypes.c_void_p(0)                                                # only some dw*_out
+    assert call(gd, None, bad) == ct.LACT_EINVAL
+    assert lib.lact_ttt_bwd(ctypes.byref(gd), None, *ptrs, ws, ctypes.c_size_t(16), None) == ct.LACT_ENOSPC
+
+    sp = lambda **kw: _abi.LactSwaProblem(*[kw.get(n, v) for n, v in
+                                            (("B", 1), ("H", 2), ("T", 1024), ("d", 128), ("window", 256),
+                                             ("dtype", 1), ("reserved", 0))])
+    assert lib.lact_swa_workspace_bytes(ctypes.byref(sp())) > 0
+    for bad_p in (sp(T=1000), sp(window=100), sp(d=96), sp(dtype=0), sp(window=0), sp(d=576)):
+        assert lib.lact_swa_workspace_bytes(ctypes.byref(bad_p)) == 0
+        assert lib.lact_swa_fwd(ctypes.byref(bad_p), *ptrs[:8], ws, big, None) == ct.LACT_EINVAL
+    p = sp()
+    bad = list(ptrs[:8])
+    bad[7] = ctypes.c_void_p(ptrs[1].value)                                    # out on k
+    assert lib.lact_swa_fwd(ctypes.byref(p), *bad, ws, big, None) == ct.LACT_EINVAL
+    assert lib.lact_swa_fwd(ctypes.byref(p), *ptrs[:8], ws, ctypes.c_size_t(16), None) == ct.LACT_ENOSPC
