@@ -576,18 +576,36 @@ struct GemmOp {
                         static_cast<int64_t>(grow) * p.ld + t.n0;
     const bool tr = p.tr_group >= 0 && (t.item / p.tr_mod) == p.tr_group;
     const float rs = (p.row_scale && valid) ? __ldg(p.row_scale + t.out_item * p.rs_item + grow) : 1.0f;
+    // cin of the next 16 columns is loaded while this step's are used, so
+    // the epilogue does not wait on one global load latency per step
+    const bool has_c = p.cin && valid;
+    float4 cn[4];
+    if (has_c) {
+      const float4* c = reinterpret_cast<const float4*>(p.cin + off);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cn[i] = c[i];
+    }
 #pragma unroll 1
     for (int j = 0; j < BN; j += 16) {
       float v[16];
+      float4 cc[4];
+      if (has_c) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cc[i] = cn[i];
+        if (j + 16 < BN) {
+          const float4* c = reinterpret_cast<const float4*>(p.cin + off + j + 16);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cn[i] = c[i];
+        }
+      }
       __syncwarp();
       tmem_ld16(tq + j, v);
       tmem_ld_wait();
       if (valid) {
-        if (p.cin) {
-          const float4* c = reinterpret_cast<const float4*>(p.cin + off + j);
+        if (has_c) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float4 x = c[i];
+            const float4 x = cc[i];
             v[4 * i + 0] = p.alpha * v[4 * i + 0] + p.beta * x.x;
             v[4 * i + 1] = p.alpha * v[4 * i + 1] + p.beta * x.y;
             v[4 * i + 2] = p.alpha * v[4 * i + 2] + p.beta * x.z;
