@@ -109,9 +109,19 @@ static void swa_run(const SwaDims& S, const SwaBufs& b, const void* q, const voi
   L(K_SWA, [&] {
     const int64_t rows = S.BH * S.T;
     const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(rows * 32, 256), 148 * 64));
-    (void)launch_pdl(k_swa_softmax, blocks, 256, 0, st, static_cast<const float*>(b.S), rows,
-                     static_cast<int>(S.nb), static_cast<int>(S.Lw), S.window,
-                     1.0f / sqrtf(static_cast<float>(S.d)), b.P);
+    const float scale = 1.0f / sqrtf(static_cast<float>(S.d));
+    const float* Sf = b.S;
+    const int nb = static_cast<int>(S.nb);
+    // rows of up to 33 x 128 scores are held in registers (read once)
+    switch (S.Lw / 128) {
+#define LACT_SWA_REG(NV) \
+      case NV: (void)launch_pdl(k_swa_softmax_reg<NV>, blocks, 256, 0, st, Sf, rows, nb, S.window, scale, b.P); break;
+      LACT_SWA_REG(2) LACT_SWA_REG(3) LACT_SWA_REG(5) LACT_SWA_REG(9) LACT_SWA_REG(17) LACT_SWA_REG(33)
+#undef LACT_SWA_REG
+      default:
+        (void)launch_pdl(k_swa_softmax, blocks, 256, 0, st, Sf, rows, nb, static_cast<int>(S.Lw), S.window, scale,
+                         b.P);
+    }
     return cudaGetLastError();
   });
   L(K_SWA_GEMM, [&] {   // out_z = P_z Vp_window(z), bf16

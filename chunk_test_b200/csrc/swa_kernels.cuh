@@ -134,4 +134,59 @@ __global__ void __launch_bounds__(256) k_swa_softmax(const float* __restrict__ S
   }
 }
 
+// The same softmax with the row held in registers: NV float4 per lane
+// (Lw = 128 * NV), so the scores are read once.
+template <int NV>
+__global__ void __launch_bounds__(256) k_swa_softmax_reg(const float* __restrict__ S, int64_t rows, int nb,
+                                                         int64_t window, float scale,
+                                                         __nv_bfloat16* __restrict__ P) {
+  griddep_launch();
+  griddep_wait();
+  constexpr int Lw = 128 * NV;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < rows;
+       w += nwarps) {
+    const int64_t z = w >> 7;
+    const int r = static_cast<int>(w & 127);
+    const int64_t m = z % nb;
+    const int64_t lo0 = window - m * 128;
+    const int64_t lo = lo0 > r + 1 ? lo0 : r + 1, hi = r + window;
+    const float* s = S + w * Lw;
+    float4 x[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) x[i] = *reinterpret_cast<const float4*>(s + 4 * lane + 128 * i);
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 4 * lane + 128 * i;
+      const float xs[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (c + e >= lo && c + e <= hi) mx = fmaxf(mx, xs[e] * scale);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 4 * lane + 128 * i;
+      float* xs = reinterpret_cast<float*>(&x[i]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float y = (c + e >= lo && c + e <= hi) ? __expf(xs[e] * scale - mx) : 0.f;
+        xs[e] = y;
+        sum += y;
+      }
+    }
+    sum = warp_sum(sum);
+    const float inv = 1.0f / sum;
+    __nv_bfloat16* p = P + w * Lw;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+      *reinterpret_cast<uint2*>(p + 4 * lane + 128 * i) =
+          make_uint2(pack_bf16x2(x[i].x * inv, x[i].y * inv), pack_bf16x2(x[i].z * inv, x[i].w * inv));
+  }
+}
+
 }  // namespace lact
