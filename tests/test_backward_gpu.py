@@ -76,6 +76,10 @@ CASES = [
               RULE_MOMENTUM, BF16), dict(per_bh=True, with_dw=True, scaled=True)),
     (Workload("bwd-bf16-d64-set", 1, 2, 1500, 300, 64, 128, 1500, UPDATE_THEN_APPLY, RULE_GD, BF16),
      dict(with_dw=True)),
+    (Workload("bwd-bf16-d256-atu-mom-mask", 1, 2, 1536, 1536, 256, 512, 256, APPLY_THEN_UPDATE,
+              RULE_MOMENTUM, BF16), dict(mask=video_update_mask(6, 1), scaled=True, with_dw=True)),
+    (Workload("bwd-bf16-d384-uta-ragged", 1, 1, 1100, 1100, 384, 768, 512, UPDATE_THEN_APPLY, RULE_GD,
+              BF16), dict(mask=[1, 0, 1], per_bh=True)),
 ]
 
 
