@@ -681,12 +681,12 @@ def run_swa(args, w: Workload):
                for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
     dom, (n_launch, ms_kind) = max(prof.items(), key=lambda kv: kv[1][1])
     roof = None
-    if dom == "swa_gemm_umma":
+    if dom in ("swa_gemm_umma", "swa_flash_umma"):
         achieved = flops * args.steps / (ms_kind / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
                 "frac": achieved / pk_sust, "kernel": dom, "launches": n_launch,
                 "avg_launch_us": 1e3 * ms_kind / n_launch, "timed": "alone (per-kernel pass)",
-                "traffic": None, "peak_source": f"{pk_src} sustained bf16",
+                "traffic": traffic_for(dom, w), "peak_source": f"{pk_src} sustained bf16",
                 "work": "algorithmic: 4 d FLOPs per (query, key) pair in the window"}
     elif dom == "swa_elem":
         Lw = window + 128
@@ -765,6 +765,7 @@ KERNEL_SOURCES = {
     "grad_umma": ("pair_kernels.cuh", "umma_kernels.cuh", "sm100.cuh"),
     "rule_renorm": ("elem_kernels.cuh", "sm100.cuh"),
     "qk_prologue": ("elem_kernels.cuh", "sm100.cuh"),
+    "swa_flash_umma": ("swa_flash.cuh", "umma_kernels.cuh", "sm100.cuh"),
 }
 
 

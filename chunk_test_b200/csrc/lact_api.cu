@@ -367,13 +367,13 @@ static cudaError_t launch_gemm_any(bool split, int bn, dim3 grid, const GemmPara
 enum Kind {
   K_INIT, K_PROLOGUE, K_BETA_MEAN, K_FWD_QUERY, K_APPLY_OUT, K_FWD_KEY, K_GRAD, K_NS_SUMSQ,
   K_NS_SCALE, K_NS_GRAM, K_NS_POLY, K_NS_UPDATE, K_RULE, K_FINALIZE, K_SIMT_GEMM, K_FWD_ELEM_F32,
-  K_APPLY_FUSED, K_KEY_GRAD, K_BWD_ELEM, K_BWD_GEMM, K_SWA, K_SWA_GEMM, K_COUNT
+  K_APPLY_FUSED, K_KEY_GRAD, K_BWD_ELEM, K_BWD_GEMM, K_SWA, K_SWA_GEMM, K_SWA_FLASH, K_COUNT
 };
 static const char* const kKindNames[K_COUNT] = {
     "init_state", "qk_prologue", "beta_mean", "fwd_query_umma", "apply_out_umma", "fwd_key_umma",
     "grad_umma", "ns_sumsq", "ns_scale", "ns_gram_umma", "ns_poly_umma", "ns_update_umma",
     "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32", "apply_fused_umma",
-    "key_grad_umma", "bwd_elem", "bwd_gemm_umma", "swa_elem", "swa_gemm_umma"};
+    "key_grad_umma", "bwd_elem", "bwd_gemm_umma", "swa_elem", "swa_gemm_umma", "swa_flash_umma"};
 
 // Optional per-launch CUDA-event pairs on the launching stream.
 struct ProfRec { int kind; cudaEvent_t a, b; };
