@@ -10,9 +10,12 @@
 //   3. k_swa_softmax: the sliding causal mask, 1/sqrt(d) and the softmax,
 //      P in bf16;
 //   4. out_z = P_z Vp_window on the tensor cores (V MN-major), bf16 out.
-// For head dims up to 256, steps 2-4 run fused in k_swa_flash (the scores
-// stay on chip, online softmax); larger head dims take the path above, whose
-// scores make a round trip through HBM (fp32 S, bf16 P).
+// For head dims up to 256 the path is two launches: k_swa_prologue_q writes
+// Qt = q' * k_scale (the key offset only adds a per-query constant to the
+// scores, which the softmax removes), and k_swa_flash reads Qt with the
+// caller's k and v as they are, the scores staying on chip (online
+// softmax).  Larger head dims take the path above, whose scores make a round
+// trip through HBM (fp32 S, bf16 P).
 #pragma once
 
 #include "swa_flash.cuh"
@@ -47,20 +50,20 @@ struct SwaBufs {
 static bool swa_fused(const SwaDims& S) { return S.d <= 256; }
 
 static void swa_plan(const SwaDims& S, Bump& bp, SwaBufs& b) {
-  const int64_t pad_rows = S.BH * (S.window + S.T) + S.tail;
   b.Qp = bp.take<__nv_bfloat16>(S.BH * S.T * S.d);
+  b.Kp = b.Vp = b.P = nullptr;
+  b.S = nullptr;
+  if (swa_fused(S)) return;
+  const int64_t pad_rows = S.BH * (S.window + S.T) + S.tail;
   b.Kp = bp.take<__nv_bfloat16>(pad_rows * S.d);
   b.Vp = bp.take<__nv_bfloat16>(pad_rows * S.d);
-  b.S = nullptr;
-  b.P = nullptr;
-  if (!swa_fused(S)) {
-    b.S = bp.take<float>(S.BH * S.T * S.Lw);
-    b.P = bp.take<__nv_bfloat16>(S.BH * S.T * S.Lw);
-  }
+  b.S = bp.take<float>(S.BH * S.T * S.Lw);
+  b.P = bp.take<__nv_bfloat16>(S.BH * S.T * S.Lw);
 }
 
 template <int D>
-static cudaError_t launch_swa_flash(const SwaDims& S, const SwaBufs& b, void* out, cudaStream_t st) {
+static cudaError_t launch_swa_flash(const SwaDims& S, const SwaBufs& b, const void* k, const void* v, void* out,
+                                    cudaStream_t st) {
   constexpr int smem = SwaCfg<D>::kSmem;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -73,9 +76,8 @@ static cudaError_t launch_swa_flash(const SwaDims& S, const SwaBufs& b, void* ou
   }
   SwaFlashParams f;
   std::memset(&f, 0, sizeof(f));
-  const int64_t Tp = S.window + S.T;
-  if (!map3d(&f.tmQ, b.Qp, S.d, S.T, S.BH, 64, 128) || !map3d(&f.tmK, b.Kp, S.d, Tp, S.BH, 64, 128) ||
-      !map3d(&f.tmV, b.Vp, S.d, Tp, S.BH, 64, 64))
+  if (!map3d(&f.tmQ, b.Qp, S.d, S.T, S.BH, 64, 128) || !map3d(&f.tmK, k, S.d, S.T, S.BH, 64, 128) ||
+      !map3d(&f.tmV, v, S.d, S.T, S.BH, 64, 64))
     return cudaErrorInvalidValue;
   f.bh_count = static_cast<int>(S.BH); f.nb = static_cast<int>(S.nb); f.window = static_cast<int>(S.window);
   f.scale = 1.0f / sqrtf(static_cast<float>(S.d));
@@ -120,6 +122,24 @@ static void swa_run(const SwaDims& S, const SwaBufs& b, const void* q, const voi
                     cudaStream_t st, Launcher& L) {
   L.st = st;
   const int64_t items = S.BH * S.nb;
+  if (swa_fused(S)) {
+    L(K_SWA, [&] {
+      const int64_t n = S.BH * S.T * (S.d / 8);
+      const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(n, 256), 148 * 32));
+      (void)launch_pdl(k_swa_prologue_q, blocks, 256, 0, st, static_cast<const __nv_bfloat16*>(q), qs, qo, ks,
+                       static_cast<int>(S.H), S.T, static_cast<int>(S.d), n, b.Qp);
+      return cudaGetLastError();
+    });
+    L(K_SWA_FLASH, [&] {
+      switch (S.d) {
+        case 64: return launch_swa_flash<64>(S, b, k, v, out, st);
+        case 128: return launch_swa_flash<128>(S, b, k, v, out, st);
+        case 192: return launch_swa_flash<192>(S, b, k, v, out, st);
+        default: return launch_swa_flash<256>(S, b, k, v, out, st);
+      }
+    });
+    return;
+  }
   L(K_SWA, [&] {
     const int64_t n = (S.BH * S.T + S.BH * S.window + S.tail) * (S.d / 8);
     const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(n, 256), 148 * 32));
@@ -129,17 +149,6 @@ static void swa_run(const SwaDims& S, const SwaBufs& b, const void* q, const voi
                      b.Qp, b.Kp, b.Vp);
     return cudaGetLastError();
   });
-  if (swa_fused(S)) {
-    L(K_SWA_FLASH, [&] {
-      switch (S.d) {
-        case 64: return launch_swa_flash<64>(S, b, out, st);
-        case 128: return launch_swa_flash<128>(S, b, out, st);
-        case 192: return launch_swa_flash<192>(S, b, out, st);
-        default: return launch_swa_flash<256>(S, b, out, st);
-      }
-    });
-    return;
-  }
   L(K_SWA_GEMM, [&] {   // S_z = Qp_z Kp_window(z)^T, fp32
     GemmParams g = gemm_params();
     const int bn = pick_bn_swa(S.Lw);

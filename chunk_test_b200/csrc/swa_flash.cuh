@@ -1,9 +1,10 @@
 // swa_flash.cuh -- fused sliding-window attention for head dims up to 256:
 // the scores and probabilities of a block of 128 queries stay on chip (TMEM
 // and shared memory) while it walks the key blocks of its window, with an
-// online softmax ("LaCT架构核心思想解析" §1.1; the layout of q', k', v is
-// the one swa_kernels.cuh describes: keys and values in padded buffers
-// [BH][w + T][d], key j at padded row w + j).
+// online softmax ("LaCT架构核心思想解析" §1.1).  Inputs: Qt [BH][T][d]
+// from k_swa_prologue_q (q' times the key scale) and the caller's k and v
+// [BH][T][d] as given; the scores Qt . k differ from q' . k' by a constant
+// per query, which the softmax removes.
 //
 // Persistent CTAs over tiles (head, 128-query block m); per tile the key
 // blocks j0..m, j0 = max(0, m - w/128), each of 128 keys.  Warps:
@@ -13,7 +14,9 @@
 //   2..5  softmax, one query row per thread: masked row max of S_j, the
 //         online rescale of the output row in TMEM when the max grows,
 //         P_j = exp(s - max) in bf16 into a swizzled K-major smem tile, and
-//         the row sum; after the last block, out = O / sum in bf16.
+//         the row sum; after the last block, out = O / sum in bf16.  The
+//         softmax is the plain one up to rounding: the reference max of a
+//         row only lags the true running max by at most 8 in log2 units.
 //   6     P V issuer: O += P_j V_j (TMEM, D columns).
 // Every wait is bounded (mbar_wait); a wait that gives up records the
 // timeout in the device status word and the CTA stops.
@@ -24,9 +27,9 @@
 namespace lact {
 
 struct SwaFlashParams {
-  CUtensorMap tmQ;   // q'  [BH][T][d],        box {64, 128}
-  CUtensorMap tmK;   // k'  [BH][w + T][d],    box {64, 128}
-  CUtensorMap tmV;   // v   [BH][w + T][d],    box {64, 64}
+  CUtensorMap tmQ;   // Qt [BH][T][d], box {64, 128}
+  CUtensorMap tmK;   // k  [BH][T][d], box {64, 128}
+  CUtensorMap tmV;   // v  [BH][T][d], box {64, 64}
   int bh_count, nb;  // heads, 128-query blocks per head
   int window;        // w (a multiple of 128)
   float scale;       // 1 / sqrt(d)
@@ -49,6 +52,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[15])));
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x by the ex2.approx instruction (-inf gives 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <int D>
 struct SwaCfg {
@@ -148,7 +158,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
         const int j0 = m - wb > 0 ? m - wb : 0;
         for (int j = j0; j <= m; ++j, ++ik) {
           const int st = ik % KS;
-          const int prow = p.window + j * 128;   // padded row of key j*128
+          const int prow = j * 128;   // first key of block j
           if (ik >= KS && !mbar_wait(&kempty[st], ((ik / KS) - 1) & 1)) { ok = false; break; }
           uint8_t* kd = smem + C::kOffK + st * C::kKBytes;
           mbar_arrive_expect_tx(&kfull[st], C::kKBytes);
@@ -216,10 +226,18 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
     }
   } else {
     // ------------------------------------------------------------ softmax
+    // One query row per thread.  The row of S_j is loaded into registers in
+    // one go, so the S buffer is released before the exponentials.  Scores
+    // stay in raw units; exp(x) is computed as 2^(x log2 e) with the ex2
+    // instruction, the scale folded into one FMA per score.  The reference
+    // max mx of a row is raised only when a block's max exceeds it by more
+    // than 8 in log2 units, so the output row is rescaled rarely and the
+    // unnormalised probabilities stay below 2^8.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t prow_s = smem_u32(smem + C::kOffP) + r * 128;
+    const float c2 = p.scale * 1.4426950408889634f;   // log2 e / sqrt(d)
     int sc = 0, pc = 0, tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
@@ -228,78 +246,81 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
       float mx = -INFINITY, sum = 0.f;
       for (int j = j0; j <= m; ++j, ++sc, ++pc) {
         const int sb = sc & 1;
-        // valid columns of this row in key block j: [lo, hi]
-        const int hi = j == m ? r : 127;
-        const int lo = (j == m - wb) ? r + 1 : 0;
         // waits are made warp-uniform: the TMEM loads and stores below are
         // warp-collective, so every lane must take the same path
         if (!__all_sync(0xffffffffu, mbar_wait(&sfull[sb], (sc >> 1) & 1))) { ok = false; break; }
         tc_fence_after();
         const uint32_t ts = tq + C::kColS + sb * 128;
-        float bm = -INFINITY;
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 16) {
-          float v[16];
-          __syncwarp();
-          tmem_ld16(ts + c0, v);
-          tmem_ld_wait();
+        float sv[128];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i >= lo && c0 + i <= hi) bm = fmaxf(bm, v[i] * p.scale);
+        for (int c0 = 0; c0 < 128; c0 += 16) tmem_ld16(ts + c0, sv + c0);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[sb]);
+        // only the diagonal block and the block at the window's start are cut
+        if (j == m || j == m - wb) {
+          const int hi = j == m ? r : 127;
+          const int lo = j == m - wb ? r + 1 : 0;
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i < lo || i > hi) sv[i] = -INFINITY;
         }
-        const float mn = fmaxf(mx, bm);
+        float b8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) b8[i] = sv[i];
+#pragma unroll
+        for (int i = 8; i < 128; ++i) b8[i & 7] = fmaxf(b8[i & 7], sv[i]);
+        const float bm = fmaxf(fmaxf(fmaxf(b8[0], b8[1]), fmaxf(b8[2], b8[3])),
+                               fmaxf(fmaxf(b8[4], b8[5]), fmaxf(b8[6], b8[7])));
+        float a = 1.0f;
+        bool grow = false;
+        if (mx == -INFINITY) {
+          mx = bm;   // no earlier key of this row: its output row and sum are zero
+        } else if ((bm - mx) * c2 > 8.0f) {
+          grow = true;
+          a = ex2_approx((mx - bm) * c2);
+          mx = bm;
+        }
+        const float off = mx == -INFINITY ? 0.f : -mx * c2;
+        uint32_t hw[64];
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float e0 = ex2_approx(fmaf(sv[2 * i], c2, off));
+          const float e1 = ex2_approx(fmaf(sv[2 * i + 1], c2, off));
+          ps[i & 3] += e0 + e1;
+          hw[i] = pack_bf16x2(e0, e1);
+        }
         // the previous block's P V has finished with O and with the P tile
         if (pc > 0 && !__all_sync(0xffffffffu, mbar_wait(pempty, (pc - 1) & 1))) { ok = false; break; }
         tc_fence_after();
-        // rescale the output row by exp(mx - mn) where the row max grew; the
-        // whole warp runs the loop when any lane needs it (factor 1 elsewhere)
-        const bool grow = j > j0 && mx != -INFINITY && mn > mx;
-        const float a = grow ? __expf(mx - mn) : 1.0f;
-        if (__any_sync(0xffffffffu, grow)) {
+        if (__any_sync(0xffffffffu, grow)) {   // the whole warp runs it; factor 1 in other rows
 #pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            float o[16];
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float o[32];
             __syncwarp();
             tmem_ld16(tq + C::kColO + c0, o);
+            tmem_ld16(tq + C::kColO + c0 + 16, o + 16);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] *= a;
+            for (int i = 0; i < 32; ++i) o[i] *= a;
             tmem_st16(tq + C::kColO + c0, o);
+            tmem_st16(tq + C::kColO + c0 + 16, o + 16);
           }
           tmem_st_wait();
         }
-        sum *= a;
-        mx = mn;
-        float ps = 0.f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 16) {
-          float v[16];
-          __syncwarp();
-          tmem_ld16(ts + c0, v);
-          tmem_ld_wait();
-          uint32_t hw[8];
+        sum = sum * a + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+        // row r of the K-major 128-byte-swizzled P tile: 64 keys per 16 KB
+        // block, 16-byte chunk g holds keys 8g..8g+7
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int c = c0 + 2 * i;
-            const float e0 = (c >= lo && c <= hi) ? __expf(v[2 * i] * p.scale - mn) : 0.f;
-            const float e1 = (c + 1 >= lo && c + 1 <= hi) ? __expf(v[2 * i + 1] * p.scale - mn) : 0.f;
-            ps += e0 + e1;
-            hw[i] = pack_bf16x2(e0, e1);
-          }
-          // row r of the K-major 128-byte-swizzled P tile: 64 keys per 16 KB block
-          const uint32_t base = prow_s + (c0 >> 6) * 16384;
-          const int ch = (c0 & 63) >> 3;   // first 16-byte chunk of these 16 keys
-          st_shared_v4(base + (((ch) ^ (r & 7)) << 4), hw[0], hw[1], hw[2], hw[3]);
-          st_shared_v4(base + (((ch + 1) ^ (r & 7)) << 4), hw[4], hw[5], hw[6], hw[7]);
-        }
-        sum += ps;
+        for (int g = 0; g < 16; ++g)
+          st_shared_v4(prow_s + (g >> 3) * 16384 + (((g & 7) ^ (r & 7)) << 4), hw[4 * g], hw[4 * g + 1],
+                       hw[4 * g + 2], hw[4 * g + 3]);
         tc_fence_before();
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&sempty[sb]);
-          mbar_arrive(pfull);
-        }
+        if (lane == 0) mbar_arrive(pfull);
       }
       if (!ok) break;
       // O is complete: out = O / sum
@@ -308,15 +329,18 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
       const float inv = sum > 0.f ? 1.0f / sum : 0.f;
       __nv_bfloat16* dst = p.out + (static_cast<int64_t>(bh) * p.T + static_cast<int64_t>(m) * 128 + r) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        float o[16];
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float o[32];
         __syncwarp();
         tmem_ld16(tq + C::kColO + c0, o);
+        tmem_ld16(tq + C::kColO + c0 + 16, o + 16);
         tmem_ld_wait();
-        st_global_v4(dst + c0, pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
-                     pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
-        st_global_v4(dst + c0 + 8, pack_bf16x2(o[8] * inv, o[9] * inv), pack_bf16x2(o[10] * inv, o[11] * inv),
-                     pack_bf16x2(o[12] * inv, o[13] * inv), pack_bf16x2(o[14] * inv, o[15] * inv));
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          st_global_v4(dst + c0 + 8 * g, pack_bf16x2(o[8 * g] * inv, o[8 * g + 1] * inv),
+                       pack_bf16x2(o[8 * g + 2] * inv, o[8 * g + 3] * inv),
+                       pack_bf16x2(o[8 * g + 4] * inv, o[8 * g + 5] * inv),
+                       pack_bf16x2(o[8 * g + 6] * inv, o[8 * g + 7] * inv));
       }
       tc_fence_before();
       __syncwarp();

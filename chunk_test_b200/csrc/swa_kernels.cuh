@@ -74,6 +74,43 @@ __global__ void __launch_bounds__(256) k_swa_prologue(const __nv_bfloat16* __res
   }
 }
 
+// Query prologue of the fused path: Qt = (q * q_scale + q_offset) * k_scale
+// per head and channel, so that Qt . k = q' . k' - q' . k_offset.  The last
+// term is the same for every key of a query and the softmax removes it, so
+// the keys and values are read as given.  Grid-stride over 16-byte vectors.
+__global__ void __launch_bounds__(256) k_swa_prologue_q(const __nv_bfloat16* __restrict__ q,
+                                                        const float* __restrict__ qs,
+                                                        const float* __restrict__ qo,
+                                                        const float* __restrict__ ks, int H, int64_t T,
+                                                        int d, int64_t n, __nv_bfloat16* __restrict__ Qt) {
+  griddep_launch();
+  griddep_wait();
+  const int nv = d >> 3;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t row = i / nv;             // bh * T + t
+    const int c = static_cast<int>(i % nv) * 8;
+    const int h = static_cast<int>((row / T) % H);
+    const uint4 qv = *reinterpret_cast<const uint4*>(q + row * d + c);
+    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+    const float4* s4 = reinterpret_cast<const float4*>(qs + h * d + c);
+    const float4* o4 = reinterpret_cast<const float4*>(qo + h * d + c);
+    const float4* k4 = reinterpret_cast<const float4*>(ks + h * d + c);
+    const float4 sa = s4[0], sb = s4[1], oa = o4[0], ob = o4[1], ka = k4[0], kb = k4[1];
+    const float sc[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+    const float of[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
+    const float kc[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+    uint32_t ow[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float q0 = __uint_as_float(qw[e] << 16), q1 = __uint_as_float(qw[e] & 0xffff0000u);
+      ow[e] = pack_bf16x2(fmaf(q0, sc[2 * e], of[2 * e]) * kc[2 * e],
+                          fmaf(q1, sc[2 * e + 1], of[2 * e + 1]) * kc[2 * e + 1]);
+    }
+    *reinterpret_cast<uint4*>(Qt + row * d + c) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  }
+}
+
 // Masked softmax of the window scores, one warp per query row.  S and P are
 // [BH * nb][128][Lw] (Lw = w + 128, a multiple of 128): row r of block z
 // (query t = m*128 + r, m = z % nb) sees padded window rows p with

@@ -278,10 +278,12 @@ int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts,
  * includes the token itself).  q, k, v, out [B, H, T, d] bf16 (device);
  * q_scale, q_offset, k_scale, k_offset [H, d] float32 (device).  Limits: d
  * a multiple of 64 up to 512, T and window multiples of 128, window <=
- * 16384, B*H <= 4096.  The scores take a round trip through the workspace
- * (fp32 scores, bf16 probabilities: B*H*T*(window+128)*6 bytes);
- * lact_swa_workspace_bytes gives its size.  Asynchronous on `stream`; the
- * error behaviour of lact_ttt_fwd. */
+ * 16384, B*H <= 4096.  For d <= 256 the scores stay on chip and the
+ * workspace holds one transformed copy of q (B*H*T*d bf16); for d = 320..512
+ * the scores take a round trip through it (fp32 scores, bf16
+ * probabilities: B*H*T*(window+128)*6 bytes, plus padded copies of k' and
+ * v).  lact_swa_workspace_bytes gives its size.  Asynchronous on `stream`;
+ * the error behaviour of lact_ttt_fwd. */
 typedef struct lact_swa_problem {
   int64_t B, H, T, d, window;
   int32_t dtype;   /* LACT_BF16 */
