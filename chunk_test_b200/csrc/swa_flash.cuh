@@ -8,8 +8,12 @@
 //
 // Persistent CTAs over tiles (head, 128-query block m); per tile the key
 // blocks j0..m, j0 = max(0, m - w/128), each of 128 keys.  Warps:
-//   0     TMA producer: q' tile once per tile; per key block its K tile
-//         (K-major operand of S) and V tile (MN-major operand of P V).
+//   0     TMA producer of the queries (once per tile) and of each key
+//         block's K tile (K-major operand of S).
+//   7     TMA producer of the V tiles (MN-major operand of P V), in two
+//         halves of 64 keys with their own barriers, so the next block's
+//         first half loads while the second half of P V runs.  Keys and
+//         values have separate producers: a K load never waits for P V.
 //   1     S issuer: S_j = Q K_j^T into one of two TMEM buffers (128 cols).
 //   2..5  softmax, one query row per thread: masked row max of S_j, the
 //         online rescale of the output row in TMEM when the max grows,
@@ -37,8 +41,9 @@ struct SwaFlashParams {
   int64_t T;
 };
 
-constexpr int kSwaThreads = 224;
+constexpr int kSwaThreads = 256;
 constexpr int kSwaPvWarp = 6;
+constexpr int kSwaVWarp = 7;
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile(
@@ -75,8 +80,9 @@ struct SwaCfg {
   static constexpr int kOffV = kOffK + kStages * kKBytes;
   static constexpr int kOffP = kOffV + kStages * kVBytes;
   static constexpr int kOffBar = kOffP + kPBytes;
-  // qfull qempty | kfull kempty vfull vempty (x stages) | sfull[2] sempty[2] | pfull pempty | ofull oempty
-  static constexpr int kBars = 2 + 4 * kStages + 4 + 2 + 2;
+  // qfull qempty | kfull kempty (x stages) | vfull vempty (x 2 halves x stages) | sfull[2] sempty[2] |
+  // pfull pempty | ofull oempty
+  static constexpr int kBars = 2 + 2 * kStages + 4 * kStages + 4 + 2 + 2;
   static constexpr int kSmem = kOffBar + kBars * 8 + 16 + 1024;
   static constexpr uint32_t kColO = 0, kColS = 256;
 };
@@ -94,9 +100,9 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
   uint64_t* qempty = bar + 1;
   uint64_t* kfull = bar + 2;
   uint64_t* kempty = kfull + KS;
-  uint64_t* vfull = kempty + KS;
-  uint64_t* vempty = vfull + KS;
-  uint64_t* sfull = vempty + KS;
+  uint64_t* vfull = kempty + KS;     // [stage * 2 + half]
+  uint64_t* vempty = vfull + 2 * KS;
+  uint64_t* sfull = vempty + 2 * KS;
   uint64_t* sempty = sfull + 2;
   uint64_t* pfull = sempty + 2;
   uint64_t* pempty = pfull + 1;
@@ -119,6 +125,8 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
     for (int i = 0; i < KS; ++i) {
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < 2 * KS; ++i) {
       mbar_init(&vfull[i], 1);
       mbar_init(&vempty[i], 1);
     }
@@ -163,12 +171,27 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
           uint8_t* kd = smem + C::kOffK + st * C::kKBytes;
           mbar_arrive_expect_tx(&kfull[st], C::kKBytes);
           for (int kb = 0; kb < C::kKb; ++kb) tma_load_3d(kd + kb * 16384, &p.tmK, &kfull[st], kb * 64, prow, bh);
-          if (ik >= KS && !mbar_wait(&vempty[st], ((ik / KS) - 1) & 1)) { ok = false; break; }
+        }
+      }
+    }
+  } else if (warp == kSwaVWarp) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0) {
+      int ik = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        const int m = tile % p.nb, bh = tile / p.nb;
+        const int j0 = m - wb > 0 ? m - wb : 0;
+        for (int j = j0; ok && j <= m; ++j, ++ik) {
+          const int st = ik % KS;
           uint8_t* vd = smem + C::kOffV + st * C::kVBytes;
-          mbar_arrive_expect_tx(&vfull[st], C::kVBytes);
-          for (int kk = 0; kk < 2; ++kk)
+          for (int h = 0; h < 2; ++h) {
+            uint64_t* full = &vfull[2 * st + h];
+            if (ik >= KS && !mbar_wait(&vempty[2 * st + h], ((ik / KS) - 1) & 1)) { ok = false; break; }
+            mbar_arrive_expect_tx(full, C::kVBytes / 2);
             for (int nb = 0; nb < C::kKb; ++nb)
-              tma_load_3d(vd + (kk * C::kKb + nb) * 8192, &p.tmV, &vfull[st], nb * 64, prow + kk * 64, bh);
+              tma_load_3d(vd + (h * C::kKb + nb) * 8192, &p.tmV, full, nb * 64, j * 128 + h * 64, bh);
+          }
         }
       }
     }
@@ -212,19 +235,21 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
           const int st = ik % KS;
           if (j == j0 && tc > 0 && !mbar_wait(oempty, (tc - 1) & 1)) { ok = false; break; }
           if (!mbar_wait(pfull, pc & 1)) { ok = false; break; }
-          if (!mbar_wait(&vfull[st], (ik / KS) & 1)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t vb = sbase + C::kOffV + st * C::kVBytes;
-          for (int kk = 0; kk < 2; ++kk)
+          for (int kk = 0; kk < 2 && ok; ++kk) {   // keys 64 kk .. 64 kk + 63
+            if (!mbar_wait(&vfull[2 * st + kk], (ik / KS) & 1)) { ok = false; break; }
+            tc_fence_after();
             mma_kblock<false, true>(tmem + C::kColO, sbase + C::kOffP + kk * 16384, 0, vb + kk * C::kKb * 8192,
                                     8192, ido, j == j0 && kk == 0);
-          umma_commit(&vempty[st]);
+            umma_commit(&vempty[2 * st + kk]);
+          }
+          if (!ok) break;
           umma_commit(pempty);
         }
         if (ok) umma_commit(ofull);
       }
     }
-  } else {
+  } else if (warp >= 2 && warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ softmax
     // One query row per thread.  The row of S_j is loaded into registers in
     // one go, so the S buffer is released before the exponentials.  Scores

@@ -75,3 +75,25 @@ def test_swa_at_the_lm760m_shape_on_sampled_rows():
     err = rel_l2(g, r)
     assert err <= 2e-2, err
     print(f"swa lm760m sampled: rel-L2 {err:.2e}")
+
+
+@pytest.mark.parametrize("d", [128, 512])
+def test_swa_with_wide_scales_and_offsets(d):
+    """Offsets of order one and scales far from one.  The fused path (d up to
+    256) drops the key offset, a constant per query in the scores, and folds
+    the key scale into the queries; the materialised path (d 512) applies
+    both to the keys.  The oracle applies them as defined."""
+    inp = make_swa_inputs(1, 2, 768, d, seed=11)
+    g = torch.Generator().manual_seed(12)
+    shape = inp["q_scale"].shape
+    inp["q_scale"] = 1.0 + 0.5 * torch.randn(shape, generator=g)
+    inp["q_offset"] = torch.randn(shape, generator=g)
+    inp["k_scale"] = 1.0 + 0.5 * torch.randn(shape, generator=g)
+    inp["k_offset"] = 2.0 * torch.randn(shape, generator=g)
+    WINDOW[0] = 256
+    got = run(inp)
+    want = so.swa_layer(inp["q"], inp["k"], inp["v"], inp["q_scale"], inp["q_offset"], inp["k_scale"],
+                        inp["k_offset"], 256)
+    err = rel_l2(got, want)
+    assert err <= 2e-2, err
+    print(f"swa wide scales d{d}: rel-L2 {err:.2e}")
