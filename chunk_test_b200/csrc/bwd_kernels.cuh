@@ -158,9 +158,13 @@ __device__ __forceinline__ float sigm(float z) { return 1.0f / (1.0f + expf(-z))
 // The second-order factors of one element: the partials of phi with respect
 // to (z1, u, z3, p, q, r), and the element's terms of dphi/dlr.
 struct HvpOut { float fz1, fu, fz3, fp, fq, fr, g1, g2, g3; };
+// FAST: the sigmoid on the fast exponential and division (relative error
+// about 1e-6, far below the bf16 rounding of the factors on the tensor-core
+// path); otherwise the accurate expf and IEEE division of the fp32 path.
+template <bool FAST = false>
 __device__ __forceinline__ HvpOut hvp_factors(float z1, float u, float z3, float pp, float qq, float rr,
                                               float e1, float e2, float e3) {
-  const float sg = 1.0f / (1.0f + expf(-z1));
+  const float sg = FAST ? sigmoidf_(z1) : 1.0f / (1.0f + expf(-z1));
   const float s = z1 * sg;
   const float sp = sg * (1.0f + z1 * (1.0f - sg));
   const float spp = sg * (1.0f - sg) * (2.0f + z1 * (1.0f - 2.0f * sg));
@@ -219,168 +223,6 @@ __global__ void __launch_bounds__(256) k_hvp_elem(float* __restrict__ Z, float* 
     o[0] = g1;
     o[1] = g2;
     o[2] = g3;
-  }
-}
-
-__device__ __forceinline__ uint2 pack4_bf16(float a, float b, float c, float d) {
-  return make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
-}
-
-// The second-order factors on row-concatenated blocks, for merged
-// contractions: in Zk = [z1 | z3 | p | r] ([BH][rows][4 dh]) and Zv = [u | q]
-// ([BH][rows][2 dh]), fp32; out Phik = [dz1 | dz3 | dp | dr] and Phiv =
-// [du | dq] in bf16 with rows n..rows-1 as zeros, and dlr.  Warps walk the
-// rows; each lane takes 4 consecutive columns per step (dh is a multiple of
-// 64).
-__global__ void __launch_bounds__(256) k_hvp_elem_cat(const float* __restrict__ Zk,
-                                                      const float* __restrict__ Zv, int BH, int64_t rows,
-                                                      int dh, int n, const float* __restrict__ lr, int64_t T,
-                                                      int64_t row0, float* __restrict__ dlr,
-                                                      __nv_bfloat16* __restrict__ Phik,
-                                                      __nv_bfloat16* __restrict__ Phiv) {
-  griddep_launch();
-  griddep_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       w < static_cast<int64_t>(BH) * rows; w += nwarps) {
-    const int64_t bh = w / rows, i = w % rows;
-    const float* zk = Zk + w * 4 * dh;
-    const float* zv = Zv + w * 2 * dh;
-    __nv_bfloat16* pk = Phik + w * 4 * dh;
-    __nv_bfloat16* pv = Phiv + w * 2 * dh;
-    if (i >= n) {
-      for (int c = 4 * lane; c < 4 * dh; c += 128) *reinterpret_cast<uint2*>(pk + c) = make_uint2(0u, 0u);
-      for (int c = 4 * lane; c < 2 * dh; c += 128) *reinterpret_cast<uint2*>(pv + c) = make_uint2(0u, 0u);
-      continue;
-    }
-    const float* l = lr + (bh * T + row0 + i) * 3;
-    const float e1 = l[0], e2 = l[1], e3 = l[2];
-    float g1 = 0.f, g2 = 0.f, g3 = 0.f;
-    for (int c = 4 * lane; c < dh; c += 128) {
-      const float4 z1 = *reinterpret_cast<const float4*>(zk + c);
-      const float4 z3 = *reinterpret_cast<const float4*>(zk + dh + c);
-      const float4 pp = *reinterpret_cast<const float4*>(zk + 2 * dh + c);
-      const float4 rr = *reinterpret_cast<const float4*>(zk + 3 * dh + c);
-      const float4 u = *reinterpret_cast<const float4*>(zv + c);
-      const float4 qq = *reinterpret_cast<const float4*>(zv + dh + c);
-      HvpOut f[4];
-      f[0] = hvp_factors(z1.x, u.x, z3.x, pp.x, qq.x, rr.x, e1, e2, e3);
-      f[1] = hvp_factors(z1.y, u.y, z3.y, pp.y, qq.y, rr.y, e1, e2, e3);
-      f[2] = hvp_factors(z1.z, u.z, z3.z, pp.z, qq.z, rr.z, e1, e2, e3);
-      f[3] = hvp_factors(z1.w, u.w, z3.w, pp.w, qq.w, rr.w, e1, e2, e3);
-      *reinterpret_cast<uint2*>(pk + c) = pack4_bf16(f[0].fz1, f[1].fz1, f[2].fz1, f[3].fz1);
-      *reinterpret_cast<uint2*>(pk + dh + c) = pack4_bf16(f[0].fz3, f[1].fz3, f[2].fz3, f[3].fz3);
-      *reinterpret_cast<uint2*>(pk + 2 * dh + c) = pack4_bf16(f[0].fp, f[1].fp, f[2].fp, f[3].fp);
-      *reinterpret_cast<uint2*>(pk + 3 * dh + c) = pack4_bf16(f[0].fr, f[1].fr, f[2].fr, f[3].fr);
-      *reinterpret_cast<uint2*>(pv + c) = pack4_bf16(f[0].fu, f[1].fu, f[2].fu, f[3].fu);
-      *reinterpret_cast<uint2*>(pv + dh + c) = pack4_bf16(f[0].fq, f[1].fq, f[2].fq, f[3].fq);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        g1 += f[e].g1;
-        g2 += f[e].g2;
-        g3 += f[e].g3;
-      }
-    }
-    g1 = warp_sum(g1);
-    g2 = warp_sum(g2);
-    g3 = warp_sum(g3);
-    if (lane == 0) {
-      float* o = dlr + (bh * T + row0 + i) * 3;
-      o[0] = g1;
-      o[1] = g2;
-      o[2] = g3;
-    }
-  }
-}
-
-// Apply backward on row-concatenated blocks: in Za = [z1 | z3]
-// ([BH][rows][2 dh]) and G = dO W2 ([BH][rows][dh], dO already scaled), fp32;
-// out Phia = [dz1 | dz3] and Hq = silu(z1) z3 in bf16, rows n..rows-1 zero.
-// Warps walk the rows, 4 columns per lane per step.
-__global__ void __launch_bounds__(256) k_apply_bwd_cat(const float* __restrict__ Za,
-                                                       const float* __restrict__ G, int BH, int64_t rows,
-                                                       int dh, int n, __nv_bfloat16* __restrict__ Phia,
-                                                       __nv_bfloat16* __restrict__ Hq) {
-  griddep_launch();
-  griddep_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       w < static_cast<int64_t>(BH) * rows; w += nwarps) {
-    const bool live = (w % rows) < n;
-    for (int c = 4 * lane; c < dh; c += 128) {
-      float4 dz1 = make_float4(0.f, 0.f, 0.f, 0.f), dz3 = dz1, hq = dz1;
-      if (live) {
-        const float4 z1 = *reinterpret_cast<const float4*>(Za + w * 2 * dh + c);
-        const float4 z3 = *reinterpret_cast<const float4*>(Za + w * 2 * dh + dh + c);
-        const float4 g = *reinterpret_cast<const float4*>(G + w * dh + c);
-        const float zz1[4] = {z1.x, z1.y, z1.z, z1.w}, zz3[4] = {z3.x, z3.y, z3.z, z3.w};
-        const float gg[4] = {g.x, g.y, g.z, g.w};
-        float a[4], b3[4], h[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float sg = 1.0f / (1.0f + expf(-zz1[e]));
-          const float s = zz1[e] * sg;
-          a[e] = gg[e] * zz3[e] * sg * (1.0f + zz1[e] * (1.0f - sg));
-          b3[e] = gg[e] * s;
-          h[e] = s * zz3[e];
-        }
-        dz1 = make_float4(a[0], a[1], a[2], a[3]);
-        dz3 = make_float4(b3[0], b3[1], b3[2], b3[3]);
-        hq = make_float4(h[0], h[1], h[2], h[3]);
-      }
-      *reinterpret_cast<uint2*>(Phia + w * 2 * dh + c) = pack4_bf16(dz1.x, dz1.y, dz1.z, dz1.w);
-      *reinterpret_cast<uint2*>(Phia + w * 2 * dh + dh + c) = pack4_bf16(dz3.x, dz3.y, dz3.z, dz3.w);
-      *reinterpret_cast<uint2*>(Hq + w * dh + c) = pack4_bf16(hq.x, hq.y, hq.z, hq.w);
-    }
-  }
-}
-
-// The keys' gradient factors of the forward recompute as bf16 operands:
-// E = (lr1 u z3 silu'(z1), lr2 silu(z1) z3, lr3 u silu(z1)) from Z = (z1, u,
-// z3), [3][BH][rows][dh]; rows n..rows-1 written as zeros.  Warps walk the
-// rows, 4 columns per lane per step.
-__global__ void __launch_bounds__(256) k_key_factors_bf16(const float* __restrict__ Z, int BH, int64_t rows,
-                                                          int dh, int n, const float* __restrict__ lr,
-                                                          int64_t T, int64_t row0,
-                                                          __nv_bfloat16* __restrict__ E) {
-  griddep_launch();
-  griddep_wait();
-  const int64_t plane = static_cast<int64_t>(BH) * rows * dh;
-  const int lane = threadIdx.x & 31;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       w < static_cast<int64_t>(BH) * rows; w += nwarps) {
-    const int64_t bh = w / rows, r = w % rows;
-    const bool live = r < n;
-    float l1 = 0.f, l2 = 0.f, l3 = 0.f;
-    if (live) {
-      const float* l = lr + (bh * T + row0 + r) * 3;
-      l1 = l[0]; l2 = l[1]; l3 = l[2];
-    }
-    for (int c = 4 * lane; c < dh; c += 128) {
-      const int64_t o = w * dh + c;
-      float e1[4] = {0.f, 0.f, 0.f, 0.f}, eh[4] = {0.f, 0.f, 0.f, 0.f}, e3[4] = {0.f, 0.f, 0.f, 0.f};
-      if (live) {
-        const float4 z1 = *reinterpret_cast<const float4*>(Z + o);
-        const float4 u = *reinterpret_cast<const float4*>(Z + plane + o);
-        const float4 z3 = *reinterpret_cast<const float4*>(Z + 2 * plane + o);
-        const float zz1[4] = {z1.x, z1.y, z1.z, z1.w}, uu[4] = {u.x, u.y, u.z, u.w};
-        const float zz3[4] = {z3.x, z3.y, z3.z, z3.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float sg = 1.0f / (1.0f + expf(-zz1[e]));
-          const float s = zz1[e] * sg;
-          e1[e] = l1 * uu[e] * zz3[e] * sg * (1.0f + zz1[e] * (1.0f - sg));
-          eh[e] = l2 * s * zz3[e];
-          e3[e] = l3 * uu[e] * s;
-        }
-      }
-      *reinterpret_cast<uint2*>(E + o) = pack4_bf16(e1[0], e1[1], e1[2], e1[3]);
-      *reinterpret_cast<uint2*>(E + plane + o) = pack4_bf16(eh[0], eh[1], eh[2], eh[3]);
-      *reinterpret_cast<uint2*>(E + 2 * plane + o) = pack4_bf16(e3[0], e3[1], e3[2], e3[3]);
-    }
   }
 }
 

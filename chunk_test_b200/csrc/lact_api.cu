@@ -206,6 +206,21 @@ static bool map3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same map without swizzle: boxes are dense row-major in shared memory
+// (used for bulk stores of narrow staging tiles).
+static bool map3d_plain(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint64_t batch,
+                        uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ launches
 // Every kernel is launched with programmatic stream serialization: the
 // next kernel of the stream may start while this one drains, does its local
@@ -367,13 +382,14 @@ static cudaError_t launch_gemm_any(bool split, int bn, dim3 grid, const GemmPara
 enum Kind {
   K_INIT, K_PROLOGUE, K_BETA_MEAN, K_FWD_QUERY, K_APPLY_OUT, K_FWD_KEY, K_GRAD, K_NS_SUMSQ,
   K_NS_SCALE, K_NS_GRAM, K_NS_POLY, K_NS_UPDATE, K_RULE, K_FINALIZE, K_SIMT_GEMM, K_FWD_ELEM_F32,
-  K_APPLY_FUSED, K_KEY_GRAD, K_BWD_ELEM, K_BWD_GEMM, K_SWA, K_SWA_GEMM, K_SWA_FLASH, K_COUNT
+  K_APPLY_FUSED, K_KEY_GRAD, K_BWD_ELEM, K_BWD_GEMM, K_SWA, K_SWA_GEMM, K_SWA_FLASH, K_BWD_KEY, K_BWD_APPLY, K_COUNT
 };
 static const char* const kKindNames[K_COUNT] = {
     "init_state", "qk_prologue", "beta_mean", "fwd_query_umma", "apply_out_umma", "fwd_key_umma",
     "grad_umma", "ns_sumsq", "ns_scale", "ns_gram_umma", "ns_poly_umma", "ns_update_umma",
     "rule_renorm", "finalize_state", "simt_gemm_f32", "fwd_elem_f32", "apply_fused_umma",
-    "key_grad_umma", "bwd_elem", "bwd_gemm_umma", "swa_elem", "swa_gemm_umma", "swa_flash_umma"};
+    "key_grad_umma", "bwd_elem", "bwd_gemm_umma", "swa_elem", "swa_gemm_umma", "swa_flash_umma",
+    "bwd_key_umma", "bwd_apply_umma"};
 
 // Optional per-launch CUDA-event pairs on the launching stream.
 struct ProfRec { int kind; cudaEvent_t a, b; };

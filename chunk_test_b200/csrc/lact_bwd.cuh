@@ -21,6 +21,7 @@
 #pragma once
 
 #include "bwd_kernels.cuh"
+#include "bwd_key_op.cuh"
 
 namespace lact {
 
@@ -42,7 +43,7 @@ struct BwdBufs {
   float *dqh, *dkh, *ofull, *part;
   // bf16 problems (tensor-core contractions): bf16 operands
   __nv_bfloat16 *qh16, *kh16, *dos16, *hist16, *op16, *Gam16;
-  __nv_bfloat16 *Bk, *Bv, *Ba;   // stacked operands of the merged contractions
+  __nv_bfloat16 *Bk, *Bv;   // stacked operands of the merged contractions
   int64_t zr;   // rows per head of the per-chunk [rows][dh] planes
 };
 
@@ -68,7 +69,6 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
     b.Gam16 = bp.take<__nv_bfloat16>(planes);
     b.Bk = bp.take<__nv_bfloat16>(4 * D.BH * D.dh * D.d);
     b.Bv = bp.take<__nv_bfloat16>(2 * D.BH * D.dh * D.d);
-    b.Ba = bp.take<__nv_bfloat16>(2 * D.BH * D.dh * D.d);
   } else {
     b.dos32 = bp.take<float>(nq);
     b.qh = bp.take<float>(nq);
@@ -85,8 +85,10 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
     b.part = bp.take<float>(rule_rows(D));
   }
   b.mnorm = bp.take<float>(D.nch * rule_rows(D));
-  b.Z = bp.take<float>((bf ? 6 : 3) * zpl);     // bf16 problems: the merged blocks [z1|z3|p|r], [u|q]
-  if (!bf) b.Pz = bp.take<float>(3 * zpl);
+  if (!bf) {
+    b.Z = bp.take<float>(3 * zpl);
+    b.Pz = bp.take<float>(3 * zpl);
+  }
   b.P = bp.take<float>(planes);
   b.A = bp.take<float>(planes);
   b.Ap = bp.take<float>(planes);
@@ -468,11 +470,24 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
       return cudaGetLastError();
     });
   }
-  // the keys' forward at a state W (bf16): out = (k^ W1^T, v W2, k^ W3^T), rows of chunk c
-  auto key_forward = [&](const B16* W, int64_t c0, int nc, float* out) {
-    tcg(KM, KM, kh, static_cast<int>(c0), 0, Wop(W, 0), 0, nc, dh, d, out, zr * D.dh, dh, false);
-    tcg(KM, MN, vv, static_cast<int>(c0), 0, Wop(W, 1), 0, nc, dh, d, out + zpl, zr * D.dh, dh, false);
-    tcg(KM, KM, kh, static_cast<int>(c0), 0, Wop(W, 2), 0, nc, dh, d, out + 2 * zpl, zr * D.dh, dh, false);
+  // The forward's fused key kernel at a state W (bf16): z1 = X W1^T, z3 = X W3^T,
+  // g = Y W2 for rows x_row0 .. x_row0 + n of X and Y ([BH][rows][d]), and the
+  // factor planes E [3][BH][zr][dh] = (lr1 g z3 silu'(z1), lr2 silu(z1) z3,
+  // lr3 g silu(z1)); lr null means unit rates.
+  auto fwd_key = [&](int kind, const B16* W, const Opnd& X, const void* Y, int x_row0, int n, const float* lr,
+                     B16* E) {
+    L(kind, [&] {
+      FwdParams f;
+      std::memset(&f, 0, sizeof(f));
+      if (!map3d(&f.tmX, X.p, D.d, X.rows, D.BH, 64, 128) || !map3d(&f.tmV, Y, D.d, X.rows, D.BH, 64, 128) ||
+          !map3d(&f.tmW, W, D.d, D.dh, 3 * D.BH, 64, 64) || !map3d(&f.tmW2, W + jst, D.dh, D.d, D.BH, 64, 64) ||
+          !map3d(&f.tmE, E, D.dh, zr, 3 * D.BH, 64, 32))
+        return cudaErrorInvalidValue;
+      f.bh_count = BH; f.n_slices = dh / 64; f.n_row_tiles = static_cast<int>(cdiv(n, 128));
+      f.x_row0 = x_row0; f.rows_valid = n; f.kb_count = d / 64; f.dh = dh; f.T = static_cast<int>(X.rows);
+      f.e = E; f.buf_rows = zr; f.lr = lr;
+      return launch_umma<FwdOp<true>>(static_cast<int64_t>(f.n_slices) * f.n_row_tiles * BH, f, st);
+    });
   };
 
   // ---- forward recompute: the states, momenta and pre-renorm row norms
@@ -483,12 +498,7 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     copy(b.hist16 + (c + 1) * planes, b.hist16 + c * planes, planes * 2);
     if (in.mask && in.mask[c] == 0) continue;
     if (mom) copy(b.mh + c * planes, b.Mm, planes * 4);
-    key_forward(b.hist16 + c * planes, c0, nc, b.Z);
-    L(K_BWD_ELEM, [&] {
-      (void)launch_pdl(k_key_factors_bf16, grid_for(zpl, 4), 256, 0, st, b.Z, BH, zr, dh, nc, in.lr, D.T, c0,
-                       b.op16);
-      return cudaGetLastError();
-    });
+    fwd_key(K_FWD_KEY, b.hist16 + c * planes, kh, in.v, static_cast<int>(c0), nc, in.lr, b.op16);
     L(K_BWD_GEMM, [&] {   // -G = E^T [k^, v, k^] over the chunk, W2's plane stored transposed
       GemmParams g = gemm_params();
       if (!map3d(&g.tmA, b.op16, dh, zr, 3 * BH, 64, 64) || !map3d(&g.tmB, b.kh16, d, D.T, BH, 64, 64) ||
@@ -532,36 +542,26 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     copy2d(dst + slot * plane, n_slots * pb, src_plane, pb, pb, D.BH);
   };
   const int64_t dh4 = 4 * D.dh, dh2 = 2 * D.dh;
-  float* Zk = b.Z;                    // [BH][zr][4 dh]
-  float* Zv = b.Z + 4 * zpl;          // [BH][zr][2 dh]
   B16* Phik = b.op16;                 // [BH][zr][4 dh]
   B16* Phiv = b.op16 + 4 * zpl;       // [BH][zr][2 dh]
   const Opnd Zk_op{Phik, dh4, zr, D.BH}, Zv_op{Phiv, dh2, zr, D.BH};
   auto apply_bwd = [&](const B16* W, int64_t qr0, int nq_c) {
     const int r0 = static_cast<int>(qr0);
-    stack_rows(b.Ba, 2, 0, W);               // [W1; W3]
-    stack_rows(b.Ba, 2, 1, W + 2 * jst);
-    const Opnd Ba_op{b.Ba, D.d, dh2, D.BH};
-    float* Za = b.Z;                          // [BH][zr][2 dh]
-    float* G = b.Z + 2 * zpl;                 // [BH][zr][dh]
-    B16* Phia = b.op16;                       // [BH][zr][2 dh]
-    B16* Hq = b.op16 + 2 * zpl;               // [BH][zr][dh]
-    tcg(KM, KM, qh, r0, 0, Ba_op, 0, nq_c, 2 * dh, d, Za, zr * dh2, dh2, false);
-    tcg(KM, MN, dos, r0, 0, Wop(W, 1), 0, nq_c, dh, d, G, zr * D.dh, dh, false);
-    L(K_BWD_ELEM, [&] {
-      (void)launch_pdl(k_apply_bwd_cat, grid_for(zpl, 4), 256, 0, st, static_cast<const float*>(Za),
-                       static_cast<const float*>(G), BH, zr, dh, nq_c, Phia, Hq);
-      return cudaGetLastError();
-    });
-    const Opnd Pa{Phia, dh2, zr, D.BH}, Hq_op{Hq, D.dh, zr, D.BH};
+    // [z1|z3] = q^ [W1; W3]^T and g = dO W2 with the factors dz1 = g z3 silu'(z1),
+    // hq = silu(z1) z3 and dz3 = g silu(z1): the fused key kernel with unit
+    // rates and dO in place of v, planes Ea = (dz1, hq, dz3)
+    B16* Ea = b.op16;
+    fwd_key(K_BWD_APPLY, W, qh, dos.p, r0, nq_c, nullptr, Ea);
+    const Opnd E1{Ea, D.dh, zr, D.BH}, Eh{Ea + zpl, D.dh, zr, D.BH}, E3{Ea + 2 * zpl, D.dh, zr, D.BH};
     // dW1 += dz1^T q^, dW3 += dz3^T q^, dW2 += dO^T hq
-    tcg(MN, MN, Pa, 0, 0, qh, r0, dh, d, nq_c, A, plane, d, true);
-    tcg(MN, MN, Pa, dh, 0, qh, r0, dh, d, nq_c, A + 2 * jst, plane, d, true);
-    tcg(MN, MN, dos, 0, r0, Hq_op, 0, d, dh, nq_c, A + jst, plane, dh, true);
-    // dq^ += [dz1|dz3] [W1; W3]
-    tcg(KM, MN, Pa, 0, 0, Ba_op, 0, nq_c, d, 2 * dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
+    tcg(MN, MN, E1, 0, 0, qh, r0, dh, d, nq_c, A, plane, d, true);
+    tcg(MN, MN, E3, 0, 0, qh, r0, dh, d, nq_c, A + 2 * jst, plane, d, true);
+    tcg(MN, MN, dos, 0, r0, Eh, 0, d, dh, nq_c, A + jst, plane, dh, true);
+    // dq^ += dz1 W1 + dz3 W3
+    tcg(KM, MN, E1, 0, 0, Wop(W, 0), 0, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
+    tcg(KM, MN, E3, 0, 0, Wop(W, 2), 0, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
     if (in.scale)   // the unscaled output hq W2^T, for the scale's gradient
-      tcg(KM, KM, Hq_op, 0, 0, Wop(W, 1), 0, nq_c, d, dh, b.ofull + qr0 * d, D.Tq * D.d, d, false);
+      tcg(KM, KM, Eh, 0, 0, Wop(W, 1), 0, nq_c, d, dh, b.ofull + qr0 * d, D.Tq * D.d, d, false);
   };
   for (int64_t c = D.nch - 1; c >= 0; --c) {
     const int64_t c0 = c * D.chunk;
@@ -596,15 +596,20 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
       stack_rows(b.Bk, 4, 3, b.Gam16 + 2 * jst);
       copy2d(b.Bv, dh2 * 2, Wp16 + jst, D.dh * 2, D.dh * 2, D.BH * D.d);
       copy2d(b.Bv + D.dh, dh2 * 2, b.Gam16 + jst, D.dh * 2, D.dh * 2, D.BH * D.d);
-      const Opnd Bk_op{b.Bk, D.d, dh4, D.BH}, Bv_op{b.Bv, dh2, D.d, D.BH};
+      const Opnd Bk_op{b.Bk, D.d, dh4, D.BH};
       const int k0 = static_cast<int>(c0);
-      tcg(KM, KM, kh, k0, 0, Bk_op, 0, nc, 4 * dh, d, Zk, zr * dh4, dh4, false);   // [z1|z3|p|r]
-      tcg(KM, MN, vv, k0, 0, Bv_op, 0, nc, 2 * dh, d, Zv, zr * dh2, dh2, false);   // [u|q]
-      L(K_BWD_ELEM, [&] {
-        (void)launch_pdl(k_hvp_elem_cat, static_cast<unsigned>(cdiv(D.BH * zr * 32, 256)), 256, 0, st,
-                         static_cast<const float*>(Zk), static_cast<const float*>(Zv), BH, zr, dh, nc, in.lr, D.T,
-                         c0, in.dlr, Phik, Phiv);
-        return cudaGetLastError();
+      // [z1|z3|p|r] = k^ Bk^T, [u|q] = v Bv and their second-order factors, one kernel
+      L(K_BWD_KEY, [&] {
+        BwdKeyParams f;
+        std::memset(&f, 0, sizeof(f));
+        if (!map3d(&f.tmX, kh.p, D.d, D.T, D.BH, 64, 128) || !map3d(&f.tmV, in.v, D.d, D.T, D.BH, 64, 128) ||
+            !map3d(&f.tmBk, b.Bk, D.d, dh4, D.BH, 64, 64) || !map3d(&f.tmBv, b.Bv, dh2, D.d, D.BH, 64, 64) ||
+            !map3d_plain(&f.tmPk, Phik, dh4, zr, D.BH, 16, 32) || !map3d_plain(&f.tmPv, Phiv, dh2, zr, D.BH, 16, 32))
+          return cudaErrorInvalidValue;
+        f.bh_count = BH; f.n_slices = dh / 64; f.n_row_tiles = static_cast<int>(cdiv(zr, 128));
+        f.kb_count = d / 64; f.x_row0 = k0; f.rows_valid = nc; f.dh = dh;
+        f.T = D.T; f.lr = in.lr; f.dlr = in.dlr;
+        return launch_umma<BwdKeyOp>(static_cast<int64_t>(f.n_slices) * f.n_row_tiles * BH, f, st);
       });
       // dW1 += dz1^T k^, dW3 += dz3^T k^, dW2 += v^T du
       tcg(MN, MN, Zk_op, 0, 0, kh, k0, dh, d, nc, Ap, plane, d, true);

@@ -19,6 +19,8 @@
 // fp32 in TMEM.  K is consumed in blocks of 64 (one 128-byte swizzle row).
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace lact {
@@ -30,8 +32,22 @@ constexpr int kEpiWarps = 4;
 constexpr int kIssuer2Warp = 6;
 
 // Block size of a kernel whose Op has kIssuers MMA issuers.
+// Epilogue warp groups of an Op: 1 unless the Op sets kEpiGroups.  Each
+// group has 4 warps (one TMEM lane quarter each) and takes its share of the
+// tile's columns; the extra groups' warps follow the issuers.
+template <class Op, class = void>
+struct EpiGroups {
+  static constexpr int value = 1;
+};
 template <class Op>
-constexpr int umma_threads() { return Op::kIssuers == 2 ? kThreads + 32 : kThreads; }
+struct EpiGroups<Op, std::void_t<decltype(Op::kEpiGroups)>> {
+  static constexpr int value = Op::kEpiGroups;
+};
+
+template <class Op>
+constexpr int umma_threads() {
+  return (Op::kIssuers == 2 ? kThreads + 32 : kThreads) + (EpiGroups<Op>::value - 1) * 32 * kEpiWarps;
+}
 
 template <int N>
 struct TmemCols {
@@ -52,6 +68,8 @@ __global__ void __launch_bounds__(umma_threads<Op>(), 1)
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int S = Op::kStages;
   constexpr int NB = Op::kAccBufs;
+  constexpr int EG = EpiGroups<Op>::value;
+  constexpr int kExtraEpi0 = Op::kIssuers == 2 ? kIssuer2Warp + 1 : 2 + kEpiWarps;   // first warp of group 1
   constexpr uint32_t kCols = TmemCols<NB * Op::kAccCols>::value;
   static_assert(NB * Op::kAccCols <= 512, "accumulator buffers must fit in TMEM");
   uint8_t* extra = smem + S * Op::kStageBytes;
@@ -78,7 +96,7 @@ __global__ void __launch_bounds__(umma_threads<Op>(), 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], Op::kIssuers);
-      mbar_init(&acc_empty[b], kEpiWarps);
+      mbar_init(&acc_empty[b], kEpiWarps * EG);
     }
     fence_barrier_init();
     Op::prefetch(p);
@@ -129,14 +147,18 @@ __global__ void __launch_bounds__(umma_threads<Op>(), 1)
         umma_commit(&acc_full[buf]);
       }
     }
-  } else if (warp < 2 + kEpiWarps) {
+  } else if (warp < 2 + kEpiWarps || (EG > 1 && warp >= kExtraEpi0)) {
+    const int group = warp < 2 + kEpiWarps ? 0 : 1 + (warp - kExtraEpi0) / kEpiWarps;
     int local = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
       const typename Op::Tile t = Op::map_tile(p, tile);
       const int buf = local % NB, use = local / NB;
       if (!mbar_wait(&acc_full[buf], use & 1)) break;
       tc_fence_after();
-      Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane, extra);
+      if constexpr (EG > 1)
+        Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane, extra, group);
+      else
+        Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane, extra);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -217,7 +239,8 @@ struct FwdParams {
   __nv_bfloat16* e;  // key tiles:   E [3][BH][buf_rows][dh]  (E1, Eh, E3)
   __nv_bfloat16* e_lo;  // split: lo parts, same layout
   int64_t buf_rows;
-  const float* lr;   // [BH, T, 3]
+  const float* lr;   // [BH, T, 3]; null: unit rates on the chunk's rows (the apply's backward:
+                     // E1 = dz1, Eh = hq, E3 = dz3 for the output gradient in place of v)
 };
 
 template <bool KMODE, bool SPLIT = false, int NSL = 64>
@@ -319,10 +342,14 @@ struct FwdOp {
       // This warp's 32 rows of E1, Eh, E3 -> swizzled staging -> TMA stores.
       float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
       if (valid) {
-        const float* l = p.lr + (static_cast<int64_t>(t.bh) * p.T + p.x_row0 + grow) * 3;
-        eta0 = l[0];
-        eta1 = l[1];
-        eta2 = l[2];
+        if (p.lr) {
+          const float* l = p.lr + (static_cast<int64_t>(t.bh) * p.T + p.x_row0 + grow) * 3;
+          eta0 = l[0];
+          eta1 = l[1];
+          eta2 = l[2];
+        } else {
+          eta0 = eta1 = eta2 = 1.0f;
+        }
       }
       const uint32_t stg = smem_u32(extra) + quarter * 3 * 4096 + lane * 128;
       if (lane == 0) bulk_wait_read_all();  // the previous tile's stores have read the staging
@@ -397,10 +424,14 @@ struct FwdOp {
     } else {
       float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
       if (valid) {
-        const float* l = p.lr + (static_cast<int64_t>(t.bh) * p.T + p.x_row0 + grow) * 3;
-        eta0 = l[0];
-        eta1 = l[1];
-        eta2 = l[2];
+        if (p.lr) {
+          const float* l = p.lr + (static_cast<int64_t>(t.bh) * p.T + p.x_row0 + grow) * 3;
+          eta0 = l[0];
+          eta1 = l[1];
+          eta2 = l[2];
+        } else {
+          eta0 = eta1 = eta2 = 1.0f;
+        }
       }
       const int64_t plane = static_cast<int64_t>(p.bh_count) * p.buf_rows * p.dh;
       const int64_t off = (static_cast<int64_t>(t.bh) * p.buf_rows + grow) * p.dh + col0;
