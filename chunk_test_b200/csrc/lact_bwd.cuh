@@ -381,20 +381,36 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     constexpr bool AMN = decltype(a_mn)::value, BMN = decltype(b_mn)::value;
     L(K_BWD_GEMM, [&] {
       GemmParams g = gemm_params();
-      // halve the N tile while the launch has too few tiles to fill the SMs
+      // Too few output tiles to fill the SMs: an accumulating contraction over
+      // a long K splits K (each split adds its part into out with atomics);
+      // otherwise the N tile is halved.
       int bn = pick_bn(N);
-      while (bn >= 128 && (bn / 2) % 64 == 0 && N % (bn / 2) == 0 &&
-             static_cast<int64_t>(N / bn) * cdiv(M, 128) * BH < 100)
-        bn /= 2;
+      const int kbt = static_cast<int>(cdiv(K, 64));
+      const int64_t tiles = static_cast<int64_t>(N / bn) * cdiv(M, 128) * BH;
+      int splits = 1;
+      if (acc && tiles < 100 && kbt >= 8)
+        splits = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sm_count() / tiles, kbt / 4)));
+      if (splits > 1) {
+        splits = static_cast<int>(cdiv(kbt, cdiv(kbt, splits)));   // no empty split
+      } else {
+        while (bn >= 128 && (bn / 2) % 64 == 0 && N % (bn / 2) == 0 &&
+               static_cast<int64_t>(N / bn) * cdiv(M, 128) * BH < 100)
+          bn /= 2;
+      }
       if (!map3d(&g.tmA, a.p, a.inner, a.rows, a.batch, 64, AMN ? 64 : 128) ||
           !map3d(&g.tmB, bo.p, bo.inner, bo.rows, bo.batch, 64, BMN ? 64 : bn))
         return cudaErrorInvalidValue;
-      g.items = BH; g.kb_count = g.kb_total = static_cast<int>(cdiv(K, 64));
+      g.items = BH; g.kb_total = kbt; g.kb_count = static_cast<int>(cdiv(kbt, splits));
       g.a_m0 = a_m0; g.a_k0 = a_k0; g.b_k0 = b_k0;
       g.zb_mod = BH; g.m_valid = M;
       g.outf = out; g.item_stride = out_item; g.ld = ld;
-      if (acc) { g.beta = 1.0f; g.cin = out; }
-      return launch_gemm<AMN, BMN>(bn, dim3(N / bn, cdiv(M, 128), BH), g, st);
+      if (splits > 1) {
+        g.red = 1;
+      } else if (acc) {
+        g.beta = 1.0f;
+        g.cin = out;
+      }
+      return launch_gemm<AMN, BMN>(bn, dim3(N / bn, cdiv(M, 128), splits * BH), g, st);
     });
   };
   const std::false_type KM;   // K-major operand

@@ -514,6 +514,8 @@ struct GemmParams {
   int a_m0;                // first M coordinate of A's map that tile row 0 reads (MN-major A:
                            // a multiple of 8, the map's inner coordinate)
   int zb_div, zb_mul;      // if zb_div > 0: B's batch = (item / zb_div) * zb_mul + item % zb_div
+  int red;                 // fp32 output added into outf with atomics (no cin): the K splits of
+                           // an item all add into output item `item`
 };
 
 template <bool A_MN, bool B_MN, int BN, bool SPLIT = false>
@@ -540,7 +542,7 @@ struct GemmOp {
     t.m0 = ((idx / p.nt_n) % p.nt_m) * kBM;
     t.item = z % p.items;
     t.split = z / p.items;
-    t.out_item = z;
+    t.out_item = p.red ? t.item : z;
     t.zb = p.zb_div > 0 ? (t.item / p.zb_div) * p.zb_mul + t.item % p.zb_div : (t.item % p.zb_mod) + p.zb_add;
     t.alt = p.alt_group >= 0 && (t.item / p.zb_mod) == p.alt_group;
     return t;
@@ -653,8 +655,17 @@ struct GemmOp {
         if (p.outf && tr) {
           float* o = p.outf + static_cast<int64_t>(t.out_item) * p.item_stride +
                      static_cast<int64_t>(t.n0 + j) * p.ld_t + grow;
+          if (p.red) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o[i * p.ld_t] = v[i];
+            for (int i = 0; i < 16; ++i) atomicAdd(o + i * p.ld_t, v[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i * p.ld_t] = v[i];
+          }
+        } else if (p.outf && p.red) {
+          float4* o = reinterpret_cast<float4*>(p.outf + off + j);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) atomicAdd(o + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
         } else if (p.outf) {
           float* o = p.outf + off + j;
 #pragma unroll
