@@ -104,10 +104,12 @@ __device__ __forceinline__ void mma_kblock_pair(uint32_t d_tmem, uint32_t a_base
 }
 
 // The pair pipeline.  Op supplies kStages, kStageBytes (per CTA; both CTAs
-// load the same number of bytes), kAccCols, kAccBufs, Tile, num_tiles()
-// (pair tiles), map_tile(p, idx, rank), num_kb(), prefetch(),
+// load the same number of bytes), kExtraBytes (shared memory for the
+// epilogue, after the ring), kAccCols, kAccBufs, Tile, num_tiles() (pair
+// tiles), map_tile(p, idx, rank), num_kb(), prefetch(),
 // load(p, t, kb, stage, bar_cluster_addr), mma(p, t, stage, tmem, kb)
-// (even CTA) and epilogue(p, t, tmem, quarter, lane).
+// (even CTA), epilogue(p, t, tmem, quarter, lane, extra) and
+// epilogue_done(lane).
 template <class Op>
 __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
     umma_pair_kernel(const __grid_constant__ typename Op::Params p) {
@@ -119,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
   constexpr int NB = Op::kAccBufs;
   constexpr uint32_t kCols = TmemCols<NB * Op::kAccCols>::value;
   static_assert(NB * Op::kAccCols <= 512, "accumulator buffers must fit in TMEM");
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Op::kStageBytes);
+  uint8_t* extra = smem + S * Op::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(extra + Op::kExtraBytes);
   uint64_t* empty = full + S;
   uint64_t* acc_full = empty + S;      // [2]
   uint64_t* acc_empty = acc_full + 2;  // [2], used in the even CTA
@@ -201,11 +204,12 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
       const int buf = local % NB, use = local / NB;
       if (!mbar_wait(&acc_full[buf], use & 1)) break;
       tc_fence_after();
-      Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane, nullptr);
+      Op::epilogue(p, t, tmem + buf * Op::kAccCols, warp & 3, lane, extra);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader + buf * 8u);
     }
+    Op::epilogue_done(lane);
   }
   tc_fence_before();
   cluster_sync_all();  // no CTA leaves while its peer may still use its memory
@@ -232,6 +236,7 @@ struct GemmPairOp {
   static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
   static constexpr int kAccCols = TmemCols<BN>::value;
   static constexpr int kAccBufs = 2;
+  static constexpr int kExtraBytes = 0;
   using Tile = typename Base::Tile;   // m0 is this CTA's first row
 
   __device__ static int num_tiles(const Params& p) { return p.n_tiles; }
@@ -273,11 +278,12 @@ struct GemmPairOp {
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter, int lane, uint8_t*) {
     Base::epilogue(p, t, tmem, quarter, lane, nullptr);
   }
+  __device__ static void epilogue_done(int) {}
 };
 
 template <class Op>
 constexpr int umma_pair_smem_bytes() {
-  return Op::kStages * Op::kStageBytes + (2 * Op::kStages + 4) * 8 + 16 + 1024;
+  return Op::kStages * Op::kStageBytes + Op::kExtraBytes + (2 * Op::kStages + 4) * 8 + 16 + 1024;
 }
 
 }  // namespace lact

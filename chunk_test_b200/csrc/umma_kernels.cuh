@@ -243,6 +243,78 @@ struct FwdParams {
                      // E1 = dz1, Eh = hq, E3 = dz3 for the output gradient in place of v)
 };
 
+// Key-tile gradient factors of 64 hidden units for one epilogue warp's 32
+// rows (row0 + 32 quarter + lane of the chunk), per token t and unit r with
+// s1 = sigmoid(z1):  E1 = lr1 u z3 s1 (1 + z1 (1 - s1)),  Eh = lr2 silu(z1) z3,
+// E3 = lr3 u silu(z1)  (unit rates when p.lr is null), in bf16 through the
+// warp's three swizzled 32 x 64 staging tiles in `extra` and bulk tensor
+// stores at columns col0 .. col0 + 63.  tz1, tz3, tu: the warp's TMEM
+// addresses of the 64 columns of z1, z3 and u.
+__device__ __forceinline__ void key_factors_tma(const FwdParams& p, int bh, int row0, int col0, uint32_t tz1,
+                                                uint32_t tz3, uint32_t tu, int quarter, int lane, uint8_t* extra) {
+  const int grow = row0 + quarter * 32 + lane;
+  const bool valid = grow < p.rows_valid;
+  float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
+  if (valid) {
+    if (p.lr) {
+      const float* l = p.lr + (static_cast<int64_t>(bh) * p.T + p.x_row0 + grow) * 3;
+      eta0 = l[0];
+      eta1 = l[1];
+      eta2 = l[2];
+    } else {
+      eta0 = eta1 = eta2 = 1.0f;
+    }
+  }
+  const uint32_t stg = smem_u32(extra) + quarter * 3 * 4096 + lane * 128;
+  if (lane == 0) bulk_wait_read_all();  // the previous tile's stores have read the staging
+  __syncwarp();
+#pragma unroll 1
+  for (int j = 0; j < 64; j += 16) {
+    float z1[16], z3[16], u[16];
+    __syncwarp();
+    tmem_ld16(tz1 + j, z1);
+    tmem_ld16(tz3 + j, z3);
+    tmem_ld16(tu + j, u);
+    tmem_ld_wait();
+    uint32_t w[3][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float e1[2], eh[2], e3[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float a = z1[2 * i + c], b = z3[2 * i + c], g = u[2 * i + c];
+        const float s = sigmoid_fast(a);
+        const float sa = a * s;
+        const float ds = fmaf(sa, 1.0f - s, s);
+        e1[c] = (eta0 * g) * (b * ds);
+        eh[c] = eta1 * (sa * b);
+        e3[c] = (eta2 * g) * sa;
+      }
+      w[0][i] = pack_bf16x2(e1[0], e1[1]);
+      w[1][i] = pack_bf16x2(eh[0], eh[1]);
+      w[2][i] = pack_bf16x2(e3[0], e3[1]);
+    }
+    // row `lane` of each staging tile; 16-byte chunk c at c ^ (lane % 8)
+    const uint32_t c0 = ((j / 8) ^ (lane & 7)) << 4, c1 = ((j / 8 + 1) ^ (lane & 7)) << 4;
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+      st_shared_v4(stg + m * 4096 + c0, w[m][0], w[m][1], w[m][2], w[m][3]);
+      st_shared_v4(stg + m * 4096 + c1, w[m][4], w[m][5], w[m][6], w[m][7]);
+    }
+  }
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    const uint8_t* src = extra + quarter * 3 * 4096;
+    const int row = row0 + quarter * 32;
+#pragma unroll
+    for (int m = 0; m < 3; ++m)
+      tma_store_3d(&p.tmE, src + m * 4096, col0, row, m * p.bh_count + bh);
+    bulk_commit_group();
+  }
+}
+
+
 template <bool KMODE, bool SPLIT = false, int NSL = 64>
 struct FwdOp {
   static_assert(KMODE || !SPLIT, "split mode is for key tiles");
@@ -339,65 +411,7 @@ struct FwdOp {
     const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const int64_t col0 = static_cast<int64_t>(t.slice) * NSL;
     if constexpr (kTmaStore) {
-      // This warp's 32 rows of E1, Eh, E3 -> swizzled staging -> TMA stores.
-      float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
-      if (valid) {
-        if (p.lr) {
-          const float* l = p.lr + (static_cast<int64_t>(t.bh) * p.T + p.x_row0 + grow) * 3;
-          eta0 = l[0];
-          eta1 = l[1];
-          eta2 = l[2];
-        } else {
-          eta0 = eta1 = eta2 = 1.0f;
-        }
-      }
-      const uint32_t stg = smem_u32(extra) + quarter * 3 * 4096 + lane * 128;
-      if (lane == 0) bulk_wait_read_all();  // the previous tile's stores have read the staging
-      __syncwarp();
-#pragma unroll 1
-      for (int j = 0; j < 64; j += 16) {
-        float z1[16], z3[16], u[16];
-        __syncwarp();
-        tmem_ld16(tq + j, z1);
-        tmem_ld16(tq + 64 + j, z3);
-        tmem_ld16(tq + 128 + j, u);
-        tmem_ld_wait();
-        uint32_t w[3][8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float e1[2], eh[2], e3[2];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const float a = z1[2 * i + c], b = z3[2 * i + c], g = u[2 * i + c];
-            const float s = sigmoid_fast(a);
-            const float sa = a * s;
-            const float ds = fmaf(sa, 1.0f - s, s);
-            e1[c] = (eta0 * g) * (b * ds);
-            eh[c] = eta1 * (sa * b);
-            e3[c] = (eta2 * g) * sa;
-          }
-          w[0][i] = pack_bf16x2(e1[0], e1[1]);
-          w[1][i] = pack_bf16x2(eh[0], eh[1]);
-          w[2][i] = pack_bf16x2(e3[0], e3[1]);
-        }
-        // row `lane` of each staging tile; 16-byte chunk c at c ^ (lane % 8)
-        const uint32_t c0 = ((j / 8) ^ (lane & 7)) << 4, c1 = ((j / 8 + 1) ^ (lane & 7)) << 4;
-#pragma unroll
-        for (int m = 0; m < 3; ++m) {
-          st_shared_v4(stg + m * 4096 + c0, w[m][0], w[m][1], w[m][2], w[m][3]);
-          st_shared_v4(stg + m * 4096 + c1, w[m][4], w[m][5], w[m][6], w[m][7]);
-        }
-      }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const uint8_t* src = extra + quarter * 3 * 4096;
-        const int row = t.row0 + quarter * 32;
-#pragma unroll
-        for (int m = 0; m < 3; ++m)
-          tma_store_3d(&p.tmE, src + m * 4096, static_cast<int>(col0), row, m * p.bh_count + t.bh);
-        bulk_commit_group();
-      }
+      key_factors_tma(p, t.bh, t.row0, static_cast<int>(col0), tq, tq + 64, tq + 128, quarter, lane, extra);
       return;
     }
     if (!KMODE) {
