@@ -285,6 +285,65 @@ __global__ void __launch_bounds__(256) k_prologue_bwd(const float* __restrict__ 
   }
 }
 
+// The same for bf16 inputs x, one warp per row with the row in registers:
+// 8 elements per lane and step, two steps at most (d a multiple of 64, at
+// most 512).  Grid-stride over the rows.
+__global__ void __launch_bounds__(256) k_prologue_bwd_bf16(const __nv_bfloat16* __restrict__ x,
+                                                           const float* __restrict__ dxh,
+                                                           float* __restrict__ dx, int64_t rows, int d) {
+  griddep_launch();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int nc = d >> 3;   // 8-element chunks per row
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
+       row += nwarps) {
+    float xv[2][8], gv[2][8];
+    float ss = 0.f, sg = 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = lane + 32 * i;
+      if (c >= nc) continue;
+      const uint4 raw = *reinterpret_cast<const uint4*>(x + row * d + 8 * c);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      const float4 g0 = *reinterpret_cast<const float4*>(dxh + row * d + 8 * c);
+      const float4 g1 = *reinterpret_cast<const float4*>(dxh + row * d + 8 * c + 4);
+      const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        xv[i][2 * e] = __uint_as_float(w[e] << 16);
+        xv[i][2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        gv[i][e] = gg[e];
+        const float s = xv[i][e] * sigm(xv[i][e]);
+        ss += s * s;
+        sg += s * gg[e];
+      }
+    }
+    ss = warp_sum(ss);
+    sg = warp_sum(sg);
+    const float n = sqrtf(ss);
+    const float inv = n > 0.f ? 1.0f / n : 0.f;
+    const float dot = sg * inv;   // <x^, dx^>
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = lane + 32 * i;
+      if (c >= nc) continue;
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float z = xv[i][e], sgz = sigm(z);
+        o[e] = (gv[i][e] - z * sgz * inv * dot) * inv * sgz * (1.0f + z * (1.0f - sgz));
+      }
+      float4* out = reinterpret_cast<float4*>(dx + row * d + 8 * c);
+      out[0] = make_float4(o[0], o[1], o[2], o[3]);
+      out[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
 // Gradient of the initial weights: A [3][BH][plane] summed over the batch
 // for an initial state shared by it (w_shared), else copied.
 __global__ void __launch_bounds__(256) k_sum_batch(const float* __restrict__ A, int B, int H,

@@ -58,8 +58,6 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
   b.zr = std::max<int64_t>(D.chunk, D.nch == 1 ? D.Tq : D.chunk);
   const int64_t zpl = D.BH * b.zr * D.dh;
   if (bf) {
-    b.q32 = bp.take<float>(nq);          // raw q, k for the prologue's backward
-    b.k32 = bp.take<float>(nk);
     b.do32 = bp.take<float>(nq);         // dout, for the scale's gradient
     b.qh16 = bp.take<__nv_bfloat16>(nq);
     b.kh16 = bp.take<__nv_bfloat16>(nk);
@@ -420,20 +418,12 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     return j == 1 ? Opnd{W + jst, D.dh, D.d, D.BH} : Opnd{W + j * jst, D.d, D.dh, D.BH};
   };
 
-  // ---- raw fp32 q, k (prologue backward), dout (scale gradient), bf16 q^, k^
-  {
-    const void* src[3] = {in.q, in.k, in.dout};
-    float* dst[3] = {b.q32, b.k32, b.do32};
-    const int64_t n[3] = {nq, nk, nq};
-    for (int i = 0; i < 3; ++i) {
-      if (i == 2 && !in.scale) continue;
-      L(K_BWD_ELEM, [&] {
-        (void)launch_pdl(k_bf16_to_f32, grid_for(n[i], 4), 256, 0, st, static_cast<const B16*>(src[i]), dst[i],
-                         n[i]);
-        return cudaGetLastError();
-      });
-    }
-  }
+  // ---- dout in fp32 (the scale's gradient), bf16 q^, k^
+  if (in.scale)
+    L(K_BWD_ELEM, [&] {
+      (void)launch_pdl(k_bf16_to_f32, grid_for(nq, 4), 256, 0, st, static_cast<const B16*>(in.dout), b.do32, nq);
+      return cudaGetLastError();
+    });
   const B16* dos16 = static_cast<const B16*>(in.dout);
   if (in.scale) {
     L(K_BWD_ELEM, [&] {
@@ -641,13 +631,13 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
 
   // ---- prologue backward, the scale's gradient, the initial weights' gradient
   L(K_BWD_ELEM, [&] {
-    (void)launch_pdl(k_prologue_bwd, static_cast<unsigned>(cdiv(D.BH * D.Tq * 32, 256)), 256, 0, st,
-                     static_cast<const float*>(b.q32), static_cast<const float*>(b.dqh), in.dq, D.BH * D.Tq, d);
+    (void)launch_pdl(k_prologue_bwd_bf16, grid_for(D.BH * D.Tq * 32, 1), 256, 0, st, static_cast<const B16*>(in.q),
+                     static_cast<const float*>(b.dqh), in.dq, D.BH * D.Tq, d);
     return cudaGetLastError();
   });
   L(K_BWD_ELEM, [&] {
-    (void)launch_pdl(k_prologue_bwd, static_cast<unsigned>(cdiv(D.BH * D.T * 32, 256)), 256, 0, st,
-                     static_cast<const float*>(b.k32), static_cast<const float*>(b.dkh), in.dk, D.BH * D.T, d);
+    (void)launch_pdl(k_prologue_bwd_bf16, grid_for(D.BH * D.T * 32, 1), 256, 0, st, static_cast<const B16*>(in.k),
+                     static_cast<const float*>(b.dkh), in.dk, D.BH * D.T, d);
     return cudaGetLastError();
   });
   if (in.scale)
