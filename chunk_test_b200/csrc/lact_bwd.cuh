@@ -379,15 +379,24 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     constexpr bool AMN = decltype(a_mn)::value, BMN = decltype(b_mn)::value;
     L(K_BWD_GEMM, [&] {
       GemmParams g = gemm_params();
-      // Too few output tiles to fill the SMs: an accumulating contraction over
-      // a long K splits K (each split adds its part into out with atomics);
-      // otherwise the N tile is halved.
+      // An accumulating contraction splits K into up to 4 parts of at least 4
+      // K blocks (each split adds its part into out with atomics) when that
+      // fills the last wave of tiles better; the others halve the N tile while
+      // they have too few tiles to fill the SMs.
       int bn = pick_bn(N);
       const int kbt = static_cast<int>(cdiv(K, 64));
       const int64_t tiles = static_cast<int64_t>(N / bn) * cdiv(M, 128) * BH;
       int splits = 1;
-      if (acc && tiles < 100 && kbt >= 8)
-        splits = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sm_count() / tiles, kbt / 4)));
+      if (acc) {
+        const int64_t sms = sm_count();
+        auto fill = [&](int64_t t) { return static_cast<double>(t) / static_cast<double>(cdiv(t, sms) * sms); };
+        double best = fill(tiles);
+        for (int sp = 2; sp <= 4 && kbt / sp >= 4; ++sp)
+          if (fill(tiles * sp) > best + 0.05) {
+            best = fill(tiles * sp);
+            splits = sp;
+          }
+      }
       if (splits > 1) {
         splits = static_cast<int>(cdiv(kbt, cdiv(kbt, splits)));   // no empty split
       } else {
