@@ -236,7 +236,7 @@ struct GemmPairOp {
   static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
   static constexpr int kAccCols = TmemCols<BN>::value;
   static constexpr int kAccBufs = 2;
-  static constexpr int kExtraBytes = 0;
+  static constexpr int kExtraBytes = Base::kExtraBytes;   // the epilogue's staging tiles
   using Tile = typename Base::Tile;   // m0 is this CTA's first row
 
   __device__ static int num_tiles(const Params& p) { return p.n_tiles; }
@@ -275,8 +275,9 @@ struct GemmPairOp {
     constexpr uint32_t id = idesc_bf16(2 * kBM, BN, A_MN, B_MN);
     mma_kblock_pair<A_MN, B_MN>(tmem, st, 8192u, st + kABytes, 8192u, id, kb == 0);
   }
-  __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter, int lane, uint8_t*) {
-    Base::epilogue(p, t, tmem, quarter, lane, nullptr);
+  __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter, int lane,
+                                  uint8_t* extra) {
+    Base::epilogue(p, t, tmem, quarter, lane, extra);
   }
   __device__ static void epilogue_done(int) {}
 };

@@ -544,7 +544,16 @@ struct GemmOp {
   static constexpr int kStages = (196608 / kStageBytes) < 6 ? (196608 / kStageBytes) : 6;
   static constexpr int kAccCols = TmemCols<BN>::value;
   static constexpr int kAccBufs = 2;
-  static constexpr int kExtraBytes = 0;
+  // Per epilogue warp: a 32-row x 16-column fp32 staging tile with a row
+  // pitch of 17 floats (a thread's row writes are conflict-free).  When the
+  // tile reads an fp32 input cin, cin and the fp32 output pass through it as
+  // 64-byte row segments, 8 rows per warp access, instead of one row (one
+  // cache line) per thread: the row-per-thread loads stalled those epilogues
+  // (Newton-Schulz update 69 -> 52.5 us).  Store-only epilogues keep the
+  // direct row stores, which measured faster there (chunk gradient 30.1 us
+  // direct, 33.8 us staged).
+  static constexpr int kStgPitch = 17;
+  static constexpr int kExtraBytes = kEpiWarps * 32 * kStgPitch * 4;
   static constexpr int kIssuers = 1;
   struct Tile { int m0, n0, item, out_item, split, zb; bool alt; };
 
@@ -614,59 +623,66 @@ struct GemmOp {
   }
   __device__ static void epilogue_done(int) {}
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter,
-                                  int lane, uint8_t*) {
+                                  int lane, uint8_t* extra) {
     const int r = quarter * 32 + lane;
     const int grow = t.m0 + r;
     const bool valid = grow < p.m_valid;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const int64_t off = static_cast<int64_t>(t.out_item) * p.item_stride +
-                        static_cast<int64_t>(grow) * p.ld + t.n0;
+    const int64_t base = static_cast<int64_t>(t.out_item) * p.item_stride + t.n0;
+    const int64_t off = base + static_cast<int64_t>(grow) * p.ld;
     const bool tr = p.tr_group >= 0 && (t.item / p.tr_mod) == p.tr_group;
     const float rs = (p.row_scale && valid) ? __ldg(p.row_scale + t.out_item * p.rs_item + grow) : 1.0f;
+    float* stg = reinterpret_cast<float*>(extra) + quarter * 32 * kStgPitch;
+    // In the coalesced passes this lane moves rows 8 k + lane / 4 (k < 4) of
+    // the warp's 32, columns 4 (lane % 4) .. + 3 of the 16.
+    const int wrow0 = t.m0 + quarter * 32, cr = lane >> 2, cc = (lane & 3) * 4;
+    const bool has_c = p.cin != nullptr;
     // cin of the next 16 columns is loaded while this step's are used, so
     // the epilogue does not wait on one global load latency per step
-    const bool has_c = p.cin && valid;
     float4 cn[4];
-    if (has_c) {
-      const float4* c = reinterpret_cast<const float4*>(p.cin + off);
+    auto load_c = [&](int j) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) cn[i] = c[i];
-    }
+      for (int k = 0; k < 4; ++k) {
+        const int rr = wrow0 + 8 * k + cr;
+        cn[k] = rr < p.m_valid ? *reinterpret_cast<const float4*>(p.cin + base + static_cast<int64_t>(rr) * p.ld + j + cc)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    if (has_c) load_c(0);
 #pragma unroll 1
     for (int j = 0; j < BN; j += 16) {
-      float v[16];
-      float4 cc[4];
+      float v[16], c[16];
       if (has_c) {
+        __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cc[i] = cn[i];
-        if (j + 16 < BN) {
-          const float4* c = reinterpret_cast<const float4*>(p.cin + off + j + 16);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) cn[i] = c[i];
+        for (int k = 0; k < 4; ++k) {
+          float* sp = stg + (8 * k + cr) * kStgPitch + cc;
+          sp[0] = cn[k].x;
+          sp[1] = cn[k].y;
+          sp[2] = cn[k].z;
+          sp[3] = cn[k].w;
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) c[i] = stg[lane * kStgPitch + i];
+        if (j + 16 < BN) load_c(j + 16);
       }
       __syncwarp();
       tmem_ld16(tq + j, v);
       tmem_ld_wait();
-      if (valid) {
-        if (has_c) {
+      if (has_c) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 x = cc[i];
-            v[4 * i + 0] = p.alpha * v[4 * i + 0] + p.beta * x.x;
-            v[4 * i + 1] = p.alpha * v[4 * i + 1] + p.beta * x.y;
-            v[4 * i + 2] = p.alpha * v[4 * i + 2] + p.beta * x.z;
-            v[4 * i + 3] = p.alpha * v[4 * i + 3] + p.beta * x.w;
-          }
-        } else if (p.alpha != 1.0f) {
+        for (int i = 0; i < 16; ++i) v[i] = p.alpha * v[i] + p.beta * c[i];
+      } else if (p.alpha != 1.0f) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] *= p.alpha;
-        }
-        if (p.row_scale) {
+        for (int i = 0; i < 16; ++i) v[i] *= p.alpha;
+      }
+      if (p.row_scale) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] *= rs;
-        }
-        if (p.outf && tr) {
+        for (int i = 0; i < 16; ++i) v[i] *= rs;
+      }
+      if (p.outf && tr) {
+        if (valid) {
           float* o = p.outf + static_cast<int64_t>(t.out_item) * p.item_stride +
                      static_cast<int64_t>(t.n0 + j) * p.ld_t + grow;
           if (p.red) {
@@ -676,17 +692,40 @@ struct GemmOp {
 #pragma unroll
             for (int i = 0; i < 16; ++i) o[i * p.ld_t] = v[i];
           }
-        } else if (p.outf && p.red) {
-          float4* o = reinterpret_cast<float4*>(p.outf + off + j);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) atomicAdd(o + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
-        } else if (p.outf) {
-          float* o = p.outf + off + j;
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            st_global_v4(o + 4 * i, __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
-                         __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
         }
+      } else if (p.outf && !has_c) {
+        if (valid) {
+          float* o = p.outf + off + j;
+          if (p.red) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              atomicAdd(reinterpret_cast<float4*>(o) + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              st_global_v4(o + 4 * i, __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
+                           __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
+          }
+        }
+      } else if (p.outf) {
+        __syncwarp();   // every lane has read its cin row from the staging tile
+#pragma unroll
+        for (int i = 0; i < 16; ++i) stg[lane * kStgPitch + i] = v[i];
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int rr = wrow0 + 8 * k + cr;
+          if (rr >= p.m_valid) continue;
+          const float* sp = stg + (8 * k + cr) * kStgPitch + cc;
+          float* o = p.outf + base + static_cast<int64_t>(rr) * p.ld + j + cc;
+          if (p.red)
+            atomicAdd(reinterpret_cast<float4*>(o), make_float4(sp[0], sp[1], sp[2], sp[3]));
+          else
+            st_global_v4(o, __float_as_uint(sp[0]), __float_as_uint(sp[1]), __float_as_uint(sp[2]),
+                         __float_as_uint(sp[3]));
+        }
+      }
+      if (valid) {
         if (p.outb) {
           uint32_t hw[8];
 #pragma unroll
