@@ -259,7 +259,12 @@ size_t lact_ttt_bwd_workspace_bytes(const lact_problem* p);
  * batch shares them), dout_scale [B,H,Tq] (required when out_scale is
  * given, else ignored).  No output may overlap an input or another output.
  * `workspace` is device scratch of lact_ttt_bwd_workspace_bytes(p) bytes,
- * 256-byte aligned.  Asynchronous on `stream`, like the forward. */
+ * 256-byte aligned.  Asynchronous on `stream`, like the forward.
+ * On bf16 problems some fp32 sums are accumulated with atomic adds: dlr
+ * across hidden-unit slices, and the contractions whose token range is
+ * split across CTAs.  Repeated calls on the same inputs can therefore
+ * differ in the last bits (the order of fp32 additions varies); the fp32
+ * path is deterministic. */
 int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts,
                  const void* q, const void* k, const void* v,
                  const float* lr, const float* beta,
