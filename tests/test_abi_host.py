@@ -206,3 +206,24 @@ def test_backward_and_attention_arguments_are_checked_without_a_gpu():
     bad[7] = ctypes.c_void_p(ptrs[1].value)                                    # out on k
     assert lib.lact_swa_fwd(ctypes.byref(p), *bad, ws, big, None) == ct.LACT_EINVAL
     assert lib.lact_swa_fwd(ctypes.byref(p), *ptrs[:8], ws, ctypes.c_size_t(16), None) == ct.LACT_ENOSPC
+
+
+def test_attention_workspace_follows_the_documented_layout():
+    """lact_swa_workspace_bytes (host arithmetic): for d up to 256 the scores
+    stay on chip and the workspace is one bf16 copy of the transformed q;
+    for larger d it also holds the fp32 scores, the bf16 probabilities
+    (B*H*T*(window+128)*6 bytes) and the zero-padded k' and v copies."""
+    lib = ct.lib()
+    sp = lambda **kw: _abi.LactSwaProblem(*[kw.get(n, v) for n, v in
+                                            (("B", 1), ("H", 2), ("T", 1024), ("d", 128), ("window", 256),
+                                             ("dtype", 1), ("reserved", 0))])
+    rup = lambda x: (x + 255) // 256 * 256
+    for B, H, T, d, w in ((1, 2, 1024, 128, 256), (2, 6, 32768, 256, 2048), (1, 1, 384, 64, 1024)):
+        got = lib.lact_swa_workspace_bytes(ctypes.byref(sp(B=B, H=H, T=T, d=d, window=w)))
+        assert got == rup(B * H * T * d * 2), (B, H, T, d, w, got)
+    B, H, T, d, w = 1, 1, 512, 512, 256
+    got = lib.lact_swa_workspace_bytes(ctypes.byref(sp(B=B, H=H, T=T, d=d, window=w)))
+    scores = B * H * T * (w + 128) * 6
+    padded = 2 * (B * H * (w + T) + w) * d * 2
+    assert got >= B * H * T * d * 2 + scores + padded
+    assert got <= B * H * T * d * 2 + scores + padded + 4 * 256
