@@ -222,6 +222,8 @@ static bool map3d_plain(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_
 }
 
 // ------------------------------------------------------------------ launches
+// Opt-in dynamic shared memory per CTA on sm_100 (227 KB).
+constexpr int kMaxSmemPerBlock = 232448;
 // Every kernel is launched with programmatic stream serialization: the
 // next kernel of the stream may start while this one drains, does its local
 // setup (barrier init, TMEM allocation, tensor-map prefetch), and waits in
@@ -258,6 +260,7 @@ static int sm_count() {
 template <class Op>
 static cudaError_t launch_umma(int64_t ntiles, const typename Op::Params& p, cudaStream_t st) {
   constexpr int smem = umma_smem_bytes<Op>();
+  static_assert(smem <= kMaxSmemPerBlock, "dynamic shared memory above the per-CTA limit");
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -276,6 +279,7 @@ static cudaError_t launch_umma(int64_t ntiles, const typename Op::Params& p, cud
 template <int D>
 static cudaError_t launch_apply(int64_t ntiles, const ApplyParams& p, cudaStream_t st) {
   constexpr int smem = ApplyCfg<D>::kSmem;
+  static_assert(smem <= kMaxSmemPerBlock, "dynamic shared memory above the per-CTA limit");
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -293,6 +297,7 @@ static cudaError_t launch_apply(int64_t ntiles, const ApplyParams& p, cudaStream
 
 static cudaError_t launch_key_grad(int64_t items, const KeyGradParams& p, cudaStream_t st) {
   constexpr int smem = KGCfg::kSmem;
+  static_assert(smem <= kMaxSmemPerBlock, "dynamic shared memory above the per-CTA limit");
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -312,6 +317,7 @@ static cudaError_t launch_key_grad(int64_t items, const KeyGradParams& p, cudaSt
 template <class Op>
 static cudaError_t launch_pair(int64_t ntiles, const typename Op::Params& p, cudaStream_t st) {
   constexpr int smem = umma_pair_smem_bytes<Op>();
+  static_assert(smem <= kMaxSmemPerBlock, "dynamic shared memory above the per-CTA limit");
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -65,6 +65,7 @@ template <int D>
 static cudaError_t launch_swa_flash(const SwaDims& S, const SwaBufs& b, const void* k, const void* v, void* out,
                                     cudaStream_t st) {
   constexpr int smem = SwaCfg<D>::kSmem;
+  static_assert(smem <= kMaxSmemPerBlock, "dynamic shared memory above the per-CTA limit");
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
