@@ -208,7 +208,8 @@ def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=N
     dL/d w_out (`dw_out`, three tensors like the forward's w_out).  Returns a
     dict of float32 tensors: dq, dk, dv, dlr, dbeta (momentum, else None),
     dw1, dw2, dw3 (shaped like w1, w2, w3) and dout_scale (when out_scale is
-    given, else None)."""
+    given, else None).  On bf16 inputs some fp32 sums are accumulated with
+    atomic adds, so repeated calls can differ in the last bits."""
     _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
     if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_contiguous():
         raise ValueError("dout must be a contiguous tensor shaped like q, in q's dtype")
