@@ -188,6 +188,120 @@ def ClockSampler(device: int):
         return SmiClockSampler(device)
 
 
+
+# ---------------------------------------------------------------- forward timing
+def forward_timing(ct, w: Workload, dev, steps: int, warmup: int, seed: int, barrier, barrier_max, local: int):
+    """Times `steps` layer forwards of workload `w` on inputs resident in HBM,
+    then the same steps again under the library's launch profiler.  Returns
+    the inputs, both pass times (max over ranks), the per-kernel profile and
+    the clock record of the first pass."""
+    inp_cpu = make_inputs(w, seed=seed)
+    inp = {k: (None if v is None else v.to(dev)) for k, v in inp_cpu.items()}
+    B, H = w.B, w.H
+    out = torch.empty_like(inp["q"])
+    w_out = (torch.empty((B * H, w.dh, w.d), device=dev), torch.empty((B * H, w.d, w.dh), device=dev),
+             torch.empty((B * H, w.dh, w.d), device=dev))
+    ws = torch.empty(ct.workspace_bytes(inp["q"], inp["k"], inp["w1"], w.chunk, w.order, w.rule),
+                     device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ct.ttt_fwd(inp["q"], inp["k"], inp["v"], inp["lr"], inp["beta"], inp["w1"], inp["w2"],
+                   inp["w3"], w.chunk, w.order, w.rule, out=out, w_out=w_out, workspace=ws,
+                   stream=stream)
+
+    for _ in range(warmup):
+        step()
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after warm-up")
+
+    # ---- timed region (device time, CUDA events on the launching stream).
+    # The K steps run exactly as a caller runs them: no events between the
+    # kernels, whose launches overlap (programmatic dependent launch).
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    ms_total = barrier_max(e0.elapsed_time(e1))
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after the timed region")
+
+    # ---- per-kernel pass: the same K steps again with a CUDA event pair around
+    # every launch (the library's launch profiler).  The profiler runs every
+    # launch alone on the caller's stream (no side-stream apply, no overlap of
+    # consecutive launches), so this pass gives each kernel's own duration
+    # (kernel shares, roofline) but not the headline time.
+    ct.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(steps):
+        step()
+    p1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ct.profile_enable(False)
+    ms_profiled = barrier_max(p0.elapsed_time(p1))
+    prof = ct.profile_read()
+    if ct.status(stream) != ct.LACT_OK:
+        raise SystemExit("device status not OK after the per-kernel pass")
+    return {"inp_cpu": inp_cpu, "inp": inp, "w_out": w_out, "stream": stream, "ms_total": ms_total,
+            "ms_profiled": ms_profiled, "prof": prof, "clocks": clk}
+
+
+def roofline_entry(prof: dict, w: Workload, steps: int):
+    """Roofline of the kernel with the largest summed duration in the
+    per-kernel pass.  Every launch there runs alone, so a tensor-core kernel
+    is measured against the burst bf16 peak; the sustained fraction is given
+    beside it."""
+    hbm, pk_burst, pk_sust, pk_src = peaks()
+    work = kernel_work(w)
+    name, (n_launch, ms_kind) = max(prof.items(), key=lambda kv: kv[1][1])
+    if name not in work:
+        return None
+    bound, amount, _ = work[name]
+    per_launch = amount * steps / n_launch
+    dur_s = ms_kind / n_launch / 1e3
+    if bound == "tensor":
+        achieved = per_launch / dur_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk_burst, "unit": "TFLOP/s",
+                "frac": achieved / pk_burst, "frac_of_sustained": achieved / pk_sust,
+                "peak_source": f"{pk_src} burst bf16 (the kernel is timed alone)"}
+    else:
+        achieved = per_launch / dur_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_source": f"{pk_src} copy bandwidth"}
+    roof.update({"kernel": name, "launches": n_launch, "avg_launch_us": 1e3 * ms_kind / n_launch,
+                 "work_per_launch": per_launch, "timed": "alone (per-kernel pass)",
+                 "traffic": traffic_for(name, w)})
+    return roof
+
+
+def config_entry(ct, idx: int, steps: int, warmup: int, dev, local: int) -> dict:
+    """One line of the `configs` record: another workload of the same layer
+    timed the same way on this GPU (inputs resident in HBM, larger than L2)."""
+    w = WORKLOADS[idx]
+    t = forward_timing(ct, w, dev, steps, warmup, 0, lambda: None, lambda x: x, local)
+    _, pk_burst, pk_sust, _ = peaks()
+    ms_step = t["ms_total"] / steps
+    tflops = step_flops(w) / (ms_step / 1e3) / 1e12
+    prof = t["prof"]
+    total = sum(x[1] for x in prof.values())
+    return {"workload": w.name, "steps": steps, "warmup": warmup, "ms_per_step": ms_step,
+            "tokens_per_s": w.tokens / (ms_step / 1e3), "algorithmic_tflops": tflops,
+            "frac_of_burst": tflops / pk_burst, "frac_of_sustained": tflops / pk_sust,
+            "roofline": roofline_entry(prof, w, steps),
+            "kernel_shares": {k: round(v[1] / total, 4) for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])},
+            "clocks": t["clocks"]}
+
 # ---------------------------------------------------------------- CPU oracle
 def oracle_sample(w: Workload, inp: dict, budget_s: float, max_heads: int):
     """Runs the oracle on whole (batch, head) sequences until `budget_s`
@@ -284,6 +398,9 @@ def main():
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "swa"],
                     help="time the layer forward (default), its backward (lact_ttt_bwd) or the "
                          "block's sliding-window attention (lact_swa_fwd, window = the chunk)")
+    ap.add_argument("--extra-steps", type=int, default=20,
+                    help="timed steps of each other bf16 workload in the `configs` record "
+                         "(1 GPU; 0 skips them)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload at this sequence length instead (a scaled case "
                          "for profiling; named in config.workload)")
@@ -319,96 +436,21 @@ def main():
             import torch.distributed as dist
             dist.barrier()
 
-    inp_cpu = make_inputs(w, seed=rank)
-    inp = {k: (None if v is None else v.to(dev)) for k, v in inp_cpu.items()}
-    B, H = w.B, w.H
-    out = torch.empty_like(inp["q"])
-    w_out = (torch.empty((B * H, w.dh, w.d), device=dev), torch.empty((B * H, w.d, w.dh), device=dev),
-             torch.empty((B * H, w.dh, w.d), device=dev))
-    ws = torch.empty(ct.workspace_bytes(inp["q"], inp["k"], inp["w1"], w.chunk, w.order, w.rule),
-                     device=dev, dtype=torch.uint8)
-    stream = torch.cuda.current_stream(dev)
-
-    def step():
-        ct.ttt_fwd(inp["q"], inp["k"], inp["v"], inp["lr"], inp["beta"], inp["w1"], inp["w2"],
-                   inp["w3"], w.chunk, w.order, w.rule, out=out, w_out=w_out, workspace=ws,
-                   stream=stream)
-
-    for _ in range(args.warmup):
-        step()
-    if ct.status(stream) != ct.LACT_OK:
-        raise SystemExit("device status not OK after warm-up")
-
-    # ---- timed region (device time, CUDA events on the launching stream).
-    # The K steps run exactly as a caller runs them: no events between the
-    # kernels, whose launches overlap (programmatic dependent launch).
-    clocks = ClockSampler(local)
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    clk = clocks.stop()
-    ms_total = barrier_max(e0.elapsed_time(e1))
-    if ct.status(stream) != ct.LACT_OK:
-        raise SystemExit("device status not OK after the timed region")
-
-    # ---- per-kernel pass: the same K steps again with a CUDA event pair around
-    # every launch (the library's launch profiler).  The profiler runs every
-    # launch alone on the caller's stream (no side-stream apply, no overlap of
-    # consecutive launches), so this pass gives each kernel's own duration
-    # (kernel shares, roofline) but not the headline time.
-    ct.profile_enable(True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    p0.record(stream)
-    for _ in range(args.steps):
-        step()
-    p1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    ct.profile_enable(False)
-    ms_profiled = barrier_max(p0.elapsed_time(p1))
-    prof = ct.profile_read()
-    if ct.status(stream) != ct.LACT_OK:
-        raise SystemExit("device status not OK after the per-kernel pass")
+    t = forward_timing(ct, w, dev, args.steps, args.warmup, rank, barrier, barrier_max, local)
+    inp_cpu, ms_total, ms_profiled, prof, clk = t["inp_cpu"], t["ms_total"], t["ms_profiled"], t["prof"], t["clocks"]
+    stream, w_out = t["stream"], t["w_out"]
 
     ms_step = ms_total / args.steps
     tok_step = w.tokens
     value = job_value(world, tok_step, args.steps, ms_total)
     hbm, pk_burst, pk_sust, pk_src = peaks()
     flops = step_flops(w)
-    launches_per_step = ct.launch_count(inp["q"], inp["k"], inp["w1"], w.chunk, w.order, w.rule)
-
-    # ---- roofline of the dominant kernel
-    work = kernel_work(w)
-    dom = max(prof.items(), key=lambda kv: kv[1][1])
-    name, (n_launch, ms_kind) = dom
-    roof = None
-    if name in work:
-        bound, amount, unit = work[name]
-        per_launch = amount * args.steps / n_launch
-        dur_s = ms_kind / n_launch / 1e3
-        if bound == "tensor":
-            achieved = per_launch / dur_s / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
-                    "frac": achieved / pk_sust}
-        else:
-            achieved = per_launch / dur_s / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                    "frac": achieved / hbm}
-        roof.update({"kernel": name, "launches": n_launch, "avg_launch_us": 1e3 * ms_kind / n_launch,
-                     "timed": "alone (per-kernel pass)",
-                     "traffic": traffic_for(name, w), "peak_source": f"{pk_src} sustained bf16"
-                     if bound == "tensor" else f"{pk_src} copy bandwidth"})
+    launches_per_step = ct.launch_count(t["inp"]["q"], t["inp"]["k"], t["inp"]["w1"], w.chunk, w.order, w.rule)
+    roof = roofline_entry(prof, w, args.steps)
     kernels = {k: {"launches": v[0], "ms": round(v[1], 4),
                    "share": round(v[1] / sum(x[1] for x in prof.values()), 4)}
                for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    del t
 
     # ---- end to end: host buffers in, results back, through the C ABI
     pin = {k: (None if v is None else v.pin_memory()) for k, v in inp_cpu.items()}
@@ -416,7 +458,6 @@ def main():
     hwo = tuple(torch.empty(t.shape, dtype=torch.float32).pin_memory() for t in w_out)
     hws = torch.empty(ct.host_workspace_bytes(pin["q"], pin["k"], pin["w1"], w.chunk, w.order,
                                               w.rule), device=dev, dtype=torch.uint8)
-    del ws
 
     def host_step():
         ct.ttt_fwd_host(pin["q"], pin["k"], pin["v"], pin["lr"], pin["beta"], pin["w1"], pin["w2"],
@@ -445,8 +486,8 @@ def main():
         "data": "synthetic (seeded normal q/k/v, softplus lr, random-init fast weights)",
         "config": workload_config(w, world),
         "tensor_peak_frac": {"algorithmic_tflops": flops / (ms_step / 1e3) / 1e12,
-                             "frac_of_sustained": flops / (ms_step / 1e3) / 1e12 / pk_sust,
                              "frac_of_burst": flops / (ms_step / 1e3) / 1e12 / pk_burst,
+                             "frac_of_sustained": flops / (ms_step / 1e3) / 1e12 / pk_sust,
                              "peak_source": pk_src},
         "roofline": roof,
         "kernels": kernels,
@@ -461,6 +502,10 @@ def main():
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk,
     }
+    if world == 1 and not args.tokens and args.extra_steps > 0:
+        # the other bf16 workloads, timed the same way (1 GPU only)
+        line["configs"] = [config_entry(ct, i, args.extra_steps, args.warmup, dev, local)
+                           for i in (2, 3, 4, 5) if i != args.workload]
     if world == 1 and rank == 0:
         tok, sec, nh = oracle_sample(w, inp_cpu, args.cpu_budget, max_heads=w.B * w.H)
         line["cpu_baseline"] = {"value": tok / sec, "unit": UNIT, "cores": blas_threads(),
@@ -540,18 +585,20 @@ def run_backward(args, w: Workload):
     dom_name, (n_launch, ms_kind) = max(prof.items(), key=lambda kv: kv[1][1])
     flops = bwd_flops(w)
     roof = None
-    _, _, pk_sust, pk_src = peaks()
+    _, pk_burst, pk_sust, pk_src = peaks()
     if dom_name in ("simt_gemm_f32", "bwd_gemm_umma"):
         # every FLOP of bwd_flops() is in these contractions
         achieved = flops * args.steps / (ms_kind / 1e3) / 1e12
         tensor = dom_name == "bwd_gemm_umma"
-        peak = pk_sust if tensor else FP32_FMA_TFLOPS
+        peak = pk_burst if tensor else FP32_FMA_TFLOPS
         roof = {"bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "kernel": dom_name, "launches": n_launch,
                 "avg_launch_us": 1e3 * ms_kind / n_launch, "timed": "alone (per-kernel pass)",
                 "traffic": None,
-                "peak_source": f"{pk_src} sustained bf16" if tensor else
+                "peak_source": f"{pk_src} burst bf16 (the kernel is timed alone)" if tensor else
                                "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz"}
+        if tensor:
+            roof["frac_of_sustained"] = achieved / pk_sust
     kernels = {k: {"launches": v[0], "ms": round(v[1], 4),
                    "share": round(v[1] / sum(x[1] for x in prof.values()), 4)}
                for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
@@ -594,6 +641,7 @@ def run_backward(args, w: Workload):
         "data": "synthetic (seeded normal q/k/v/dout, softplus lr, random-init fast weights)",
         "config": dict(workload_config(w, 1), **{"pass": "backward (lact_ttt_bwd)"}),
         "peak_frac": {"algorithmic_tflops": flops / (ms_step / 1e3) / 1e12,
+                      "frac_of_burst_bf16": flops / (ms_step / 1e3) / 1e12 / pk_burst,
                       "frac_of_sustained_bf16": flops / (ms_step / 1e3) / 1e12 / pk_sust,
                       "frac_of_fp32_fma": flops / (ms_step / 1e3) / 1e12 / FP32_FMA_TFLOPS},
         "roofline": roof,
@@ -673,8 +721,7 @@ def run_swa(args, w: Workload):
     torch.cuda.synchronize(dev)
     prof = ct.profile_read()
     ct.profile_enable(False)
-    _, _, pk_sust, pk_src = peaks()
-    hbm, *_ = peaks()
+    hbm, pk_burst, pk_sust, pk_src = peaks()
     flops = swa_flops(B, H, T, d, window)
     kernels = {k: {"launches": v[0], "ms": round(v[1], 4),
                    "share": round(v[1] / sum(x[1] for x in prof.values()), 4)}
@@ -683,10 +730,11 @@ def run_swa(args, w: Workload):
     roof = None
     if dom in ("swa_gemm_umma", "swa_flash_umma"):
         achieved = flops * args.steps / (ms_kind / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
-                "frac": achieved / pk_sust, "kernel": dom, "launches": n_launch,
-                "avg_launch_us": 1e3 * ms_kind / n_launch, "timed": "alone (per-kernel pass)",
-                "traffic": traffic_for(dom, w), "peak_source": f"{pk_src} sustained bf16",
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk_burst, "unit": "TFLOP/s",
+                "frac": achieved / pk_burst, "frac_of_sustained": achieved / pk_sust, "kernel": dom,
+                "launches": n_launch, "avg_launch_us": 1e3 * ms_kind / n_launch,
+                "timed": "alone (per-kernel pass)", "traffic": traffic_for(dom, w),
+                "peak_source": f"{pk_src} burst bf16 (the kernel is timed alone)",
                 "work": "algorithmic: 4 d FLOPs per (query, key) pair in the window"}
     elif dom == "swa_elem":
         Lw = window + 128
@@ -727,6 +775,7 @@ def run_swa(args, w: Workload):
                    "window": window, "pass": "sliding-window attention (lact_swa_fwd)",
                    "l2": "inputs and scores larger than L2, no flush"},
         "peak_frac": {"algorithmic_tflops": flops / (ms_step / 1e3) / 1e12,
+                      "frac_of_burst_bf16": flops / (ms_step / 1e3) / 1e12 / pk_burst,
                       "frac_of_sustained_bf16": flops / (ms_step / 1e3) / 1e12 / pk_sust},
         "roofline": roof, "kernels": kernels,
         "gpu_launches": sum(v[0] for v in prof.values()),

@@ -329,9 +329,13 @@ __global__ void __launch_bounds__(256) k_finalize_state(const float* __restrict_
 }
 
 // beta_bar[bh][c] = mean of beta over chunk c's tokens (one warp per entry).
+// With `sums` set the kernel writes the sum instead, and the token count at
+// beta_bar[BH * nch + w]: context-parallel ranks each hold a share of every
+// chunk, so their sums and counts are added over the ranks first and
+// k_beta_div forms the mean.
 __global__ void __launch_bounds__(256) k_beta_mean(const float* __restrict__ beta, int BH, int64_t T,
                                                    int64_t chunk, int nch,
-                                                   float* __restrict__ beta_bar) {
+                                                   float* __restrict__ beta_bar, int sums) {
   griddep_launch();
   griddep_wait();
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -343,7 +347,22 @@ __global__ void __launch_bounds__(256) k_beta_mean(const float* __restrict__ bet
   float s = 0.f;
   for (int64_t t = t0 + lane; t < t1; t += 32) s += b[t];
   s = warp_sum(s);
-  if (lane == 0) beta_bar[w] = s / static_cast<float>(t1 - t0);
+  if (lane != 0) return;
+  if (sums) {
+    beta_bar[w] = s;
+    beta_bar[static_cast<int64_t>(BH) * nch + w] = static_cast<float>(t1 - t0);
+  } else {
+    beta_bar[w] = s / static_cast<float>(t1 - t0);
+  }
+}
+
+// beta_bar[i] /= beta_bar[n + i]: the mean of beta over a chunk whose sum and
+// token count were added over the context-parallel ranks.
+__global__ void __launch_bounds__(256) k_beta_div(float* __restrict__ beta_bar, int64_t n) {
+  griddep_launch();
+  griddep_wait();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) beta_bar[i] = beta_bar[i] / beta_bar[n + i];
 }
 
 // ---------------------------------------------------------------------------

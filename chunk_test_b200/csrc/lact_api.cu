@@ -143,7 +143,7 @@ static void plan(const Dims& D, Bump& bp, Bufs& b) {
   b.P = bp.take<float>((bf ? D.splits : 1) * planes);
   if (D.rule == LACT_RULE_MOMENTUM) {
     b.Mm = bp.take<float>(planes);
-    b.bbar = bp.take<float>(D.BH * D.nch);
+    b.bbar = bp.take<float>(2 * D.BH * D.nch);   // sums, then token counts (context parallelism)
   }
   if (!D.fused_kg) b.E = bp.take<uint8_t>(3 * D.BH * D.key_rows * D.dh * esz);
   if (D.split) b.E_lo = bp.take<uint8_t>(3 * D.BH * D.key_rows * D.dh * esz);
@@ -568,13 +568,22 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
   // q^, k^ = silu + L2 norm rows.
   L(K_PROLOGUE, [&] { return launch_prologue(D, b, in, st); });
   if (D.rule == LACT_RULE_MOMENTUM) {
+    // With context parallelism: per-chunk sums and token counts, added over
+    // the ranks, then divided on the device.
+    const int sums = in.allreduce ? 1 : 0;
+    const int64_t w = D.BH * D.nch;
     L(K_BETA_MEAN, [&] {
-      const int64_t w = D.BH * D.nch;
       (void)launch_pdl(k_beta_mean, static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st, in.beta, BH, D.T, D.chunk,
-                                                                            static_cast<int>(D.nch), b.bbar);
+                       static_cast<int>(D.nch), b.bbar, sums);
       return cudaGetLastError();
     });
-    reduce(b.bbar, D.BH * D.nch, LACT_REDUCE_MEAN);   // equal shares: mean of the ranks' means
+    if (sums) {
+      reduce(b.bbar, 2 * w, LACT_REDUCE_SUM);
+      L(K_BETA_MEAN, [&] {
+        (void)launch_pdl(k_beta_div, static_cast<unsigned>(cdiv(w, 256)), 256, 0, st, b.bbar, w);
+        return cudaGetLastError();
+      });
+    }
   }
 
   bool join_before_rule = false, side_used = false;
@@ -937,8 +946,15 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
     if (upd) ++ver;
   }
 
-  if (side_used && L.err == LACT_OK && cudaStreamWaitEvent(main_st, side->join[last_join], 0) != cudaSuccess)
-    L.err = LACT_ECUDA;   // the last chunks' applies are done before the call's work ends
+  // The last chunks' applies are done before the call's work ends, also when
+  // a launch failed after an apply was forked: the side stream may still read
+  // or write the caller's buffers, which the caller may free once the call
+  // returns.  The first error code is kept.
+  if (side_used) {
+    const bool joined_ok = cudaEventRecord(side->join[last_join], side->side) == cudaSuccess &&
+                           cudaStreamWaitEvent(main_st, side->join[last_join], 0) == cudaSuccess;
+    if (!joined_ok && L.err == LACT_OK) L.err = LACT_ECUDA;
+  }
   L(K_FINALIZE, [&] {
     (void)launch_pdl(k_finalize_state, state_blocks, 256, 0, st, b.Wm, BH, d, dh, in.w1o, in.w2o, in.w3o,
                      static_cast<const float*>(b.Mm), in.m1, in.m2, in.m3);
@@ -1039,34 +1055,30 @@ static int input_bytes(const Dims& D, size_t sz[8]) {
 
 // Scratch of lact_ttt_fwd_noalloc: a file-scope device buffer, so callers
 // that may not allocate still get a workspace.  Host code must not use the
-// symbol itself as a device address; the address is looked up per device.
+// symbol itself as a device address; the address is looked up for the
+// current device.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[LACT_NOALLOC_SCRATCH_BYTES];
-static std::mutex g_noalloc_mu;
-static void* g_noalloc_addr[64];
 
-// Device address of g_noalloc_scratch on the current device (looked up once
-// per device, with that device current).
+// Device address of g_noalloc_scratch on the current device.  Looked up on
+// every call (a lookup allocates nothing): after a device reset the module
+// is loaded again and the buffer may sit at another address, so a cached
+// address could go stale.
 static int noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LACT_ECUDA;
-  if (dev < 0 || dev >= 64) return LACT_ENODEV;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LACT_ECUDA;
-    g_noalloc_addr[dev] = ptr;
-  }
-  *out = g_noalloc_addr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LACT_ECUDA;
+  *out = ptr;
   return LACT_OK;
 }
 
 // One thread waits on a barrier that expects one arrival nobody makes.
-__global__ void k_selftest_wait() {
+// The budget is the kernel's own argument, so calls running at the same
+// time keep their normal budget.
+__global__ void k_selftest_wait(long long budget) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_barrier_init();
-    mbar_wait(&bar, 0);
+    mbar_wait_for(&bar, 0, budget);
   }
 }
 
@@ -1093,7 +1105,11 @@ int64_t lact_ttt_launch_count_ex(const lact_problem* p, const lact_fwd_opts* opt
   plan(D, bp, b);
   Inputs in;
   std::memset(&in, 0, sizeof(in));
-  in.mask = opts ? opts->update_mask : nullptr;   // the only option that changes the launches
+  // the options that change the launches: the update mask, and the
+  // context-parallel hook (the momentum rule's beta means then take a
+  // second kernel)
+  in.mask = opts ? opts->update_mask : nullptr;
+  in.allreduce = opts ? opts->allreduce : nullptr;
   Launcher L{true, nullptr};
   run(D, b, in, nullptr, L, nullptr);
   return L.count;
@@ -1335,14 +1351,8 @@ int lact_device_check(void) {
 int lact_selftest_wait_timeout(int64_t budget_cycles, void* stream) {
   if (budget_cycles < 1 || budget_cycles > (int64_t(1) << 31)) return LACT_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long normal = kDefaultWaitBudget, b = budget_cycles;
-  if (cudaMemcpyToSymbolAsync(g_wait_budget, &b, sizeof(b), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return LACT_ECUDA;
-  k_selftest_wait<<<1, 32, 0, st>>>();
+  k_selftest_wait<<<1, 32, 0, st>>>(static_cast<long long>(budget_cycles));
   const cudaError_t e = cudaGetLastError();
-  if (cudaMemcpyToSymbolAsync(g_wait_budget, &normal, sizeof(normal), 0, cudaMemcpyHostToDevice, st) !=
-      cudaSuccess)
-    return LACT_ECUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return LACT_ECUDA;
   return e == cudaSuccess ? LACT_OK : LACT_ECUDA;
 }

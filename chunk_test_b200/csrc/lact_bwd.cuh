@@ -189,7 +189,7 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
     L(K_BETA_MEAN, [&] {
       const int64_t w = D.BH * D.nch;
       (void)launch_pdl(k_beta_mean, static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st, in.beta, BH, D.T,
-                       D.chunk, static_cast<int>(D.nch), b.bbar);
+                       D.chunk, static_cast<int>(D.nch), b.bbar, 0);
       return cudaGetLastError();
     });
   }
@@ -481,7 +481,7 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     L(K_BETA_MEAN, [&] {
       const int64_t w = D.BH * D.nch;
       (void)launch_pdl(k_beta_mean, static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st, in.beta, BH, D.T,
-                       D.chunk, static_cast<int>(D.nch), b.bbar);
+                       D.chunk, static_cast<int>(D.nch), b.bbar, 0);
       return cudaGetLastError();
     });
   }

@@ -22,7 +22,6 @@ __device__ int g_status;
 // waits more than a millisecond or so; hitting the budget means a lost
 // arrival, and the kernel then stops issuing work and returns.
 constexpr long long kDefaultWaitBudget = 1000000000LL;
-__device__ long long g_wait_budget = kDefaultWaitBudget;
 
 constexpr int kStatusTimeout = 1;
 
@@ -71,11 +70,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// g_wait_budget cycles, records kStatusTimeout and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// `budget` cycles, records kStatusTimeout and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, long long budget) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  const long long budget = g_wait_budget;
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > budget) {
       atomicExch(&g_status, kStatusTimeout);
@@ -83,6 +81,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kDefaultWaitBudget);
 }
 
 // ------------------------------------------------------------------ TMA

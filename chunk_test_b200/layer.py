@@ -51,6 +51,48 @@ def _check(q, k, v, lr, beta, w1, w2, w3, device_kind):
     for name, t in (("lr", lr), ("beta", beta), ("w1", w1), ("w2", w2), ("w3", w3)):
         if t is not None and t.dtype != torch.float32:
             raise TypeError(f"{name} must be float32")
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, H, T, d] tensors")
+    B, H, _, d = q.shape
+    T = k.shape[2]
+    if tuple(k.shape) != (B, H, T, d) or tuple(v.shape) != (B, H, T, d):
+        raise ValueError("k and v must be [B, H, T, d] with q's B, H and d")
+    if tuple(lr.shape) != (B, H, T, 3):
+        raise ValueError("lr must be [B, H, T, 3]")
+    if beta is not None and tuple(beta.shape) != (B, H, T):
+        raise ValueError("beta must be [B, H, T]")
+    if w1.dim() != 3:
+        raise ValueError("w1 must be [H or B*H, dh, d]")
+    hw, dh = w1.shape[0], w1.shape[1]
+    if tuple(w1.shape) != (hw, dh, d) or tuple(w3.shape) != (hw, dh, d) or tuple(w2.shape) != (hw, d, dh):
+        raise ValueError("w1, w3 must be [Hw, dh, d] and w2 [Hw, d, dh] with one Hw")
+
+
+def _check_outputs(q, w1, out, w_out, device_kind):
+    """The caller-given outputs: `out` shaped like q in q's dtype, `w_out`
+    three float32 tensors [B*H, dh, d], [B*H, d, dh], [B*H, dh, d]; all
+    contiguous and on q's device.  The library checks only for null
+    pointers, so a wrong size here would let the kernels write past the
+    buffer."""
+    B, H, _, d = q.shape
+    dh = w1.shape[1]
+    if (out.device != q.device or out.dtype != q.dtype or tuple(out.shape) != tuple(q.shape)
+            or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous tensor shaped like q, in q's dtype, on q's device")
+    if w_out is None or len(w_out) != 3:
+        raise ValueError("w_out must hold three tensors")
+    shapes = ((B * H, dh, d), (B * H, d, dh), (B * H, dh, d))
+    for i, (t, shp) in enumerate(zip(w_out, shapes)):
+        if (t.device.type != device_kind or t.device != q.device or t.dtype != torch.float32
+                or tuple(t.shape) != shp or not t.is_contiguous()):
+            raise ValueError(f"w_out[{i}] must be a contiguous float32 {list(shp)} tensor on q's device")
+
+
+def _check_workspace(ws, device, need):
+    if ws.device != device or ws.dtype != torch.uint8 or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor on the device of the call")
+    if ws.numel() < need:
+        raise ValueError(f"workspace holds {ws.numel()} bytes; the call needs {need}")
 
 
 def workspace_bytes(q, k, w1, chunk, order, rule) -> int:
@@ -94,18 +136,19 @@ def _hook(py_fn, device, errors: list):
 
 
 def torch_distributed_allreduce(group=None):
-    """A context-parallel hook for ttt_fwd(allreduce=...): all-reduce over the
-    torch.distributed process group `group` (NCCL for CUDA tensors), enqueued
-    on the layer's stream, so that the layer's later kernels see the sum (or
-    the mean, for REDUCE_MEAN)."""
+    """A context-parallel hook for ttt_fwd(allreduce=...): a sum all-reduce
+    over the torch.distributed process group `group` (NCCL for CUDA tensors),
+    enqueued on the layer's stream, so that the layer's later kernels see the
+    sum.  The library asks only for sums (any mean it needs it forms on the
+    device from summed sums and counts)."""
     import torch.distributed as dist
 
     def fn(buf, op, stream=None):
+        if op != _abi.REDUCE_SUM:
+            raise ValueError(f"unsupported reduction op {op}")
         ctx = torch.cuda.stream(stream) if (stream is not None and buf.is_cuda) else _nullctx()
         with ctx:
             dist.all_reduce(buf, op=dist.ReduceOp.SUM, group=group)
-            if op == _abi.REDUCE_MEAN:
-                buf.div_(dist.get_world_size(group))
 
     return fn
 
@@ -178,11 +221,13 @@ def ttt_fwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out=None, w_ou
         w_out = (torch.empty((B * H, dh, d), device=q.device, dtype=torch.float32),
                  torch.empty((B * H, d, dh), device=q.device, dtype=torch.float32),
                  torch.empty((B * H, dh, d), device=q.device, dtype=torch.float32))
+    _check_outputs(q, w1, out, w_out, "cuda")
     need = _abi.workspace_bytes(p)
     if need == 0:
         raise LactError(_abi.LACT_EINVAL, "lact_ttt_workspace_bytes")
     if workspace is None:
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    _check_workspace(workspace, q.device, need)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     rc = _abi.lib().lact_ttt_fwd_ex(
@@ -288,6 +333,7 @@ def ttt_fwd_noalloc(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out, w
     lact_ttt_fwd_noalloc in include/lact.h for its size and sharing rules).
     `out` and `w_out` must be given (pre-allocated by the caller)."""
     _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
+    _check_outputs(q, w1, out, w_out, "cuda")
     p = make_problem(q, k, w1, chunk, order, rule)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
@@ -307,7 +353,11 @@ def ttt_fwd_host(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, *, out, w_ou
     they are valid.  `workspace` is a device uint8 tensor of
     host_workspace_bytes() bytes."""
     _check(q, k, v, lr, beta, w1, w2, w3, "cpu")
+    _check_outputs(q, w1, out, w_out, "cpu")
     p = make_problem(q, k, w1, chunk, order, rule)
+    if workspace.device.type != "cuda":
+        raise ValueError("workspace must be a CUDA tensor")
+    _check_workspace(workspace, workspace.device, _abi.host_workspace_bytes(p))
     if stream is None:
         stream = torch.cuda.current_stream(workspace.device)
     rc = _abi.lib().lact_ttt_fwd_host(

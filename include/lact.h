@@ -207,9 +207,10 @@ int lact_ttt_fwd_ex(const lact_problem* p, const lact_fwd_opts* opts,
  * exceeds the buffer.  It calls no cudaMalloc, cudaFree or other allocating
  * routine.
  *
- * The first call on a device looks up the buffer's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the one buffer and it keeps
+ * Every call looks up the buffer's device address on the current device
+ * (cudaGetSymbolAddress, which allocates nothing); the first call on a
+ * device may load the library's device code there, so make it before any
+ * stream capture.  All calls share the one buffer and it keeps
  * the previous call's contents (the forward never relies on its contents at
  * entry): calls that can overlap on the GPU (different streams, or several
  * host threads) race on it and must be serialised by the caller. */

@@ -60,8 +60,7 @@ class EmulatedGroup:
                 total = self.bufs[0].clone()
                 for b in self.bufs[1:]:
                     total += b                        # the same order on every rank
-                if op == ct.REDUCE_MEAN:
-                    total /= self.n
+                assert op == ct.REDUCE_SUM            # the library asks only for sums
                 done = torch.cuda.Event()
                 done.record(stream)
             self.done[rank] = done

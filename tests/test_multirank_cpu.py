@@ -130,25 +130,40 @@ def _cp_hook_worker(rank, world, port, outdir):
         fn = ct.torch_distributed_allreduce()
         a = torch.arange(6, dtype=torch.float32) + 10.0 * rank
         fn(a, ct.REDUCE_SUM)
-        b = torch.full((4,), 1.0 + rank)
-        fn(b, ct.REDUCE_MEAN)
+        # a per-chunk mean over ranks that hold unequal shares: the library
+        # sums the (sum, count) pairs and divides on the device
+        sums = torch.tensor([3.0 * (rank + 1), 5.0, 2.0 * (rank + 1), 1.0 + rank])
+        fn(sums, ct.REDUCE_SUM)
+        try:
+            fn(torch.ones(2), ct.REDUCE_MEAN)
+            rejected = False
+        except ValueError:
+            rejected = True
         with open(os.path.join(outdir, f"cp{rank}.json"), "w") as f:
-            json.dump({"sum": a.tolist(), "mean": b.tolist()}, f)
+            json.dump({"sum": a.tolist(), "pairs": sums.tolist(), "mean_rejected": rejected}, f)
     finally:
         dist.destroy_process_group()
 
 
-def test_context_parallel_hook_sums_and_averages_over_ranks():
+def test_context_parallel_hook_sums_over_ranks():
     """The torch.distributed hook that the layer calls between a chunk's
-    gradient and its rule: a sum over the ranks in place (gradients), or the
-    mean (the per-chunk beta means of equal shares)."""
+    gradient and its rule: a sum over the ranks in place (the gradient
+    planes, and the per-chunk beta sums and token counts whose quotient the
+    library forms on the device).  The hook performs no other arithmetic and
+    refuses any other op."""
     with tempfile.TemporaryDirectory() as d:
         mp.start_processes(_cp_hook_worker, args=(2, _free_port(), d), nprocs=2, join=True,
                            start_method="spawn")
         res = [json.load(open(os.path.join(d, f"cp{r}.json"))) for r in range(2)]
     for r in res:
         assert r["sum"] == [10.0 + 2 * i for i in range(6)]
-        assert r["mean"] == [1.5] * 4
+        # rank r held [3 (r + 1), 5, 2 (r + 1), 1 + r]: the sums add element-wise
+        assert r["pairs"] == [9.0, 10.0, 6.0, 3.0]
+        assert r["mean_rejected"]
+    # the mean of beta over a chunk split 1 : 2 between the ranks is the
+    # quotient of the summed pair, not the mean of the two ranks' means
+    total_sum, total_count = res[0]["pairs"][2], res[0]["pairs"][3]
+    assert total_sum / total_count == (2.0 + 4.0) / (1.0 + 2.0)
 
 
 @pytest.mark.parametrize("rule", [0, 1, 2])
