@@ -221,6 +221,20 @@ static bool map3d_plain(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 map over [batch][rows][inner] (dense), 32 x 32 boxes with
+// 128-byte swizzle (the fp32 staging tiles of bulk-store epilogues).
+static bool map3d_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint64_t batch) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner * 4, inner * rows * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ launches
 // Opt-in dynamic shared memory per CTA on sm_100 (227 KB).
 constexpr int kMaxSmemPerBlock = 232448;
@@ -756,8 +770,17 @@ static void run(const Dims& D, const Bufs& b, const Inputs& in, cudaStream_t mai
           if (D.rule != LACT_RULE_MUON) {  // W2's gradient straight into its [d, dh] layout
             g.tr_group = 1; g.tr_mod = BH; g.ld_t = dh;
           }
-          if (!D.split && (D.bn == 128 || D.bn == 256))   // 256-row pair tiles over dh
+          if (!D.split && (D.bn == 128 || D.bn == 256)) {  // 256-row pair tiles over dh
+            // the partial planes leave through bulk tensor stores: W1's and
+            // W3's as [dh, d], W2's transposed into [d, dh]
+            const uint64_t nplanes = static_cast<uint64_t>(splits) * 3 * BH;
+            if (g.tr_group == 1) {
+              if (!map3d_f32(&g.tmOut, b.P, d, dh, nplanes) || !map3d_f32(&g.tmOutT, b.P, dh, d, nplanes))
+                return cudaErrorInvalidValue;
+              g.out_tma = 1;
+            }
             return launch_gemm_pair<true, true>(D.bn, dim3(d / D.bn, cdiv(dh, 256), splits * 3 * BH), g, st);
+          }
           return launch_gemm_any<true, true>(D.split, D.bn, dim3(d / D.bn, cdiv(dh, 128), splits * 3 * BH), g, st);
         });
       } else if (!bf) {

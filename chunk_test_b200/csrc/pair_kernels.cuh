@@ -157,24 +157,31 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
   griddep_wait();  // after the local setup, before any global access
 
   if (warp == 0) {
-    if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      for (int tile = pair; ok && tile < ntiles; tile += npairs) {
-        const typename Op::Tile t = Op::map_tile(p, tile, rank);
-        const int nkb = Op::num_kb(p, t);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % S;
-          if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) { ok = false; break; }
-          if (leader) mbar_arrive_expect_tx(&full[s], 2u * Op::kStageBytes);
-          Op::load(p, t, kb, smem + s * Op::kStageBytes, mapa_rank(smem_u32(&full[s]), 0));
+    // The whole warp produces: lane 0 waits for the slot (and, in the even
+    // CTA, posts the stage's bytes of both CTAs), then the copies are spread
+    // over the lanes.
+    int it = 0;
+    bool ok = true;
+    LaneIssue li(lane);   // one running count: successive copies rotate over the lanes
+    for (int tile = pair; ok && tile < ntiles; tile += npairs) {
+      const typename Op::Tile t = Op::map_tile(p, tile, rank);
+      const int nkb = Op::num_kb(p, t);
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % S;
+        if (lane == 0) {
+          if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) ok = false;
+          else if (leader) mbar_arrive_expect_tx(&full[s], 2u * Op::kStageBytes);
         }
+        ok = warp_bcast(ok);
+        if (!ok) break;
+        Op::load(p, t, kb, smem + s * Op::kStageBytes, mapa_rank(smem_u32(&full[s]), 0), li);
       }
-      // Every stage release (including the last S, committed by the even
-      // CTA's MMAs) has landed before this CTA may leave.
+    }
+    // Every stage release (including the last S, committed by the even
+    // CTA's MMAs) has landed before this CTA may leave.
+    if (lane == 0)
       for (int i = it > S ? it - S : 0; ok && i < it; ++i)
         if (!mbar_wait(&empty[i % S], (i / S) & 1)) ok = false;
-    }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       int it = 0, local = 0;
@@ -236,7 +243,11 @@ struct GemmPairOp {
   static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
   static constexpr int kAccCols = TmemCols<BN>::value;
   static constexpr int kAccBufs = 2;
-  static constexpr int kExtraBytes = Base::kExtraBytes;   // the epilogue's staging tiles
+  // The epilogue's staging: per epilogue warp two 32 x 32 fp32 tiles (the
+  // bulk-store path) or the generic path's tile, whichever is larger.
+  static constexpr int kStgBytes = 2 * 32 * 32 * 4;
+  static constexpr int kExtraBytes =
+      kEpiWarps * kStgBytes > Base::kExtraBytes ? kEpiWarps * kStgBytes : Base::kExtraBytes;
   using Tile = typename Base::Tile;   // m0 is this CTA's first row
 
   __device__ static int num_tiles(const Params& p) { return p.n_tiles; }
@@ -252,23 +263,24 @@ struct GemmPairOp {
     tma_prefetch_map(&p.tmB);
     if (p.alt_group >= 0) tma_prefetch_map(&p.tmB2);
   }
-  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint32_t bar) {
+  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint32_t bar, LaneIssue& li) {
     const int kk = (t.split * p.kb_count + kb) * kBK;
     const int ak = p.a_k0 + kk, bk = p.b_k0 + kk;
     const int half = (t.m0 / kBM) & 1;  // this CTA's rank in the pair
     const int n0 = t.n0 + half * kHalfN;
     if (A_MN) {
-      tma_load_3d_pair(st, &p.tmA, bar, t.m0, ak, t.item);
-      tma_load_3d_pair(st + 8192, &p.tmA, bar, t.m0 + 64, ak, t.item);
+      if (li.mine()) tma_load_3d_pair(st, &p.tmA, bar, t.m0, ak, t.item);
+      if (li.mine()) tma_load_3d_pair(st + 8192, &p.tmA, bar, t.m0 + 64, ak, t.item);
     } else {
-      tma_load_3d_pair(st, &p.tmA, bar, ak, t.m0, t.item);
+      if (li.mine()) tma_load_3d_pair(st, &p.tmA, bar, ak, t.m0, t.item);
     }
     const CUtensorMap* mb = t.alt ? &p.tmB2 : &p.tmB;
     if (B_MN) {
 #pragma unroll
-      for (int b = 0; b < kHalfN / 64; ++b) tma_load_3d_pair(st + kABytes + b * 8192, mb, bar, n0 + b * 64, bk, t.zb);
+      for (int b = 0; b < kHalfN / 64; ++b)
+        if (li.mine()) tma_load_3d_pair(st + kABytes + b * 8192, mb, bar, n0 + b * 64, bk, t.zb);
     } else {
-      tma_load_3d_pair(st + kABytes, mb, bar, bk, n0, t.zb);
+      if (li.mine()) tma_load_3d_pair(st + kABytes, mb, bar, bk, n0, t.zb);
     }
   }
   __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {
@@ -277,9 +289,57 @@ struct GemmPairOp {
   }
   __device__ static void epilogue(const Params& p, const Tile& t, uint32_t tmem, int quarter, int lane,
                                   uint8_t* extra) {
-    Base::epilogue(p, t, tmem, quarter, lane, extra);
+    if (!p.out_tma) {
+      Base::epilogue(p, t, tmem, quarter, lane, extra);
+      return;
+    }
+    // The warp's 32 rows leave in 32-column pieces: TMEM -> registers ->
+    // a swizzled 4 KB staging tile -> one bulk tensor store, two tiles in
+    // flight per warp.  Row-per-thread global stores (one cache line per
+    // thread per instruction) took about 6 us per 128 x 256 fp32 tile.
+    const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool tr = p.tr_group >= 0 && (t.item / p.tr_mod) == p.tr_group;
+    uint8_t* stg = extra + quarter * kStgBytes;
+    const uint32_t sb = smem_u32(stg);
+    const int row0 = t.m0 + quarter * 32;
+#pragma unroll 1
+    for (int j = 0; j < BN; j += 32) {
+      const int slot = (j >> 5) & 1;
+      float v[32];
+      __syncwarp();
+      tmem_ld16(tq + j, v);
+      tmem_ld16(tq + j + 16, v + 16);
+      tmem_ld_wait();
+      if (lane == 0) bulk_wait_read_le1();  // the store that last used this slot has read it
+      __syncwarp();
+      const uint32_t tb = sb + slot * 4096;
+      if (!tr) {
+        // row `lane` (an output row), 16-byte chunk c at c ^ (lane % 8)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(tb + lane * 128 + ((c ^ (lane & 7)) << 4), __float_as_uint(v[4 * c]),
+                       __float_as_uint(v[4 * c + 1]), __float_as_uint(v[4 * c + 2]), __float_as_uint(v[4 * c + 3]));
+      } else {
+        // transposed: staging row i holds output column n0 + j + i, element
+        // `lane` of it this thread's row; 16-byte chunk lane / 4 at (lane / 4) ^ (i % 8)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          st_shared_f32(tb + i * 128 + (((lane >> 2) ^ (i & 7)) << 4) + (lane & 3) * 4, v[i]);
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (!tr)
+          tma_store_3d(&p.tmOut, stg + slot * 4096, t.n0 + j, row0, t.out_item);
+        else
+          tma_store_3d(&p.tmOutT, stg + slot * 4096, row0, t.n0 + j, t.out_item);
+        bulk_commit_group();
+      }
+    }
   }
-  __device__ static void epilogue_done(int) {}
+  __device__ static void epilogue_done(int lane) {
+    if (lane == 0) bulk_wait_all();
+  }
 };
 
 template <class Op>

@@ -102,6 +102,26 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Spreads the bulk tensor copies of one pipeline stage over the lanes of a
+// producer warp: the i-th copy of the stage is issued by lane i % 32.  One
+// thread's bulk copies complete roughly one at a time on B200 (about 0.6 us
+// each, nearly independent of their size up to 64 KB: one lane streams about
+// 26 GB/s in 16 KB boxes), while copies issued from different lanes overlap
+// (four lanes: about 90 GB/s per SM), so a stage of several copies is issued
+// by as many lanes.
+struct LaneIssue {
+  int lane;
+  int next;
+  __device__ __forceinline__ explicit LaneIssue(int l) : lane(l), next(0) {}
+  __device__ __forceinline__ bool mine() { return (next++ & 31) == lane; }
+  __device__ __forceinline__ void load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+    if (mine()) tma_load_3d(dst, map, bar, x, y, z);
+  }
+};
+
+// Broadcast of lane 0's value to the whole warp.
+__device__ __forceinline__ bool warp_bcast(bool v) { return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0; }
+
 // 3-D tiled store from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
   asm volatile(
@@ -118,12 +138,20 @@ __device__ __forceinline__ void bulk_commit_group() {
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// Wait until at most one committed bulk store still reads its shared-memory
+// source (a two-slot staging ring may rewrite the older slot).
+__device__ __forceinline__ void bulk_wait_read_le1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 // Wait until every committed bulk store has completed.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
@@ -151,6 +179,15 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// CTA-wide barrier for warp-specialized kernels.  Roles run by one lane (an
+// MMA issuer) bring the other 31 lanes of their warp to the barrier long
+// before that lane; the warp is reconverged first so that the aligned
+// barrier is reached by whole warps, as its definition requires.
+__device__ __forceinline__ void cta_sync_converged() {
+  __syncwarp();
+  __syncthreads();
 }
 
 // D[tmem] (+)= A[smem] * B[smem]; kind::f16 (bf16 in, fp32 accumulate).
