@@ -121,44 +121,31 @@ __global__ void __launch_bounds__(kApplyThreads, 1) k_apply(const __grid_constan
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // The whole warp: lane 0 waits for each slot and posts its bytes, the
-    // copies rotate over the lanes.
-    int ia = 0, ib = 0, tc = 0;
-    bool ok = true;
-    LaneIssue li(lane);
-    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
-      const int rt = tile % p.n_row_tiles, bh = tile / p.n_row_tiles;
-      const int row = p.q_row0 + rt * kBM;
-      if (lane == 0) {
-        if (tc > 0 && !mbar_wait(qempty, (tc - 1) & 1)) ok = false;
-        else mbar_arrive_expect_tx(qfull, C::kQBytes);
-      }
-      ok = warp_bcast(ok);
-      if (!ok) break;
-      for (int kb = 0; kb < C::kKb; ++kb) li.load_3d(smem + kb * 16384, &p.tmQ, qfull, kb * 64, row, bh);
-      for (int s = 0; ok && s < S; ++s) {
-        for (int kb = 0; kb < C::kKb; ++kb, ++ia) {
-          const int st = ia % C::kAStages;
-          if (lane == 0) {
-            if (ia >= C::kAStages && !mbar_wait(&aempty[st], ((ia / C::kAStages) - 1) & 1)) ok = false;
-            else mbar_arrive_expect_tx(&afull[st], C::kABytes);
+    if (lane == 0) {
+      int ia = 0, ib = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
+        const int rt = tile % p.n_row_tiles, bh = tile / p.n_row_tiles;
+        const int row = p.q_row0 + rt * kBM;
+        if (tc > 0 && !mbar_wait(qempty, (tc - 1) & 1)) break;
+        mbar_arrive_expect_tx(qfull, C::kQBytes);
+        for (int kb = 0; kb < C::kKb; ++kb) tma_load_3d(smem + kb * 16384, &p.tmQ, qfull, kb * 64, row, bh);
+        for (int s = 0; ok && s < S; ++s) {
+          for (int kb = 0; kb < C::kKb; ++kb, ++ia) {
+            const int st = ia % C::kAStages;
+            if (ia >= C::kAStages && !mbar_wait(&aempty[st], ((ia / C::kAStages) - 1) & 1)) { ok = false; break; }
+            uint8_t* dst = smem + C::kOffA + st * C::kABytes;
+            mbar_arrive_expect_tx(&afull[st], C::kABytes);
+            tma_load_3d(dst, &p.tmW, &afull[st], kb * 64, s * 64, bh);                       // W1_s
+            tma_load_3d(dst + 8192, &p.tmW, &afull[st], kb * 64, s * 64, 2 * p.bh_count + bh);  // W3_s
           }
-          ok = warp_bcast(ok);
           if (!ok) break;
-          uint8_t* dst = smem + C::kOffA + st * C::kABytes;
-          li.load_3d(dst, &p.tmW, &afull[st], kb * 64, s * 64, bh);                       // W1_s
-          li.load_3d(dst + 8192, &p.tmW, &afull[st], kb * 64, s * 64, 2 * p.bh_count + bh);  // W3_s
+          const int st = ib % C::kBStages;
+          if (ib >= C::kBStages && !mbar_wait(&bempty[st], ((ib / C::kBStages) - 1) & 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bfull[st], C::kBBytes);
+          tma_load_3d(smem + C::kOffB + st * C::kBBytes, &p.tmW2, &bfull[st], s * 64, 0, bh);   // W2[:, s]
+          ++ib;
         }
-        if (!ok) break;
-        const int st = ib % C::kBStages;
-        if (lane == 0) {
-          if (ib >= C::kBStages && !mbar_wait(&bempty[st], ((ib / C::kBStages) - 1) & 1)) ok = false;
-          else mbar_arrive_expect_tx(&bfull[st], C::kBBytes);
-        }
-        ok = warp_bcast(ok);
-        if (!ok) break;
-        li.load_3d(smem + C::kOffB + st * C::kBBytes, &p.tmW2, &bfull[st], s * 64, 0, bh);   // W2[:, s]
-        ++ib;
       }
     }
   } else if (warp == 1) {

@@ -76,14 +76,14 @@ struct BwdKeyOp {
     tma_prefetch_map(&p.tmBk);
     tma_prefetch_map(&p.tmBv);
   }
-  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar, LaneIssue& li) {
+  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
     const int k = kb * kBK, row = p.x_row0 + t.row0, hs = t.slice * 64;
-    li.load_3d(st, &p.tmX, bar, k, row, t.bh);
-    li.load_3d(st + kOffV, &p.tmV, bar, k, row, t.bh);
+    tma_load_3d(st, &p.tmX, bar, k, row, t.bh);
+    tma_load_3d(st + kOffV, &p.tmV, bar, k, row, t.bh);
 #pragma unroll
-    for (int g = 0; g < 4; ++g) li.load_3d(st + kOffBk + g * kSBytes, &p.tmBk, bar, k, g * p.dh + hs, t.bh);
-    li.load_3d(st + kOffBv, &p.tmBv, bar, hs, k, t.bh);
-    li.load_3d(st + kOffBv + kSBytes, &p.tmBv, bar, p.dh + hs, k, t.bh);
+    for (int g = 0; g < 4; ++g) tma_load_3d(st + kOffBk + g * kSBytes, &p.tmBk, bar, k, g * p.dh + hs, t.bh);
+    tma_load_3d(st + kOffBv, &p.tmBv, bar, hs, k, t.bh);
+    tma_load_3d(st + kOffBv + kSBytes, &p.tmBv, bar, p.dh + hs, k, t.bh);
   }
   __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb, int issuer) {
     const bool f = kb == 0;

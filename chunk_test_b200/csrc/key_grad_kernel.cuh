@@ -127,40 +127,31 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // The whole warp: lane 0 waits for each slot and posts its bytes, the
-    // copies rotate over the lanes.
-    int it = 0, ic = 0;
-    bool ok = true;
-    LaneIssue li(lane);
-    for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
-      int bh, s, t0, t1;
-      item_range(item, bh, s, t0, t1);
-      if (t0 >= t1) continue;
-      if (lane == 0) {
-        if (ic > 0 && !mbar_wait(wempty, (ic - 1) & 1)) ok = false;
-        else mbar_arrive_expect_tx(wfull, 49152);
-      }
-      ok = warp_bcast(ok);
-      if (!ok) break;
-      ++ic;
-      li.load_3d(smem + C::kOffW13, &p.tmW, wfull, 0, 0, bh);                          // W1 0-63
-      li.load_3d(smem + C::kOffW13 + 8192, &p.tmW, wfull, 0, 0, 2 * p.bh_count + bh);  // W3 0-63
-      li.load_3d(smem + C::kOffW13 + 16384, &p.tmW, wfull, 0, 64, bh);                 // W1 64-127
-      li.load_3d(smem + C::kOffW13 + 24576, &p.tmW, wfull, 0, 64, 2 * p.bh_count + bh);
-      li.load_3d(smem + C::kOffW2, &p.tmW2, wfull, 0, 0, bh);                          // W2[:, 0-63]
-      li.load_3d(smem + C::kOffW2 + 8192, &p.tmW2, wfull, 64, 0, bh);                  // W2[:, 64-127]
-      for (int t = t0; t < t1; ++t, ++it) {
-        const int slot = it & 1;
-        if (lane == 0) {
-          if (it >= 2 && !mbar_wait(&tempty[slot], ((it >> 1) - 1) & 1)) ok = false;
-          else mbar_arrive_expect_tx(&tfull[slot], C::kSlot);
+    if (lane == 0) {
+      int it = 0, ic = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        int bh, s, t0, t1;
+        item_range(item, bh, s, t0, t1);
+        if (t0 >= t1) continue;
+        if (ic > 0 && !mbar_wait(wempty, (ic - 1) & 1)) break;
+        ++ic;
+        mbar_arrive_expect_tx(wfull, 49152);
+        tma_load_3d(smem + C::kOffW13, &p.tmW, wfull, 0, 0, bh);                          // W1 0-63
+        tma_load_3d(smem + C::kOffW13 + 8192, &p.tmW, wfull, 0, 0, 2 * p.bh_count + bh);  // W3 0-63
+        tma_load_3d(smem + C::kOffW13 + 16384, &p.tmW, wfull, 0, 64, bh);                 // W1 64-127
+        tma_load_3d(smem + C::kOffW13 + 24576, &p.tmW, wfull, 0, 64, 2 * p.bh_count + bh);
+        tma_load_3d(smem + C::kOffW2, &p.tmW2, wfull, 0, 0, bh);                          // W2[:, 0-63]
+        tma_load_3d(smem + C::kOffW2 + 8192, &p.tmW2, wfull, 64, 0, bh);                  // W2[:, 64-127]
+        for (int t = t0; t < t1; ++t, ++it) {
+          const int slot = it & 1;
+          if (it >= 2 && !mbar_wait(&tempty[slot], ((it >> 1) - 1) & 1)) { ok = false; break; }
+          uint8_t* dst = smem + C::kOffRing + slot * C::kSlot;
+          const int row = p.x_row0 + t * kBM;
+          mbar_arrive_expect_tx(&tfull[slot], C::kSlot);
+          tma_load_3d(dst, &p.tmK, &tfull[slot], 0, row, bh);
+          tma_load_3d(dst + 16384, &p.tmV, &tfull[slot], 0, row, bh);
         }
-        ok = warp_bcast(ok);
-        if (!ok) break;
-        uint8_t* dst = smem + C::kOffRing + slot * C::kSlot;
-        const int row = p.x_row0 + t * kBM;
-        li.load_3d(dst, &p.tmK, &tfull[slot], 0, row, bh);
-        li.load_3d(dst + 16384, &p.tmV, &tfull[slot], 0, row, bh);
       }
     }
   } else if (warp >= 2) {

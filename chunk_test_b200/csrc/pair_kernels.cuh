@@ -157,31 +157,24 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
   griddep_wait();  // after the local setup, before any global access
 
   if (warp == 0) {
-    // The whole warp produces: lane 0 waits for the slot (and, in the even
-    // CTA, posts the stage's bytes of both CTAs), then the copies are spread
-    // over the lanes.
-    int it = 0;
-    bool ok = true;
-    LaneIssue li(lane);   // one running count: successive copies rotate over the lanes
-    for (int tile = pair; ok && tile < ntiles; tile += npairs) {
-      const typename Op::Tile t = Op::map_tile(p, tile, rank);
-      const int nkb = Op::num_kb(p, t);
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % S;
-        if (lane == 0) {
-          if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) ok = false;
-          else if (leader) mbar_arrive_expect_tx(&full[s], 2u * Op::kStageBytes);
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < ntiles; tile += npairs) {
+        const typename Op::Tile t = Op::map_tile(p, tile, rank);
+        const int nkb = Op::num_kb(p, t);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % S;
+          if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full[s], 2u * Op::kStageBytes);
+          Op::load(p, t, kb, smem + s * Op::kStageBytes, mapa_rank(smem_u32(&full[s]), 0));
         }
-        ok = warp_bcast(ok);
-        if (!ok) break;
-        Op::load(p, t, kb, smem + s * Op::kStageBytes, mapa_rank(smem_u32(&full[s]), 0), li);
       }
-    }
-    // Every stage release (including the last S, committed by the even
-    // CTA's MMAs) has landed before this CTA may leave.
-    if (lane == 0)
+      // Every stage release (including the last S, committed by the even
+      // CTA's MMAs) has landed before this CTA may leave.
       for (int i = it > S ? it - S : 0; ok && i < it; ++i)
         if (!mbar_wait(&empty[i % S], (i / S) & 1)) ok = false;
+    }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       int it = 0, local = 0;
@@ -263,24 +256,23 @@ struct GemmPairOp {
     tma_prefetch_map(&p.tmB);
     if (p.alt_group >= 0) tma_prefetch_map(&p.tmB2);
   }
-  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint32_t bar, LaneIssue& li) {
+  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint32_t bar) {
     const int kk = (t.split * p.kb_count + kb) * kBK;
     const int ak = p.a_k0 + kk, bk = p.b_k0 + kk;
     const int half = (t.m0 / kBM) & 1;  // this CTA's rank in the pair
     const int n0 = t.n0 + half * kHalfN;
     if (A_MN) {
-      if (li.mine()) tma_load_3d_pair(st, &p.tmA, bar, t.m0, ak, t.item);
-      if (li.mine()) tma_load_3d_pair(st + 8192, &p.tmA, bar, t.m0 + 64, ak, t.item);
+      tma_load_3d_pair(st, &p.tmA, bar, t.m0, ak, t.item);
+      tma_load_3d_pair(st + 8192, &p.tmA, bar, t.m0 + 64, ak, t.item);
     } else {
-      if (li.mine()) tma_load_3d_pair(st, &p.tmA, bar, ak, t.m0, t.item);
+      tma_load_3d_pair(st, &p.tmA, bar, ak, t.m0, t.item);
     }
     const CUtensorMap* mb = t.alt ? &p.tmB2 : &p.tmB;
     if (B_MN) {
 #pragma unroll
-      for (int b = 0; b < kHalfN / 64; ++b)
-        if (li.mine()) tma_load_3d_pair(st + kABytes + b * 8192, mb, bar, n0 + b * 64, bk, t.zb);
+      for (int b = 0; b < kHalfN / 64; ++b) tma_load_3d_pair(st + kABytes + b * 8192, mb, bar, n0 + b * 64, bk, t.zb);
     } else {
-      if (li.mine()) tma_load_3d_pair(st + kABytes, mb, bar, bk, n0, t.zb);
+      tma_load_3d_pair(st + kABytes, mb, bar, bk, n0, t.zb);
     }
   }
   __device__ static void mma(const Params&, const Tile&, uint32_t st, uint32_t tmem, int kb) {

@@ -102,26 +102,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Spreads the bulk tensor copies of one pipeline stage over the lanes of a
-// producer warp: the i-th copy of the stage is issued by lane i % 32.  One
-// thread's bulk copies complete roughly one at a time on B200 (about 0.6 us
-// each, nearly independent of their size up to 64 KB: one lane streams about
-// 26 GB/s in 16 KB boxes), while copies issued from different lanes overlap
-// (four lanes: about 90 GB/s per SM), so a stage of several copies is issued
-// by as many lanes.
-struct LaneIssue {
-  int lane;
-  int next;
-  __device__ __forceinline__ explicit LaneIssue(int l) : lane(l), next(0) {}
-  __device__ __forceinline__ bool mine() { return (next++ & 31) == lane; }
-  __device__ __forceinline__ void load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
-    if (mine()) tma_load_3d(dst, map, bar, x, y, z);
-  }
-};
-
-// Broadcast of lane 0's value to the whole warp.
-__device__ __forceinline__ bool warp_bcast(bool v) { return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0; }
-
 // 3-D tiled store from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
   asm volatile(

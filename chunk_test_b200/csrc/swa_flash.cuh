@@ -155,55 +155,43 @@ __global__ void __launch_bounds__(kSwaThreads, 1) k_swa_flash(const __grid_const
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // The whole warp: lane 0 waits for each slot and posts its bytes, the
-    // copies rotate over the lanes.
-    int ik = 0, tc = 0;
-    bool ok = true;
-    LaneIssue li(lane);
-    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
-      const int m = tile % p.nb, bh = tile / p.nb;
-      if (lane == 0) {
-        if (tc > 0 && !mbar_wait(qempty, (tc - 1) & 1)) ok = false;
-        else mbar_arrive_expect_tx(qfull, C::kQBytes);
-      }
-      ok = warp_bcast(ok);
-      if (!ok) break;
-      for (int kb = 0; kb < C::kKb; ++kb) li.load_3d(smem + kb * 16384, &p.tmQ, qfull, kb * 64, m * 128, bh);
-      const int j0 = m - wb > 0 ? m - wb : 0;
-      for (int j = j0; j <= m; ++j, ++ik) {
-        const int st = ik % KS;
-        const int prow = j * 128;   // first key of block j
-        if (lane == 0) {
-          if (ik >= KS && !mbar_wait(&kempty[st], ((ik / KS) - 1) & 1)) ok = false;
-          else mbar_arrive_expect_tx(&kfull[st], C::kKBytes);
+    if (lane == 0) {
+      int ik = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
+        const int m = tile % p.nb, bh = tile / p.nb;
+        if (tc > 0 && !mbar_wait(qempty, (tc - 1) & 1)) break;
+        mbar_arrive_expect_tx(qfull, C::kQBytes);
+        for (int kb = 0; kb < C::kKb; ++kb) tma_load_3d(smem + kb * 16384, &p.tmQ, qfull, kb * 64, m * 128, bh);
+        const int j0 = m - wb > 0 ? m - wb : 0;
+        for (int j = j0; j <= m; ++j, ++ik) {
+          const int st = ik % KS;
+          const int prow = j * 128;   // first key of block j
+          if (ik >= KS && !mbar_wait(&kempty[st], ((ik / KS) - 1) & 1)) { ok = false; break; }
+          uint8_t* kd = smem + C::kOffK + st * C::kKBytes;
+          mbar_arrive_expect_tx(&kfull[st], C::kKBytes);
+          for (int kb = 0; kb < C::kKb; ++kb) tma_load_3d(kd + kb * 16384, &p.tmK, &kfull[st], kb * 64, prow, bh);
         }
-        ok = warp_bcast(ok);
-        if (!ok) break;
-        uint8_t* kd = smem + C::kOffK + st * C::kKBytes;
-        for (int kb = 0; kb < C::kKb; ++kb) li.load_3d(kd + kb * 16384, &p.tmK, &kfull[st], kb * 64, prow, bh);
       }
     }
   } else if (warp == kSwaVWarp) {
     // ------------------------------------------------------------ V producer
-    int ik = 0;
-    bool ok = true;
-    LaneIssue li(lane);
-    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-      const int m = tile % p.nb, bh = tile / p.nb;
-      const int j0 = m - wb > 0 ? m - wb : 0;
-      for (int j = j0; ok && j <= m; ++j, ++ik) {
-        const int st = ik % KS;
-        uint8_t* vd = smem + C::kOffV + st * C::kVBytes;
-        for (int h = 0; h < 2; ++h) {
-          uint64_t* full = &vfull[2 * st + h];
-          if (lane == 0) {
-            if (ik >= KS && !mbar_wait(&vempty[2 * st + h], ((ik / KS) - 1) & 1)) ok = false;
-            else mbar_arrive_expect_tx(full, C::kVBytes / 2);
+    if (lane == 0) {
+      int ik = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        const int m = tile % p.nb, bh = tile / p.nb;
+        const int j0 = m - wb > 0 ? m - wb : 0;
+        for (int j = j0; ok && j <= m; ++j, ++ik) {
+          const int st = ik % KS;
+          uint8_t* vd = smem + C::kOffV + st * C::kVBytes;
+          for (int h = 0; h < 2; ++h) {
+            uint64_t* full = &vfull[2 * st + h];
+            if (ik >= KS && !mbar_wait(&vempty[2 * st + h], ((ik / KS) - 1) & 1)) { ok = false; break; }
+            mbar_arrive_expect_tx(full, C::kVBytes / 2);
+            for (int nb = 0; nb < C::kKb; ++nb)
+              tma_load_3d(vd + (h * C::kKb + nb) * 8192, &p.tmV, full, nb * 64, j * 128 + h * 64, bh);
           }
-          ok = warp_bcast(ok);
-          if (!ok) break;
-          for (int nb = 0; nb < C::kKb; ++nb)
-            li.load_3d(vd + (h * C::kKb + nb) * 8192, &p.tmV, full, nb * 64, j * 128 + h * 64, bh);
         }
       }
     }

@@ -112,23 +112,18 @@ __global__ void __launch_bounds__(umma_threads<Op>(), 1)
   griddep_wait();  // after the local setup, before any global access
 
   if (warp == 0) {
-    // The whole warp produces: lane 0 waits for the slot and posts the
-    // stage's bytes, then the stage's copies are spread over the lanes.
-    int it = 0;
-    bool ok = true;
-    LaneIssue li(lane);   // one running count: successive copies rotate over the lanes
-    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-      const typename Op::Tile t = Op::map_tile(p, tile);
-      const int nkb = Op::num_kb(p, t);
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % S;
-        if (lane == 0) {
-          if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) ok = false;
-          else mbar_arrive_expect_tx(&full[s], Op::stage_bytes(p, t));
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        const typename Op::Tile t = Op::map_tile(p, tile);
+        const int nkb = Op::num_kb(p, t);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % S;
+          if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], Op::stage_bytes(p, t));
+          Op::load(p, t, kb, smem + s * Op::kStageBytes, &full[s]);
         }
-        ok = warp_bcast(ok);
-        if (!ok) break;
-        Op::load(p, t, kb, smem + s * Op::kStageBytes, &full[s], li);
       }
     }
   } else if (warp == 1 || (Op::kIssuers == 2 && warp == kIssuer2Warp)) {
@@ -369,23 +364,23 @@ struct FwdOp {
       tma_prefetch_map(&p.tmW2lo);
     }
   }
-  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar, LaneIssue& li) {
+  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
     const int k = kb * kBK, row = p.x_row0 + t.row0, hs = t.slice * NSL;
     const int z1 = t.bh, z3 = 2 * p.bh_count + t.bh;
-    li.load_3d(st, &p.tmX, bar, k, row, t.bh);
-    li.load_3d(st + kOffW, &p.tmW, bar, k, hs, z1);                 // W1 rows of the slice
-    li.load_3d(st + kOffW + kWBytes, &p.tmW, bar, k, hs, z3);       // W3 rows of the slice
+    tma_load_3d(st, &p.tmX, bar, k, row, t.bh);
+    tma_load_3d(st + kOffW, &p.tmW, bar, k, hs, z1);                 // W1 rows of the slice
+    tma_load_3d(st + kOffW + kWBytes, &p.tmW, bar, k, hs, z3);       // W3 rows of the slice
     if (SPLIT) {
-      li.load_3d(st + kOffXlo, &p.tmXlo, bar, k, row, t.bh);
-      li.load_3d(st + kOffWlo, &p.tmWlo, bar, k, hs, z1);
-      li.load_3d(st + kOffWlo + kWBytes, &p.tmWlo, bar, k, hs, z3);
+      tma_load_3d(st + kOffXlo, &p.tmXlo, bar, k, row, t.bh);
+      tma_load_3d(st + kOffWlo, &p.tmWlo, bar, k, hs, z1);
+      tma_load_3d(st + kOffWlo + kWBytes, &p.tmWlo, bar, k, hs, z3);
     }
     if (KMODE) {
-      li.load_3d(st + kOffV, &p.tmV, bar, k, row, t.bh);
+      tma_load_3d(st + kOffV, &p.tmV, bar, k, row, t.bh);
 #pragma unroll
       for (int b = 0; b < NSL / 64; ++b) {                           // W2[k.., hs..]: MN blocks of 64
-        li.load_3d(st + kOffW2 + b * 8192, &p.tmW2, bar, hs + 64 * b, k, t.bh);
-        if (SPLIT) li.load_3d(st + kOffW2 + kWBytes + b * 8192, &p.tmW2lo, bar, hs + 64 * b, k, t.bh);
+        tma_load_3d(st + kOffW2 + b * 8192, &p.tmW2, bar, hs + 64 * b, k, t.bh);
+        if (SPLIT) tma_load_3d(st + kOffW2 + kWBytes + b * 8192, &p.tmW2lo, bar, hs + 64 * b, k, t.bh);
       }
     }
   }
@@ -597,33 +592,31 @@ struct GemmOp {
       tma_prefetch_map(&p.tmBlo);
     }
   }
-  __device__ static void load_a(const CUtensorMap* m, uint8_t* dst, uint64_t* bar, int m0, int ak, int z,
-                                 LaneIssue& li) {
+  __device__ static void load_a(const CUtensorMap* m, uint8_t* dst, uint64_t* bar, int m0, int ak, int z) {
     if (A_MN) {
-      li.load_3d(dst, m, bar, m0, ak, z);
-      li.load_3d(dst + 8192, m, bar, m0 + 64, ak, z);
+      tma_load_3d(dst, m, bar, m0, ak, z);
+      tma_load_3d(dst + 8192, m, bar, m0 + 64, ak, z);
     } else {
-      li.load_3d(dst, m, bar, ak, m0, z);
+      tma_load_3d(dst, m, bar, ak, m0, z);
     }
   }
-  __device__ static void load_b(const CUtensorMap* m, uint8_t* dst, uint64_t* bar, int n0, int bk, int z,
-                                 LaneIssue& li) {
+  __device__ static void load_b(const CUtensorMap* m, uint8_t* dst, uint64_t* bar, int n0, int bk, int z) {
     if (B_MN) {
 #pragma unroll
-      for (int b = 0; b < BN / 64; ++b) li.load_3d(dst + b * 8192, m, bar, n0 + b * 64, bk, z);
+      for (int b = 0; b < BN / 64; ++b) tma_load_3d(dst + b * 8192, m, bar, n0 + b * 64, bk, z);
     } else {
-      li.load_3d(dst, m, bar, bk, n0, z);
+      tma_load_3d(dst, m, bar, bk, n0, z);
     }
   }
-  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar, LaneIssue& li) {
+  __device__ static void load(const Params& p, const Tile& t, int kb, uint8_t* st, uint64_t* bar) {
     const int kk = (t.split * p.kb_count + kb) * kBK;
     const int ak = p.a_k0 + kk, bk = p.b_k0 + kk;
     const int am = t.m0 + p.a_m0;
-    load_a(&p.tmA, st, bar, am, ak, t.item, li);
-    load_b(t.alt ? &p.tmB2 : &p.tmB, st + kOffB, bar, t.n0, bk, t.zb, li);
+    load_a(&p.tmA, st, bar, am, ak, t.item);
+    load_b(t.alt ? &p.tmB2 : &p.tmB, st + kOffB, bar, t.n0, bk, t.zb);
     if (SPLIT) {
-      load_a(&p.tmAlo, st + kABytes, bar, am, ak, t.item, li);
-      if (!t.alt) load_b(&p.tmBlo, st + kOffB + kBBytes, bar, t.n0, bk, t.zb, li);
+      load_a(&p.tmAlo, st + kABytes, bar, am, ak, t.item);
+      if (!t.alt) load_b(&p.tmBlo, st + kOffB + kBBytes, bar, t.n0, bk, t.zb);
     }
   }
   __device__ static void mma(const Params&, const Tile& t, uint32_t st, uint32_t tmem, int kb, int) {
