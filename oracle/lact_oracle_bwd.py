@@ -11,9 +11,10 @@ torch.autograd, a library routine, as one step.  The pins check this forward
 against the numpy oracle and the gradients against central finite
 differences.
 
-Covered: the GD and momentum rules, both orders, the per-chunk update mask,
-the output scale, shared or per-(b, h) initial weights.  The Muon rule's
-backward (through the Newton-Schulz iteration) is not covered.
+Covered: the GD, momentum and Muon rules (the Muon backward runs through
+the Frobenius normalisation and the five Newton-Schulz steps), both orders,
+the per-chunk update mask, the output scale, shared or per-(b, h) initial
+weights.
 """
 from __future__ import annotations
 
@@ -21,7 +22,12 @@ import numpy as np
 import torch
 
 APPLY_THEN_UPDATE, UPDATE_THEN_APPLY = 0, 1
-RULE_GD, RULE_MOMENTUM = 0, 1
+RULE_GD, RULE_MOMENTUM, RULE_MUON = 0, 1, 2
+
+# Newton-Schulz quintic of the Muon rule (R7): coefficients, steps, eps.
+NS_COEFFS = (3.4445, -4.7750, 2.0315)
+NS_STEPS = 5
+NS_EPS = 1e-7
 
 
 def _t(x):
@@ -63,6 +69,22 @@ def _chunk_grads(W1, W2, W3, K, V, lr):
     return G1, G2, G3
 
 
+def _newton_schulz5(G):
+    """Muon's orthogonalised update of a gradient matrix [P2 §2.2.1]
+    eqs. 9-10: X = G / (||G||_F + eps), then five times
+    X <- a X + (b A + c A A) X with A = X X^T, X oriented so that A is the
+    smaller Gram matrix (the same result in exact arithmetic either way)."""
+    a, b, c = NS_COEFFS
+    X = G / (G.norm() + NS_EPS)
+    transposed = X.shape[0] > X.shape[1]
+    if transposed:
+        X = X.T
+    for _ in range(NS_STEPS):
+        A = X @ X.T
+        X = a * X + (b * A + c * (A @ A)) @ X
+    return X.T if transposed else X
+
+
 def _renorm(W_new, W_old):
     """Each row of W_new scaled to the norm its row had before (R4, R5)."""
     return W_new * (W_old.norm(dim=1, keepdim=True) / W_new.norm(dim=1, keepdim=True))
@@ -92,8 +114,10 @@ def head_forward(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule, update_mask=
                 U = M
             elif rule == RULE_GD:
                 U = G
+            elif rule == RULE_MUON:
+                U = tuple(_newton_schulz5(g) for g in G)
             else:
-                raise ValueError("the backward oracle covers GD and momentum")
+                raise ValueError(f"unknown rule {rule}")
             W = tuple(_renorm(w - u, w) for w, u in zip(W, U))
         if order == UPDATE_THEN_APPLY:
             outs.append(_fast_net(*W, qh[rows]))

@@ -9,7 +9,7 @@ import pytest
 
 import oracle
 from oracle import lact_oracle_bwd as ob
-from oracle import APPLY_THEN_UPDATE, UPDATE_THEN_APPLY, RULE_GD, RULE_MOMENTUM
+from oracle import APPLY_THEN_UPDATE, UPDATE_THEN_APPLY, RULE_GD, RULE_MOMENTUM, RULE_MUON
 
 RNG = np.random.default_rng(99)
 
@@ -39,6 +39,8 @@ CASES = [
     (APPLY_THEN_UPDATE, RULE_MOMENTUM, None, False),
     (UPDATE_THEN_APPLY, RULE_MOMENTUM, [1, 0, 1, 1], False),
     (APPLY_THEN_UPDATE, RULE_MOMENTUM, [0, 1, 1, 0], True),
+    (APPLY_THEN_UPDATE, RULE_MUON, None, False),
+    (UPDATE_THEN_APPLY, RULE_MUON, [1, 1, 0, 1], True),
 ]
 
 
@@ -69,13 +71,22 @@ def test_gradients_match_central_differences(order, rule, mask, scaled):
                          out_scale=scale)
     names = ["q", "k", "v", "lr", "w1", "w2", "w3"] + (["beta"] if rule == RULE_MOMENTUM else [])
     eps = 1e-6
+
+    def loss_at(delta, t):
+        return _numpy_loss(dict(p, **{n: p[n] + t * delta[n] for n in names}), 3, order, rule, dout, dw,
+                           mask, scale)
+
     for only in names + [None]:
         delta = {n: (RNG.standard_normal(p[n].shape) if (only is None or n == only) else 0 * p[n])
                  for n in names}
-        plus = dict(p, **{n: p[n] + eps * delta[n] for n in names})
-        minus = dict(p, **{n: p[n] - eps * delta[n] for n in names})
-        fd = (_numpy_loss(plus, 3, order, rule, dout, dw, mask, scale)
-              - _numpy_loss(minus, 3, order, rule, dout, dw, mask, scale)) / (2 * eps)
+        if rule == RULE_MUON:
+            # five Newton-Schulz quintic steps compose to a polynomial of very
+            # high degree: the fourth-order stencil keeps the truncation error
+            # below the tolerance (the second-order one misses by ~1e-6)
+            fd = (-loss_at(delta, 2 * eps) + 8 * loss_at(delta, eps) - 8 * loss_at(delta, -eps)
+                  + loss_at(delta, -2 * eps)) / (12 * eps)
+        else:
+            fd = (loss_at(delta, eps) - loss_at(delta, -eps)) / (2 * eps)
         an = sum((g["d" + n] * delta[n]).sum() for n in names)
         assert an == pytest.approx(fd, rel=1e-6, abs=1e-8), (only, an, fd)
     if scaled:
@@ -95,3 +106,20 @@ def test_without_updates_only_the_apply_has_gradients():
     for n in ("dk", "dv", "dlr", "dbeta"):
         assert np.all(g[n] == 0), n
     assert np.any(g["dq"] != 0) and np.any(g["dw2"] != 0)
+
+
+def test_muon_with_zero_rates_has_no_path_through_the_update():
+    """lr = 0: every chunk gradient is zero, the Frobenius normalisation maps
+    it to zero (R7's eps) and no state moves, so out = f_{W0}(q^): the rates
+    still get a gradient (the Newton-Schulz map's derivative at zero is
+    1 / eps times the identity) while k and v get none through the apply."""
+    p = _problem(T=9)
+    p["lr"] = np.zeros_like(p["lr"])
+    dout = RNG.standard_normal(p["q"].shape)
+    g = ob.ttt_layer_bwd(**p, chunk=3, order=APPLY_THEN_UPDATE, rule=RULE_MUON, dout=dout)
+    want = oracle.ttt_layer_ex(p["q"], p["k"], p["v"], p["lr"], p["beta"], p["w1"], p["w2"], p["w3"],
+                               3, APPLY_THEN_UPDATE, RULE_MUON)
+    np.testing.assert_allclose(g["out"], want[0], rtol=1e-12, atol=1e-13)
+    for a, b in zip((g["w1o"], g["w2o"], g["w3o"]), (p["w1"], p["w2"], p["w3"])):
+        np.testing.assert_allclose(a, np.concatenate([b]), rtol=1e-12, atol=1e-13)
+    assert np.all(np.isfinite(g["dlr"])) and np.any(g["dlr"] != 0)
