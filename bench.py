@@ -525,14 +525,28 @@ def main():
 FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def bwd_flops(w: Workload) -> float:
-    """Algorithmic FLOPs of lact_ttt_bwd, all in its contractions: per key
+def bwd_flops(w: Workload) -> dict:
+    """Algorithmic FLOPs of lact_ttt_bwd by where they run.  "layer": per key
     token per head 12 d dh to recompute the forward's updates (keys' forward
     6, gradient 6) and 30 d dh in the reverse loop (keys' forward again 6,
     (p, q, r) 6, the weight gradients 6, dk 8, dv 4); per query token per head
     16 d dh for the apply's backward (its forward 6, the weight gradients 6,
-    dq 4)."""
-    return w.B * w.H * w.d * w.dh * (42.0 * w.T + 16.0 * w.Tq)
+    dq 4).  "ns" (Muon only, fp32 on the CUDA cores): per chunk and matrix,
+    with m = max(d, dh), n = min(d, dh), two passes of the five Newton-Schulz
+    steps (4 m n^2 + 2 n^3 each: the Gram, its square, the update) and one
+    pass of their vector-Jacobian product (6 m n^2 + 4 n^3 each)."""
+    layer = w.B * w.H * w.d * w.dh * (42.0 * w.T + 16.0 * w.Tq)
+    ns = 0.0
+    if w.rule == RULE_MUON:
+        m, n = max(w.d, w.dh), min(w.d, w.dh)
+        ns = w.B * w.H * 3 * w.n_chunks * 5 * (14.0 * m * n * n + 8.0 * n ** 3)
+    return {"layer": layer, "ns": ns}
+
+
+def bwd_on_tc(w: Workload) -> bool:
+    """Whether lact_ttt_bwd runs the layer's contractions on the tensor cores:
+    bf16 GD and momentum problems; Muon ones run in fp32 on the CUDA cores."""
+    return w.dtype == BF16 and w.rule != RULE_MUON
 
 
 def run_backward(args, w: Workload):
@@ -541,8 +555,6 @@ def run_backward(args, w: Workload):
     world, rank, local = dist_env()
     if world > 1:
         raise SystemExit("--pass bwd runs on one GPU")
-    if w.rule == RULE_MUON:
-        raise SystemExit("the backward covers GD and momentum")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     inp_cpu = make_inputs(w, seed=0)
@@ -583,11 +595,17 @@ def run_backward(args, w: Workload):
     ct.profile_enable(False)
     launches_per_step = sum(v[0] for v in prof.values()) // args.steps
     dom_name, (n_launch, ms_kind) = max(prof.items(), key=lambda kv: kv[1][1])
-    flops = bwd_flops(w)
+    fl = bwd_flops(w)
     roof = None
     _, pk_burst, pk_sust, pk_src = peaks()
     if dom_name in ("simt_gemm_f32", "bwd_gemm_umma"):
-        # every FLOP of bwd_flops() is in these contractions
+        # the layer's contractions run in bwd_gemm_umma on bf16 GD / momentum
+        # workloads and in simt_gemm_f32 otherwise (fp32, and every Muon
+        # workload); the Newton-Schulz ones in simt_gemm_f32
+        if dom_name == "bwd_gemm_umma":
+            flops = fl["layer"]
+        else:
+            flops = fl["ns"] + (0.0 if bwd_on_tc(w) else fl["layer"])
         achieved = flops * args.steps / (ms_kind / 1e3) / 1e12
         tensor = dom_name == "bwd_gemm_umma"
         peak = pk_burst if tensor else FP32_FMA_TFLOPS
@@ -632,18 +650,18 @@ def run_backward(args, w: Workload):
     h2d = sum(t.numel() * t.element_size() for t in pin.values() if t is not None) + \
         pdout.numel() * pdout.element_size()
     d2h = sum(t.numel() * t.element_size() for t in hgrad.values() if t is not None)
-    tok = w.tokens
+    tok, total = w.tokens, fl["layer"] + fl["ns"]
     line = {
         "metric": "TTT-layer backward tokens/s at 1 B200", "value": tok / (ms_step / 1e3),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == BF16 else "f32",
+        "dtype": "bf16" if bwd_on_tc(w) else "f32",
         "data": "synthetic (seeded normal q/k/v/dout, softplus lr, random-init fast weights)",
         "config": dict(workload_config(w, 1), **{"pass": "backward (lact_ttt_bwd)"}),
-        "peak_frac": {"algorithmic_tflops": flops / (ms_step / 1e3) / 1e12,
-                      "frac_of_burst_bf16": flops / (ms_step / 1e3) / 1e12 / pk_burst,
-                      "frac_of_sustained_bf16": flops / (ms_step / 1e3) / 1e12 / pk_sust,
-                      "frac_of_fp32_fma": flops / (ms_step / 1e3) / 1e12 / FP32_FMA_TFLOPS},
+        "peak_frac": {"algorithmic_tflops": total / (ms_step / 1e3) / 1e12,
+                      "frac_of_burst_bf16": total / (ms_step / 1e3) / 1e12 / pk_burst,
+                      "frac_of_sustained_bf16": total / (ms_step / 1e3) / 1e12 / pk_sust,
+                      "frac_of_fp32_fma": total / (ms_step / 1e3) / 1e12 / FP32_FMA_TFLOPS},
         "roofline": roof,
         "kernels": kernels,
         "gpu_launches": launches_per_step * args.steps,

@@ -371,4 +371,85 @@ __global__ void __launch_bounds__(256) k_sum_batch(const float* __restrict__ A, 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Muon rule backward: the vector-Jacobian product of
+//   U = NS5(S / (||S||_F + eps))     ("大块测试时训练（LaCT）技术解析" §2.2.1,
+//                                     eqs. 9-10; five steps of
+//   X <- a X + X (b A + c A A),  A = X^T X)
+// runs as fp32 batched GEMMs (k_simt_gemm) over the kept iterates; these
+// kernels are its elementwise and layout steps.
+// ---------------------------------------------------------------------------
+
+// out[p][c][r] = in[p][r][c] for `nplanes` planes of rows x cols (32 x 32
+// tiles through shared memory).  grid (cdiv(cols, 32), cdiv(rows, 32),
+// nplanes), block (32, 8).
+__global__ void __launch_bounds__(256) k_transpose_planes(const float* __restrict__ in, float* __restrict__ out,
+                                                          int rows, int cols) {
+  griddep_launch();
+  griddep_wait();
+  __shared__ float tile[32][33];
+  const int64_t base = static_cast<int64_t>(blockIdx.z) * rows * cols;
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = in[base + static_cast<int64_t>(r) * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) out[base + static_cast<int64_t>(c) * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+// M <- M + M^T for `items` n x n matrices, in place: one thread per pair
+// (i <= j).
+__global__ void __launch_bounds__(256) k_sym_add(float* __restrict__ M, int n, int64_t items) {
+  griddep_launch();
+  griddep_wait();
+  const int64_t per = static_cast<int64_t>(n) * n;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < items * per; t += stride) {
+    const int64_t item = t / per, e = t % per;
+    const int i = static_cast<int>(e / n), j = static_cast<int>(e % n);
+    if (i > j) continue;
+    float* m = M + item * per;
+    const float s = m[static_cast<int64_t>(i) * n + j] + m[static_cast<int64_t>(j) * n + i];
+    m[static_cast<int64_t>(i) * n + j] = s;
+    m[static_cast<int64_t>(j) * n + i] = s;
+  }
+}
+
+// The normalisation's VJP, one block per matrix: with n = ||S||_F (from the
+// forward's fixed-order partial sums of squares, `part`) and Y0 = dL/dX0,
+//   dL/dS = Y0 / (n + eps) - <Y0, S> / (n (n + eps)^2) S     (n > 0)
+//   dL/dS = Y0 / eps                                         (S = 0)
+__global__ void __launch_bounds__(1024) k_ns_norm_vjp(const float* __restrict__ S, const float* __restrict__ Y0,
+                                                     const float* __restrict__ part, int nblk, float eps,
+                                                     int64_t plane, float* __restrict__ out) {
+  griddep_launch();
+  griddep_wait();
+  __shared__ float red[32];
+  __shared__ float coef[2];
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * plane;
+  float dot = 0.f;
+  for (int64_t e = threadIdx.x; e < plane; e += blockDim.x) dot = fmaf(Y0[base + e], S[base + e], dot);
+  dot = warp_sum(dot);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dot;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) {
+      float ss = 0.f;
+      for (int i = 0; i < nblk; ++i) ss += part[static_cast<int64_t>(blockIdx.x) * nblk + i];
+      const float nrm = sqrtf(ss), den = nrm + eps;
+      coef[0] = 1.0f / den;
+      coef[1] = nrm > 0.f ? v / (nrm * den * den) : 0.f;
+    }
+  }
+  __syncthreads();
+  const float c0 = coef[0], c1 = coef[1];
+  for (int64_t e = threadIdx.x; e < plane; e += blockDim.x) out[base + e] = c0 * Y0[base + e] - c1 * S[base + e];
+}
+
 }  // namespace lact

@@ -1264,7 +1264,7 @@ int lact_ttt_fwd_host(const lact_problem* p, const void* q, const void* k, const
 
 size_t lact_ttt_bwd_workspace_bytes(const lact_problem* p) {
   Dims D;
-  if (validate(p, D) != LACT_OK || D.rule == LACT_RULE_MUON) return 0;
+  if (validate(p, D) != LACT_OK) return 0;
   return bwd_workspace_bytes(D);
 }
 
@@ -1277,7 +1277,6 @@ int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts, const void* q
   Dims D;
   int rc = validate(p, D);
   if (rc != LACT_OK) return rc;
-  if (D.rule == LACT_RULE_MUON) return LACT_EINVAL;
   if (opts && (opts->m1 || opts->m2 || opts->m3 || opts->allreduce)) return LACT_EINVAL;
   const float* scale = opts ? opts->out_scale : nullptr;
   const bool mom = D.rule == LACT_RULE_MOMENTUM;

@@ -13,6 +13,18 @@
 //      contractions;
 //   3. the prologue's backward gives dq and dk; the initial weights'
 //      gradient is summed over the batch when the batch shares it.
+// Muon: the recompute keeps each chunk's update direction S (its negated
+// gradient, all three planes as [dh, d]); the reverse loop takes the renorm
+// backward's gradient with respect to the update, re-runs the five
+// Newton-Schulz steps on S keeping their iterates, and walks their
+// vector-Jacobian product back to S (ns_keep, ns_vjp), in fp32 on the CUDA
+// cores.  bf16 Muon problems take the fp32 path whole, on fp32 copies of
+// their inputs: the iteration's Jacobian magnifies operand rounding (rounding
+// only the chunk gradient to bf16 moves the exact backward by a few percent),
+// so bf16 operands would not hold the bf16 tolerance.  The rule kernel applies the orthogonalised
+// direction as GD applies S, so the renorm backward's GD output is the
+// gradient with respect to that direction in GD's sign, and the (linear) VJP
+// carries it to the gradient with respect to the chunk's gradient.
 // fp32 problems run every contraction as a batched k_simt_gemm over the B*H
 // heads in fp32.  bf16 problems run them on the tensor cores (GemmOp, bf16
 // operands through TMA, fp32 accumulation); the elementwise kernels write
@@ -44,16 +56,25 @@ struct BwdBufs {
   // bf16 problems (tensor-core contractions): bf16 operands
   __nv_bfloat16 *qh16, *kh16, *dos16, *hist16, *op16, *Gam16;
   __nv_bfloat16 *Bk, *Bv;   // stacked operands of the merged contractions
+  // Muon: per-chunk directions [nch][3BH][dh][d]; Newton-Schulz iterates
+  // X0..X5 (planes), Gram matrices A0..A4 and polynomials B0..B4
+  // ([3BH][d][d] each), two [d][d] temporaries, two VJP planes, the update in
+  // the weights' layout, the norms' partial sums
+  float *Phist, *nsX, *nsA, *nsB, *nsT, *nsY, *dir, *nspart;
   int64_t zr;   // rows per head of the per-chunk [rows][dh] planes
 };
 
 static int64_t rule_rows(const Dims& D) { return 2 * D.BH * D.dh + D.BH * D.d; }
 
+// bf16 problems run their contractions on the tensor cores, except under
+// Muon (fp32 on the CUDA cores, see above).
+static bool bwd_on_tc(const Dims& D) { return D.dtype == LACT_BF16 && D.rule != LACT_RULE_MUON; }
+
 static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
   std::memset(&b, 0, sizeof(b));
   const int64_t planes = 3 * D.BH * D.dh * D.d;
   const int64_t nq = D.BH * D.Tq * D.d, nk = D.BH * D.T * D.d;
-  const bool bf = D.dtype == LACT_BF16;
+  const bool bf = bwd_on_tc(D);
   const bool mom = D.rule == LACT_RULE_MOMENTUM;
   b.zr = std::max<int64_t>(D.chunk, D.nch == 1 ? D.Tq : D.chunk);
   const int64_t zpl = D.BH * b.zr * D.dh;
@@ -68,6 +89,12 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
     b.Bk = bp.take<__nv_bfloat16>(4 * D.BH * D.dh * D.d);
     b.Bv = bp.take<__nv_bfloat16>(2 * D.BH * D.dh * D.d);
   } else {
+    if (D.dtype == LACT_BF16) {   // fp32 copies of the inputs
+      b.q32 = bp.take<float>(nq);
+      b.k32 = bp.take<float>(nk);
+      b.v32 = bp.take<float>(nk);
+      b.do32 = bp.take<float>(nq);
+    }
     b.dos32 = bp.take<float>(nq);
     b.qh = bp.take<float>(nq);
     b.kh = bp.take<float>(nk);
@@ -83,6 +110,17 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
     b.part = bp.take<float>(rule_rows(D));
   }
   b.mnorm = bp.take<float>(D.nch * rule_rows(D));
+  if (D.rule == LACT_RULE_MUON) {
+    const int64_t grams = 3 * D.BH * D.d * D.d;
+    b.Phist = bp.take<float>(D.nch * planes);
+    b.nsX = bp.take<float>(6 * planes);
+    b.nsA = bp.take<float>(5 * grams);
+    b.nsB = bp.take<float>(5 * grams);
+    b.nsT = bp.take<float>(2 * grams);
+    b.nsY = bp.take<float>(2 * planes);
+    b.dir = bp.take<float>(planes);
+    b.nspart = bp.take<float>(3 * D.BH * kNsBlocks);
+  }
   if (!bf) {
     b.Z = bp.take<float>(3 * zpl);
     b.Pz = bp.take<float>(3 * zpl);
@@ -106,10 +144,133 @@ static unsigned grid_for(int64_t n, int per_thread = 1) {
   return static_cast<unsigned>(std::min<int64_t>(std::max<int64_t>(cdiv(n, 256LL * per_thread), 1), 148 * 32));
 }
 
+// ------------------------------------------------------------------ Muon
+// C[item] = alpha * A(item) B(item)^T + beta * cin over the 3 BH matrices,
+// fp32 on the CUDA cores (k_simt_gemm indexing).
+static void ns_gemm(const Dims& D, Launcher& L, cudaStream_t st, const float* A, int64_t a_item, int64_t a_m,
+                    int64_t a_k, const float* B, int64_t b_item, int64_t b_n, int64_t b_k, int M, int N, int K,
+                    float alpha, float beta, const float* cin, float* out, int64_t out_item, int64_t ld) {
+  L(K_SIMT_GEMM, [&] {
+    SimtGemmParams s = simt_params();
+    s.A = A; s.a_item = a_item; s.a_m = a_m; s.a_k = a_k;
+    s.B = B; s.b_item = b_item; s.b_n = b_n; s.b_k = b_k;
+    s.M = M; s.N = N; s.K = K; s.alpha = alpha; s.beta = beta; s.cin = cin;
+    s.outf = out; s.item_stride = out_item; s.ld = ld;
+    return simt(s, static_cast<int>(3 * D.BH), st);
+  });
+}
+
+// W2's planes between the weights' layout [d, dh] and the Newton-Schulz
+// layout [dh, d] (the other two planes are copied): dst = src with plane
+// group 1 transposed; `to_ns` picks the direction.
+static void ns_relayout(const Dims& D, Launcher& L, cudaStream_t st, const float* src, float* dst, bool to_ns) {
+  const int64_t plane = D.dh * D.d, jst = D.BH * plane;
+  if (!L.dry && L.err == LACT_OK) {
+    if (cudaMemcpyAsync(dst, src, static_cast<size_t>(jst) * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dst + 2 * jst, src + 2 * jst, static_cast<size_t>(jst) * 4, cudaMemcpyDeviceToDevice,
+                        st) != cudaSuccess)
+      L.err = LACT_ECUDA;
+  }
+  const int rows = static_cast<int>(to_ns ? D.d : D.dh), cols = static_cast<int>(to_ns ? D.dh : D.d);
+  L(K_BWD_ELEM, [&] {
+    (void)launch_pdl(k_transpose_planes, dim3(cdiv(cols, 32), cdiv(rows, 32), D.BH), dim3(32, 8), 0, st,
+                     src + jst, dst + jst, rows, cols);
+    return cudaGetLastError();
+  });
+}
+
+// The Newton-Schulz steps on S ([3BH][dh][d]), keeping X0..X5, A0..A4 and
+// B0..B4 and the norms' partial sums:
+//   X0 = S / (||S||_F + eps);  A = X^T X;  B = b A + c A A;  X <- a X + X B
+// (the forward's arithmetic, "大块测试时训练（LaCT）技术解析" §2.2.1).
+static void ns_keep(const Dims& D, const BwdBufs& b, const float* S, cudaStream_t st, Launcher& L) {
+  const int d = static_cast<int>(D.d), dh = static_cast<int>(D.dh), n3 = static_cast<int>(3 * D.BH);
+  const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane, dd = D.d * D.d, grams = n3 * dd;
+  L(K_NS_SUMSQ, [&] {
+    (void)launch_pdl(k_ns_sumsq, dim3(kNsBlocks, n3), 256, 0, st, S, 1, planes, plane, b.nsX, b.nspart);
+    return cudaGetLastError();
+  });
+  L(K_NS_SCALE, [&] {
+    (void)launch_pdl(k_ns_scale, dim3(kNsBlocks, n3), 256, 0, st, b.nsX, static_cast<__nv_bfloat16*>(nullptr),
+                     static_cast<__nv_bfloat16*>(nullptr), plane, static_cast<const float*>(b.nspart), kNsBlocks,
+                     kNsEps);
+    return cudaGetLastError();
+  });
+  for (int k = 0; k < kNsSteps; ++k) {
+    const float* X = b.nsX + k * planes;
+    float* A = b.nsA + k * grams;
+    float* B = b.nsB + k * grams;
+    ns_gemm(D, L, st, X, plane, 1, d, X, plane, 1, d, d, d, dh, 1.0f, 0.0f, nullptr, A, dd, d);        // X^T X
+    ns_gemm(D, L, st, A, dd, d, 1, A, dd, 1, d, d, d, d, kNsC, kNsB, A, B, dd, d);                       // c A A + b A
+    ns_gemm(D, L, st, X, plane, d, 1, B, dd, 1, d, dh, d, d, 1.0f, kNsA, X, b.nsX + (k + 1) * planes, plane,
+            d);                                                                                          // X B + a X
+  }
+}
+
+// dL/dS = VJP of S -> X5 at the iterates ns_keep kept, applied to Y
+// (= dL/dX5, [3BH][dh][d], b.nsY; overwritten), written to `out`.  One step
+// back, with Y = dL/dX' for X' = a X + X B, B = b A + c A A, A = X^T X:
+//   dB = X^T Y,  dA = b dB + c (dB A + A dB),  dL/dX = a Y + Y B + X (dA + dA^T)
+// (A and B are symmetric).  Then the normalisation's VJP (k_ns_norm_vjp).
+static void ns_vjp(const Dims& D, const BwdBufs& b, const float* S, float* out, cudaStream_t st, Launcher& L) {
+  const int d = static_cast<int>(D.d), dh = static_cast<int>(D.dh), n3 = static_cast<int>(3 * D.BH);
+  const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane, dd = D.d * D.d, grams = n3 * dd;
+  float* Y = b.nsY;
+  float* Yn = b.nsY + planes;
+  float* dB = b.nsT;
+  float* T = b.nsT + grams;
+  for (int k = kNsSteps - 1; k >= 0; --k) {
+    const float* X = b.nsX + k * planes;
+    const float* A = b.nsA + k * grams;
+    const float* B = b.nsB + k * grams;
+    ns_gemm(D, L, st, X, plane, 1, d, Y, plane, 1, d, d, d, dh, 1.0f, 0.0f, nullptr, dB, dd, d);       // X^T Y
+    ns_gemm(D, L, st, dB, dd, d, 1, A, dd, 1, d, d, d, d, kNsC, kNsB, dB, T, dd, d);                    // c dB A + b dB
+    ns_gemm(D, L, st, A, dd, d, 1, dB, dd, 1, d, d, d, d, kNsC, 1.0f, T, T, dd, d);                     // + c A dB
+    L(K_BWD_ELEM, [&] {
+      (void)launch_pdl(k_sym_add, grid_for(grams, 1), 256, 0, st, T, d, static_cast<int64_t>(n3));
+      return cudaGetLastError();
+    });
+    ns_gemm(D, L, st, Y, plane, d, 1, B, dd, 1, d, dh, d, d, 1.0f, kNsA, Y, Yn, plane, d);              // Y B + a Y
+    ns_gemm(D, L, st, X, plane, d, 1, T, dd, 1, d, dh, d, d, 1.0f, 1.0f, Yn, Yn, plane, d);             // + X (dA + dA^T)
+    std::swap(Y, Yn);
+  }
+  L(K_BWD_ELEM, [&] {
+    (void)launch_pdl(k_ns_norm_vjp, static_cast<unsigned>(n3), 1024, 0, st, S, static_cast<const float*>(Y),
+                     static_cast<const float*>(b.nspart), kNsBlocks, kNsEps, plane, out);
+    return cudaGetLastError();
+  });
+}
+
+// Forward recompute, Muon: the chunk's direction S (= b.P, [dh, d] planes)
+// kept for the reverse loop, and its orthogonalised update in the weights'
+// layout (b.dir) for the rule kernel.
+static void muon_forward_step(const Dims& D, const BwdBufs& b, int64_t c, cudaStream_t st, Launcher& L) {
+  const int64_t planes = 3 * D.BH * D.dh * D.d;
+  float* S = b.Phist + c * planes;
+  if (!L.dry && L.err == LACT_OK &&
+      cudaMemcpyAsync(S, b.P, static_cast<size_t>(planes) * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    L.err = LACT_ECUDA;
+  ns_keep(D, b, S, st, L);
+  ns_relayout(D, L, st, b.nsX + kNsSteps * planes, b.dir, false);
+}
+
+// Reverse loop, Muon: b.Gam holds the gradient with respect to the update
+// (the renorm backward's GD output, weights' layout); replaced by the
+// gradient with respect to the chunk's negated gradient S.
+static void muon_backward_step(const Dims& D, const BwdBufs& b, int64_t c, cudaStream_t st, Launcher& L) {
+  const int64_t planes = 3 * D.BH * D.dh * D.d;
+  const float* S = b.Phist + c * planes;
+  ns_relayout(D, L, st, b.Gam, b.nsY, true);
+  ns_keep(D, b, S, st, L);
+  ns_vjp(D, b, S, b.dir, st, L);
+  ns_relayout(D, L, st, b.dir, b.Gam, false);
+}
+
 // fp32 problems: every contraction on the CUDA cores in fp32.
 static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaStream_t st, Launcher& L) {
   L.st = st;
   const bool mom = D.rule == LACT_RULE_MOMENTUM;
+  const bool muon = D.rule == LACT_RULE_MUON;
   const int BH = static_cast<int>(D.BH), d = static_cast<int>(D.d), dh = static_cast<int>(D.dh);
   const int64_t plane = D.dh * D.d, planes = 3 * D.BH * plane, jst = D.BH * plane;
   const int64_t nq = D.BH * D.Tq * D.d, nk = D.BH * D.T * D.d;
@@ -138,11 +299,23 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
     });
   };
 
-  // ---- the scaled output gradient, zeroed accumulators
+  // ---- fp32 inputs (copies of bf16 ones), the scaled output gradient, zeroed accumulators
   const float* q32 = static_cast<const float*>(in.q);
   const float* k32 = static_cast<const float*>(in.k);
   const float* v32 = static_cast<const float*>(in.v);
   const float* do32 = static_cast<const float*>(in.dout);
+  if (D.dtype == LACT_BF16) {
+    const void* src[4] = {in.q, in.k, in.v, in.dout};
+    float* dst[4] = {b.q32, b.k32, b.v32, b.do32};
+    const int64_t n[4] = {nq, nk, nk, nq};
+    for (int i = 0; i < 4; ++i)
+      L(K_BWD_ELEM, [&] {
+        (void)launch_pdl(k_bf16_to_f32, grid_for(n[i], 4), 256, 0, st, static_cast<const __nv_bfloat16*>(src[i]),
+                         dst[i], n[i]);
+        return cudaGetLastError();
+      });
+    q32 = b.q32; k32 = b.k32; v32 = b.v32; do32 = b.do32;
+  }
   const float* dos = do32;
   if (in.scale) {
     L(K_BWD_ELEM, [&] {
@@ -220,13 +393,14 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
       s.zb_mod = BH; s.alt_b = 1;
       s.M = dh; s.N = d; s.K = nc;
       s.outf = b.P; s.item_stride = plane; s.ld = d;
-      s.tr_group = 1; s.tr_mod = BH; s.ld_t = dh;
+      if (!muon) { s.tr_group = 1; s.tr_mod = BH; s.ld_t = dh; }   // Muon keeps [dh, d] planes
       return simt(s, 3 * BH, st);
     });
+    if (muon) muon_forward_step(D, b, c, st, L);
     L(K_RULE, [&] {
       RuleParams r;
       std::memset(&r, 0, sizeof(r));
-      r.Wm = Wn; r.S = b.P; r.splits = 1; r.split_stride = planes;
+      r.Wm = Wn; r.S = muon ? b.dir : b.P; r.splits = 1; r.split_stride = planes;
       r.Mm = mom ? b.Mm : nullptr; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch);
       r.chunk_idx = static_cast<int>(c); r.rule = D.rule; r.BH = BH; r.dh = dh; r.d = d;
       r.nrm_out = b.mnorm + c * rows_all;
@@ -275,12 +449,13 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
         RenormBwdParams r;
         std::memset(&r, 0, sizeof(r));
         r.A = A; r.Wc = Wc; r.Wp = Wp; r.mnorm = b.mnorm + c * rows_all; r.Gam = b.Gam; r.Ap = Ap;
-        r.rule = D.rule; r.Bm = b.Bm; r.Mprev = mom ? b.mh + c * planes : nullptr; r.beta_bar = b.bbar;
-        r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c); r.part = b.part;
+        r.rule = muon ? LACT_RULE_GD : D.rule; r.Bm = b.Bm; r.Mprev = mom ? b.mh + c * planes : nullptr;
+        r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c); r.part = b.part;
         r.BH = BH; r.dh = dh; r.d = d;
         (void)launch_pdl(k_renorm_bwd, static_cast<unsigned>(cdiv(rows_all * 32, 256)), 256, 0, st, r);
         return cudaGetLastError();
       });
+      if (muon) muon_backward_step(D, b, c, st, L);   // through the Newton-Schulz steps
       if (mom)
         L(K_BWD_ELEM, [&] {
           (void)launch_pdl(k_head_dbeta, static_cast<unsigned>(BH), 256, 0, st, b.part, BH, dh, d, D.T, c0, nc,
@@ -664,7 +839,7 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
 }
 
 static void run_bwd(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaStream_t st, Launcher& L) {
-  if (D.dtype == LACT_BF16) run_bwd_tc(D, b, in, st, L);
+  if (bwd_on_tc(D)) run_bwd_tc(D, b, in, st, L);
   else run_bwd_f32(D, b, in, st, L);
 }
 

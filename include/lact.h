@@ -237,8 +237,8 @@ int lact_ttt_fwd_host(const lact_problem* p,
                       void* out, float* w1_out, float* w2_out, float* w3_out,
                       void* workspace, size_t workspace_bytes, void* stream);
 
-/* Device scratch bytes lact_ttt_bwd needs for problem *p (0 if *p is invalid
- * or uses the Muon rule).  Pure host arithmetic. */
+/* Device scratch bytes lact_ttt_bwd needs for problem *p (0 if *p is
+ * invalid).  Pure host arithmetic. */
 size_t lact_ttt_bwd_workspace_bytes(const lact_problem* p);
 
 /* The layer's backward: the gradients of a scalar loss L with respect to
@@ -249,9 +249,15 @@ size_t lact_ttt_bwd_workspace_bytes(const lact_problem* p);
  * are kept in the workspace), then a reverse chunk loop takes, per chunk,
  * the apply's backward, the renorm and rule backward, and the backward of
  * the chunk gradient (its second-order terms: [P2 §2.1] eqs. 4-5 written as
- * functions of W, k, v and lr).  Rules: GD and momentum (LACT_EINVAL for
- * Muon).  Options: update_mask and out_scale; the momentum buffers and the
- * all-reduce hook are not supported (LACT_EINVAL).
+ * functions of W, k, v and lr).  Rules: GD, momentum and Muon; for Muon the
+ * rule backward is the vector-Jacobian product of the Frobenius
+ * normalisation and the five Newton-Schulz steps ([P2 §2.2.1] eqs. 9-10),
+ * recomputed per chunk from the kept chunk gradient.  A Muon problem runs
+ * its whole backward in fp32 on the CUDA cores, bf16 inputs included (read
+ * as fp32): the iteration's Jacobian magnifies bf16 operand rounding past
+ * the bf16 tolerance.  GD and momentum bf16 problems run their contractions
+ * on the tensor cores (bf16 operands, fp32 accumulation).  Options: update_mask and out_scale; the
+ * momentum buffers and the all-reduce hook are not supported (LACT_EINVAL).
  * Layouts: the inputs as in lact_ttt_fwd; dout [B,H,Tq,d] in the problem's
  * dtype; dw*_out in the layouts of w*_out, or NULL (zero).  Outputs, all
  * float32 device buffers: dq [B,H,Tq,d], dk, dv [B,H,T,d], dlr [B,H,T,3],

@@ -4,7 +4,7 @@ autograd oracle (oracle/lact_oracle_bwd.py).
 Every gradient (q, k, v, lr, beta, the initial weights, the output scale) is
 compared by relative L2 over all heads: <= 1e-4 for fp32 workloads, <= 2e-2
 for bf16 ones (the backward computes in fp32 in both; the oracle reads the
-same bf16-rounded inputs).  Cases span the two orders, GD and momentum, a
+same bf16-rounded inputs).  Cases span the two orders, GD, momentum and Muon, a
 ragged last chunk, masks, the output scale, given final-weight gradients,
 shared and per-(b, h) initial weights and a single chunk with separate
 queries; the full-size 760M LM shape is checked on sampled heads.
@@ -15,7 +15,8 @@ import torch
 
 import chunk_test_b200 as ct
 from oracle import lact_oracle_bwd as ob
-from lact_inputs import (APPLY_THEN_UPDATE, BF16, F32, RULE_GD, RULE_MOMENTUM, UPDATE_THEN_APPLY,
+from lact_inputs import (APPLY_THEN_UPDATE, BF16, F32, RULE_GD, RULE_MOMENTUM, RULE_MUON,
+                         UPDATE_THEN_APPLY,
                          WORKLOADS, Workload, make_inputs, make_out_scale, make_output_grads,
                          video_update_mask)
 
@@ -80,6 +81,16 @@ CASES = [
               RULE_MOMENTUM, BF16), dict(mask=video_update_mask(6, 1), scaled=True, with_dw=True)),
     (Workload("bwd-bf16-d384-uta-ragged", 1, 1, 1100, 1100, 384, 768, 512, UPDATE_THEN_APPLY, RULE_GD,
               BF16), dict(mask=[1, 0, 1], per_bh=True)),
+    # Muon: the vector-Jacobian product through five Newton-Schulz steps and
+    # the Frobenius normalisation, in fp32 on both launch paths.
+    (Workload("bwd-f32-atu-muon", 1, 2, 768, 768, 64, 128, 256, APPLY_THEN_UPDATE, RULE_MUON, F32),
+     dict(scaled=True, with_dw=True)),
+    (Workload("bwd-f32-uta-muon-mask", 2, 1, 700, 700, 32, 64, 128, UPDATE_THEN_APPLY, RULE_MUON, F32),
+     dict(mask=[1, 1, 0, 1, 1, 1], per_bh=True)),
+    (Workload("bwd-bf16-d128-atu-muon", 1, 2, 1024, 1024, 128, 256, 256, APPLY_THEN_UPDATE, RULE_MUON,
+              BF16), dict(with_dw=True)),
+    (Workload("bwd-bf16-d384-atu-muon", 1, 1, 1024, 1024, 384, 768, 512, APPLY_THEN_UPDATE, RULE_MUON,
+              BF16), dict(scaled=True)),
 ]
 
 
