@@ -91,14 +91,15 @@ def _renorm(W_new, W_old):
 
 
 def head_forward(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule, update_mask=None,
-                 out_scale=None):
+                 out_scale=None, M0=None):
     """The layer for one (batch, head) in torch fp64: returns out [Tq, d],
-    the final (W1, W2, W3) and the final momentum (zeros for GD)."""
+    the final (W1, W2, W3) and the final momentum (zeros for GD).  M0: the
+    momentum before the first chunk (R15), zeros if None."""
     T, Tq = k.shape[0], q.shape[0]
     starts = list(range(0, T, chunk))
     qh, kh = _prologue(q), _prologue(k)
     W = (W1, W2, W3)
-    M = tuple(torch.zeros_like(w) for w in W)
+    M = tuple(torch.zeros_like(w) for w in W) if M0 is None else tuple(M0)
     outs = []
     for ci, c0 in enumerate(starts):
         c1 = min(c0 + chunk, T)
@@ -128,7 +129,7 @@ def head_forward(q, k, v, lr, beta, W1, W2, W3, chunk, order, rule, update_mask=
 
 
 def ttt_layer_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, dw=None,
-                  update_mask=None, out_scale=None, heads=None):
+                  update_mask=None, out_scale=None, heads=None, m_in=None, dm=None):
     """Gradients of sum(out * dout) + sum_j <w_j_out, dw_j> over the layer's
     inputs, on the ABI layout (q [B,H,Tq,d]; k, v [B,H,T,d]; lr [B,H,T,3];
     beta [B,H,T] or None; w1, w3 [Hw,dh,d], w2 [Hw,d,dh] with Hw = H or B*H;
@@ -138,11 +139,23 @@ def ttt_layer_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, dw=No
     shape of the initial weights: summed over the batch when they are
     shared), dout_scale (or None) and, for the forward check, out and the
     final weights (w1o, w2o, w3o).  heads: optional (b, h) pairs; the others
-    are left as NaN (the initial-weight gradients then sum only those)."""
+    are left as NaN (the initial-weight gradients then sum only those).
+
+    Momentum in/out (R15, momentum rule): m_in = (m1, m2, m3), each [B*H]
+    in the layout of w*_out, the momentum before the first chunk (zeros if
+    None); dm = the gradients of the final momentum, added to the loss as
+    sum_j <m_j_out, dm_j>.  With either given, the dict also holds dm1,
+    dm2, dm3 (the gradients of m_in) and the final momentum (m1o, m2o,
+    m3o)."""
     q, k, v, lr, beta = _t(q), _t(k), _t(v), _t(lr), _t(beta)
     w1, w2, w3, dout = _t(w1), _t(w2), _t(w3), _t(dout)
     dw = None if dw is None else tuple(_t(x) for x in dw)
     out_scale = _t(out_scale)
+    with_m = m_in is not None or dm is not None
+    if with_m and rule != RULE_MOMENTUM:
+        raise ValueError("momentum in/out needs the momentum rule")
+    m_in = None if m_in is None else tuple(_t(x) for x in m_in)
+    dm = None if dm is None else tuple(_t(x) for x in dm)
     B, H, Tq, d = q.shape
     T = k.shape[2]
     dh = w1.shape[1]
@@ -157,6 +170,10 @@ def ttt_layer_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, dw=No
         "w2o": torch.full((B * H, d, dh), nan, dtype=torch.float64),
         "w3o": torch.full((B * H, dh, d), nan, dtype=torch.float64),
     }
+    if with_m:
+        for j, shp in ((1, (dh, d)), (2, (d, dh)), (3, (dh, d))):
+            res[f"dm{j}"] = torch.full((B * H,) + shp, nan, dtype=torch.float64)
+            res[f"m{j}o"] = torch.full((B * H,) + shp, nan, dtype=torch.float64)
     todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
     mask = None if update_mask is None else [int(x) for x in update_mask]
     for b, h in todo:
@@ -165,20 +182,28 @@ def ttt_layer_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, dw=No
                   None if beta is None else beta[b, h].clone(),
                   w1[wi].clone(), w2[wi].clone(), w3[wi].clone(),
                   None if out_scale is None else out_scale[b, h].clone()]
+        bh = b * H + h
+        M0 = None
+        if with_m:
+            M0 = [torch.zeros_like(x) if m_in is None else m_in[j][bh].clone()
+                  for j, x in enumerate((w1[wi], w2[wi], w3[wi]))]
+            leaves += M0
         for x in leaves:
             if x is not None:
                 x.requires_grad_(True)
-        qq, kk, vv, ll, bb, W1, W2, W3, ss = leaves
-        out, W, _ = head_forward(qq, kk, vv, ll, bb, W1, W2, W3, chunk, order, rule, mask, ss)
+        qq, kk, vv, ll, bb, W1, W2, W3, ss = leaves[:9]
+        out, W, M = head_forward(qq, kk, vv, ll, bb, W1, W2, W3, chunk, order, rule, mask, ss, M0)
         loss = (out * dout[b, h]).sum()
         if dw is not None:
-            loss = loss + sum((wf * g[b * H + h]).sum() for wf, g in zip(W, dw))
+            loss = loss + sum((wf * g[bh]).sum() for wf, g in zip(W, dw))
+        if dm is not None:
+            loss = loss + sum((mf * g[bh]).sum() for mf, g in zip(M, dm))
         want = [x for x in leaves if x is not None]
         grads = torch.autograd.grad(loss, want, allow_unused=True)
         it = iter(grads)
         g = {}
-        for name, x in zip(("dq", "dk", "dv", "dlr", "dbeta", "dw1", "dw2", "dw3", "dout_scale"),
-                           leaves):
+        for name, x in zip(("dq", "dk", "dv", "dlr", "dbeta", "dw1", "dw2", "dw3", "dout_scale",
+                            "dm1", "dm2", "dm3"), leaves):
             if x is not None:
                 gx = next(it)
                 g[name] = torch.zeros_like(x) if gx is None else gx
@@ -192,5 +217,9 @@ def ttt_layer_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, dw=No
         res["dw2"][wi] += g["dw2"]
         res["dw3"][wi] += g["dw3"]
         res["out"][b, h] = out.detach()
-        res["w1o"][b * H + h], res["w2o"][b * H + h], res["w3o"][b * H + h] = (x.detach() for x in W)
+        res["w1o"][bh], res["w2o"][bh], res["w3o"][bh] = (x.detach() for x in W)
+        if with_m:
+            for j in range(3):
+                res[f"dm{j + 1}"][bh] = g[f"dm{j + 1}"]
+                res[f"m{j + 1}o"][bh] = M[j].detach()
     return {k_: (None if v_ is None else v_.numpy()) for k_, v_ in res.items()}

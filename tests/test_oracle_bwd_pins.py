@@ -26,11 +26,14 @@ def _problem(B=1, H=2, T=12, Tq=None, d=4, dh=6, beta=True, w_per_bh=False, lr_s
         w3=RNG.standard_normal((Hw, dh, d)) / d ** 0.5)
 
 
-def _numpy_loss(p, chunk, order, rule, dout, dw, mask=None, scale=None):
-    out, w1o, w2o, w3o, *_ = oracle.ttt_layer_ex(p["q"], p["k"], p["v"], p["lr"], p["beta"], p["w1"],
-                                                 p["w2"], p["w3"], chunk, order, rule,
-                                                 update_mask=mask, out_scale=scale)
-    return (out * dout).sum() + sum((a * b).sum() for a, b in zip((w1o, w2o, w3o), dw))
+def _numpy_loss(p, chunk, order, rule, dout, dw, mask=None, scale=None, m_in=None, dm=None):
+    out, w1o, w2o, w3o, m1o, m2o, m3o = oracle.ttt_layer_ex(
+        p["q"], p["k"], p["v"], p["lr"], p["beta"], p["w1"], p["w2"], p["w3"], chunk, order, rule,
+        update_mask=mask, out_scale=scale, m_in=m_in)
+    loss = (out * dout).sum() + sum((a * b).sum() for a, b in zip((w1o, w2o, w3o), dw))
+    if dm is not None:
+        loss = loss + sum((a * b).sum() for a, b in zip((m1o, m2o, m3o), dm))
+    return loss
 
 
 CASES = [
@@ -123,3 +126,50 @@ def test_muon_with_zero_rates_has_no_path_through_the_update():
     for a, b in zip((g["w1o"], g["w2o"], g["w3o"]), (p["w1"], p["w2"], p["w3"])):
         np.testing.assert_allclose(a, np.concatenate([b]), rtol=1e-12, atol=1e-13)
     assert np.all(np.isfinite(g["dlr"])) and np.any(g["dlr"] != 0)
+
+
+@pytest.mark.parametrize("order,mask", [(APPLY_THEN_UPDATE, None), (UPDATE_THEN_APPLY, [1, 0, 1, 1])])
+def test_momentum_in_and_out_gradients_match_central_differences(order, mask):
+    """R15: with an initial momentum M_0 handed in and a loss on the final
+    momentum, the gradient of M_0 (and every other input) matches central
+    differences of the numpy oracle's forward run from M_0."""
+    p = _problem(B=2, T=11)
+    dout = RNG.standard_normal(p["q"].shape)
+    dw = (RNG.standard_normal((4, 6, 4)), RNG.standard_normal((4, 4, 6)), RNG.standard_normal((4, 6, 4)))
+    m_in = (RNG.standard_normal((4, 6, 4)), RNG.standard_normal((4, 4, 6)), RNG.standard_normal((4, 6, 4)))
+    dm = (RNG.standard_normal((4, 6, 4)), RNG.standard_normal((4, 4, 6)), RNG.standard_normal((4, 6, 4)))
+    g = ob.ttt_layer_bwd(**p, chunk=3, order=order, rule=RULE_MOMENTUM, dout=dout, dw=dw, update_mask=mask,
+                         m_in=m_in, dm=dm)
+    want = oracle.ttt_layer_ex(p["q"], p["k"], p["v"], p["lr"], p["beta"], p["w1"], p["w2"], p["w3"], 3,
+                               order, RULE_MOMENTUM, update_mask=mask, m_in=m_in)
+    for a, b in zip((g["m1o"], g["m2o"], g["m3o"]), want[4:7]):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    names = ["q", "k", "v", "lr", "beta", "w1", "w2", "w3"]
+    eps = 1e-6
+    for only in ["m", "beta", None]:
+        delta = {n: (RNG.standard_normal(p[n].shape) if only is None or n == only else 0 * p[n])
+                 for n in names}
+        dmv = tuple(RNG.standard_normal(m.shape) if only in ("m", None) else 0 * m for m in m_in)
+
+        def loss_at(t):
+            return _numpy_loss(dict(p, **{n: p[n] + t * delta[n] for n in names}), 3, order, RULE_MOMENTUM,
+                               dout, dw, mask, None, tuple(m + t * e for m, e in zip(m_in, dmv)), dm)
+
+        fd = (loss_at(eps) - loss_at(-eps)) / (2 * eps)
+        an = sum((g["d" + n] * delta[n]).sum() for n in names)
+        an += sum((g[f"dm{j + 1}"] * dmv[j]).sum() for j in range(3))
+        assert an == pytest.approx(fd, rel=1e-6, abs=1e-8), (only, an, fd)
+
+
+def test_momentum_gradient_passes_through_masked_chunks():
+    """Every chunk masked: the momentum is handed through untouched, so the
+    gradient of M_0 is the gradient given for the final momentum."""
+    p = _problem(T=9)
+    dout = RNG.standard_normal(p["q"].shape)
+    m_in = (RNG.standard_normal((2, 6, 4)), RNG.standard_normal((2, 4, 6)), RNG.standard_normal((2, 6, 4)))
+    dm = (RNG.standard_normal((2, 6, 4)), RNG.standard_normal((2, 4, 6)), RNG.standard_normal((2, 6, 4)))
+    g = ob.ttt_layer_bwd(**p, chunk=3, order=APPLY_THEN_UPDATE, rule=RULE_MOMENTUM, dout=dout,
+                         update_mask=[0, 0, 0], m_in=m_in, dm=dm)
+    for j in range(3):
+        np.testing.assert_array_equal(g[f"dm{j + 1}"], dm[j])
+        np.testing.assert_array_equal(g[f"m{j + 1}o"], m_in[j])
