@@ -42,6 +42,13 @@ class LactFwdOpts(ctypes.Structure):
     ]
 
 
+class LactBwdMomentum(ctypes.Structure):
+    """lact_bwd_momentum: dL/dM_final in (dm*_out, 0 = zero) and dL/dM_0 out
+    (dm*), all device float32 pointers."""
+    _fields_ = [("dm1_out", ctypes.c_void_p), ("dm2_out", ctypes.c_void_p), ("dm3_out", ctypes.c_void_p),
+                ("dm1", ctypes.c_void_p), ("dm2", ctypes.c_void_p), ("dm3", ctypes.c_void_p)]
+
+
 class LactSwaProblem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("T", ctypes.c_int64),
                 ("d", ctypes.c_int64), ("window", ctypes.c_int64), ("dtype", ctypes.c_int32),
@@ -66,6 +73,8 @@ SIGNATURES = {
     "lact_ttt_bwd_workspace_bytes": (ctypes.c_size_t, [_P]),
     "lact_ttt_bwd": (ctypes.c_int, [_P, ctypes.POINTER(LactFwdOpts)] + [_vp] * 21
                      + [_vp, ctypes.c_size_t, _vp]),
+    "lact_ttt_bwd_ex": (ctypes.c_int, [_P, ctypes.POINTER(LactFwdOpts), ctypes.POINTER(LactBwdMomentum)]
+                        + [_vp] * 21 + [_vp, ctypes.c_size_t, _vp]),
     "lact_ttt_host_workspace_bytes": (ctypes.c_size_t, [_P]),
     "lact_ttt_fwd_host": (ctypes.c_int, [_P] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]),
     "lact_swa_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(LactSwaProblem)]),

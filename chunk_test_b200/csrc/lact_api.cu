@@ -1274,12 +1274,30 @@ int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts, const void* q
                  const float* dw3_out, float* dq, float* dk, float* dv, float* dlr, float* dbeta,
                  float* dw1, float* dw2, float* dw3, float* dout_scale, void* workspace,
                  size_t workspace_bytes_, void* stream) {
+  return lact_ttt_bwd_ex(p, opts, nullptr, q, k, v, lr, beta, w1, w2, w3, dout, dw1_out, dw2_out, dw3_out, dq,
+                         dk, dv, dlr, dbeta, dw1, dw2, dw3, dout_scale, workspace, workspace_bytes_, stream);
+}
+
+int lact_ttt_bwd_ex(const lact_problem* p, const lact_fwd_opts* opts, const lact_bwd_momentum* mg,
+                    const void* q, const void* k, const void* v, const float* lr, const float* beta,
+                    const float* w1, const float* w2, const float* w3, const void* dout, const float* dw1_out,
+                    const float* dw2_out, const float* dw3_out, float* dq, float* dk, float* dv, float* dlr,
+                    float* dbeta, float* dw1, float* dw2, float* dw3, float* dout_scale, void* workspace,
+                    size_t workspace_bytes_, void* stream) {
   Dims D;
   int rc = validate(p, D);
   if (rc != LACT_OK) return rc;
-  if (opts && (opts->m1 || opts->m2 || opts->m3 || opts->allreduce)) return LACT_EINVAL;
+  if (opts && opts->allreduce) return LACT_EINVAL;
   const float* scale = opts ? opts->out_scale : nullptr;
   const bool mom = D.rule == LACT_RULE_MOMENTUM;
+  const float* m0[3] = {opts ? opts->m1 : nullptr, opts ? opts->m2 : nullptr, opts ? opts->m3 : nullptr};
+  const float* dmf[3] = {mg ? mg->dm1_out : nullptr, mg ? mg->dm2_out : nullptr, mg ? mg->dm3_out : nullptr};
+  float* dm0[3] = {mg ? mg->dm1 : nullptr, mg ? mg->dm2 : nullptr, mg ? mg->dm3 : nullptr};
+  const bool any_m0 = m0[0] || m0[1] || m0[2], any_dmf = dmf[0] || dmf[1] || dmf[2];
+  if ((any_m0 || mg) && !mom) return LACT_EINVAL;
+  if (any_m0 && !(m0[0] && m0[1] && m0[2])) return LACT_EINVAL;
+  if (any_dmf && !(dmf[0] && dmf[1] && dmf[2])) return LACT_EINVAL;
+  if (mg && !(dm0[0] && dm0[1] && dm0[2])) return LACT_EINVAL;
   const size_t e = D.dtype == LACT_BF16 ? 2 : 4;
   const size_t nq = static_cast<size_t>(D.BH * D.Tq * D.d), nk = static_cast<size_t>(D.BH * D.T * D.d);
   const size_t hw = static_cast<size_t>(D.w_shared ? D.H : D.BH) * D.d * D.dh * 4;
@@ -1289,11 +1307,15 @@ int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts, const void* q
                      {lr, static_cast<size_t>(D.BH * D.T) * 12, true}, {beta, static_cast<size_t>(D.BH * D.T) * 4, mom},
                      {w1, hw, true}, {w2, hw, true}, {w3, hw, true}, {dout, nq * e, true},
                      {dw1_out, wo, false}, {dw2_out, wo, false}, {dw3_out, wo, false},
-                     {scale, static_cast<size_t>(D.BH * D.Tq) * 4, false}};
+                     {scale, static_cast<size_t>(D.BH * D.Tq) * 4, false},
+                     {m0[0], wo, false}, {m0[1], wo, false}, {m0[2], wo, false},
+                     {dmf[0], wo, false}, {dmf[1], wo, false}, {dmf[2], wo, false}};
+  const bool with_dm = mg != nullptr;
   const Buf outs[] = {{dq, nq * 4, true}, {dk, nk * 4, true}, {dv, nk * 4, true},
                       {dlr, static_cast<size_t>(D.BH * D.T) * 12, true},
                       {dbeta, static_cast<size_t>(D.BH * D.T) * 4, mom}, {dw1, hw, true}, {dw2, hw, true},
-                      {dw3, hw, true}, {dout_scale, static_cast<size_t>(D.BH * D.Tq) * 4, scale != nullptr}};
+                      {dw3, hw, true}, {dout_scale, static_cast<size_t>(D.BH * D.Tq) * 4, scale != nullptr},
+                      {dm0[0], wo, with_dm}, {dm0[1], wo, with_dm}, {dm0[2], wo, with_dm}};
   for (const Buf& b : ins)
     if ((b.need && !b.p) || (b.p && !aligned16(b.p) && b.p != scale)) return LACT_EINVAL;
   for (const Buf& b : outs)
@@ -1314,7 +1336,8 @@ int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts, const void* q
   BwdBufs b;
   plan_bwd(D, bp, b);
   BwdInputs in{q, k, v, lr, beta, w1, w2, w3, dout, dw1_out, dw2_out, dw3_out,
-               opts ? opts->update_mask : nullptr, scale, dq, dk, dv, dlr, dbeta, dw1, dw2, dw3, dout_scale};
+               opts ? opts->update_mask : nullptr, scale, dq, dk, dv, dlr, dbeta, dw1, dw2, dw3, dout_scale,
+               {m0[0], m0[1], m0[2]}, {dmf[0], dmf[1], dmf[2]}, {dm0[0], dm0[1], dm0[2]}};
   Launcher L{false, static_cast<cudaStream_t>(stream)};
   run_bwd(D, b, in, static_cast<cudaStream_t>(stream), L);
   return L.err;

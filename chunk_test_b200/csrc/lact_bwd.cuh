@@ -45,6 +45,9 @@ struct BwdInputs {
   const uint8_t* mask;
   const float* scale;
   float *dq, *dk, *dv, *dlr, *dbeta, *dw1, *dw2, *dw3, *dscale;
+  const float* m0[3];    // momentum: M_0 (the layouts of w*_out), or null (zeros)
+  const float* dmf[3];   // momentum: dL/dM_final, or null (zero)
+  float* dm0[3];         // momentum: out dL/dM_0, or null
 };
 
 struct BwdBufs {
@@ -329,7 +332,12 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
   zero(in.dv, nk * 4);
   zero(b.dqh, nq * 4);
   zero(b.dkh, nk * 4);
-  if (mom) zero(b.Bm, planes * 4);
+  if (mom) {   // dL/dM after the last chunk
+    for (int j = 0; j < 3; ++j) {
+      if (in.dmf[j]) copy(b.Bm + j * jst, in.dmf[j], jst * 4);
+      else zero(b.Bm + j * jst, jst * 4);
+    }
+  }
   const float* dwf[3] = {in.dw1f, in.dw2f, in.dw3f};
   for (int j = 0; j < 3; ++j) {
     if (dwf[j]) copy(b.A + j * jst, dwf[j], jst * 4);
@@ -354,8 +362,7 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
     (void)launch_pdl(k_init_state, blocks, 256, 0, st, in.w1, in.w2, in.w3, static_cast<int>(D.H), D.w_shared,
                      BH, d, dh, b.hist, static_cast<__nv_bfloat16*>(nullptr),
                      static_cast<__nv_bfloat16*>(nullptr), mom ? b.Mm : nullptr,
-                     static_cast<const float*>(nullptr), static_cast<const float*>(nullptr),
-                     static_cast<const float*>(nullptr));
+                     in.m0[0], in.m0[1], in.m0[2]);
     return cudaGetLastError();
   });
   if (mom) {
@@ -512,6 +519,9 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
                      static_cast<int>(D.B), static_cast<int>(D.H), plane, D.w_shared, in.dw1, in.dw2, in.dw3);
     return cudaGetLastError();
   });
+  if (mom)   // after chunk 0, B holds dL/dM_0
+    for (int j = 0; j < 3; ++j)
+      if (in.dm0[j]) copy(in.dm0[j], b.Bm + j * jst, jst * 4);
 }
 
 // One bf16 operand: a dense [batch][rows][inner] tensor.
@@ -623,7 +633,12 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
   zero(in.dv, nk * 4);
   zero(b.dqh, nq * 4);
   zero(b.dkh, nk * 4);
-  if (mom) zero(b.Bm, planes * 4);
+  if (mom) {   // dL/dM after the last chunk
+    for (int j = 0; j < 3; ++j) {
+      if (in.dmf[j]) copy(b.Bm + j * jst, in.dmf[j], jst * 4);
+      else zero(b.Bm + j * jst, jst * 4);
+    }
+  }
   const float* dwf[3] = {in.dw1f, in.dw2f, in.dw3f};
   for (int j = 0; j < 3; ++j) {
     if (dwf[j]) copy(b.A + j * jst, dwf[j], jst * 4);
@@ -648,8 +663,7 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(cdiv(planes, 1024), 148 * 16));
     (void)launch_pdl(k_init_state, blocks, 256, 0, st, in.w1, in.w2, in.w3, static_cast<int>(D.H), D.w_shared,
                      BH, d, dh, b.hist, b.hist16, static_cast<B16*>(nullptr), mom ? b.Mm : nullptr,
-                     static_cast<const float*>(nullptr), static_cast<const float*>(nullptr),
-                     static_cast<const float*>(nullptr));
+                     in.m0[0], in.m0[1], in.m0[2]);
     return cudaGetLastError();
   });
   if (mom) {
@@ -836,6 +850,9 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
                      static_cast<int>(D.B), static_cast<int>(D.H), plane, D.w_shared, in.dw1, in.dw2, in.dw3);
     return cudaGetLastError();
   });
+  if (mom)   // after chunk 0, B holds dL/dM_0
+    for (int j = 0; j < 3; ++j)
+      if (in.dm0[j]) copy(in.dm0[j], b.Bm + j * jst, jst * 4);
 }
 
 static void run_bwd(const Dims& D, const BwdBufs& b, const BwdInputs& in, cudaStream_t st, Launcher& L) {

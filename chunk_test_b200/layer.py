@@ -246,20 +246,43 @@ def bwd_workspace_bytes(q, k, w1, chunk, order, rule) -> int:
     return _abi.bwd_workspace_bytes(make_problem(q, k, w1, chunk, order, rule))
 
 
+def _check_momentum(name, ms, q, dh, d):
+    B, H = q.shape[0], q.shape[1]
+    shapes = ((B * H, dh, d), (B * H, d, dh), (B * H, dh, d))
+    if len(ms) != 3:
+        raise ValueError(f"{name} must be three tensors (m1, m2, m3)")
+    for m, shp in zip(ms, shapes):
+        if (m.device != q.device or m.dtype != torch.float32 or not m.is_contiguous()
+                or tuple(m.shape) != shp):
+            raise ValueError(f"{name} must be contiguous float32 tensors on q's device shaped {shapes}")
+
+
 def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=None,
-            update_mask=None, out_scale=None, workspace=None, stream=None):
-    """The layer's backward on the current CUDA device (lact_ttt_bwd): the
-    gradients of a loss given dL/d out (`dout`, like q) and optionally
-    dL/d w_out (`dw_out`, three tensors like the forward's w_out).  Returns a
-    dict of float32 tensors: dq, dk, dv, dlr, dbeta (momentum, else None),
-    dw1, dw2, dw3 (shaped like w1, w2, w3) and dout_scale (when out_scale is
-    given, else None).  On bf16 inputs some fp32 sums are accumulated with
-    atomic adds, so repeated calls can differ in the last bits."""
+            update_mask=None, out_scale=None, m_in=None, dm_out=None, momentum_grads=False,
+            workspace=None, stream=None):
+    """The layer's backward on the current CUDA device (lact_ttt_bwd, or
+    lact_ttt_bwd_ex for the momentum gradients): the gradients of a loss
+    given dL/d out (`dout`, like q) and optionally dL/d w_out (`dw_out`,
+    three tensors like the forward's w_out).  Returns a dict of float32
+    tensors: dq, dk, dv, dlr, dbeta (momentum, else None), dw1, dw2, dw3
+    (shaped like w1, w2, w3) and dout_scale (when out_scale is given, else
+    None).  Momentum rule: `m_in` is the momentum the forward started from
+    (the three tensors its m_inout held before the call), `dm_out` the
+    gradient of the final momentum it wrote; with either given or
+    `momentum_grads` set the dict also holds dm1, dm2, dm3, the gradients
+    of m_in.  On bf16 inputs some fp32 sums are accumulated with atomic
+    adds, so repeated calls can differ in the last bits."""
     _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
     if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_contiguous():
         raise ValueError("dout must be a contiguous tensor shaped like q, in q's dtype")
+    dh, d = w1.shape[1], w1.shape[2]
+    if m_in is not None:
+        _check_momentum("m_in", m_in, q, dh, d)
+    if dm_out is not None:
+        _check_momentum("dm_out", dm_out, q, dh, d)
+    want_dm = momentum_grads or m_in is not None or dm_out is not None
     p = make_problem(q, k, w1, chunk, order, rule)
-    opts, _keep = _options(p, update_mask, out_scale, None, q)
+    opts, _keep = _options(p, update_mask, out_scale, m_in, q)
     f32 = dict(device=q.device, dtype=torch.float32)
     res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
            "dv": torch.empty(v.shape, **f32), "dlr": torch.empty(lr.shape, **f32),
@@ -275,14 +298,24 @@ def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=N
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     dw = (None, None, None) if dw_out is None else tuple(dw_out)
-    rc = _abi.lib().lact_ttt_bwd(
-        ctypes.byref(p), None if opts is None else ctypes.byref(opts), _ptr(q), _ptr(k), _ptr(v),
+    mg = None
+    if want_dm:
+        B, H = q.shape[0], q.shape[1]
+        res["dm1"] = torch.empty((B * H, dh, d), **f32)
+        res["dm2"] = torch.empty((B * H, d, dh), **f32)
+        res["dm3"] = torch.empty((B * H, dh, d), **f32)
+        dmo = (None, None, None) if dm_out is None else tuple(dm_out)
+        mg = _abi.LactBwdMomentum(*(None if x is None else x.data_ptr()
+                                    for x in dmo + (res["dm1"], res["dm2"], res["dm3"])))
+    rc = _abi.lib().lact_ttt_bwd_ex(
+        ctypes.byref(p), None if opts is None else ctypes.byref(opts), None if mg is None else ctypes.byref(mg),
+        _ptr(q), _ptr(k), _ptr(v),
         _ptr(lr), _ptr(beta), _ptr(w1), _ptr(w2), _ptr(w3), _ptr(dout), *(_ptr(x) for x in dw),
         _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dlr"]), _ptr(res["dbeta"]),
         _ptr(res["dw1"]), _ptr(res["dw2"]), _ptr(res["dw3"]), _ptr(res["dout_scale"]),
         _ptr(workspace), ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
     if rc != _abi.LACT_OK:
-        raise LactError(rc, "lact_ttt_bwd")
+        raise LactError(rc, "lact_ttt_bwd_ex")
     return res
 
 

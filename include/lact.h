@@ -256,8 +256,11 @@ size_t lact_ttt_bwd_workspace_bytes(const lact_problem* p);
  * its whole backward in fp32 on the CUDA cores, bf16 inputs included (read
  * as fp32): the iteration's Jacobian magnifies bf16 operand rounding past
  * the bf16 tolerance.  GD and momentum bf16 problems run their contractions
- * on the tensor cores (bf16 operands, fp32 accumulation).  Options: update_mask and out_scale; the
- * momentum buffers and the all-reduce hook are not supported (LACT_EINVAL).
+ * on the tensor cores (bf16 operands, fp32 accumulation).  Options:
+ * update_mask, out_scale, and m1/m2/m3, which the backward READS as the
+ * momentum the forward started from (M_0; the forward overwrote its copy,
+ * so the caller keeps one); their gradient comes from lact_ttt_bwd_ex.  The
+ * all-reduce hook is not supported (LACT_EINVAL).
  * Layouts: the inputs as in lact_ttt_fwd; dout [B,H,Tq,d] in the problem's
  * dtype; dw*_out in the layouts of w*_out, or NULL (zero).  Outputs, all
  * float32 device buffers: dq [B,H,Tq,d], dk, dv [B,H,T,d], dlr [B,H,T,3],
@@ -281,6 +284,38 @@ int lact_ttt_bwd(const lact_problem* p, const lact_fwd_opts* opts,
                  float* dq, float* dk, float* dv, float* dlr, float* dbeta,
                  float* dw1, float* dw2, float* dw3, float* dout_scale,
                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Momentum gradients of the backward (R15 resume, momentum rule): the
+ * gradient with respect to the final momentum the forward wrote into
+ * m1/m2/m3 (dm*_out: all three or none, NULL = zero), and the output, the
+ * gradient with respect to the momentum it started from (dm*: all three
+ * required).  Layouts: dm1, dm3 [B*H, dh, d], dm2 [B*H, d, dh] float32,
+ * 16-byte aligned device buffers, like m1/m2/m3.  Carrying the momentum
+ * back through a masked chunk is the identity; through an updated chunk c,
+ * M_c = mean(beta over c) M_{c-1} + G_c gives dL/dM_{c-1} = mean(beta) dL/dM_c. */
+typedef struct lact_bwd_momentum {
+  const float* dm1_out;
+  const float* dm2_out;
+  const float* dm3_out;
+  float* dm1;
+  float* dm2;
+  float* dm3;
+} lact_bwd_momentum;
+
+/* lact_ttt_bwd that also returns the momentum gradients (`mg`, or NULL for
+ * lact_ttt_bwd's behaviour).  With `mg` the rule must be
+ * LACT_RULE_MOMENTUM; opts->m1/m2/m3 give M_0 (zeros if absent).
+ * LACT_EINVAL also for: only some of the dm* or dm*_out buffers,
+ * misaligned ones, or outputs that overlap any other argument. */
+int lact_ttt_bwd_ex(const lact_problem* p, const lact_fwd_opts* opts, const lact_bwd_momentum* mg,
+                    const void* q, const void* k, const void* v,
+                    const float* lr, const float* beta,
+                    const float* w1, const float* w2, const float* w3,
+                    const void* dout, const float* dw1_out, const float* dw2_out,
+                    const float* dw3_out,
+                    float* dq, float* dk, float* dv, float* dlr, float* dbeta,
+                    float* dw1, float* dw2, float* dw3, float* dout_scale,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* Sliding-window attention, the other half of the LaCT block ([P1 §1.1]):
  * per head and channel learnable scales and offsets on the queries and

@@ -23,7 +23,9 @@ Option inputs (their own generator, so the layer inputs above do not move):
   update mask: the chunk pattern of an autoregressive video sequence whose
       noisy chunks precede each clean one, [noisy x k, clean] repeated
       ("LaCT架构核心思想解析" §3.2: one noisy copy per clean chunk, or two in
-      the teacher-forcing sequence).
+      the teacher-forcing sequence);
+  momentum (m1, m2, m3) in the final weights' layouts ~ N(0, 0.01/row length),
+      a momentum handed in from an earlier call, or a final momentum's gradient.
 """
 from __future__ import annotations
 
@@ -144,6 +146,20 @@ def make_output_grads(w: Workload, seed: int = 0, with_weights: bool = False):
         dws = (torch.randn((BH, w.dh, w.d), generator=g), torch.randn((BH, w.d, w.dh), generator=g),
                torch.randn((BH, w.dh, w.d), generator=g))
     return dout, dws
+
+
+def make_momentum(w: Workload, seed: int = 0):
+    """A seeded momentum state (m1, m2, m3) fp32 in the layouts of the final
+    weights [B*H, dh, d], [B*H, d, dh], [B*H, dh, d]: N(0,1) scaled by
+    0.1/sqrt(row length), rows a tenth of the initial weights' norm (a
+    momentum that leaves the renormalised rows well away from zero); used as
+    a momentum handed in and as the gradient of a final momentum."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(40_000 + seed)
+    BH = w.B * w.H
+    return (0.1 * torch.randn((BH, w.dh, w.d), generator=g) / w.d ** 0.5,
+            0.1 * torch.randn((BH, w.d, w.dh), generator=g) / w.dh ** 0.5,
+            0.1 * torch.randn((BH, w.dh, w.d), generator=g) / w.d ** 0.5)
 
 
 def make_swa_inputs(B: int, H: int, T: int, d: int, seed: int = 0) -> dict:

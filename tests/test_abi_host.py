@@ -181,8 +181,26 @@ def test_backward_and_attention_arguments_are_checked_without_a_gpu():
     # the Muon backward keeps every chunk's direction and the Newton-Schulz iterates
     assert _abi.bwd_workspace_bytes(_prob(WORKLOADS[1], rule=2)) > _abi.bwd_workspace_bytes(gd)
     call = lambda p, o, a: lib.lact_ttt_bwd(ctypes.byref(p), o, *a, ws, big, None)
-    m_opts = _abi.LactFwdOpts(None, None, 13 * G, 14 * G, 15 * G)
-    assert call(_prob(WORKLOADS[1], rule=1), ctypes.byref(m_opts), ptrs) == ct.LACT_EINVAL
+    # momentum in/out (lact_ttt_bwd_ex): M_0 in opts, the gradients in a
+    # lact_bwd_momentum; every buffer in a slot of its own
+    mom = _prob(WORKLOADS[1], rule=1)
+    m_in = _abi.LactFwdOpts(None, None, 30 * G, 31 * G, 32 * G)
+    mg_ok = _abi.LactBwdMomentum(33 * G, 34 * G, 35 * G, 36 * G, 37 * G, 38 * G)
+    call_ex = lambda p, o, mg, a: lib.lact_ttt_bwd_ex(ctypes.byref(p), o, mg, *a, ws, big, None)
+    assert call_ex(gd, None, ctypes.byref(mg_ok), ptrs) == ct.LACT_EINVAL        # momentum grads with GD
+    assert call(gd, ctypes.byref(m_in), ptrs) == ct.LACT_EINVAL                  # M_0 with GD
+    some = _abi.LactFwdOpts(None, None, 30 * G, 0, 32 * G)
+    assert call(mom, ctypes.byref(some), ptrs) == ct.LACT_EINVAL                 # only some of M_0
+    for bad_mg in (_abi.LactBwdMomentum(33 * G, 34 * G, 35 * G, 36 * G, 0, 38 * G),   # a dM_0 missing
+                   _abi.LactBwdMomentum(33 * G, 0, 35 * G, 36 * G, 37 * G, 38 * G),   # only some dM_final
+                   _abi.LactBwdMomentum(33 * G, 34 * G, 35 * G, 36 * G + 8, 37 * G, 38 * G),  # misaligned
+                   _abi.LactBwdMomentum(33 * G, 34 * G, 35 * G, 13 * G, 37 * G, 38 * G),  # dM_0 on dq
+                   _abi.LactBwdMomentum(33 * G, 34 * G, 35 * G, 30 * G, 37 * G, 38 * G),  # dM_0 on M_0
+                   _abi.LactBwdMomentum(33 * G, 34 * G, 35 * G, 36 * G, 36 * G, 38 * G)):  # dM_0s overlap
+        assert call_ex(mom, ctypes.byref(m_in), ctypes.byref(bad_mg), ptrs) == ct.LACT_EINVAL
+    hook = _abi.LactFwdOpts(None, None, None, None, None)
+    hook.allreduce = _abi.ALLREDUCE_FN(lambda *a: 0)
+    assert call(mom, ctypes.byref(hook), ptrs) == ct.LACT_EINVAL                 # no all-reduce hook
     bad = list(ptrs)
     bad[0] = ctypes.c_void_p(0)                                                # q missing
     assert call(gd, None, bad) == ct.LACT_EINVAL

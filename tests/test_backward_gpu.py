@@ -17,13 +17,13 @@ import chunk_test_b200 as ct
 from oracle import lact_oracle_bwd as ob
 from lact_inputs import (APPLY_THEN_UPDATE, BF16, F32, RULE_GD, RULE_MOMENTUM, RULE_MUON,
                          UPDATE_THEN_APPLY,
-                         WORKLOADS, Workload, make_inputs, make_out_scale, make_output_grads,
-                         video_update_mask)
+                         WORKLOADS, Workload, make_inputs, make_momentum, make_out_scale,
+                         make_output_grads, video_update_mask)
 
 pytestmark = pytest.mark.gpu
 
 TOL = {F32: 1e-4, BF16: 2e-2}
-NAMES = ("dq", "dk", "dv", "dlr", "dbeta", "dw1", "dw2", "dw3", "dout_scale")
+NAMES = ("dq", "dk", "dv", "dlr", "dbeta", "dw1", "dw2", "dw3", "dout_scale", "dm1", "dm2", "dm3")
 
 
 def rel_l2(got, want):
@@ -32,22 +32,32 @@ def rel_l2(got, want):
     return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
 
 
-def run_both(w, seed, *, per_bh=False, mask=None, scaled=False, with_dw=False, heads=None):
+def run_both(w, seed, *, per_bh=False, mask=None, scaled=False, with_dw=False, heads=None, m_in=False,
+             dm=False, mgrads=False):
     inp = make_inputs(w, seed=seed)
     if per_bh:
         for n in ("w1", "w2", "w3"):
             inp[n] = torch.cat([inp[n] * (1.0 + 0.1 * b) for b in range(w.B)], dim=0).contiguous()
     dout, dws = make_output_grads(w, seed=seed, with_weights=with_dw)
     scale = make_out_scale(w, seed=seed) if scaled else None
+    m0 = make_momentum(w, seed=seed) if m_in else None
+    dmf = make_momentum(w, seed=seed + 1) if dm else None
     dev = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
     got = ct.ttt_bwd(dev["q"], dev["k"], dev["v"], dev["lr"], dev["beta"], dev["w1"], dev["w2"],
                      dev["w3"], w.chunk, w.order, w.rule, dout.cuda(),
                      dw_out=None if dws is None else tuple(x.cuda() for x in dws),
-                     update_mask=mask, out_scale=None if scale is None else scale.cuda())
+                     update_mask=mask, out_scale=None if scale is None else scale.cuda(),
+                     m_in=None if m0 is None else tuple(x.cuda() for x in m0),
+                     dm_out=None if dmf is None else tuple(x.cuda() for x in dmf), momentum_grads=mgrads)
     assert ct.status() == ct.LACT_OK
     want = ob.ttt_layer_bwd(inp["q"], inp["k"], inp["v"], inp["lr"], inp["beta"], inp["w1"],
                             inp["w2"], inp["w3"], w.chunk, w.order, w.rule, dout, dw=dws,
-                            update_mask=mask, out_scale=scale, heads=heads)
+                            update_mask=mask, out_scale=scale, heads=heads, m_in=m0, dm=dmf)
+    if mgrads and want.get("dm1") is None:   # the gradient of a zero M_0 (the oracle's zeros)
+        want = ob.ttt_layer_bwd(inp["q"], inp["k"], inp["v"], inp["lr"], inp["beta"], inp["w1"],
+                                inp["w2"], inp["w3"], w.chunk, w.order, w.rule, dout, dw=dws,
+                                update_mask=mask, out_scale=scale, heads=heads,
+                                m_in=tuple(torch.zeros_like(x) for x in make_momentum(w, seed=seed)))
     return got, want
 
 
@@ -81,6 +91,13 @@ CASES = [
               RULE_MOMENTUM, BF16), dict(mask=video_update_mask(6, 1), scaled=True, with_dw=True)),
     (Workload("bwd-bf16-d384-uta-ragged", 1, 1, 1100, 1100, 384, 768, 512, UPDATE_THEN_APPLY, RULE_GD,
               BF16), dict(mask=[1, 0, 1], per_bh=True)),
+    # momentum handed in and out (M_0 in, dL/dM_final in, dL/dM_0 out)
+    (Workload("bwd-f32-atu-mom-inout", 1, 2, 768, 768, 64, 128, 256, APPLY_THEN_UPDATE, RULE_MOMENTUM, F32),
+     dict(m_in=True, dm=True, with_dw=True, mask=[1, 0, 1])),
+    (Workload("bwd-bf16-d128-uta-mom-inout", 1, 2, 1024, 1024, 128, 256, 256, UPDATE_THEN_APPLY,
+              RULE_MOMENTUM, BF16), dict(m_in=True, dm=True, per_bh=True)),
+    (Workload("bwd-bf16-d256-atu-mom-grads", 1, 2, 1536, 1536, 256, 512, 512, APPLY_THEN_UPDATE,
+              RULE_MOMENTUM, BF16), dict(mgrads=True, scaled=True)),
     # Muon: the vector-Jacobian product through five Newton-Schulz steps and
     # the Frobenius normalisation, in fp32 on both launch paths.
     (Workload("bwd-f32-atu-muon", 1, 2, 768, 768, 64, 128, 256, APPLY_THEN_UPDATE, RULE_MUON, F32),
