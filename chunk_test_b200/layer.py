@@ -118,8 +118,8 @@ class _CudaBuf:
 
 def _hook(py_fn, device, errors: list):
     """C hook (lact_allreduce_fn) around py_fn(buf, op, stream): buf is a
-    float32 tensor aliasing the library's buffer, op REDUCE_SUM or
-    REDUCE_MEAN, stream the torch stream of the call.  An exception is kept
+    float32 tensor aliasing the library's buffer, op the reduction (the
+    library asks for REDUCE_SUM only), stream the torch stream of the call.  An exception is kept
     in `errors` and reported to the library as a failure."""
 
     def c_fn(ptr, count, op, stream_ptr, user):

@@ -126,8 +126,10 @@ int lact_ttt_fwd(const lact_problem* p,
  * work already enqueued on `stream`:
  *   - after each chunk's gradient, on its partial gradient planes, op SUM
  *     (the summed gradient is then the whole chunk's);
- *   - once before the chunk loop (momentum rule), on the per-chunk means of
- *     beta [B*H, nchunks], op MEAN (equal shares: the mean of the means).
+ *   - once before the chunk loop (momentum rule), on the per-chunk sums of
+ *     beta and their token counts [2, B*H, nchunks], op SUM (the library
+ *     then divides each sum by its count on the device: the mean of beta
+ *     over the whole chunk).
  * The hook must reduce the buffer in place over the ranks so that work
  * enqueued on `stream` after it returns sees the result (for example NCCL on
  * that stream), and return 0; any other value stops the call with
@@ -136,6 +138,8 @@ int lact_ttt_fwd(const lact_problem* p,
  * its own queries.  Every rank must make the same sequence of calls with
  * the same problem shape and options (the hook is called the same number of
  * times with the same counts on every rank). */
+/* Reduction ops a hook may be asked for.  The library asks for SUM only;
+ * MEAN is kept so that hooks written against it keep their meaning. */
 enum { LACT_REDUCE_SUM = 0, LACT_REDUCE_MEAN = 1 };
 typedef int (*lact_allreduce_fn)(float* data, int64_t count, int op, void* stream, void* user);
 
