@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(256) k_rowdot(const float* __restrict__ a, con
 
 struct RenormBwdParams {
   const float* A;       // dL/dW^c            [3][BH][plane]
+  float* A2;            // or null: a second part of dL/dW^c (the ranks' summed
+                        // own contributions), added to A and then cleared
   const float* Wc;      // W^c (after renorm)
   const float* Wp;      // W^{c-1}
   const float* mnorm;   // |W'_r| per row (rule row order)
@@ -91,7 +93,7 @@ __global__ void __launch_bounds__(256) k_renorm_bwd(const RenormBwdParams p) {
   for (int c = lane; c < r.len; c += 32) {
     const int64_t o = r.base + c;
     nn += p.Wp[o] * p.Wp[o];
-    wa += p.Wc[o] * p.A[o];
+    wa += p.Wc[o] * (p.A2 ? p.A[o] + p.A2[o] : p.A[o]);
   }
   nn = warp_sum(nn);
   wa = warp_sum(wa);
@@ -105,7 +107,12 @@ __global__ void __launch_bounds__(256) k_renorm_bwd(const RenormBwdParams p) {
   for (int c = lane; c < r.len; c += 32) {
     const int64_t o = r.base + c;
     const float u = p.Wc[o] * inv_n;
-    const float D = g * (p.A[o] - u * dot);
+    float a = p.A[o];
+    if (p.A2) {
+      a += p.A2[o];
+      p.A2[o] = 0.f;
+    }
+    const float D = g * (a - u * dot);
     p.Ap[o] = D + dot * p.Wp[o] * inv_n;
     float gam;
     if (p.rule == 1) {
@@ -126,9 +133,12 @@ __global__ void __launch_bounds__(256) k_renorm_bwd(const RenormBwdParams p) {
 }
 
 // Momentum: dL/dbeta_bar_c = sum over the head's rows of <E, M^{c-1}>, spread
-// over the chunk's tokens (beta_bar is their mean).  One block per head.
+// over the chunk's tokens (beta_bar is their mean): n local tokens, of
+// count[bh] in the whole chunk (the ranks' summed counts under context
+// parallelism; n when count is null).  One block per head.
 __global__ void __launch_bounds__(256) k_head_dbeta(const float* __restrict__ part, int BH, int dh,
                                                     int d, int64_t T, int64_t c0, int n,
+                                                    const float* __restrict__ count, int64_t count_stride,
                                                     float* __restrict__ dbeta) {
   griddep_launch();
   griddep_wait();
@@ -149,7 +159,7 @@ __global__ void __launch_bounds__(256) k_head_dbeta(const float* __restrict__ pa
     if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
     __syncthreads();
   }
-  const float per = red[0] / static_cast<float>(n);
+  const float per = red[0] / (count ? count[bh * count_stride] : static_cast<float>(n));
   for (int t = threadIdx.x; t < n; t += 256) dbeta[static_cast<int64_t>(bh) * T + c0 + t] = per;
 }
 
@@ -368,6 +378,24 @@ __global__ void __launch_bounds__(256) k_sum_batch(const float* __restrict__ A, 
       acc = src[hw * plane + off];
     }
     (j == 0 ? d1 : (j == 1 ? d2 : d3))[e] = acc;
+  }
+}
+
+// A += B over n floats (16-byte steps when n is a multiple of 4).
+__global__ void __launch_bounds__(256) k_add_planes(float* __restrict__ A, const float* __restrict__ B, int64_t n) {
+  griddep_launch();
+  griddep_wait();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (n % 4 == 0) {
+    for (int64_t i = t0; i < n / 4; i += stride) {
+      float4 a = reinterpret_cast<float4*>(A)[i];
+      const float4 b = reinterpret_cast<const float4*>(B)[i];
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+      reinterpret_cast<float4*>(A)[i] = a;
+    }
+  } else {
+    for (int64_t i = t0; i < n; i += stride) A[i] += B[i];
   }
 }
 

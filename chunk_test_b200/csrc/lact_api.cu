@@ -1287,7 +1287,6 @@ int lact_ttt_bwd_ex(const lact_problem* p, const lact_fwd_opts* opts, const lact
   Dims D;
   int rc = validate(p, D);
   if (rc != LACT_OK) return rc;
-  if (opts && opts->allreduce) return LACT_EINVAL;
   const float* scale = opts ? opts->out_scale : nullptr;
   const bool mom = D.rule == LACT_RULE_MOMENTUM;
   const float* m0[3] = {opts ? opts->m1 : nullptr, opts ? opts->m2 : nullptr, opts ? opts->m3 : nullptr};
@@ -1337,7 +1336,8 @@ int lact_ttt_bwd_ex(const lact_problem* p, const lact_fwd_opts* opts, const lact
   plan_bwd(D, bp, b);
   BwdInputs in{q, k, v, lr, beta, w1, w2, w3, dout, dw1_out, dw2_out, dw3_out,
                opts ? opts->update_mask : nullptr, scale, dq, dk, dv, dlr, dbeta, dw1, dw2, dw3, dout_scale,
-               {m0[0], m0[1], m0[2]}, {dmf[0], dmf[1], dmf[2]}, {dm0[0], dm0[1], dm0[2]}};
+               {m0[0], m0[1], m0[2]}, {dmf[0], dmf[1], dmf[2]}, {dm0[0], dm0[1], dm0[2]},
+               opts ? opts->allreduce : nullptr, opts ? opts->allreduce_user : nullptr};
   Launcher L{false, static_cast<cudaStream_t>(stream)};
   run_bwd(D, b, in, static_cast<cudaStream_t>(stream), L);
   return L.err;

@@ -25,6 +25,15 @@
 // direction as GD applies S, so the renorm backward's GD output is the
 // gradient with respect to that direction in GD's sign, and the (linear) VJP
 // carries it to the gradient with respect to the chunk's gradient.
+// Context parallelism (the all-reduce hook): every rank holds the same
+// states, so dL/dW^c is the sum over the ranks of their own contributions
+// (the apply's backward on their queries, the chunk gradient's
+// second-order terms on their keys, their dL/dw_out) plus the part carried
+// through the renorm backward, which every rank computes alike from the
+// summed gradient.  The own contributions accumulate in Aloc, are summed
+// over the ranks before each renorm backward (which reads and clears them)
+// and once after the loop; the recompute sums each chunk's gradient and the
+// beta sums and counts as the forward does.
 // fp32 problems run every contraction as a batched k_simt_gemm over the B*H
 // heads in fp32.  bf16 problems run them on the tensor cores (GemmOp, bf16
 // operands through TMA, fp32 accumulation); the elementwise kernels write
@@ -48,6 +57,8 @@ struct BwdInputs {
   const float* m0[3];    // momentum: M_0 (the layouts of w*_out), or null (zeros)
   const float* dmf[3];   // momentum: dL/dM_final, or null (zero)
   float* dm0[3];         // momentum: out dL/dM_0, or null
+  lact_allreduce_fn allreduce;   // context parallelism: the ranks' sum, or null
+  void* allreduce_user;
 };
 
 struct BwdBufs {
@@ -55,6 +66,7 @@ struct BwdBufs {
   float *hist, *mh, *Mm, *mnorm, *bbar;
   float *Z, *Pz, *E, *P;
   float *A, *Ap, *Gam, *Bm;
+  float* Aloc;   // context parallelism: this rank's own contributions to dL/dW
   float *dqh, *dkh, *ofull, *part;
   // bf16 problems (tensor-core contractions): bf16 operands
   __nv_bfloat16 *qh16, *kh16, *dos16, *hist16, *op16, *Gam16;
@@ -108,7 +120,7 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
   if (mom) {
     b.mh = bp.take<float>(D.nch * planes);
     b.Mm = bp.take<float>(planes);
-    b.bbar = bp.take<float>(D.BH * D.nch);
+    b.bbar = bp.take<float>(2 * D.BH * D.nch);   // means, then (context parallel) token counts
     b.Bm = bp.take<float>(planes);
     b.part = bp.take<float>(rule_rows(D));
   }
@@ -130,6 +142,7 @@ static void plan_bwd(const Dims& D, Bump& bp, BwdBufs& b) {
   }
   b.P = bp.take<float>(planes);
   b.A = bp.take<float>(planes);
+  b.Aloc = bp.take<float>(planes);
   b.Ap = bp.take<float>(planes);
   b.dqh = bp.take<float>(nq);
   b.dkh = bp.take<float>(nk);
@@ -287,6 +300,12 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
   auto copy = [&](void* dst, const void* src, int64_t bytes) {
     if (!L.dry) memop(cudaMemcpyAsync(dst, src, static_cast<size_t>(bytes), cudaMemcpyDeviceToDevice, st));
   };
+  const bool cp = in.allreduce != nullptr;
+  auto reduce = [&](float* data, int64_t count) {   // in place over the ranks, op SUM
+    if (!cp || L.dry || L.err != LACT_OK) return;
+    if (in.allreduce(data, count, LACT_REDUCE_SUM, static_cast<void*>(st), in.allreduce_user) != 0)
+      L.err = LACT_ECOMM;
+  };
   // one batched fp32 GEMM over the heads (see k_simt_gemm for the indexing)
   auto gemm = [&](const float* A, int64_t a_item, int64_t a_m, int64_t a_k, const float* B, int64_t b_item,
                   int64_t b_n, int64_t b_k, int M, int N, int K, float* out, int64_t out_item, int64_t ld,
@@ -338,10 +357,13 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
       else zero(b.Bm + j * jst, jst * 4);
     }
   }
+  if (mom && in.dmf[0]) reduce(b.Bm, planes);   // the ranks' gradients of the final momentum
   const float* dwf[3] = {in.dw1f, in.dw2f, in.dw3f};
+  float* dw_init = cp ? b.Aloc : b.A;   // dL/dw_out is this rank's own
+  if (cp) zero(b.A, planes * 4);
   for (int j = 0; j < 3; ++j) {
-    if (dwf[j]) copy(b.A + j * jst, dwf[j], jst * 4);
-    else zero(b.A + j * jst, jst * 4);
+    if (dwf[j]) copy(dw_init + j * jst, dwf[j], jst * 4);
+    else zero(dw_init + j * jst, jst * 4);
   }
 
   // ---- forward recompute: q^, k^ (fp32), initial state, beta means
@@ -365,13 +387,20 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
                      in.m0[0], in.m0[1], in.m0[2]);
     return cudaGetLastError();
   });
-  if (mom) {
+  if (mom) {   // per-chunk beta means (context parallel: sums and counts over the ranks)
+    const int64_t w = D.BH * D.nch;
     L(K_BETA_MEAN, [&] {
-      const int64_t w = D.BH * D.nch;
       (void)launch_pdl(k_beta_mean, static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st, in.beta, BH, D.T,
-                       D.chunk, static_cast<int>(D.nch), b.bbar, 0);
+                       D.chunk, static_cast<int>(D.nch), b.bbar, cp ? 1 : 0);
       return cudaGetLastError();
     });
+    if (cp) {
+      reduce(b.bbar, 2 * w);
+      L(K_BETA_MEAN, [&] {
+        (void)launch_pdl(k_beta_div, static_cast<unsigned>(cdiv(w, 256)), 256, 0, st, b.bbar, w);
+        return cudaGetLastError();
+      });
+    }
   }
   // the keys' forward at state W: Z = (k^ W1^T, v W2, k^ W3^T), rows of chunk c
   auto key_forward = [&](const float* W, int64_t c0, int nc, float* Zout) {
@@ -403,6 +432,7 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
       if (!muon) { s.tr_group = 1; s.tr_mod = BH; s.ld_t = dh; }   // Muon keeps [dh, d] planes
       return simt(s, 3 * BH, st);
     });
+    reduce(b.P, planes);   // the whole chunk's gradient
     if (muon) muon_forward_step(D, b, c, st, L);
     L(K_RULE, [&] {
       RuleParams r;
@@ -429,11 +459,12 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
       (void)launch_pdl(k_apply_bwd_elem, grid_for(zpl, 4), 256, 0, st, b.Z, zpl);
       return cudaGetLastError();
     });
-    // dW1 += dz1^T q^, dW3 += dz3^T q^, dW2 += dO^T hq
+    // dW1 += dz1^T q^, dW3 += dz3^T q^, dW2 += dO^T hq (this rank's own part)
+    float* Aq = cp ? b.Aloc : A;
     for (int j = 0; j < 3; j += 2)
-      gemm(b.Z + j * zpl, zr * D.dh, 1, dh, b.qh + qr0 * d, D.Tq * D.d, 1, d, dh, d, nq_c, A + j * jst, plane, d,
+      gemm(b.Z + j * zpl, zr * D.dh, 1, dh, b.qh + qr0 * d, D.Tq * D.d, 1, d, dh, d, nq_c, Aq + j * jst, plane, d,
            true);
-    gemm(dos + qr0 * d, D.Tq * D.d, 1, d, b.Z + zpl, zr * D.dh, 1, dh, d, dh, nq_c, A + jst, plane, dh, true);
+    gemm(dos + qr0 * d, D.Tq * D.d, 1, d, b.Z + zpl, zr * D.dh, 1, dh, d, dh, nq_c, Aq + jst, plane, dh, true);
     // dq^ += dz1 W1 + dz3 W3
     for (int j = 0; j < 3; j += 2)
       gemm(b.Z + j * zpl, zr * D.dh, dh, 1, W + j * jst, plane, 1, d, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d,
@@ -452,10 +483,11 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
     const bool upd = !in.mask || in.mask[c] != 0;
     if (D.order == LACT_UPDATE_THEN_APPLY) apply_bwd(Wc, qr0, nq_c);
     if (upd) {
+      reduce(b.Aloc, planes);   // the ranks' own contributions to dL/dW^c
       L(K_BWD_ELEM, [&] {
         RenormBwdParams r;
         std::memset(&r, 0, sizeof(r));
-        r.A = A; r.Wc = Wc; r.Wp = Wp; r.mnorm = b.mnorm + c * rows_all; r.Gam = b.Gam; r.Ap = Ap;
+        r.A = A; r.A2 = cp ? b.Aloc : nullptr; r.Wc = Wc; r.Wp = Wp; r.mnorm = b.mnorm + c * rows_all; r.Gam = b.Gam; r.Ap = Ap;
         r.rule = muon ? LACT_RULE_GD : D.rule; r.Bm = b.Bm; r.Mprev = mom ? b.mh + c * planes : nullptr;
         r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch); r.chunk_idx = static_cast<int>(c); r.part = b.part;
         r.BH = BH; r.dh = dh; r.d = d;
@@ -466,7 +498,7 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
       if (mom)
         L(K_BWD_ELEM, [&] {
           (void)launch_pdl(k_head_dbeta, static_cast<unsigned>(BH), 256, 0, st, b.part, BH, dh, d, D.T, c0, nc,
-                           in.dbeta);
+                           cp ? static_cast<const float*>(b.bbar + D.BH * D.nch + c) : nullptr, D.nch, in.dbeta);
           return cudaGetLastError();
         });
       // the keys' forward at W^{c-1}, and (p, q, r) = (k^ Gam1^T, v Gam2, k^ Gam3^T)
@@ -477,11 +509,12 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
                          zr, dh, nc, in.lr, D.T, c0, in.dlr);
         return cudaGetLastError();
       });
-      // dW1 += dz1^T k^, dW3 += dz3^T k^, dW2 += v^T du
+      // dW1 += dz1^T k^, dW3 += dz3^T k^, dW2 += v^T du (this rank's own part)
+      float* Ak = cp ? b.Aloc : Ap;
       for (int j = 0; j < 3; j += 2)
-        gemm(b.Z + j * zpl, zr * D.dh, 1, dh, b.kh + c0 * d, D.T * D.d, 1, d, dh, d, nc, Ap + j * jst, plane, d,
+        gemm(b.Z + j * zpl, zr * D.dh, 1, dh, b.kh + c0 * d, D.T * D.d, 1, d, dh, d, nc, Ak + j * jst, plane, d,
              true);
-      gemm(v32 + c0 * d, D.T * D.d, 1, d, b.Z + zpl, zr * D.dh, 1, dh, d, dh, nc, Ap + jst, plane, dh, true);
+      gemm(v32 + c0 * d, D.T * D.d, 1, d, b.Z + zpl, zr * D.dh, 1, dh, d, dh, nc, Ak + jst, plane, dh, true);
       // dk^ += dz1 W1 + dz3 W3 + dp Gam1 + dr Gam3
       for (int j = 0; j < 3; j += 2) {
         gemm(b.Z + j * zpl, zr * D.dh, dh, 1, Wp + j * jst, plane, 1, d, nc, d, dh, b.dkh + c0 * d, D.T * D.d, d,
@@ -514,6 +547,13 @@ static void run_bwd_f32(const Dims& D, const BwdBufs& b, const BwdInputs& in, cu
                        in.dscale, D.BH * D.Tq, d);
       return cudaGetLastError();
     });
+  if (cp) {   // the own contributions left after chunk 0, summed over the ranks
+    reduce(b.Aloc, planes);
+    L(K_BWD_ELEM, [&] {
+      (void)launch_pdl(k_add_planes, grid_for(planes, 4), 256, 0, st, A, static_cast<const float*>(b.Aloc), planes);
+      return cudaGetLastError();
+    });
+  }
   L(K_BWD_ELEM, [&] {
     (void)launch_pdl(k_sum_batch, grid_for(planes, 4), 256, 0, st, static_cast<const float*>(A),
                      static_cast<int>(D.B), static_cast<int>(D.H), plane, D.w_shared, in.dw1, in.dw2, in.dw3);
@@ -555,6 +595,12 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
   };
   auto copy = [&](void* dst, const void* src, int64_t bytes) {
     if (!L.dry) memop(cudaMemcpyAsync(dst, src, static_cast<size_t>(bytes), cudaMemcpyDeviceToDevice, st));
+  };
+  const bool cp = in.allreduce != nullptr;
+  auto reduce = [&](float* data, int64_t count) {   // in place over the ranks, op SUM
+    if (!cp || L.dry || L.err != LACT_OK) return;
+    if (in.allreduce(data, count, LACT_REDUCE_SUM, static_cast<void*>(st), in.allreduce_user) != 0)
+      L.err = LACT_ECOMM;
   };
   // out[item] (+)= A(item) B(item)^T with A [M x K], B [N x K] per head, both
   // bf16 through TMA: K-major A read from row a_m0, MN-major operands from K
@@ -639,10 +685,13 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
       else zero(b.Bm + j * jst, jst * 4);
     }
   }
+  if (mom && in.dmf[0]) reduce(b.Bm, planes);   // the ranks' gradients of the final momentum
   const float* dwf[3] = {in.dw1f, in.dw2f, in.dw3f};
+  float* dw_init = cp ? b.Aloc : b.A;   // dL/dw_out is this rank's own
+  if (cp) zero(b.A, planes * 4);
   for (int j = 0; j < 3; ++j) {
-    if (dwf[j]) copy(b.A + j * jst, dwf[j], jst * 4);
-    else zero(b.A + j * jst, jst * 4);
+    if (dwf[j]) copy(dw_init + j * jst, dwf[j], jst * 4);
+    else zero(dw_init + j * jst, jst * 4);
   }
   L(K_PROLOGUE, [&] {
     constexpr int ROWS = 4;
@@ -666,13 +715,20 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
                      in.m0[0], in.m0[1], in.m0[2]);
     return cudaGetLastError();
   });
-  if (mom) {
+  if (mom) {   // per-chunk beta means (context parallel: sums and counts over the ranks)
+    const int64_t w = D.BH * D.nch;
     L(K_BETA_MEAN, [&] {
-      const int64_t w = D.BH * D.nch;
       (void)launch_pdl(k_beta_mean, static_cast<unsigned>(cdiv(w * 32, 256)), 256, 0, st, in.beta, BH, D.T,
-                       D.chunk, static_cast<int>(D.nch), b.bbar, 0);
+                       D.chunk, static_cast<int>(D.nch), b.bbar, cp ? 1 : 0);
       return cudaGetLastError();
     });
+    if (cp) {
+      reduce(b.bbar, 2 * w);
+      L(K_BETA_MEAN, [&] {
+        (void)launch_pdl(k_beta_div, static_cast<unsigned>(cdiv(w, 256)), 256, 0, st, b.bbar, w);
+        return cudaGetLastError();
+      });
+    }
   }
   // The forward's fused key kernel at a state W (bf16): z1 = X W1^T, z3 = X W3^T,
   // g = Y W2 for rows x_row0 .. x_row0 + n of X and Y ([BH][rows][d]), and the
@@ -716,6 +772,7 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
       g.tr_group = 1; g.tr_mod = BH; g.ld_t = dh;
       return launch_gemm<true, true>(bn, dim3(d / bn, cdiv(dh, 128), 3 * BH), g, st);
     });
+    reduce(b.P, planes);   // the whole chunk's gradient
     L(K_RULE, [&] {
       RuleParams r;
       std::memset(&r, 0, sizeof(r));
@@ -757,10 +814,11 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     B16* Ea = b.op16;
     fwd_key(K_BWD_APPLY, W, qh, dos.p, r0, nq_c, nullptr, Ea);
     const Opnd E1{Ea, D.dh, zr, D.BH}, Eh{Ea + zpl, D.dh, zr, D.BH}, E3{Ea + 2 * zpl, D.dh, zr, D.BH};
-    // dW1 += dz1^T q^, dW3 += dz3^T q^, dW2 += dO^T hq
-    tcg(MN, MN, E1, 0, 0, qh, r0, dh, d, nq_c, A, plane, d, true);
-    tcg(MN, MN, E3, 0, 0, qh, r0, dh, d, nq_c, A + 2 * jst, plane, d, true);
-    tcg(MN, MN, dos, 0, r0, Eh, 0, d, dh, nq_c, A + jst, plane, dh, true);
+    // dW1 += dz1^T q^, dW3 += dz3^T q^, dW2 += dO^T hq (this rank's own part)
+    float* Aq = cp ? b.Aloc : A;
+    tcg(MN, MN, E1, 0, 0, qh, r0, dh, d, nq_c, Aq, plane, d, true);
+    tcg(MN, MN, E3, 0, 0, qh, r0, dh, d, nq_c, Aq + 2 * jst, plane, d, true);
+    tcg(MN, MN, dos, 0, r0, Eh, 0, d, dh, nq_c, Aq + jst, plane, dh, true);
     // dq^ += dz1 W1 + dz3 W3
     tcg(KM, MN, E1, 0, 0, Wop(W, 0), 0, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
     tcg(KM, MN, E3, 0, 0, Wop(W, 2), 0, nq_c, d, dh, b.dqh + qr0 * d, D.Tq * D.d, d, true);
@@ -777,10 +835,11 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
     const bool upd = !in.mask || in.mask[c] != 0;
     if (D.order == LACT_UPDATE_THEN_APPLY) apply_bwd(Wc16, qr0, nq_c);
     if (upd) {
+      reduce(b.Aloc, planes);   // the ranks' own contributions to dL/dW^c
       L(K_BWD_ELEM, [&] {
         RenormBwdParams r;
         std::memset(&r, 0, sizeof(r));
-        r.A = A; r.Wc = b.hist + (c + 1) * planes; r.Wp = b.hist + c * planes; r.mnorm = b.mnorm + c * rows_all;
+        r.A = A; r.A2 = cp ? b.Aloc : nullptr; r.Wc = b.hist + (c + 1) * planes; r.Wp = b.hist + c * planes; r.mnorm = b.mnorm + c * rows_all;
         r.Gam16 = b.Gam16; r.Ap = Ap; r.rule = D.rule; r.Bm = b.Bm;
         r.Mprev = mom ? b.mh + c * planes : nullptr; r.beta_bar = b.bbar; r.nch = static_cast<int>(D.nch);
         r.chunk_idx = static_cast<int>(c); r.part = b.part; r.BH = BH; r.dh = dh; r.d = d;
@@ -790,7 +849,7 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
       if (mom)
         L(K_BWD_ELEM, [&] {
           (void)launch_pdl(k_head_dbeta, static_cast<unsigned>(BH), 256, 0, st, b.part, BH, dh, d, D.T, c0, nc,
-                           in.dbeta);
+                           cp ? static_cast<const float*>(b.bbar + D.BH * D.nch + c) : nullptr, D.nch, in.dbeta);
           return cudaGetLastError();
         });
       // stacked operands: Bk = [W1; W3; Gam1; Gam3] [BH][4 dh][d], Bv = [W2 | Gam2] [BH][d][2 dh]
@@ -815,10 +874,11 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
         f.T = D.T; f.lr = in.lr; f.dlr = in.dlr;
         return launch_umma<BwdKeyOp>(static_cast<int64_t>(f.n_slices) * f.n_row_tiles * BH, f, st);
       });
-      // dW1 += dz1^T k^, dW3 += dz3^T k^, dW2 += v^T du
-      tcg(MN, MN, Zk_op, 0, 0, kh, k0, dh, d, nc, Ap, plane, d, true);
-      tcg(MN, MN, Zk_op, dh, 0, kh, k0, dh, d, nc, Ap + 2 * jst, plane, d, true);
-      tcg(MN, MN, vv, 0, k0, Zv_op, 0, d, dh, nc, Ap + jst, plane, dh, true);
+      // dW1 += dz1^T k^, dW3 += dz3^T k^, dW2 += v^T du (this rank's own part)
+      float* Ak = cp ? b.Aloc : Ap;
+      tcg(MN, MN, Zk_op, 0, 0, kh, k0, dh, d, nc, Ak, plane, d, true);
+      tcg(MN, MN, Zk_op, dh, 0, kh, k0, dh, d, nc, Ak + 2 * jst, plane, d, true);
+      tcg(MN, MN, vv, 0, k0, Zv_op, 0, d, dh, nc, Ak + jst, plane, dh, true);
       // dk^ += [dz1|dz3|dp|dr] [W1; W3; Gam1; Gam3],  dv += [du|dq] [W2 | Gam2]^T
       tcg(KM, MN, Zk_op, 0, 0, Bk_op, 0, nc, d, 4 * dh, b.dkh + c0 * d, D.T * D.d, d, true);
       tcg(KM, KM, Zv_op, 0, 0, Opnd{b.Bv, dh2, D.d, D.BH}, 0, nc, d, 2 * dh, in.dv + c0 * d, D.T * D.d, d, true);
@@ -845,6 +905,13 @@ static void run_bwd_tc(const Dims& D, const BwdBufs& b, const BwdInputs& in, cud
                        D.BH * D.Tq, d);
       return cudaGetLastError();
     });
+  if (cp) {   // the own contributions left after chunk 0, summed over the ranks
+    reduce(b.Aloc, planes);
+    L(K_BWD_ELEM, [&] {
+      (void)launch_pdl(k_add_planes, grid_for(planes, 4), 256, 0, st, A, static_cast<const float*>(b.Aloc), planes);
+      return cudaGetLastError();
+    });
+  }
   L(K_BWD_ELEM, [&] {
     (void)launch_pdl(k_sum_batch, grid_for(planes, 4), 256, 0, st, static_cast<const float*>(A),
                      static_cast<int>(D.B), static_cast<int>(D.H), plane, D.w_shared, in.dw1, in.dw2, in.dw3);

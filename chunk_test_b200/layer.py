@@ -259,7 +259,7 @@ def _check_momentum(name, ms, q, dh, d):
 
 def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=None,
             update_mask=None, out_scale=None, m_in=None, dm_out=None, momentum_grads=False,
-            workspace=None, stream=None):
+            allreduce=None, workspace=None, stream=None):
     """The layer's backward on the current CUDA device (lact_ttt_bwd, or
     lact_ttt_bwd_ex for the momentum gradients): the gradients of a loss
     given dL/d out (`dout`, like q) and optionally dL/d w_out (`dw_out`,
@@ -270,8 +270,12 @@ def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=N
     (the three tensors its m_inout held before the call), `dm_out` the
     gradient of the final momentum it wrote; with either given or
     `momentum_grads` set the dict also holds dm1, dm2, dm3, the gradients
-    of m_in.  On bf16 inputs some fp32 sums are accumulated with atomic
-    adds, so repeated calls can differ in the last bits."""
+    of m_in.  `allreduce`: the context-parallel hook of ttt_fwd; each rank
+    passes its own tokens (and its own dout, dw_out and dm_out, the
+    gradients of its share of the loss) and gets the gradients of its own
+    tokens and, alike on every rank, of the shared initial state.  On bf16
+    inputs some fp32 sums are accumulated with atomic adds, so repeated
+    calls can differ in the last bits."""
     _check(q, k, v, lr, beta, w1, w2, w3, "cuda")
     if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_contiguous():
         raise ValueError("dout must be a contiguous tensor shaped like q, in q's dtype")
@@ -282,7 +286,8 @@ def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=N
         _check_momentum("dm_out", dm_out, q, dh, d)
     want_dm = momentum_grads or m_in is not None or dm_out is not None
     p = make_problem(q, k, w1, chunk, order, rule)
-    opts, _keep = _options(p, update_mask, out_scale, m_in, q)
+    errors = []
+    opts, _keep = _options(p, update_mask, out_scale, m_in, q, allreduce, errors)
     f32 = dict(device=q.device, dtype=torch.float32)
     res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
            "dv": torch.empty(v.shape, **f32), "dlr": torch.empty(lr.shape, **f32),
@@ -314,6 +319,8 @@ def ttt_bwd(q, k, v, lr, beta, w1, w2, w3, chunk, order, rule, dout, *, dw_out=N
         _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dlr"]), _ptr(res["dbeta"]),
         _ptr(res["dw1"]), _ptr(res["dw2"]), _ptr(res["dw3"]), _ptr(res["dout_scale"]),
         _ptr(workspace), ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
+    if errors:
+        raise errors[0]
     if rc != _abi.LACT_OK:
         raise LactError(rc, "lact_ttt_bwd_ex")
     return res

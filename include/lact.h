@@ -261,10 +261,19 @@ size_t lact_ttt_bwd_workspace_bytes(const lact_problem* p);
  * as fp32): the iteration's Jacobian magnifies bf16 operand rounding past
  * the bf16 tolerance.  GD and momentum bf16 problems run their contractions
  * on the tensor cores (bf16 operands, fp32 accumulation).  Options:
- * update_mask, out_scale, and m1/m2/m3, which the backward READS as the
+ * update_mask, out_scale, m1/m2/m3, which the backward READS as the
  * momentum the forward started from (M_0; the forward overwrote its copy,
- * so the caller keeps one); their gradient comes from lact_ttt_bwd_ex.  The
- * all-reduce hook is not supported (LACT_EINVAL).
+ * so the caller keeps one; their gradient comes from lact_ttt_bwd_ex), and
+ * the all-reduce hook.  Context parallelism: each rank passes the inputs of
+ * its forward call and the gradients of its own share of the loss (dout for
+ * its queries, its part of dw*_out and dm*_out); it gets the gradients of
+ * its own tokens, and the gradients of the shared initial weights and
+ * momentum, the same on every rank.  The hook is called (op SUM) on each
+ * updated chunk's gradient and the beta sums and counts, as in the
+ * forward's recompute; then in the reverse loop before each updated
+ * chunk's renorm backward and once after the loop, on the ranks' own
+ * contributions to the weights' gradient [3*B*H*d*dh floats]; and once on
+ * dm*_out when given.
  * Layouts: the inputs as in lact_ttt_fwd; dout [B,H,Tq,d] in the problem's
  * dtype; dw*_out in the layouts of w*_out, or NULL (zero).  Outputs, all
  * float32 device buffers: dq [B,H,Tq,d], dk, dv [B,H,T,d], dlr [B,H,T,3],

@@ -198,9 +198,6 @@ def test_backward_and_attention_arguments_are_checked_without_a_gpu():
                    _abi.LactBwdMomentum(33 * G, 34 * G, 35 * G, 30 * G, 37 * G, 38 * G),  # dM_0 on M_0
                    _abi.LactBwdMomentum(33 * G, 34 * G, 35 * G, 36 * G, 36 * G, 38 * G)):  # dM_0s overlap
         assert call_ex(mom, ctypes.byref(m_in), ctypes.byref(bad_mg), ptrs) == ct.LACT_EINVAL
-    hook = _abi.LactFwdOpts(None, None, None, None, None)
-    hook.allreduce = _abi.ALLREDUCE_FN(lambda *a: 0)
-    assert call(mom, ctypes.byref(hook), ptrs) == ct.LACT_EINVAL                 # no all-reduce hook
     bad = list(ptrs)
     bad[0] = ctypes.c_void_p(0)                                                # q missing
     assert call(gd, None, bad) == ct.LACT_EINVAL

@@ -13,6 +13,12 @@ another; every barrier has a timeout, so a rank that fails ends the test
 instead of hanging it.  Checked: the ranks' outputs, put back in token
 order, and the final weights match the unsharded oracle within the usual
 tolerances, and both ranks end with bit-identical weights.
+
+The backward under the same sharding: each rank's loss is its queries'
+<out, dout> plus its share of <w_out, dw> and <m_out, dm>; the ranks'
+gradients of their own tokens, put back in token order, and their gradients
+of the shared initial state (both ranks alike, bit for bit) match the
+unsharded autograd oracle.
 """
 import threading
 
@@ -22,8 +28,9 @@ import torch
 
 import chunk_test_b200 as ct
 import oracle
+from oracle import lact_oracle_bwd as ob
 from lact_inputs import (APPLY_THEN_UPDATE, BF16, F32, RULE_GD, RULE_MOMENTUM, RULE_MUON,
-                         UPDATE_THEN_APPLY, Workload, make_inputs)
+                         UPDATE_THEN_APPLY, Workload, make_inputs, make_momentum, make_output_grads)
 
 pytestmark = pytest.mark.gpu
 
@@ -143,3 +150,88 @@ def test_two_ranks_match_the_unsharded_layer(w):
     for j, name in enumerate(("w1", "w2", "w3")):
         errs[name] = rel_l2(results[0][1 + j].numpy(), want[1 + j])
     assert max(errs.values()) <= TOL[w.dtype], errs
+
+
+BWD_CASES = [
+    (Workload("cp-bwd-f32-gd-causal", 1, 2, 1024, 1024, 64, 128, 256, APPLY_THEN_UPDATE, RULE_GD, F32), {}),
+    (Workload("cp-bwd-f32-momentum-uta", 2, 1, 768, 768, 32, 64, 256, UPDATE_THEN_APPLY, RULE_MOMENTUM, F32),
+     dict(mask=[1, 0, 1], mom_io=True)),
+    (Workload("cp-bwd-f32-muon", 1, 2, 768, 768, 64, 128, 256, APPLY_THEN_UPDATE, RULE_MUON, F32), {}),
+    (Workload("cp-bwd-bf16-d256-causal", 1, 2, 2048, 2048, 256, 512, 512, APPLY_THEN_UPDATE, RULE_GD, BF16),
+     {}),
+    (Workload("cp-bwd-bf16-d128-momentum", 1, 2, 1536, 1536, 128, 256, 512, APPLY_THEN_UPDATE,
+              RULE_MOMENTUM, BF16), dict(mom_io=True)),
+    (Workload("cp-bwd-bf16-d64-set", 1, 2, 2048, 512, 64, 128, 2048, UPDATE_THEN_APPLY, RULE_GD, BF16), {}),
+]
+
+
+@pytest.mark.parametrize("w,kw", BWD_CASES, ids=lambda x: x.name if hasattr(x, "name") else "")
+def test_two_ranks_backward_matches_the_unsharded_gradients(w, kw):
+    world = 2
+    mask, mom_io = kw.get("mask"), kw.get("mom_io", False)
+    inp = make_inputs(w, seed=23)
+    dout, dws = make_output_grads(w, seed=23, with_weights=True)
+    m_in = make_momentum(w, seed=23) if mom_io else None
+    dm = make_momentum(w, seed=24) if mom_io else None
+    want = ob.ttt_layer_bwd(inp["q"], inp["k"], inp["v"], inp["lr"], inp["beta"], inp["w1"], inp["w2"],
+                            inp["w3"], w.chunk, w.order, w.rule, dout, dw=dws, update_mask=mask,
+                            m_in=m_in, dm=dm)
+    single = w.chunk >= w.T
+    kidx = [shard_index(w.T, w.chunk, world, r) for r in range(world)]
+    qidx = ([np.arange(r * w.Tq // world, (r + 1) * w.Tq // world) for r in range(world)] if single
+            else kidx)
+    group = EmulatedGroup(world)
+    results, errors = [None] * world, []
+
+    def rank_main(r):
+        try:
+            torch.cuda.set_device(0)
+            st = torch.cuda.Stream()
+            with torch.cuda.stream(st):
+                dev = {}
+                for name in ("k", "v", "lr", "beta"):
+                    t = inp[name]
+                    dev[name] = None if t is None else t[:, :, kidx[r]].contiguous().cuda()
+                dev["q"] = inp["q"][:, :, qidx[r]].contiguous().cuda()
+                for name in ("w1", "w2", "w3"):
+                    dev[name] = inp[name].cuda()
+                half = lambda xs: None if xs is None else tuple((0.5 * x).cuda() for x in xs)  # noqa: E731
+                res = ct.ttt_bwd(dev["q"], dev["k"], dev["v"], dev["lr"], dev["beta"], dev["w1"], dev["w2"],
+                                 dev["w3"], w.chunk // world, w.order, w.rule,
+                                 dout[:, :, qidx[r]].contiguous().cuda(), dw_out=half(dws), update_mask=mask,
+                                 m_in=None if m_in is None else tuple(x.cuda() for x in m_in),
+                                 dm_out=half(dm), stream=st, allreduce=group.hook(r))
+                assert ct.status(st) == ct.LACT_OK
+                st.synchronize()
+                results[r] = {k_: (None if v_ is None else v_.cpu()) for k_, v_ in res.items()}
+        except BaseException as e:  # noqa: BLE001
+            errors.append(e)
+            group.barrier.abort()
+
+    threads = [threading.Thread(target=rank_main, args=(r,)) for r in range(world)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=600)
+    assert not errors, errors
+    n_upd = w.n_chunks if mask is None else sum(mask)
+    mom = w.rule == RULE_MOMENTUM
+    # recompute: each chunk's gradient (+ the beta sums); reverse loop: the own
+    # contributions before each renorm and once at the end (+ dL/dM_final)
+    assert group.calls == [2 * n_upd + 1 + (1 if mom else 0) + (1 if mom_io else 0)] * world
+    tol = TOL[w.dtype]
+    errs = {}
+    for name, idx, full in (("dq", qidx, want["dq"]), ("dk", kidx, want["dk"]), ("dv", kidx, want["dv"]),
+                            ("dlr", kidx, want["dlr"]), ("dbeta", kidx, want["dbeta"])):
+        if full is None:
+            continue
+        got = np.zeros_like(full)
+        for r in range(world):
+            got[:, :, idx[r]] = results[r][name].numpy()
+        errs[name] = rel_l2(got, full)
+    shared = ["dw1", "dw2", "dw3"] + (["dm1", "dm2", "dm3"] if mom_io else [])
+    for name in shared:
+        errs[name] = rel_l2(results[0][name].numpy(), want[name])
+        assert torch.equal(results[0][name], results[1][name]), f"{name} differs between the ranks"
+    assert max(errs.values()) <= tol, f"{w.name}: {errs}"
+    print(w.name, {k_: f"{v_:.1e}" for k_, v_ in errs.items()})
