@@ -580,15 +580,50 @@ __global__ void __launch_bounds__(256) k_ns_sumsq(const float* __restrict__ S, i
   griddep_wait();
   __shared__ float red[9];
   const int item = blockIdx.y;
-  const int64_t per = (plane + gridDim.x - 1) / gridDim.x;
-  const int64_t e0 = blockIdx.x * per, e1 = (e0 + per < plane) ? e0 + per : plane;
   const int64_t base = static_cast<int64_t>(item) * plane;
   float ss = 0.f;
-  for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
-    float s = 0.f;
-    for (int i = 0; i < splits; ++i) s += S[i * split_stride + base + e];
-    Y[base + e] = s;
-    ss += s * s;
+  if ((plane & 3) == 0 && (split_stride & 3) == 0) {
+    // 16-byte steps, four vectors in flight per thread
+    const int64_t nv = plane >> 2, sv = split_stride >> 2;
+    const int64_t per = (nv + gridDim.x - 1) / gridDim.x;
+    const int64_t v0 = blockIdx.x * per, v1 = (v0 + per < nv) ? v0 + per : nv;
+    const float4* Sv = reinterpret_cast<const float4*>(S + base);
+    float4* Yv = reinterpret_cast<float4*>(Y + base);
+    for (int64_t v = v0 + threadIdx.x; v < v1; v += 4 * 256) {
+      float4 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t vv = v + u * 256;
+        x[u] = vv < v1 ? Sv[vv] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int i = 1; i < splits; ++i) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t vv = v + u * 256;
+          if (vv < v1) {
+            const float4 y = Sv[i * sv + vv];
+            x[u].x += y.x; x[u].y += y.y; x[u].z += y.z; x[u].w += y.w;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t vv = v + u * 256;
+        if (vv < v1) {
+          Yv[vv] = x[u];
+          ss += x[u].x * x[u].x + x[u].y * x[u].y + x[u].z * x[u].z + x[u].w * x[u].w;
+        }
+      }
+    }
+  } else {
+    const int64_t per = (plane + gridDim.x - 1) / gridDim.x;
+    const int64_t e0 = blockIdx.x * per, e1 = (e0 + per < plane) ? e0 + per : plane;
+    for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
+      float s = 0.f;
+      for (int i = 0; i < splits; ++i) s += S[i * split_stride + base + e];
+      Y[base + e] = s;
+      ss += s * s;
+    }
   }
   ss = block_sum_256(ss, red);
   if (threadIdx.x == 0) part[static_cast<int64_t>(item) * gridDim.x + blockIdx.x] = ss;
@@ -609,13 +644,51 @@ __global__ void __launch_bounds__(256) k_ns_scale(float* __restrict__ Y,
     sc = 1.0f / (sqrtf(s) + eps);
   }
   __syncthreads();
-  const int64_t per = (plane + gridDim.x - 1) / gridDim.x;
-  const int64_t e0 = blockIdx.x * per, e1 = (e0 + per < plane) ? e0 + per : plane;
+  const float c = sc;
   const int64_t base = static_cast<int64_t>(item) * plane;
-  for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
-    const float y = Y[base + e] * sc;
-    Y[base + e] = y;
-    store_shadow(Yb, Yb_lo, base + e, y);
+  if ((plane & 3) == 0) {
+    // 16-byte steps, four vectors in flight per thread; the bf16 copies as 8-byte stores
+    const int64_t nv = plane >> 2;
+    const int64_t per = (nv + gridDim.x - 1) / gridDim.x;
+    const int64_t v0 = blockIdx.x * per, v1 = (v0 + per < nv) ? v0 + per : nv;
+    float4* Yv = reinterpret_cast<float4*>(Y + base);
+    for (int64_t v = v0 + threadIdx.x; v < v1; v += 4 * 256) {
+      float4 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t vv = v + u * 256;
+        x[u] = vv < v1 ? Yv[vv] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t vv = v + u * 256;
+        if (vv >= v1) continue;
+        const float4 y = make_float4(x[u].x * c, x[u].y * c, x[u].z * c, x[u].w * c);
+        Yv[vv] = y;
+        if (Yb) {
+          uint2 hi;
+          hi.x = pack_bf16x2(y.x, y.y);
+          hi.y = pack_bf16x2(y.z, y.w);
+          *reinterpret_cast<uint2*>(Yb + base + 4 * vv) = hi;
+          if (Yb_lo) {
+            const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162*>(&hi.x);
+            const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162*>(&hi.y);
+            uint2 lo;
+            lo.x = pack_bf16x2(y.x - __low2float(h0), y.y - __high2float(h0));
+            lo.y = pack_bf16x2(y.z - __low2float(h1), y.w - __high2float(h1));
+            *reinterpret_cast<uint2*>(Yb_lo + base + 4 * vv) = lo;
+          }
+        }
+      }
+    }
+  } else {
+    const int64_t per = (plane + gridDim.x - 1) / gridDim.x;
+    const int64_t e0 = blockIdx.x * per, e1 = (e0 + per < plane) ? e0 + per : plane;
+    for (int64_t e = e0 + threadIdx.x; e < e1; e += 256) {
+      const float y = Y[base + e] * c;
+      Y[base + e] = y;
+      store_shadow(Yb, Yb_lo, base + e, y);
+    }
   }
 }
 

@@ -37,7 +37,7 @@ static inline int64_t rup(int64_t a, int64_t b) { return cdiv(a, b) * b; }
 constexpr float kNsA = 3.4445f, kNsB = -4.7750f, kNsC = 2.0315f;
 constexpr int kNsSteps = 5;
 constexpr float kNsEps = 1e-7f;
-constexpr int kNsBlocks = 16;  // partial-sum blocks per matrix for ||G||_F
+constexpr int kNsBlocks = 64;  // partial-sum blocks per matrix for ||G||_F
 
 struct Dims {
   int64_t B, H, BH, T, Tq, d, dh, chunk, nch;
