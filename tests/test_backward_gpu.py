@@ -118,15 +118,18 @@ def test_backward_parity(w, kw):
     print(w.name, {k: f"{v:.1e}" for k, v in errs.items()})
 
 
-def test_backward_at_the_lm760m_shape_on_sampled_heads():
-    """The 760M LM workload (B=2, H=6, T=32768, d=256, dh=512, chunk 2048),
-    two sampled heads against the oracle; dW0 sums over the batch, so it is
-    checked on a run of those two heads' batch rows only."""
-    w = WORKLOADS[2]
-    heads = [(0, 0), (1, 5)]
+@pytest.mark.parametrize("idx", [2, 3, 4], ids=["lm760m-gd", "lm3b-momentum", "lm3b-muon"])
+def test_backward_at_full_shapes_on_sampled_heads(idx):
+    """The full LM workloads (760M: B=2, H=6, d=256, dh=512, chunk 2048, GD;
+    3B: B=1, H=8, d=384, dh=768, chunk 4096, momentum and Muon; T=32768),
+    two sampled heads against the autograd oracle on the gradients of the
+    per-token inputs (dW0 sums over the batch, and over heads that share
+    it, so it is left to the cases above)."""
+    w = WORKLOADS[idx]
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
     got, want = run_both(w, seed=0, heads=heads)
     errs = {}
-    for n in ("dq", "dk", "dv", "dlr"):
+    for n in ("dq", "dk", "dv", "dlr") + (("dbeta",) if w.rule == RULE_MOMENTUM else ()):
         g = np.stack([got[n][b, h].cpu().numpy() for b, h in heads])
         r = np.stack([want[n][b, h] for b, h in heads])
         errs[n] = rel_l2(g, r)
