@@ -14,13 +14,16 @@
 // The k^ / v tiles serve twice: as the K-major A operand of the forward and,
 // viewed MN-major (d contiguous), as the B operand of the gradients.
 //
-// Warps: 0 TMA producer, 1 TMEM allocator, 2..17 epilogue (four warps per
-// 32-lane TMEM quarter, each taking 16 of every 64 columns).  The epilogue
-// group issues the MMAs itself: after a named barrier that follows its TMEM
-// reads (or its shared-memory writes), one elected thread issues exactly the
-// MMAs those reads or writes unblocked (Z_1 after Z_0 is read; the next
-// tile's DH and Z_0 after Z_1 and DH are read; the gradients after E is
-// written), so no hand-off to another warp sits on the per-tile chain.
+// Warps: 0 TMA producer, 1 TMEM allocator and MMA issuer, 2..17 epilogue
+// (four warps per 32-lane TMEM quarter, each taking 16 of every 64
+// columns).  The issuer runs each MMA group as soon as the epilogue's
+// mbarrier arrivals free its inputs: Z_1 once Z_0 is read (zempty), the
+// next tile's DH and Z_0 once Z_1 and DH are read (zempty), the gradients
+// once E is written (efull), an item's first gradient once the previous
+// item's accumulators are read (gempty).  An MMA issue holds its thread
+// until the tensor core takes it; issued from an epilogue thread (measured:
+// about 3.6K of a tile's 7K cycles, 24 of them for the gradients alone),
+// that wait held back the whole epilogue group at its next barrier.
 #pragma once
 
 #include "apply_kernel.cuh"
@@ -74,7 +77,6 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
   uint64_t* tempty = bar + 4;       // [2]
   uint64_t* zfull = bar + 6;
   uint64_t* zempty = bar + 7;
-  uint64_t* dhempty = bar + 8;
   uint64_t* efull = bar + 9;
   uint64_t* eempty = bar + 10;
   uint64_t* gfull = bar + 11;
@@ -96,7 +98,6 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
     for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 1); }
     mbar_init(zfull, 1);
     mbar_init(zempty, kKGEpiWarps);
-    mbar_init(dhempty, kKGEpiWarps);
     mbar_init(efull, kKGEpiWarps);
     mbar_init(eempty, 1);
     mbar_init(gfull, 1);
@@ -124,6 +125,11 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
     t0 = s * tps;
     t1 = t0 + tps < p.n_tiles ? t0 + tps : p.n_tiles;
   };
+
+  constexpr uint32_t idf = idesc_bf16(kBM, 128, false, false);   // Z_h
+  constexpr uint32_t idd = idesc_bf16(kBM, 128, false, true);    // DH (W2 MN-major)
+  constexpr uint32_t idg = idesc_bf16(kBM, 64, true, true);      // gradients
+  const uint32_t sb = smem_u32(smem);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -154,13 +160,75 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
         }
       }
     }
-  } else if (warp >= 2) {
-    // ------------------------------------------------------------ epilogue + MMA issue
-    constexpr uint32_t idf = idesc_bf16(kBM, 128, false, false);   // Z_h
-    constexpr uint32_t idd = idesc_bf16(kBM, 128, false, true);    // DH (W2 MN-major)
-    constexpr uint32_t idg = idesc_bf16(kBM, 64, true, true);      // gradients
-    const uint32_t sb = smem_u32(smem);
-    const bool leader = warp == 2 && lane == 0;
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, ic = 0, zr = 0, g = 0;
+      bool ok = true;
+      // DH and Z_0 of the tile in ring slot `slot` (after its k^ / v landed)
+      auto first_half = [&](int it_) -> bool {
+        const int slot = it_ & 1;
+        if (!mbar_wait(&tfull[slot], (it_ >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
+        mma_kblock<false, true>(tmem + C::kColD, vx, 0, sb + C::kOffW2, 8192u, idd, true);
+        mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13, 0, idf, true);
+        umma_commit(zfull);
+        return true;
+      };
+      for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        int bh, s, t0, t1;
+        item_range(item, bh, s, t0, t1);
+        if (t0 >= t1) continue;
+        // the weights of this item; the Z / DH buffers free (the previous
+        // tile's last reads, zempty phase zr - 1)
+        ok = mbar_wait(wfull, ic & 1) && (zr == 0 || mbar_wait(zempty, (zr - 1) & 1)) && first_half(it);
+        for (int t = t0; ok && t < t1; ++t, ++it, ++g) {
+          const int slot = it & 1;
+          const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
+          // Z_1 once Z_0 is read
+          if (!mbar_wait(zempty, zr & 1)) { ok = false; break; }
+          ++zr;
+          tc_fence_after();
+          mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13 + 16384, 0, idf, true);
+          umma_commit(zfull);
+          // the next tile's DH and Z_0 once Z_1 and DH are read
+          if (t + 1 < t1) {
+            if (!mbar_wait(zempty, zr & 1)) { ok = false; break; }
+            ++zr;
+            if (!first_half(it + 1)) { ok = false; break; }
+          }
+          // the gradients once E is written (and, for an item's first tile,
+          // once the previous item's accumulators are read)
+          if (!mbar_wait(efull, g & 1)) { ok = false; break; }
+          const bool first = t == t0;
+          if (first && ic > 0 && !mbar_wait(gempty, (ic - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {   // two 64-token halves of the tile
+            const uint32_t ko = kk * 8192;   // 64 token rows x 128 B
+            mma_kblock<true, true>(tmem + C::kColG, sb + C::kOffE + ko, 16384u, kx + ko, 8192u, idg,
+                                   first && kk == 0);
+            mma_kblock<true, true>(tmem + C::kColG + 64, sb + C::kOffE + 2 * C::kEBytes + ko, 16384u,
+                                   kx + ko, 8192u, idg, first && kk == 0);
+            mma_kblock<true, true>(tmem + C::kColG + 128, sb + C::kOffE + C::kEBytes + ko, 16384u,
+                                   vx + ko, 8192u, idg, first && kk == 0);
+          }
+          umma_commit(eempty);
+          umma_commit(&tempty[slot]);
+          if (t == t1 - 1) {
+            umma_commit(gfull);
+            umma_commit(wempty);
+          }
+        }
+        // the last tile's second Z read frees the buffers for the next item
+        // (its zempty phase is waited at the next item's start)
+        if (ok) ++zr;
+        ++ic;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;                 // 0..15
     const int quarter = warp & 3;
     const int cg = ew >> 2;                  // which 16 of every 64 columns
@@ -169,40 +237,13 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
     const int64_t plane = 128 * 64;
     const uint32_t erow = sb + C::kOffE + r * 128;
     const uint32_t sw0 = ((2 * cg) ^ (r & 7)) << 4, sw1 = ((2 * cg + 1) ^ (r & 7)) << 4;
-    // Named barrier over the epilogue group that also ANDs everyone's `ok`:
-    // a bounded wait that gave up in any thread makes the whole group leave
-    // together, so no thread is left at a barrier the others skipped.
-    auto group_and = [](bool v) -> bool {
-      int out;
-      asm volatile(
-          "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
-          "bar.red.and.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
-          : "=r"(out)
-          : "r"(static_cast<int>(v)), "n"(kKGEpiWarps * 32)
-          : "memory");
-      return out != 0;
-    };
-    // Leader: the forward MMAs of one token tile's first half (DH and Z_0).
-    auto issue_first_half = [&](int it) -> bool {
-      const int slot = it & 1;
-      if (!mbar_wait(&tfull[slot], (it >> 1) & 1)) return false;
-      tc_fence_after();
-      const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
-      mma_kblock<false, true>(tmem + C::kColD, vx, 0, sb + C::kOffW2, 8192u, idd, true);
-      mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13, 0, idf, true);
-      umma_commit(zfull);
-      return true;
-    };
-    int it = 0, ic = 0, zc = 0, g = 0;
+    int ic = 0, zc = 0, g = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
       int bh, s, t0, t1;
       item_range(item, bh, s, t0, t1);
       if (t0 >= t1) continue;
-      if (leader) ok = mbar_wait(wfull, ic & 1) && issue_first_half(it);
-      for (int t = t0; t < t1; ++t, ++it, ++g) {
-        const int slot = it & 1;
-        const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
+      for (int t = t0; ok && t < t1; ++t, ++g) {
         const int grow = t * kBM + r;
         float eta0 = 0.f, eta1 = 0.f, eta2 = 0.f;
         if (grow < p.rows_valid) {
@@ -212,7 +253,7 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
           eta2 = l[2];
         }
         for (int h = 0; h < 2; ++h, ++zc) {
-          ok = mbar_wait(zfull, zc & 1) && ok;
+          if (!mbar_wait(zfull, zc & 1)) { ok = false; break; }
           tc_fence_after();
           float z1[16], z3[16], u[16];
           const int c = cg * 16;
@@ -222,17 +263,8 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
           tmem_ld16(tq + C::kColD + h * 64 + c, u);
           tmem_ld_wait();
           tc_fence_before();
-          ok = group_and(ok);  // every read of Z_h (and, for h = 1, of DH) is done
-          if (!ok) break;
-          if (leader) {
-            tc_fence_after();
-            if (h == 0) {  // Z_1 into the freed Z buffer
-              mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13 + 16384, 0, idf, true);
-              umma_commit(zfull);
-            } else if (t + 1 < t1) {  // the next tile's DH and Z_0
-              if (!issue_first_half(it + 1)) ok = false;
-            }
-          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(zempty);   // Z_h (and, for h = 1, DH) read
           uint32_t e1w[8], ehw[8], e3w[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -251,7 +283,7 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
             ehw[i] = pack_bf16x2(vh[0], vh[1]);
             e3w[i] = pack_bf16x2(v3[0], v3[1]);
           }
-          if (h == 0 && g > 0) ok = mbar_wait(eempty, (g - 1) & 1) && ok;
+          if (h == 0 && g > 0 && !mbar_wait(eempty, (g - 1) & 1)) { ok = false; break; }
           // Row r of MN block h of each factor; 16-byte chunk c sits at c ^ (r % 8).
           const uint32_t rb = erow + h * 16384;
           st_shared_v4(rb + sw0, e1w[0], e1w[1], e1w[2], e1w[3]);
@@ -261,33 +293,14 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
           st_shared_v4(rb + 2 * C::kEBytes + sw0, e3w[0], e3w[1], e3w[2], e3w[3]);
           st_shared_v4(rb + 2 * C::kEBytes + sw1, e3w[4], e3w[5], e3w[6], e3w[7]);
         }
-        fence_async_smem();
-        ok = group_and(ok);  // every factor of this tile is in shared memory
         if (!ok) break;
-        if (leader) {
-          tc_fence_after();
-          const bool first = t == t0;
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {   // two 64-token halves of the tile
-            const uint32_t ko = kk * 8192;   // 64 token rows x 128 B
-            mma_kblock<true, true>(tmem + C::kColG, sb + C::kOffE + ko, 16384u, kx + ko, 8192u, idg,
-                                   first && kk == 0);
-            mma_kblock<true, true>(tmem + C::kColG + 64, sb + C::kOffE + 2 * C::kEBytes + ko, 16384u,
-                                   kx + ko, 8192u, idg, first && kk == 0);
-            mma_kblock<true, true>(tmem + C::kColG + 128, sb + C::kOffE + C::kEBytes + ko, 16384u,
-                                   vx + ko, 8192u, idg, first && kk == 0);
-          }
-          umma_commit(eempty);
-          umma_commit(&tempty[slot]);
-          if (t == t1 - 1) {
-            umma_commit(gfull);
-            umma_commit(wempty);
-          }
-        }
+        fence_async_smem();   // the gradient MMAs read E through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(efull);
       }
       if (!ok) break;
       // this item's partial gradients: TMEM lane = hidden unit
-      ok = mbar_wait(gfull, ic & 1);
+      if (!mbar_wait(gfull, ic & 1)) break;
       tc_fence_after();
       const int hr = r;  // hidden row of the gradient tile
       float* base = p.P + static_cast<int64_t>(s) * 3 * p.bh_count * plane;
@@ -312,7 +325,8 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
         }
       }
       tc_fence_before();
-      ok = group_and(ok);  // the gradient accumulator may be overwritten by the next item
+      __syncwarp();
+      if (lane == 0) mbar_arrive(gempty);   // the accumulators may be overwritten by the next item
       ++ic;
     }
   }
