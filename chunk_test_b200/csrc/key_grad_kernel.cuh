@@ -14,16 +14,19 @@
 // The k^ / v tiles serve twice: as the K-major A operand of the forward and,
 // viewed MN-major (d contiguous), as the B operand of the gradients.
 //
-// Warps: 0 TMA producer, 1 TMEM allocator and MMA issuer, 2..17 epilogue
-// (four warps per 32-lane TMEM quarter, each taking 16 of every 64
-// columns).  The issuer runs each MMA group as soon as the epilogue's
-// mbarrier arrivals free its inputs: Z_1 once Z_0 is read (zempty), the
-// next tile's DH and Z_0 once Z_1 and DH are read (zempty), the gradients
-// once E is written (efull), an item's first gradient once the previous
-// item's accumulators are read (gempty).  An MMA issue holds its thread
-// until the tensor core takes it; issued from an epilogue thread (measured:
-// about 3.6K of a tile's 7K cycles, 24 of them for the gradients alone),
-// that wait held back the whole epilogue group at its next barrier.
+// Warps: 0 TMA producer, 1 TMEM allocator and forward MMA issuer, 2..17
+// epilogue (four warps per 32-lane TMEM quarter, each taking 16 of every 64
+// columns), 18 gradient MMA issuer.  Each issuer runs an MMA group as soon
+// as the epilogue's mbarrier arrivals free its inputs: warp 1 Z_1 once Z_0
+// is read (zempty) and the next tile's DH and Z_0 once Z_1 and DH are read
+// (zempty); warp 18 the gradients once E is written (efull), an item's
+// first once the previous item's accumulators are read (gempty).  An MMA
+// issue holds its thread until the tensor core takes it, and one thread
+// keeps the tensor core fed only part of the time with these small MMAs
+// (measured: about 90 cycles per N = 64 gradient MMA), so the two streams
+// come from two warps, which overlap each other's gaps; issued from an
+// epilogue thread (about 3.6K of a tile's 7K cycles) the waits held back
+// the whole epilogue group at its next barrier.
 #pragma once
 
 #include "apply_kernel.cuh"
@@ -45,7 +48,8 @@ struct KeyGradParams {
   float* P;           // partial gradients [splits][3][BH][plane], W2's in [d, dh]
 };
 
-constexpr int kKGThreads = 576;   // 18 warps
+constexpr int kKGThreads = 608;   // 19 warps
+constexpr int kKGGradWarp = 18;
 constexpr int kKGEpiWarps = 16;
 
 struct KGCfg {
@@ -95,7 +99,8 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
   if (warp == 0 && lane == 0) {
     mbar_init(wfull, 1);
     mbar_init(wempty, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 1); }
+    // a ring slot is free once both issuers' MMAs that read it are done
+    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 2); }
     mbar_init(zfull, 1);
     mbar_init(zempty, kKGEpiWarps);
     mbar_init(efull, kKGEpiWarps);
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int it = 0, ic = 0, zr = 0, g = 0;
+      int it = 0, ic = 0, zr = 0;
       bool ok = true;
       // DH and Z_0 of the tile in ring slot `slot` (after its k^ / v landed)
       auto first_half = [&](int it_) -> bool {
@@ -183,26 +188,51 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
         // the weights of this item; the Z / DH buffers free (the previous
         // tile's last reads, zempty phase zr - 1)
         ok = mbar_wait(wfull, ic & 1) && (zr == 0 || mbar_wait(zempty, (zr - 1) & 1)) && first_half(it);
-        for (int t = t0; ok && t < t1; ++t, ++it, ++g) {
+        for (int t = t0; ok && t < t1; ++t, ++it) {
           const int slot = it & 1;
-          const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
+          const uint32_t kx = sb + C::kOffRing + slot * C::kSlot;
           // Z_1 once Z_0 is read
           if (!mbar_wait(zempty, zr & 1)) { ok = false; break; }
           ++zr;
           tc_fence_after();
           mma_kblock<false, false>(tmem + C::kColZ, kx, 0, sb + C::kOffW13 + 16384, 0, idf, true);
           umma_commit(zfull);
+          umma_commit(&tempty[slot]);          // this issuer's reads of the slot are issued
+          if (t == t1 - 1) umma_commit(wempty);  // and of the item's weights
           // the next tile's DH and Z_0 once Z_1 and DH are read
           if (t + 1 < t1) {
             if (!mbar_wait(zempty, zr & 1)) { ok = false; break; }
             ++zr;
             if (!first_half(it + 1)) { ok = false; break; }
           }
-          // the gradients once E is written (and, for an item's first tile,
-          // once the previous item's accumulators are read)
-          if (!mbar_wait(efull, g & 1)) { ok = false; break; }
+        }
+        // the last tile's second Z read frees the buffers for the next item
+        // (its zempty phase is waited at the next item's start)
+        if (ok) ++zr;
+        ++ic;
+      }
+    }
+  } else if (warp == kKGGradWarp) {
+    // ------------------------------------------------------------ gradient MMA issuer
+    if (lane == 0) {
+      int it = 0, ic = 0, g = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        int bh, s, t0, t1;
+        item_range(item, bh, s, t0, t1);
+        if (t0 >= t1) continue;
+        for (int t = t0; ok && t < t1; ++t, ++it, ++g) {
+          const int slot = it & 1;
+          const uint32_t kx = sb + C::kOffRing + slot * C::kSlot, vx = kx + 16384;
           const bool first = t == t0;
-          if (first && ic > 0 && !mbar_wait(gempty, (ic - 1) & 1)) { ok = false; break; }
+          // E written; the slot's k^ / v landed (its phase is already
+          // complete: the epilogue read this tile's Z); for an item's first
+          // tile, the previous item's accumulators read
+          if (!mbar_wait(efull, g & 1) || !mbar_wait(&tfull[slot], (it >> 1) & 1) ||
+              (first && ic > 0 && !mbar_wait(gempty, (ic - 1) & 1))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {   // two 64-token halves of the tile
@@ -216,14 +246,8 @@ __global__ void __launch_bounds__(kKGThreads, 1) k_key_grad64(const __grid_const
           }
           umma_commit(eempty);
           umma_commit(&tempty[slot]);
-          if (t == t1 - 1) {
-            umma_commit(gfull);
-            umma_commit(wempty);
-          }
+          if (t == t1 - 1) umma_commit(gfull);
         }
-        // the last tile's second Z read frees the buffers for the next item
-        // (its zempty phase is waited at the next item's start)
-        if (ok) ++zr;
         ++ic;
       }
     }
