@@ -86,7 +86,10 @@ def test_roofline_entry_divides_by_the_burst_peak(tmp_path, monkeypatch):
 
 
 def test_measured_peaks_file_holds_the_burst_and_sustained_figures():
-    with open(bench.os.path.join(bench.ROOT, "MEASURED_PEAKS.json")) as f:
+    path = bench.os.path.join(bench.ROOT, "MEASURED_PEAKS.json")
+    if not bench.os.path.exists(path):
+        pytest.skip("no measured peaks on this machine (the bench then uses its stated fallback)")
+    with open(path) as f:
         p = json.load(f)
     hbm, burst, sust, src = bench.peaks()
     assert src == "measured" and burst == p["bf16_tflops"] and sust == p["bf16_tflops_sustained"]
